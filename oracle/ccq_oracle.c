@@ -19,6 +19,7 @@
 #include <stdlib.h>
 #include <string.h>
 #include <fenv.h>
+#include <limits.h>
 
 /* ------------------------------------------------------------------------------------------
  * Convolutional-code codebook, [CCQ] §3.1 "Definition of Convolutional Code Codebook", Fig. 1.
@@ -95,9 +96,11 @@ float oracle_bf16_to_float(uint16_t b)
 int32_t oracle_cluster_code(uint8_t q, float code_scale, float code_zero)
 {
     float t = fmaf((float)q, code_scale, code_zero);
-    if (!(t == t)) return 0; /* NaN: not produced by any encoder; defined as code 0 */
-    if (t >= 2147483520.0f) return (int32_t)0x7FFFFF80; /* largest float below 2^31 */
-    if (t <= -2147483648.0f) return (int32_t)0x80000000;
+    /* Outside the int32 range (never produced by an encoder) the rounded value saturates to the
+     * nearest int32 and NaN gives 0; only the low 15 bits of the code are used afterwards. */
+    if (!(t == t)) return 0;
+    if (t >= 2147483648.0f) return INT32_MAX;
+    if (t < -2147483648.0f) return INT32_MIN;
     int old = fegetround();
     fesetround(FE_TONEAREST);
     float r = nearbyintf(t);
