@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Benchmark: one CCQ W2A16 MoE FFN layer, decode-sized (32 tokens, hidden 8192, 64 experts of
+gate/up 8192x3584x2 and down 3584x8192, all CCQ W2 group 64, top-8 uniform routing with softmax
+weights from N(0,1) logits, SiLU-gated, BF16 activations).
+
+A step is one full layer forward through the C ABI (routing, activation packing, gate/up matmul
+with the SiLU gate, group sums, down matmul with routing weights, top-k combine) over one batch.
+`value` is whole-job tokens/s (every rank runs its own replica of the layer: the path has no
+exchange step), timed with CUDA events over exactly --steps steps after --warmup steps, max over
+ranks.  `--impl reference` times the CPU oracle on a bounded sample of the same workload.
+
+Launch: python bench.py --gpus N --steps K --warmup W  (N > 1: under torch.distributed.run).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+T, H, I, E, TOPK = 32, 8192, 3584, 64, 8
+DISTINCT = 2          # experts encoded from N(0, 0.02) weights; the rest are device copies of them
+NOMINAL_HBM_GBS = 8000.0
+METRIC = "W2A16 MoE layer tokens/s; packed-weight HBM GB/s (% of 8 TB/s), 1 B200"
+WORKLOAD = "moe_ffn_decode_T32_H8192_I3584_E64_top8_ccq_w2_g64"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def config_dict():
+    return {
+        "workload": WORKLOAD,
+        "tokens": T, "hidden": H, "intermediate": I, "experts": E, "topk": TOPK,
+        "weight_format": "CCQ (6,4,3) code cluster, 4 weights/byte, fp32 group-64 scales",
+        "routing": "uniform distinct top-8, softmax of N(0,1) logits",
+        "weights": f"N(0,0.02) encoded by ccq_encode_host for {DISTINCT} experts, copied to all {E}",
+        "l2": "inputs larger than L2: ~1.74 GB of packed weights touched per step vs 126 MB L2",
+        "parallelism": "replicas",
+    }
+
+
+# ------------------------------------------------------------------------------------------------
+# inputs
+# ------------------------------------------------------------------------------------------------
+def make_layer(ccq, torch, device):
+    import synth
+
+    def enc(rows, cols, seed):
+        w = synth.weights_normal(rows, cols, seed)
+        c, s, a, b, _ = ccq.ccq_encode_host(w, 64, 0, 0)
+        return c, s, a, b
+
+    parts13 = [enc(2 * I, H, 3100 + e) for e in range(DISTINCT)]
+    parts2 = [enc(H, I, 3200 + e) for e in range(DISTINCT)]
+
+    def stack(parts, n, k):
+        codes = torch.empty((E * n, k // 4), dtype=torch.uint8, device=device)
+        scales = torch.empty((E * n, k // 64), dtype=torch.float32, device=device)
+        alpha = torch.empty((E * n,), dtype=torch.float32, device=device)
+        beta = torch.empty((E * n,), dtype=torch.float32, device=device)
+        dev = [tuple(torch.from_numpy(a).to(device) for a in p) for p in parts]
+        for e in range(E):
+            c, s, a, b = dev[e % len(dev)]
+            codes[e * n:(e + 1) * n].copy_(c)
+            scales[e * n:(e + 1) * n].copy_(s)
+            alpha[e * n:(e + 1) * n].copy_(a)
+            beta[e * n:(e + 1) * n].copy_(b)
+        return ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, n, k, codes, scales, alpha, beta, experts=E, device=device)
+
+    W13 = stack(parts13, 2 * I, H)
+    W2 = stack(parts2, H, I)
+    return W13, W2
+
+
+def touched_bytes(ids):
+    """Algorithmic packed-weight bytes of one step: codes + scales + alpha/beta of touched experts."""
+    per13 = 2 * I * (H // 4) + 2 * I * (H // 64) * 4 + 2 * I * 8
+    per2 = H * (I // 4) + H * (I // 64) * 4 + H * 8
+    ne = len(set(int(v) for v in np.asarray(ids).ravel()))
+    return ne * per13, ne * per2, ne
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of the same layer
+# ------------------------------------------------------------------------------------------------
+def oracle_sample(n_experts: int = 1):
+    """Time the oracle on `n_experts` experts of the decode layer (decode their weights, run every
+    (token, expert) pair routed to them), and scale to the layer by the touched-expert count."""
+    import oracle
+    import synth
+
+    x = synth.activations(T, H, 3302)
+    ids, rw = synth.routing_uniform(T, E, TOPK, 3303)
+    xb = synth.bf16_bits(x)
+    touched = sorted(set(int(v) for v in ids.ravel()))
+    c13, s13, a13, b13 = synth.w2_format_random(2 * I, H, 3304)
+    c2, s2, a2, b2 = synth.w2_format_random(H, I, 3305)
+    pairs = 0
+    t0 = time.perf_counter()
+    for e in touched[:n_experts]:
+        d13 = oracle.dequant_w2(c13, s13, a13, b13)
+        d2 = oracle.dequant_w2(c2, s2, a2, b2)
+        toks = [t for t in range(T) if e in ids[t]]
+        pairs += len(toks)
+        out = oracle.expert_ffn_f64(xb[toks], d13, d2, round_h=True)
+        del out
+    dt = time.perf_counter() - t0
+    layer_s = dt * len(touched) / n_experts
+    cores = os.cpu_count() or 1
+    sample = (f"{n_experts} of {len(touched)} touched experts ({pairs} of {T * TOPK} token-expert pairs): "
+              f"oracle decode + fp64 expert FFN, scaled by touched experts")
+    return T / layer_s, cores, sample, dt
+
+
+# ------------------------------------------------------------------------------------------------
+# reference arm (the oracle, on host cores)
+# ------------------------------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, cores, sample, dt = oracle_sample(1)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * T / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------------
+def run_ours(args, rank, world, local):
+    import torch
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        pg = dist
+    import extreme_bit_weight_b200 as ccq
+    import synth
+
+    # CPU baseline first (rank 0, N = 1 only), before any large GPU allocation
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        oracle.build()
+        v, cores, sample, dt = oracle_sample(2)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    W13, W2 = make_layer(ccq, torch, device)
+    x_host = synth.activations(T, H, 3002 + 17 * rank)
+    ids_np, rw_np = synth.routing_uniform(T, E, TOPK, 3003 + 17 * rank)
+    x = x_host.to(device)
+    ids = torch.from_numpy(ids_np).to(device)
+    rw = torch.from_numpy(rw_np).to(device)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+    ws = ccq.workspace(ccq.ccq_moe_workspace_size(T, TOPK, H, I, E), device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        ccq.ccq_moe_w2a16_forward(W13, W2, x, ids, rw, y=y, ws=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    assert ccq.ccq_check_device_error(ws, stream) == ccq.CCQ_OK
+
+    # ---- device-timed region: exactly K steps, events around every step's kernels ----
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ccq.CCQ_MOE_TRACE_POINTS)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(device)
+    clocks.start()
+    time.sleep(0.3)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(K):
+        ccq.ccq_moe_w2a16_forward_traced(W13, W2, x, ids, rw, y, ws, evs[k], stream=stream)
+    stop.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    if pg:
+        pg.barrier()
+    total_ms = start.elapsed_time(stop)
+    gemm1_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    gemm2_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in evs)
+    if pg:
+        t = torch.tensor([total_ms], device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    value = world * T / (ms_per_step * 1e-3)
+
+    # ---- end to end: pinned host inputs in, result out, through the same public call ----
+    xp = x_host.pin_memory()
+    idp = torch.from_numpy(ids_np).pin_memory()
+    rwp = torch.from_numpy(rw_np).pin_memory()
+    yp = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    K2 = max(1, min(K, 500))
+
+    def e2e_step():
+        x.copy_(xp, non_blocking=True)
+        ids.copy_(idp, non_blocking=True)
+        rw.copy_(rwp, non_blocking=True)
+        step()
+        yp.copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    if pg:
+        pg.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(K2):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = a.elapsed_time(b) / K2
+    if pg:
+        t = torch.tensor([e2e_ms], device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = xp.numel() * 2 + idp.numel() * 4 + rwp.numel() * 4
+    d2h = yp.numel() * 2
+
+    b13, b2, ne = touched_bytes(ids_np)
+    hbm, src = peaks()
+    ach13 = b13 / (gemm1_ms * 1e-3) / 1e9
+    layer_gbs = (b13 + b2) / (ms_per_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(),
+        "packed_weight_gbs": layer_gbs, "packed_weight_pct_of_8tbs": 100.0 * layer_gbs / NOMINAL_HBM_GBS,
+        "touched_experts": ne,
+        "roofline": {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (gate/up, SiLU epilogue)",
+                     "achieved": ach13, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "unit": "GB/s",
+                     "frac": ach13 / hbm, "traffic": None, "launch_ms": gemm1_ms,
+                     "algorithmic_bytes_per_launch": b13,
+                     "down_kernel": {"achieved": b2 / (gemm2_ms * 1e-3) / 1e9, "launch_ms": gemm2_ms,
+                                     "algorithmic_bytes_per_launch": b2}},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 6 * K,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

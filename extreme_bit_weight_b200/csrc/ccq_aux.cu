@@ -1,0 +1,267 @@
+// Auxiliary kernels of libccq (sm_100a): exact BF16 dequantization (inspection / tests),
+// activation packing into the decode-sized kernel's operand layout, split-K reduction, and the
+// MoE routing / combine steps around the expert matmuls.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ccq.h"
+#include "ccq_device.cuh"
+#include "ccq_kernels.cuh"
+
+namespace ccq {
+namespace {
+
+// ------------------------------------------------------------------------------------------------
+// Exact dequantization (CCQ §3.5 Algorithm 3 for W2; signed nibbles for W4).  One thread per
+// stored byte.  The code is rounded with cvt.rni (round to nearest even, saturating at the int32
+// range, NaN -> 0), so this kernel is exact for any alpha/beta, unlike the fast path.
+// ------------------------------------------------------------------------------------------------
+__global__ void dequant_w2_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales,
+                                  const float *__restrict__ alpha, const float *__restrict__ beta, int rows,
+                                  int K, uint16_t *__restrict__ out) {
+    const size_t nbytes = (size_t)rows * (K / 4);
+    const int kb = K / 4, ng = K / 64;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < nbytes;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int r = (int)(idx / kb), j = (int)(idx % kb);
+        const float t = __fmaf_rn((float)codes[idx], __ldg(alpha + r), __ldg(beta + r));
+        const uint32_t C = (uint32_t)__float2int_rn(t);
+        const float s = bf16_bits_to_float(float_to_bf16_bits(__ldg(scales + (size_t)r * ng + (4 * j) / 64)));
+        uint16_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int u = (int)((C >> (9 - 3 * i)) & 0x3Fu);
+            o[i] = float_to_bf16_bits(__fmul_rn((float)(u - 32), s));
+        }
+        uint2 v;
+        v.x = (uint32_t)o[0] | ((uint32_t)o[1] << 16);
+        v.y = (uint32_t)o[2] | ((uint32_t)o[3] << 16);
+        *reinterpret_cast<uint2 *>(out + (size_t)r * K + 4 * j) = v;
+    }
+}
+
+__global__ void dequant_w4_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales, int rows,
+                                  int K, uint16_t *__restrict__ out) {
+    const size_t nbytes = (size_t)rows * (K / 2);
+    const int kb = K / 2;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < nbytes;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int r = (int)(idx / kb), j = (int)(idx % kb);
+        const uint32_t b = codes[idx];
+        const float s = bf16_bits_to_float(float_to_bf16_bits(__ldg(scales + r)));
+        const int q0 = (int)((b & 0xFu) ^ 8u) - 8, q1 = (int)((b >> 4) ^ 8u) - 8;
+        const uint32_t v = (uint32_t)float_to_bf16_bits(__fmul_rn((float)q0, s)) |
+                           ((uint32_t)float_to_bf16_bits(__fmul_rn((float)q1, s)) << 16);
+        *reinterpret_cast<uint32_t *>(out + (size_t)r * K + 2 * j) = v;
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Activation operand packing.  One thread per (operand row p, 64-column group G): reads the
+// group's 64 BF16 values of source row tok_of[p] (or p), writes them in the XA order and the
+// group sum -160 * sum (fp32, summed in column order).
+// ------------------------------------------------------------------------------------------------
+__global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__restrict__ tok_of, int P_valid,
+                               int P, int K, uint16_t *__restrict__ xa, float *__restrict__ gsum) {
+    const int ng = K / 64, ld = gsum_ld(K);
+    const size_t total = (size_t)P_valid * ng;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int pr = (int)(idx / ng), G = (int)(idx % ng);
+        const int src = tok_of ? __ldg(tok_of + pr) : pr;
+        const uint4 *row = reinterpret_cast<const uint4 *>(x + (size_t)src * K + (size_t)G * 64);
+        uint16_t v[64];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            uint4 w = __ldg(row + q);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                v[q * 8 + 2 * h] = (uint16_t)(ws[h] & 0xFFFFu);
+                v[q * 8 + 2 * h + 1] = (uint16_t)(ws[h] >> 16);
+            }
+        }
+        float sum = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 64; ++k) sum += bf16_bits_to_float(v[k]);
+        gsum[(size_t)pr * ld + G] = -160.0f * sum;
+        // 16 runs of 4 values: (i, tig) -> j = 0..3 contiguous
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int tig = 0; tig < 4; ++tig) {
+                uint2 o;
+                o.x = (uint32_t)v[16 * tig + 0 + i] | ((uint32_t)v[16 * tig + 4 + i] << 16);
+                o.y = (uint32_t)v[16 * tig + 8 + i] | ((uint32_t)v[16 * tig + 12 + i] << 16);
+                *reinterpret_cast<uint2 *>(xa + xa_index((size_t)pr, (size_t)G * 64 + 16 * tig + i, (size_t)P)) = o;
+            }
+    }
+}
+
+__global__ void gsum_from_xa_kernel(const uint16_t *__restrict__ xa, int P_valid, int P, int K,
+                                    float *__restrict__ gsum) {
+    const int ng = K / 64, ld = gsum_ld(K);
+    const size_t total = (size_t)P_valid * ng;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int pr = (int)(idx / ng), G = (int)(idx % ng);
+        float sum = 0.0f;
+        for (int k = 0; k < 64; ++k)
+            sum += bf16_bits_to_float(xa[xa_index((size_t)pr, (size_t)G * 64 + k, (size_t)P)]);
+        gsum[(size_t)pr * ld + G] = -160.0f * sum;
+    }
+}
+
+__global__ void splitk_reduce_kernel(const float *__restrict__ partial, int ksplit, size_t split_stride, int M,
+                                     int N, uint16_t *__restrict__ y) {
+    const size_t total = (size_t)M * N;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        float s = 0.0f;
+        for (int k = 0; k < ksplit; ++k) s += partial[(size_t)k * split_stride + idx];
+        y[idx] = float_to_bf16_bits(s);
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// MoE routing.  One CTA.  Pass 1 validates each (token, slot) pair (expert id in [0,E) and not a
+// repeat within its token) and counts pairs per expert; a scan gives each expert's contiguous
+// segment of operand rows; pass 2 places each valid pair in its expert's segment.  The order
+// inside a segment does not affect any result (every operand row is computed independently).
+// Invalid pairs get inv = -1 and are reported in the error word.
+// ------------------------------------------------------------------------------------------------
+__global__ void moe_route_kernel(const int *__restrict__ ids, const float *__restrict__ rw, int T, int topk,
+                                 int E, int *__restrict__ seg_off, int *__restrict__ cursor,
+                                 int *__restrict__ tok_of, float *__restrict__ rw_perm, int *__restrict__ inv,
+                                 uint32_t *err) {
+    extern __shared__ int sh[];
+    int *cnt = sh;          // [E]
+    int *off = sh + E;      // [E+1]
+    for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    const int npairs = T * topk;
+    for (int q = threadIdx.x; q < npairs; q += blockDim.x) {
+        const int t = q / topk, j = q % topk;
+        const int e = ids[q];
+        bool ok = (e >= 0 && e < E);
+        if (!ok) record_error(err, DEV_ERR_BAD_EXPERT, (uint32_t)q);
+        if (ok)
+            for (int jj = 0; jj < j; ++jj)
+                if (ids[t * topk + jj] == e) {
+                    ok = false;
+                    record_error(err, DEV_ERR_DUP_EXPERT, (uint32_t)q);
+                    break;
+                }
+        inv[q] = ok ? -2 : -1;  // -2: valid, not yet placed
+        if (ok) atomicAdd(&cnt[e], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int s = 0;
+        for (int i = 0; i < E; ++i) {
+            off[i] = s;
+            s += cnt[i];
+        }
+        off[E] = s;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) seg_off[i] = off[i];
+    for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    for (int q = threadIdx.x; q < npairs; q += blockDim.x) {
+        if (inv[q] != -2) continue;
+        const int e = ids[q];
+        const int pos = off[e] + atomicAdd(&cnt[e], 1);
+        tok_of[pos] = q / topk;
+        rw_perm[pos] = rw[q];
+        inv[q] = pos;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < E; i += blockDim.x) cursor[i] = cnt[i];
+}
+
+// y[t] = bf16( sum_j slot[inv[t][j]] ), fixed j order, fp32; invalid pairs skipped.
+__global__ void moe_combine_kernel(const float *__restrict__ slot, const int *__restrict__ inv, int T, int topk,
+                                   int H, uint16_t *__restrict__ y) {
+    const int H4 = H / 4;
+    const size_t total = (size_t)T * H4;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int t = (int)(idx / H4), c4 = (int)(idx % H4);
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < topk; ++j) {
+            const int pr = __ldg(inv + t * topk + j);
+            if (pr < 0) continue;
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(slot + (size_t)pr * H) + c4);
+            s.x += v.x;
+            s.y += v.y;
+            s.z += v.z;
+            s.w += v.w;
+        }
+        uint2 o;
+        o.x = pack_bf16x2(s.x, s.y);
+        o.y = pack_bf16x2(s.z, s.w);
+        *reinterpret_cast<uint2 *>(y + (size_t)t * H + 4 * c4) = o;
+    }
+}
+
+inline int grid_for(size_t work, int threads) {
+    size_t b = (work + threads - 1) / threads;
+    if (b > 148 * 16) b = 148 * 16;
+    return b < 1 ? 1 : (int)b;
+}
+
+}  // namespace
+
+cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, const float *alpha,
+                           const float *beta, int rows, int K, uint16_t *out, cudaStream_t s) {
+    if (rows == 0) return cudaSuccess;
+    if (fmt == CCQ_FMT_W2_CCQ_G64) {
+        dequant_w2_kernel<<<grid_for((size_t)rows * K / 4, 256), 256, 0, s>>>(codes, scales, alpha, beta, rows, K, out);
+    } else {
+        dequant_w4_kernel<<<grid_for((size_t)rows * K / 2, 256), 256, 0, s>>>(codes, scales, rows, K, out);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, uint16_t *xa,
+                           float *gsum, cudaStream_t s) {
+    if (P_valid <= 0) return cudaSuccess;
+    pack_xa_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(x, tok_of, P_valid, P, K, xa, gsum);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float *gsum, cudaStream_t s) {
+    if (P_valid <= 0) return cudaSuccess;
+    gsum_from_xa_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(xa, P_valid, P, K, gsum);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_splitk_reduce(const float *partial, int ksplit, size_t split_stride, int M, int N,
+                                 uint16_t *y, cudaStream_t s) {
+    if ((size_t)M * N == 0) return cudaSuccess;
+    splitk_reduce_kernel<<<grid_for((size_t)M * N, 256), 256, 0, s>>>(partial, ksplit, split_stride, M, N, y);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_moe_route(const int *ids, const float *rw, int T, int topk, int E, int *seg_off, int *cursor,
+                             int *tok_of, float *rw_perm, int *inv, uint32_t *err, cudaStream_t s) {
+    const size_t sh = sizeof(int) * (2 * (size_t)E + 1);
+    if (sh > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
+        if (e != cudaSuccess) return e;
+    }
+    moe_route_kernel<<<1, 1024, sh, s>>>(ids, rw, T, topk, E, seg_off, cursor, tok_of, rw_perm, inv, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_moe_combine(const float *slot, const int *inv, int T, int topk, int H, uint16_t *y,
+                               cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    moe_combine_kernel<<<grid_for((size_t)T * (H / 4), 256), 256, 0, s>>>(slot, inv, T, topk, H, y);
+    return cudaGetLastError();
+}
+
+}  // namespace ccq

@@ -1,0 +1,371 @@
+// C ABI of libccq: argument validation, workspace layout, TMA descriptor encoding and dispatch.
+// Declarations and the contract of every entry point are in include/ccq.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "../../include/ccq.h"
+#include "ccq_device.cuh"
+#include "ccq_kernels.cuh"
+
+using namespace ccq;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const cuuint64_t *dims,
+              const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+ccq_status check_weight(const ccq_weight *w, int experts) {
+    if (!w || experts <= 0) return CCQ_ERR_INVALID_ARG;
+    if (w->fmt != CCQ_FMT_W2_CCQ_G64 && w->fmt != CCQ_FMT_W4_PER_CHANNEL) return CCQ_ERR_UNSUPPORTED;
+    if (w->n <= 0 || w->k <= 0 || w->n % 16 || w->k % 64) return CCQ_ERR_INVALID_ARG;
+    if (!w->codes || !w->scales || !aligned16(w->codes) || !aligned16(w->scales)) return CCQ_ERR_INVALID_ARG;
+    if (w->fmt == CCQ_FMT_W2_CCQ_G64) {
+        if (w->group != 64) return CCQ_ERR_UNSUPPORTED;
+        if (!w->alpha || !w->beta) return CCQ_ERR_INVALID_ARG;
+    }
+    if ((size_t)experts * w->n > (size_t)INT32_MAX) return CCQ_ERR_INVALID_ARG;
+    return CCQ_OK;
+}
+
+// --- decode-sized path ----------------------------------------------------------------------
+int pick_nt(double rows_per_expert) {
+    if (rows_per_expert <= 8.0) return 1;
+    if (rows_per_expert <= 16.0) return 2;
+    return 4;
+}
+
+struct DecodeMaps {
+    CUtensorMap codes, xa, gs;
+};
+
+bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t *xa, const float *gs, int P,
+                 int nt) {
+    const int K = w->k;
+    const cuuint64_t rows = (cuuint64_t)experts * w->n;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)(K / 4), rows};
+        cuuint64_t str[1] = {(cuuint64_t)(K / 4)};
+        cuuint32_t box[2] = {128, 128};
+        if (!make_map(&m.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w->codes, dims, str, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return false;
+    }
+    {
+        cuuint64_t dims[3] = {16, (cuuint64_t)P, (cuuint64_t)(K / 16)};
+        cuuint64_t str[2] = {32, (cuuint64_t)P * 32};
+        cuuint32_t box[3] = {16, (cuuint32_t)(8 * nt), 32};
+        if (!make_map(&m.xa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, xa, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return false;
+    }
+    {
+        const int ld = gsum_ld(K);
+        cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)P};
+        cuuint64_t str[1] = {(cuuint64_t)ld * 4};
+        cuuint32_t box[2] = {8, (cuuint32_t)(8 * nt)};
+        if (!make_map(&m.gs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, gs, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return false;
+    }
+    return true;
+}
+
+struct GemmWs {
+    size_t xa, gs, partial, total;
+    int P, ksplit, spp, row_blocks, nt;
+};
+
+GemmWs gemm_layout(const ccq_weight *w, int m) {
+    GemmWs L{};
+    L.P = (m + 3) & ~3;
+    L.nt = pick_nt((double)m);
+    const int K = w->k, N = w->n;
+    const int nst = ceil_div(K, 512);
+    L.row_blocks = ceil_div(N, 256);
+    int want = std::max(1, ceil_div(2 * 148, L.row_blocks));
+    want = std::min(want, nst);
+    L.spp = ceil_div(nst, want);
+    L.ksplit = ceil_div(nst, L.spp);
+    size_t off = 0;
+    L.xa = off;
+    off = up256(off + (size_t)L.P * K * 2);
+    L.gs = off;
+    off = up256(off + (size_t)L.P * gsum_ld(K) * 4);
+    L.partial = off;
+    if (L.ksplit > 1) off = up256(off + (size_t)L.ksplit * m * N * 4);
+    L.total = off;
+    return L;
+}
+
+struct MoeWs {
+    size_t err, seg, cursor, tok, rwp, inv, xa_x, gs_x, xa_h, gs_h, slot, total;
+    int P;
+};
+
+MoeWs moe_layout(int T, int topk, int H, int I, int E) {
+    MoeWs L{};
+    const int pairs = T * topk;
+    L.P = (pairs + 3) & ~3;
+    size_t off = 0;
+    L.err = off; off = up256(off + 16);
+    L.seg = off; off = up256(off + sizeof(int) * (size_t)(E + 1));
+    L.cursor = off; off = up256(off + sizeof(int) * (size_t)E);
+    L.tok = off; off = up256(off + sizeof(int) * (size_t)L.P);
+    L.rwp = off; off = up256(off + sizeof(float) * (size_t)L.P);
+    L.inv = off; off = up256(off + sizeof(int) * (size_t)pairs);
+    L.xa_x = off; off = up256(off + (size_t)L.P * H * 2);
+    L.gs_x = off; off = up256(off + (size_t)L.P * gsum_ld(H) * 4);
+    L.xa_h = off; off = up256(off + (size_t)L.P * I * 2);
+    L.gs_h = off; off = up256(off + (size_t)L.P * gsum_ld(I) * 4);
+    L.slot = off; off = up256(off + (size_t)L.P * H * 4);
+    L.total = off;
+    return L;
+}
+
+inline ccq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CCQ_OK : CCQ_ERR_CUDA; }
+
+inline cudaError_t trace(void *const *events, int i, cudaStream_t s) {
+    if (!events || !events[i]) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ccq_status_string(ccq_status s) {
+    switch (s) {
+        case CCQ_OK: return "ok";
+        case CCQ_ERR_INVALID_ARG: return "invalid argument";
+        case CCQ_ERR_UNSUPPORTED: return "unsupported format or shape";
+        case CCQ_ERR_CUDA: return "CUDA runtime error";
+        case CCQ_ERR_DEVICE_CHECK: return "device-side check failed (invalid routing entry)";
+        case CCQ_ERR_TIMEOUT: return "bounded device wait timed out";
+    }
+    return "unknown status";
+}
+
+const char *ccq_build_info(void) {
+    return "libccq: sm_100a; decode-sized path = register decode -> mma.sync m16n8k16 bf16, TMA-staged";
+}
+
+ccq_status ccq_dequant_bf16(const ccq_weight *w, int32_t num_experts, void *out_bf16, ccq_stream_t stream) {
+    ccq_status st = check_weight(w, num_experts);
+    if (st != CCQ_OK) return st;
+    if (!out_bf16 || !aligned16(out_bf16)) return CCQ_ERR_INVALID_ARG;
+    return cuda_status(launch_dequant(w->fmt, w->codes, w->scales, w->alpha, w->beta, num_experts * w->n, w->k,
+                                      static_cast<uint16_t *>(out_bf16), (cudaStream_t)stream));
+}
+
+size_t ccq_gemm_workspace_size(const ccq_weight *w, int32_t m) {
+    if (!w || m <= 0 || w->n <= 0 || w->k <= 0) return 0;
+    return gemm_layout(w, m).total;
+}
+
+ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, void *y_bf16, void *ws,
+                          size_t ws_bytes, ccq_stream_t stream) {
+    ccq_status st = check_weight(w, 1);
+    if (st != CCQ_OK) return st;
+    if (m < 0) return CCQ_ERR_INVALID_ARG;
+    if (m == 0) return CCQ_OK;
+    if (!x_bf16 || !y_bf16 || !aligned16(x_bf16) || !aligned16(y_bf16)) return CCQ_ERR_INVALID_ARG;
+    if (w->fmt != CCQ_FMT_W2_CCQ_G64) return CCQ_ERR_UNSUPPORTED;
+    const GemmWs L = gemm_layout(w, m);
+    if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return CCQ_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    uint16_t *xa = reinterpret_cast<uint16_t *>(base + L.xa);
+    float *gs = reinterpret_cast<float *>(base + L.gs);
+    cudaError_t e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), nullptr, m, L.P, w->k, xa, gs, s);
+    if (e != cudaSuccess) return CCQ_ERR_CUDA;
+    DecodeMaps maps;
+    if (!decode_maps(maps, w, 1, xa, gs, L.P, L.nt)) return CCQ_ERR_CUDA;
+    DecodeGemmParams p{};
+    p.scales = w->scales;
+    p.alpha = w->alpha;
+    p.beta = w->beta;
+    p.N = w->n;
+    p.K = w->k;
+    p.row_block_stride = 256;
+    p.half_stride = 128;
+    p.num_stages = ceil_div(w->k, 512);
+    p.stages_per_split = L.spp;
+    p.seg_off = nullptr;
+    p.M = m;
+    p.P = L.P;
+    p.out_ld = w->n;
+    p.err = nullptr;
+    if (L.ksplit > 1) {
+        p.mode = EPI_PARTIAL_F32;
+        p.out = base + L.partial;
+        p.out_split_stride = (size_t)m * w->n;
+    } else {
+        p.mode = EPI_BF16;
+        p.out = y_bf16;
+    }
+    e = launch_decode_gemm_w2(p, maps.codes, maps.xa, maps.gs, L.row_blocks, L.ksplit, 1, L.nt, s);
+    if (e != cudaSuccess) return CCQ_ERR_CUDA;
+    if (L.ksplit > 1) {
+        e = launch_splitk_reduce(reinterpret_cast<const float *>(base + L.partial), L.ksplit, (size_t)m * w->n, m,
+                                 w->n, static_cast<uint16_t *>(y_bf16), s);
+        if (e != cudaSuccess) return CCQ_ERR_CUDA;
+    }
+    return CCQ_OK;
+}
+
+size_t ccq_moe_workspace_size(int32_t T, int32_t topk, int32_t H, int32_t I, int32_t num_experts) {
+    if (T <= 0 || topk <= 0 || H <= 0 || I <= 0 || num_experts <= 0) return 0;
+    return moe_layout(T, topk, H, I, num_experts).total;
+}
+
+ccq_status ccq_moe_w2a16_forward(const ccq_weight *w13, const ccq_weight *w2, int32_t num_experts,
+                                 const void *x_bf16, int32_t T, const int32_t *expert_ids,
+                                 const float *routing_w, int32_t topk, void *y_bf16, void *ws, size_t ws_bytes,
+                                 ccq_stream_t stream) {
+    return ccq_moe_w2a16_forward_traced(w13, w2, num_experts, x_bf16, T, expert_ids, routing_w, topk, y_bf16, ws,
+                                        ws_bytes, stream, nullptr);
+}
+
+ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight *w2, int32_t num_experts,
+                                        const void *x_bf16, int32_t T, const int32_t *expert_ids,
+                                        const float *routing_w, int32_t topk, void *y_bf16, void *ws,
+                                        size_t ws_bytes, ccq_stream_t stream, void *const *events) {
+    ccq_status st = check_weight(w13, num_experts);
+    if (st != CCQ_OK) return st;
+    st = check_weight(w2, num_experts);
+    if (st != CCQ_OK) return st;
+    if (T < 0 || topk <= 0 || topk > 64) return CCQ_ERR_INVALID_ARG;
+    const int H = w13->k, I = w13->n / 2;
+    if (w13->n % 2 || w2->n != H || w2->k != I || I % 64) return CCQ_ERR_INVALID_ARG;
+    if (T == 0) return CCQ_OK;
+    if (!x_bf16 || !y_bf16 || !expert_ids || !routing_w || !aligned16(x_bf16) || !aligned16(y_bf16))
+        return CCQ_ERR_INVALID_ARG;
+    if (x_bf16 == y_bf16) return CCQ_ERR_INVALID_ARG;
+    if (w13->fmt != CCQ_FMT_W2_CCQ_G64 || w2->fmt != CCQ_FMT_W2_CCQ_G64) return CCQ_ERR_UNSUPPORTED;
+    const MoeWs L = moe_layout(T, topk, H, I, num_experts);
+    if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return CCQ_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    uint32_t *err = reinterpret_cast<uint32_t *>(base + L.err);
+    int *seg = reinterpret_cast<int *>(base + L.seg);
+    int *cursor = reinterpret_cast<int *>(base + L.cursor);
+    int *tok = reinterpret_cast<int *>(base + L.tok);
+    float *rwp = reinterpret_cast<float *>(base + L.rwp);
+    int *inv = reinterpret_cast<int *>(base + L.inv);
+    uint16_t *xa_x = reinterpret_cast<uint16_t *>(base + L.xa_x);
+    float *gs_x = reinterpret_cast<float *>(base + L.gs_x);
+    uint16_t *xa_h = reinterpret_cast<uint16_t *>(base + L.xa_h);
+    float *gs_h = reinterpret_cast<float *>(base + L.gs_h);
+    float *slot = reinterpret_cast<float *>(base + L.slot);
+    const int pairs = T * topk;
+
+    cudaError_t e = trace(events, 0, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(base + L.err, 0, 16, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(base + L.tok, 0, sizeof(int) * (size_t)L.P, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(base + L.rwp, 0, sizeof(float) * (size_t)L.P, s);
+    if (e == cudaSuccess)
+        e = launch_moe_route(expert_ids, routing_w, T, topk, num_experts, seg, cursor, tok, rwp, inv, err, s);
+    if (e == cudaSuccess) e = trace(events, 1, s);
+    if (e == cudaSuccess) e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), tok, pairs, L.P, H, xa_x, gs_x, s);
+    if (e == cudaSuccess) e = trace(events, 2, s);
+    if (e != cudaSuccess) return CCQ_ERR_CUDA;
+    const int nt = pick_nt((double)pairs / num_experts);
+
+    // gate/up projection with the SiLU gate fused in its epilogue -> h (activation operand layout)
+    DecodeMaps m1;
+    if (!decode_maps(m1, w13, num_experts, xa_x, gs_x, L.P, nt)) return CCQ_ERR_CUDA;
+    DecodeGemmParams p1{};
+    p1.scales = w13->scales;
+    p1.alpha = w13->alpha;
+    p1.beta = w13->beta;
+    p1.N = w13->n;
+    p1.K = H;
+    p1.row_block_stride = 128;
+    p1.half_stride = I;
+    p1.num_stages = ceil_div(H, 512);
+    p1.stages_per_split = p1.num_stages;
+    p1.seg_off = seg;
+    p1.P = L.P;
+    p1.mode = EPI_GATEUP;
+    p1.out = xa_h;
+    p1.h_P = L.P;
+    p1.I = I;
+    p1.err = err;
+    e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, ceil_div(I, 128), 1, num_experts, nt, s);
+    if (e == cudaSuccess) e = trace(events, 3, s);
+    if (e == cudaSuccess) e = launch_gsum_from_xa(xa_h, pairs, L.P, I, gs_h, s);
+    if (e == cudaSuccess) e = trace(events, 4, s);
+    if (e != cudaSuccess) return CCQ_ERR_CUDA;
+
+    // down projection, scaled by each pair's routing weight -> fp32 slots
+    DecodeMaps m2;
+    if (!decode_maps(m2, w2, num_experts, xa_h, gs_h, L.P, nt)) return CCQ_ERR_CUDA;
+    DecodeGemmParams p2{};
+    p2.scales = w2->scales;
+    p2.alpha = w2->alpha;
+    p2.beta = w2->beta;
+    p2.N = H;
+    p2.K = I;
+    p2.row_block_stride = 256;
+    p2.half_stride = 128;
+    p2.num_stages = ceil_div(I, 512);
+    p2.stages_per_split = p2.num_stages;
+    p2.seg_off = seg;
+    p2.P = L.P;
+    p2.mode = EPI_DOWN;
+    p2.out = slot;
+    p2.out_ld = H;
+    p2.rw = rwp;
+    p2.err = err;
+    e = launch_decode_gemm_w2(p2, m2.codes, m2.xa, m2.gs, ceil_div(H, 256), 1, num_experts, nt, s);
+    if (e == cudaSuccess) e = trace(events, 5, s);
+    if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
+    if (e == cudaSuccess) e = trace(events, 6, s);
+    return cuda_status(e);
+}
+
+ccq_status ccq_check_device_error(void *ws, ccq_stream_t stream) {
+    if (!ws) return CCQ_ERR_INVALID_ARG;
+    uint32_t h[2] = {0, 0};
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(h, ws, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return CCQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return CCQ_ERR_CUDA;
+    if (h[0] == 0) return CCQ_OK;
+    if (cudaMemsetAsync(ws, 0, sizeof(h), s) != cudaSuccess) return CCQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return CCQ_ERR_CUDA;
+    return (h[0] & DEV_ERR_TIMEOUT) ? CCQ_ERR_TIMEOUT : CCQ_ERR_DEVICE_CHECK;
+}
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// Kernel parameter blocks and launchers shared between the CUDA translation units of libccq.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ccq {
+
+// Epilogue modes of the decode-sized grouped kernel.
+enum EpiMode : int {
+    EPI_PARTIAL_F32 = 0,  // out_f32[ks][m][n] = partial sum over this CTA's k range
+    EPI_BF16 = 1,         // out_bf16[m][n] = bf16(acc)
+    EPI_GATEUP = 2,       // h = bf16(SiLU(acc_gate) * acc_up) written in the activation-operand layout
+    EPI_DOWN = 3          // slot_f32[p][n] = routing_w[p] * acc
+};
+
+// Activation-operand ("XA") layout used by the decode-sized kernel.  For an operand of P rows and
+// K columns (K % 64 == 0), element (p, k) with G = k/64, r = k%64, tig = r/16, j = (r/4)%4, i = r%4
+// sits at  ((((G*4 + i)*P + p)*4 + tig)*4 + j).  Rows of one 16-column block are thus grouped by
+// the state window i they meet in the decoded weights, which makes every mma B fragment one
+// contiguous, bank-conflict-free 8-byte shared-memory read.  Alongside it, gsum[p][G] holds
+// -160 * sum_{k in group G} x[p][k] (fp32, row pitch gsum_ld = round_up(K/64, 4)).
+__host__ __device__ inline size_t xa_index(size_t p, size_t k, size_t P) {
+    size_t G = k >> 6, r = k & 63, tig = r >> 4, j = (r >> 2) & 3, i = r & 3;
+    return ((((G * 4 + i) * P + p) * 4 + tig) * 4 + j);
+}
+__host__ __device__ inline int gsum_ld(int K) { return ((K / 64) + 3) & ~3; }
+
+struct DecodeGemmParams {
+    const float *scales;  // [rows_total][K/64]
+    const float *alpha;   // [rows_total]
+    const float *beta;    // [rows_total]
+    int N;                // rows per expert
+    int K;                // columns
+    int row_block_stride; // rows between consecutive row blocks
+    int half_stride;      // row offset of the CTA's second 128-row half
+    int stages_per_split; // 512-column stages per k split
+    int num_stages;       // ceil(K/512)
+    // tokens
+    const int *seg_off;   // [E+1] row offsets into the activation operand; NULL: one segment [0, M)
+    int M;
+    int P;                // rows of the activation operand
+    // epilogue
+    int mode;
+    void *out;
+    int out_ld;           // leading dimension of out (elements)
+    size_t out_split_stride; // EPI_PARTIAL_F32: elements between k splits
+    const float *rw;      // EPI_DOWN: routing weight per operand row
+    int h_P;              // EPI_GATEUP: rows of the H operand (== P)
+    int I;                // EPI_GATEUP: gate rows per expert
+    uint32_t *err;
+};
+
+cudaError_t launch_decode_gemm_w2(const DecodeGemmParams &p, const CUtensorMap &tm_codes,
+                                  const CUtensorMap &tm_xa, const CUtensorMap &tm_gs, int row_blocks,
+                                  int ksplit, int experts, int nt, cudaStream_t s);
+
+cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, const float *alpha,
+                           const float *beta, int rows, int K, uint16_t *out, cudaStream_t s);
+
+// x (BF16 [rows][K], row r taken from x[tok_of ? tok_of[p] : p]) -> XA operand + group sums.
+cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, uint16_t *xa,
+                           float *gsum, cudaStream_t s);
+// group sums of an operand already in XA layout (rows [0, P_valid))
+cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float *gsum, cudaStream_t s);
+
+cudaError_t launch_splitk_reduce(const float *partial, int ksplit, size_t split_stride, int M, int N,
+                                 uint16_t *y, cudaStream_t s);
+
+// MoE routing: counts, offsets, placement, inverse map; validates ids.
+cudaError_t launch_moe_route(const int *ids, const float *rw, int T, int topk, int E, int *seg_off,
+                             int *cursor, int *tok_of, float *rw_perm, int *inv, uint32_t *err,
+                             cudaStream_t s);
+cudaError_t launch_moe_combine(const float *slot, const int *inv, int T, int topk, int H, uint16_t *y,
+                               cudaStream_t s);
+
+}  // namespace ccq

@@ -1,0 +1,239 @@
+"""GPU parity of libccq against the CPU oracle (B200, through the C ABI).
+
+Bars: decoded BF16 weights bit-exact; matmul and MoE outputs max|d|/max|ref| <= 1e-2 (the stated
+tolerance; fp32 accumulation), with a tighter regression guard where the arithmetic allows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def ccq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import extreme_bit_weight_b200 as m
+
+    return m
+
+
+def rel_err(y, ref):
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.max(np.abs(y - ref)) / max(np.max(np.abs(ref)), 1e-30))
+
+
+def bits_of(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def w2_weight(ccq, codes, scales, alpha, beta, experts=1):
+    n = codes.shape[-2] if codes.ndim == 3 else codes.shape[0] // experts
+    k = codes.shape[-1] * 4
+    return ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, n, k, codes, scales, alpha, beta, experts=experts)
+
+
+# ----------------------------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------------------------
+def test_dequant_small_linear_bitexact(ccq):
+    # single linear M=4, K=N=256, weights N(0, 0.02) encoded by the oracle
+    w = synth.weights_normal(256, 256, 1001)
+    codes, scales, alpha, beta = oracle.encode_w2(w, 64)
+    W = w2_weight(ccq, codes, scales, alpha, beta)
+    got = bits_of(ccq.ccq_dequant_bf16(W))[0]
+    assert np.array_equal(got, oracle.dequant_w2(codes, scales, alpha, beta))
+
+
+@pytest.mark.parametrize("n,k,E", [(16, 64, 1), (48, 192, 3), (272, 576, 2), (1024, 8192, 1)])
+def test_dequant_random_format_bitexact(ccq, n, k, E):
+    codes, scales, alpha, beta = synth.w2_format_random(n * E, k, 1100 + n + k)
+    W = w2_weight(ccq, codes, scales, alpha, beta, experts=E)
+    got = bits_of(ccq.ccq_dequant_bf16(W)).reshape(n * E, k)
+    assert np.array_equal(got, oracle.dequant_w2(codes, scales, alpha, beta))
+
+
+def test_dequant_outside_fast_domain_bitexact(ccq):
+    # negative, huge and fractional code parameters: the exact decode still matches the definition
+    n, k = 64, 128
+    g = synth.rng(1200)
+    codes = g.integers(0, 256, size=(n, k // 4), dtype=np.uint8)
+    alpha = np.concatenate([g.normal(0, 300, 32), g.normal(0, 1e7, 32)]).astype(np.float32)
+    beta = np.concatenate([g.normal(0, 1e5, 32), g.normal(0, 3e9, 32)]).astype(np.float32)
+    alpha[0], beta[0] = 0.5, 0.5  # exact ties
+    scales = (g.random((n, k // 64)) * 2 - 1).astype(np.float32)
+    W = w2_weight(ccq, codes, scales, alpha, beta)
+    got = bits_of(ccq.ccq_dequant_bf16(W))[0]
+    assert np.array_equal(got, oracle.dequant_w2(codes, scales, alpha, beta))
+
+
+def test_dequant_w4_bitexact(ccq):
+    codes, scales = synth.w4_format_random(96, 320, 1300)
+    W = ccq.CcqWeight(ccq.CCQ_FMT_W4_PER_CHANNEL, 96, 320, codes, scales)
+    got = bits_of(ccq.ccq_dequant_bf16(W))[0]
+    assert np.array_equal(got, oracle.dequant_w4(codes, scales))
+
+
+# ----------------------------------------------------------------------------------------------
+# decode-sized matmul
+# ----------------------------------------------------------------------------------------------
+def test_gemm_one_hot_identity(ccq):
+    # x = I_K: y[m][n] = w[n][m], so every weight the fused kernel decodes is observed exactly
+    n, k = 272, 320
+    codes, scales, alpha, beta = synth.w2_format_random(n, k, 1400)
+    W = w2_weight(ccq, codes, scales, alpha, beta)
+    x = synth.one_hot_rows(k).cuda()
+    y = ccq.ccq_w2a16_gemm(W, x).float().cpu().numpy()
+    ref = oracle.bf16_to_f64(oracle.dequant_w2(codes, scales, alpha, beta)).T
+    assert np.array_equal(y, ref.astype(np.float32))
+
+
+def test_gemm_small_linear(ccq):
+    w = synth.weights_normal(256, 256, 1001)
+    codes, scales, alpha, beta = oracle.encode_w2(w, 64)
+    W = w2_weight(ccq, codes, scales, alpha, beta)
+    x = synth.activations(4, 256, 1002)
+    y = ccq.ccq_w2a16_gemm(W, x.cuda()).float().cpu().numpy()
+    ref = oracle.gemm_f64(synth.bf16_bits(x), oracle.dequant_w2(codes, scales, alpha, beta))
+    e = rel_err(y, ref)
+    assert e <= TOL
+    assert e <= 4e-3  # fp32 accumulation + one BF16 output rounding
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 16, 64), (3, 48, 192), (8, 256, 512), (9, 272, 576), (17, 128, 1088),
+                                   (33, 256, 1024), (1, 8192, 8192), (16, 8192, 8192)])
+def test_gemm_shapes(ccq, m, n, k):
+    codes, scales, alpha, beta = synth.w2_format_random(n, k, 1500 + m + n + k)
+    W = w2_weight(ccq, codes, scales, alpha, beta)
+    x = synth.activations(m, k, 1501 + m)
+    y = ccq.ccq_w2a16_gemm(W, x.cuda()).float().cpu().numpy()
+    ref = oracle.gemm_f64(synth.bf16_bits(x), oracle.dequant_w2(codes, scales, alpha, beta))
+    e = rel_err(y, ref)
+    assert e <= TOL
+    assert e <= 4e-3
+
+
+def test_gemm_m0_and_determinism(ccq):
+    codes, scales, alpha, beta = synth.w2_format_random(256, 1024, 1600)
+    W = w2_weight(ccq, codes, scales, alpha, beta)
+    x = synth.activations(16, 1024, 1601).cuda()
+    y0 = ccq.ccq_w2a16_gemm(W, x[:0])
+    assert y0.shape == (0, 256)
+    a = bits_of(ccq.ccq_w2a16_gemm(W, x))
+    b = bits_of(ccq.ccq_w2a16_gemm(W, x))
+    assert np.array_equal(a, b)
+
+
+# ----------------------------------------------------------------------------------------------
+# MoE FFN
+# ----------------------------------------------------------------------------------------------
+def moe_weights(ccq, E, H, I, seed):
+    c13, s13, a13, b13 = synth.w2_format_random(E * 2 * I, H, seed)
+    c2, s2, a2, b2 = synth.w2_format_random(E * H, I, seed + 1)
+    W13 = ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, 2 * I, H, c13, s13, a13, b13, experts=E)
+    W2 = ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, H, I, c2, s2, a2, b2, experts=E)
+    dec13 = oracle.dequant_w2(c13, s13, a13, b13).reshape(E, 2 * I, H)
+    dec2 = oracle.dequant_w2(c2, s2, a2, b2).reshape(E, H, I)
+    return W13, W2, dec13, dec2
+
+
+def run_moe(ccq, W13, W2, x, ids, rw):
+    ids_t = torch.from_numpy(np.ascontiguousarray(ids, np.int32)).cuda()
+    rw_t = torch.from_numpy(np.ascontiguousarray(rw, np.float32)).cuda()
+    T, H = x.shape
+    ws = ccq.workspace(ccq.ccq_moe_workspace_size(T, ids.shape[1], H, W13.n // 2, W13.experts))
+    y = ccq.ccq_moe_w2a16_forward(W13, W2, x.cuda(), ids_t, rw_t, ws=ws)
+    st = ccq.ccq_check_device_error(ws)
+    return y.float().cpu().numpy(), st
+
+
+@pytest.mark.parametrize("T,E,topk", [(5, 8, 2), (40, 4, 1), (24, 16, 4)])
+def test_moe_small_full(ccq, T, E, topk):
+    H, I = 256, 128
+    W13, W2, d13, d2 = moe_weights(ccq, E, H, I, 2000 + T)
+    x = synth.activations(T, H, 2002 + T)
+    ids, rw = synth.routing_uniform(T, E, topk, 2003 + T)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    xb = synth.bf16_bits(x)
+    ref = oracle.moe_f64(xb, d13, d2, ids, rw, round_h=True)
+    ref64 = oracle.moe_f64(xb, d13, d2, ids, rw, round_h=False)
+    assert rel_err(y, ref) <= TOL
+    assert rel_err(y, ref64) <= TOL
+
+
+def test_moe_skewed_and_empty_experts(ccq):
+    # every token on expert 2 (more tokens than one mma tile), experts 0,1,3..7 empty except one pair
+    H, I, E, T = 256, 192, 8, 37
+    W13, W2, d13, d2 = moe_weights(ccq, E, H, I, 2100)
+    x = synth.activations(T, H, 2101)
+    ids = np.full((T, 2), 2, np.int32)
+    ids[:, 1] = 5
+    rw = np.full((T, 2), 0.5, np.float32)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    ref = oracle.moe_f64(synth.bf16_bits(x), d13, d2, ids, rw, round_h=True)
+    assert rel_err(y, ref) <= TOL
+
+
+def test_moe_invalid_ids_reported_and_skipped(ccq):
+    H, I, E, T = 256, 128, 6, 7
+    W13, W2, d13, d2 = moe_weights(ccq, E, H, I, 2200)
+    x = synth.activations(T, H, 2201)
+    ids, rw = synth.routing_uniform(T, E, 3, 2202)
+    ids[1, 0] = E        # out of range
+    ids[3, 2] = -1       # out of range
+    ids[4, 1] = ids[4, 0]  # repeated within a token
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_ERR_DEVICE_CHECK
+    keep = ids.copy()
+    keep[1, 0] = -1
+    keep[3, 2] = -1
+    keep[4, 1] = -1
+    ref = oracle.moe_f64(synth.bf16_bits(x), d13, d2, keep, rw, round_h=True)
+    assert rel_err(y, ref) <= TOL
+
+
+def test_moe_token_permutation_invariance(ccq):
+    H, I, E, T = 256, 128, 8, 16
+    W13, W2, _, _ = moe_weights(ccq, E, H, I, 2300)
+    x = synth.activations(T, H, 2301)
+    ids, rw = synth.routing_uniform(T, E, 2, 2302)
+    y, _ = run_moe(ccq, W13, W2, x, ids, rw)
+    perm = synth.rng(2303).permutation(T)
+    yp, _ = run_moe(ccq, W13, W2, x[perm], ids[perm], rw[perm])
+    assert np.array_equal(yp, y[perm])
+
+
+def test_moe_decode_layer_full_size_sampled(ccq):
+    # the decode-sized MoE layer: 32 tokens, hidden 8192, 64 experts of 8192x3584x2 / 3584x8192,
+    # top-8 uniform routing with softmax weights; checked on sampled tokens against the oracle
+    T, H, I, E, topk = 32, 8192, 3584, 64, 8
+    c13, s13, a13, b13 = synth.w2_format_random(E * 2 * I, H, 3000)
+    c2, s2, a2, b2 = synth.w2_format_random(E * H, I, 3001)
+    W13 = ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, 2 * I, H, c13, s13, a13, b13, experts=E)
+    W2 = ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, H, I, c2, s2, a2, b2, experts=E)
+    x = synth.activations(T, H, 3002)
+    ids, rw = synth.routing_uniform(T, E, topk, 3003)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    xb = synth.bf16_bits(x)
+    sample = [0, 13, 31]
+    ref = np.zeros((len(sample), H))
+    for e in sorted({int(ids[t, j]) for t in sample for j in range(topk)}):
+        d13 = oracle.dequant_w2(c13[e * 2 * I:(e + 1) * 2 * I], s13[e * 2 * I:(e + 1) * 2 * I],
+                                a13[e * 2 * I:(e + 1) * 2 * I], b13[e * 2 * I:(e + 1) * 2 * I])
+        d2 = oracle.dequant_w2(c2[e * H:(e + 1) * H], s2[e * H:(e + 1) * H], a2[e * H:(e + 1) * H],
+                               b2[e * H:(e + 1) * H])
+        for si, t in enumerate(sample):
+            for j in range(topk):
+                if ids[t, j] == e:
+                    ref[si] += float(rw[t, j]) * oracle.expert_ffn_f64(xb[t:t + 1], d13, d2, round_h=True)[0]
+    assert rel_err(y[sample], ref) <= TOL
