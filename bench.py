@@ -40,7 +40,19 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    ap.add_argument("--profile-small", action="store_true",
+                    help="8 tokens over 16 experts (same tokens per expert, 442 MB of weights): for ncu captures")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
+                    help="decode: 32 tokens, uniform routing (the headline line); prefill: 4096 tokens, "
+                         "Zipf(1.1) routing, 1%% of channels x20 (tcgen05 path, tensor roofline)")
+    args = ap.parse_args()
+    global T, E, WORKLOAD
+    if args.workload == "prefill":
+        T = 4096
+        WORKLOAD = "moe_ffn_prefill_T4096_zipf1.1_H8192_I3584_E64_top8_ccq_w2_g64"
+    if args.profile_small:
+        T, E = (8, 16) if args.workload == "decode" else (512, 16)
+    return args
 
 
 def dist_env():
@@ -59,12 +71,24 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured bf16_tflops (burst)"
+    return 1590.0, "fallback"
+
+
 def config_dict():
+    prefill = WORKLOAD.startswith("moe_ffn_prefill")
     return {
         "workload": WORKLOAD,
         "tokens": T, "hidden": H, "intermediate": I, "experts": E, "topk": TOPK,
         "weight_format": "CCQ (6,4,3) code cluster, 4 weights/byte, fp32 group-64 scales",
-        "routing": "uniform distinct top-8, softmax of N(0,1) logits",
+        "routing": ("Zipf(1.1) expert popularity, top-8 by Gumbel-max; " if prefill else "uniform distinct top-8, ")
+                   + "softmax of N(0,1) logits",
+        "activations": "BF16 N(0,1)" + (", 1% of channels x20" if prefill else ""),
         "weights": f"N(0,0.02) encoded by ccq_encode_host for {DISTINCT} experts, copied to all {E}",
         "l2": "inputs larger than L2: ~1.74 GB of packed weights touched per step vs 126 MB L2",
         "parallelism": "replicas",
@@ -168,32 +192,54 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------------
 # CPU baseline: the oracle on a bounded sample of the same layer
 # ------------------------------------------------------------------------------------------------
-def oracle_sample(n_experts: int = 1):
-    """Time the oracle on `n_experts` experts of the decode layer (decode their weights, run every
-    (token, expert) pair routed to them), and scale to the layer by the touched-expert count."""
-    import oracle
-    import synth
+_ORACLE_INPUTS = None
 
-    x = synth.activations(T, H, 3302)
-    ids, rw = synth.routing_uniform(T, E, TOPK, 3303)
-    xb = synth.bf16_bits(x)
+
+def _oracle_inputs():
+    global _ORACLE_INPUTS
+    if _ORACLE_INPUTS is None:
+        import synth
+
+        x = synth.activations(T, H, 3302)
+        ids, rw = synth.routing_uniform(T, E, TOPK, 3303)
+        w13 = synth.w2_format_random(2 * I, H, 3304)
+        w2 = synth.w2_format_random(H, I, 3305)
+        _ORACLE_INPUTS = (synth.bf16_bits(x), ids, rw, w13, w2)
+    return _ORACLE_INPUTS
+
+
+def oracle_sample(n_experts: int = 1, row_frac: float = 1.0):
+    """Time the oracle on `n_experts` experts of the decode layer: decode their weights (the first
+    `row_frac` of the rows of each projection) and run every (token, expert) pair routed to them
+    through the fp64 expert FFN on those rows; scale to the whole layer by the touched-expert count
+    and 1/row_frac."""
+    import oracle
+
+    xb, ids, rw, (c13, s13, a13, b13), (c2, s2, a2, b2) = _oracle_inputs()
     touched = sorted(set(int(v) for v in ids.ravel()))
-    c13, s13, a13, b13 = synth.w2_format_random(2 * I, H, 3304)
-    c2, s2, a2, b2 = synth.w2_format_random(H, I, 3305)
+    rg = max(1, int(round(row_frac * I)))   # gate rows, and the same number of up rows
+    r2 = max(16, int(round(row_frac * H)))  # down rows
+    g13 = np.concatenate([np.arange(rg), I + np.arange(rg)])
+    r13 = 2 * rg
     pairs = 0
     t0 = time.perf_counter()
     for e in touched[:n_experts]:
-        d13 = oracle.dequant_w2(c13, s13, a13, b13)
-        d2 = oracle.dequant_w2(c2, s2, a2, b2)
+        d13 = oracle.dequant_w2(c13[g13], s13[g13], a13[g13], b13[g13])
+        d2 = oracle.dequant_w2(c2[:r2], s2[:r2], a2[:r2], b2[:r2])
         toks = [t for t in range(T) if e in ids[t]]
         pairs += len(toks)
-        out = oracle.expert_ffn_f64(xb[toks], d13, d2, round_h=True)
+        gu = oracle.gemm_f64(xb[toks], d13)                       # gate | up rows of the slice
+        h = oracle.silu_f64(gu[:, :r13 // 2]) * gu[:, r13 // 2:]
+        hb = oracle.bf16_bits(h.astype(np.float32))
+        out = oracle.gemm_f64(hb, np.ascontiguousarray(d2[:, :r13 // 2]))
         del out
     dt = time.perf_counter() - t0
-    layer_s = dt * len(touched) / n_experts
+    frac = min(1.0, (r13 * H + r2 * I) / (3.0 * I * H))  # share of the expert's weights sampled
+    layer_s = dt * len(touched) / n_experts / frac
     cores = os.cpu_count() or 1
-    sample = (f"{n_experts} of {len(touched)} touched experts ({pairs} of {T * TOPK} token-expert pairs): "
-              f"oracle decode + fp64 expert FFN, scaled by touched experts")
+    sample = (f"{n_experts} of {len(touched)} touched experts, {100 * frac:.1f}% of their weight rows "
+              f"({pairs} of {T * TOPK} token-expert pairs): oracle decode + fp64 expert FFN, "
+              f"scaled by touched experts and rows")
     return T / layer_s, cores, sample, dt
 
 
@@ -206,9 +252,13 @@ def run_reference(args, rank, world):
     import oracle
 
     oracle.build()
+    # size each step so the whole run takes about 90 s of host time
+    _, _, _, dt_full = oracle_sample(1, 0.05)
+    per_step = 90.0 / max(1, args.warmup + args.steps)
+    frac = float(min(1.0, max(0.002, 0.05 * per_step / max(dt_full, 1e-6))))
     vals = []
     for i in range(args.warmup + args.steps):
-        v, cores, sample, dt = oracle_sample(1)
+        v, cores, sample, dt = oracle_sample(1, frac)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
@@ -249,12 +299,16 @@ def run_ours(args, rank, world, local):
         import oracle
 
         oracle.build()
-        v, cores, sample, dt = oracle_sample(2)
+        v, cores, sample, dt = oracle_sample(16)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
 
     W13, W2 = make_layer(ccq, torch, device)
-    x_host = synth.activations(T, H, 3002 + 17 * rank)
-    ids_np, rw_np = synth.routing_uniform(T, E, TOPK, 3003 + 17 * rank)
+    prefill = args.workload == "prefill"
+    x_host = synth.activations(T, H, 3002 + 17 * rank, outlier_frac=0.01 if prefill else 0.0)
+    if prefill:
+        ids_np, rw_np = synth.routing_zipf(T, E, TOPK, 3003 + 17 * rank, s=1.1)
+    else:
+        ids_np, rw_np = synth.routing_uniform(T, E, TOPK, 3003 + 17 * rank)
     x = x_host.to(device)
     ids = torch.from_numpy(ids_np).to(device)
     rw = torch.from_numpy(rw_np).to(device)
@@ -273,6 +327,9 @@ def run_ours(args, rank, world, local):
     # ---- device-timed region: exactly K steps, events around every step's kernels ----
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ccq.CCQ_MOE_TRACE_POINTS)] for _ in range(K)]
+    for row in evs:  # torch creates an event on its first record; libccq re-records the same handles
+        for ev in row:
+            ev.record(stream)
     clocks = ClockSampler(local)
     if pg:
         pg.barrier()
@@ -335,13 +392,26 @@ def run_ours(args, rank, world, local):
     hbm, src = peaks()
     ach13 = b13 / (gemm1_ms * 1e-3) / 1e9
     layer_gbs = (b13 + b2) / (ms_per_step * 1e-3) / 1e9
+    valid_pairs = int(np.sum(ids_np >= 0))
+    flops13 = 2.0 * valid_pairs * (2 * I) * H
+    flops2 = 2.0 * valid_pairs * H * I
+    roofline_tensor = None
+    if prefill:
+        tf, tsrc = tensor_peak()
+        roofline_tensor = {"bound": "tensor", "kernel": "tc_gemm_w2_kernel (gate/up, SiLU epilogue)",
+                           "achieved": flops13 / (gemm1_ms * 1e-3) / 1e12, "peak": tf, "peak_source": tsrc,
+                           "unit": "TFLOP/s", "frac": flops13 / (gemm1_ms * 1e-3) / 1e12 / tf, "traffic": None,
+                           "launch_ms": gemm1_ms, "algorithmic_flops_per_launch": flops13,
+                           "down_kernel": {"achieved": flops2 / (gemm2_ms * 1e-3) / 1e12, "launch_ms": gemm2_ms,
+                                           "algorithmic_flops_per_launch": flops2},
+                           "layer_tflops": (flops13 + flops2) / (ms_per_step * 1e-3) / 1e12}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(),
         "packed_weight_gbs": layer_gbs, "packed_weight_pct_of_8tbs": 100.0 * layer_gbs / NOMINAL_HBM_GBS,
         "touched_experts": ne,
-        "roofline": {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (gate/up, SiLU epilogue)",
+        "roofline": roofline_tensor or {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (gate/up, SiLU epilogue)",
                      "achieved": ach13, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "unit": "GB/s",
                      "frac": ach13 / hbm, "traffic": None, "launch_ms": gemm1_ms,
                      "algorithmic_bytes_per_launch": b13,

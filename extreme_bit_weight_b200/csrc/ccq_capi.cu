@@ -69,7 +69,8 @@ int pick_nt(double rows_per_expert) {
 }
 
 struct DecodeMaps {
-    CUtensorMap codes, xa, gs;
+    CUtensorMap codes, xa, gs, sc;
+    bool tma_scales;
 };
 
 bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t *xa, const float *gs, int P,
@@ -99,16 +100,40 @@ bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t
         if (!make_map(&m.gs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, gs, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return false;
     }
+    // group scales [rows][K/64] fp32: staged by TMA when the row pitch is a multiple of 16 bytes
+    m.tma_scales = (K / 64) % 4 == 0;
+    if (m.tma_scales) {
+        cuuint64_t dims[2] = {(cuuint64_t)(K / 64), rows};
+        cuuint64_t str[1] = {(cuuint64_t)(K / 64) * 4};
+        cuuint32_t box[2] = {8, 128};
+        if (!make_map(&m.sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, w->scales, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return false;
+    } else {
+        m.sc = m.gs;  // unused
+    }
     return true;
 }
 
+// Token counts above these run on the tcgen05 kernel (dense GEMM: m; MoE: mean rows per expert).
+constexpr int kTcMinM = 48;
+constexpr double kTcMinRowsPerExpert = 48.0;
+constexpr int kTcMT = 2;  // 128-token sub-tiles per tcgen05 tile
+
 struct GemmWs {
-    size_t xa, gs, partial, total;
+    size_t xa, gs, partial, xt, total;
     int P, ksplit, spp, row_blocks, nt;
+    bool tc;
 };
 
 GemmWs gemm_layout(const ccq_weight *w, int m) {
     GemmWs L{};
+    if (m >= kTcMinM) {
+        L.tc = true;
+        L.P = m;
+        L.xt = 0;
+        L.total = up256((size_t)m * w->k * 2);
+        return L;
+    }
     L.P = (m + 3) & ~3;
     L.nt = pick_nt((double)m);
     const int K = w->k, N = w->n;
@@ -130,14 +155,17 @@ GemmWs gemm_layout(const ccq_weight *w, int m) {
 }
 
 struct MoeWs {
-    size_t err, seg, cursor, tok, rwp, inv, xa_x, gs_x, xa_h, gs_h, slot, total;
-    int P;
+    size_t err, seg, cursor, tok, rwp, inv, xa_x, gs_x, xa_h, gs_h, tiles, tcount, slot, total;
+    int P, max_tiles;
+    bool tc;
 };
 
 MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     MoeWs L{};
     const int pairs = T * topk;
     L.P = (pairs + 3) & ~3;
+    L.tc = (double)pairs / E >= kTcMinRowsPerExpert;
+    L.max_tiles = L.P / (128 * kTcMT) + E + 1;
     size_t off = 0;
     L.err = off; off = up256(off + 16);
     L.seg = off; off = up256(off + sizeof(int) * (size_t)(E + 1));
@@ -145,13 +173,46 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     L.tok = off; off = up256(off + sizeof(int) * (size_t)L.P);
     L.rwp = off; off = up256(off + sizeof(float) * (size_t)L.P);
     L.inv = off; off = up256(off + sizeof(int) * (size_t)pairs);
+    // activation operand of the first projection and of the second (XA + group sums for the
+    // decode-sized kernel, the plain permuted-column layout for the tcgen05 kernel)
     L.xa_x = off; off = up256(off + (size_t)L.P * H * 2);
-    L.gs_x = off; off = up256(off + (size_t)L.P * gsum_ld(H) * 4);
+    L.gs_x = off; if (!L.tc) off = up256(off + (size_t)L.P * gsum_ld(H) * 4);
     L.xa_h = off; off = up256(off + (size_t)L.P * I * 2);
-    L.gs_h = off; off = up256(off + (size_t)L.P * gsum_ld(I) * 4);
+    L.gs_h = off; if (!L.tc) off = up256(off + (size_t)L.P * gsum_ld(I) * 4);
+    L.tiles = off; if (L.tc) off = up256(off + sizeof(int2) * (size_t)L.max_tiles);
+    L.tcount = off; if (L.tc) off = up256(off + 16);
     L.slot = off; off = up256(off + (size_t)L.P * H * 4);
     L.total = off;
     return L;
+}
+
+bool tc_maps(CUtensorMap &ta, CUtensorMap &tcodes, const ccq_weight *w, int experts, const uint16_t *a, int P) {
+    const int K = w->k;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)P};
+        cuuint64_t str[1] = {(cuuint64_t)K * 2};
+        cuuint32_t box[2] = {64, 128};
+        if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return false;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)experts * w->n};
+        cuuint64_t str[1] = {(cuuint64_t)(K / 4)};
+        cuuint32_t box[2] = {64, 128};
+        if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w->codes, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
+            return false;
+    }
+    return true;
+}
+
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            n = 148;
+    }
+    return n;
 }
 
 inline ccq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CCQ_OK : CCQ_ERR_CUDA; }
@@ -178,7 +239,8 @@ const char *ccq_status_string(ccq_status s) {
 }
 
 const char *ccq_build_info(void) {
-    return "libccq: sm_100a; decode-sized path = register decode -> mma.sync m16n8k16 bf16, TMA-staged";
+    return "libccq: sm_100a; decode-sized path: register decode -> mma.sync m16n8k16 bf16 (TMA-staged); "
+           "prefill path: decode -> swizzled smem -> tcgen05.mma kind::f16, TMEM fp32 accumulators";
 }
 
 ccq_status ccq_dequant_bf16(const ccq_weight *w, int32_t num_experts, void *out_bf16, ccq_stream_t stream) {
@@ -206,6 +268,30 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
     if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return CCQ_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     uint8_t *base = static_cast<uint8_t *>(ws);
+    if (L.tc) {
+        uint16_t *xt = reinterpret_cast<uint16_t *>(base + L.xt);
+        cudaError_t e = launch_pack_xt(static_cast<const uint16_t *>(x_bf16), nullptr, m, w->k, xt, s);
+        if (e != cudaSuccess) return CCQ_ERR_CUDA;
+        CUtensorMap ta, tcodes;
+        if (!tc_maps(ta, tcodes, w, 1, xt, m)) return CCQ_ERR_CUDA;
+        TcGemmParams p{};
+        p.scales = w->scales;
+        p.alpha = w->alpha;
+        p.beta = w->beta;
+        p.N = w->n;
+        p.K = w->k;
+        p.row_block_stride = 256;
+        p.half_stride = 128;
+        p.n_tiles = ceil_div(w->n, 256);
+        p.m_tile = 128 * kTcMT;
+        p.static_tiles = ceil_div(m, p.m_tile);
+        p.M = m;
+        p.mode = EPI_BF16;
+        p.out = y_bf16;
+        p.out_ld = w->n;
+        const int grid = std::min(sm_count(), p.static_tiles * p.n_tiles);
+        return cuda_status(launch_tc_gemm_w2(p, ta, tcodes, kTcMT, grid, s));
+    }
     uint16_t *xa = reinterpret_cast<uint16_t *>(base + L.xa);
     float *gs = reinterpret_cast<float *>(base + L.gs);
     cudaError_t e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), nullptr, m, L.P, w->k, xa, gs, s);
@@ -235,7 +321,8 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
         p.mode = EPI_BF16;
         p.out = y_bf16;
     }
-    e = launch_decode_gemm_w2(p, maps.codes, maps.xa, maps.gs, L.row_blocks, L.ksplit, 1, L.nt, s);
+    p.tma_scales = maps.tma_scales;
+    e = launch_decode_gemm_w2(p, maps.codes, maps.xa, maps.gs, maps.sc, L.row_blocks, L.ksplit, 1, L.nt, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     if (L.ksplit > 1) {
         e = launch_splitk_reduce(reinterpret_cast<const float *>(base + L.partial), L.ksplit, (size_t)m * w->n, m,
@@ -298,7 +385,60 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     if (e == cudaSuccess)
         e = launch_moe_route(expert_ids, routing_w, T, topk, num_experts, seg, cursor, tok, rwp, inv, err, s);
     if (e == cudaSuccess) e = trace(events, 1, s);
-    if (e == cudaSuccess) e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), tok, pairs, L.P, H, xa_x, gs_x, s);
+    if (e != cudaSuccess) return CCQ_ERR_CUDA;
+    if (L.tc) {
+        // prefill-sized: tcgen05 grouped GEMMs over (expert, 256-token tile) entries
+        int2 *tiles = reinterpret_cast<int2 *>(base + L.tiles);
+        int *tcount = reinterpret_cast<int *>(base + L.tcount);
+        e = launch_pack_xt(static_cast<const uint16_t *>(x_bf16), tok, pairs, H, xa_x, s);
+        if (e == cudaSuccess) e = launch_build_tiles(seg, num_experts, 128 * kTcMT, tiles, tcount, s);
+        if (e == cudaSuccess) e = trace(events, 2, s);
+        if (e != cudaSuccess) return CCQ_ERR_CUDA;
+        CUtensorMap ta1, tc1, ta2, tc2;
+        if (!tc_maps(ta1, tc1, w13, num_experts, xa_x, L.P) || !tc_maps(ta2, tc2, w2, num_experts, xa_h, L.P))
+            return CCQ_ERR_CUDA;
+        TcGemmParams q1{};
+        q1.scales = w13->scales;
+        q1.alpha = w13->alpha;
+        q1.beta = w13->beta;
+        q1.N = w13->n;
+        q1.K = H;
+        q1.row_block_stride = 128;
+        q1.half_stride = I;
+        q1.n_tiles = ceil_div(I, 128);
+        q1.tile_list = tiles;
+        q1.tile_count = tcount;
+        q1.m_tile = 128 * kTcMT;
+        q1.seg_off = seg;
+        q1.mode = EPI_GATEUP;
+        q1.out = xa_h;
+        q1.out_ld = I;
+        q1.I = I;
+        q1.err = err;
+        e = launch_tc_gemm_w2(q1, ta1, tc1, kTcMT, std::min(sm_count(), L.max_tiles * q1.n_tiles), s);
+        if (e == cudaSuccess) e = trace(events, 3, s);
+        if (e == cudaSuccess) e = trace(events, 4, s);
+        TcGemmParams q2 = q1;
+        q2.scales = w2->scales;
+        q2.alpha = w2->alpha;
+        q2.beta = w2->beta;
+        q2.N = H;
+        q2.K = I;
+        q2.row_block_stride = 256;
+        q2.half_stride = 128;
+        q2.n_tiles = ceil_div(H, 256);
+        q2.mode = EPI_DOWN;
+        q2.out = slot;
+        q2.out_ld = H;
+        q2.rw = rwp;
+        q2.I = 0;
+        if (e == cudaSuccess) e = launch_tc_gemm_w2(q2, ta2, tc2, kTcMT, std::min(sm_count(), L.max_tiles * q2.n_tiles), s);
+        if (e == cudaSuccess) e = trace(events, 5, s);
+        if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
+        if (e == cudaSuccess) e = trace(events, 6, s);
+        return cuda_status(e);
+    }
+    e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), tok, pairs, L.P, H, xa_x, gs_x, s);
     if (e == cudaSuccess) e = trace(events, 2, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     const int nt = pick_nt((double)pairs / num_experts);
@@ -323,7 +463,8 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p1.h_P = L.P;
     p1.I = I;
     p1.err = err;
-    e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, ceil_div(I, 128), 1, num_experts, nt, s);
+    p1.tma_scales = m1.tma_scales;
+    e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), 1, num_experts, nt, s);
     if (e == cudaSuccess) e = trace(events, 3, s);
     if (e == cudaSuccess) e = launch_gsum_from_xa(xa_h, pairs, L.P, I, gs_h, s);
     if (e == cudaSuccess) e = trace(events, 4, s);
@@ -349,7 +490,8 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p2.out_ld = H;
     p2.rw = rwp;
     p2.err = err;
-    e = launch_decode_gemm_w2(p2, m2.codes, m2.xa, m2.gs, ceil_div(H, 256), 1, num_experts, nt, s);
+    p2.tma_scales = m2.tma_scales;
+    e = launch_decode_gemm_w2(p2, m2.codes, m2.xa, m2.gs, m2.sc, ceil_div(H, 256), 1, num_experts, nt, s);
     if (e == cudaSuccess) e = trace(events, 5, s);
     if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
     if (e == cudaSuccess) e = trace(events, 6, s);

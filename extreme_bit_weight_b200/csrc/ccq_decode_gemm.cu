@@ -34,20 +34,24 @@
 namespace ccq {
 namespace {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kRowWarps = 8;                       // warps per 16-row slot set (256 rows per CTA)
+constexpr int kConsumerWarps = 2 * kRowWarps;       // two warps per row slot: groups 0-3 / 4-7 of a stage
+constexpr int kThreads = kConsumerWarps * 32;       // lane 0 of warp 0 also issues the TMA loads
 constexpr int kCodeTileBytes = 128 * 128;  // [128 rows][128 B] = 8 groups of 16 bytes
 
 template <int NT>
 struct Smem {
     static constexpr int MP = 8 * NT;
-    static constexpr int kStages = NT >= 4 ? 3 : 4;  // ring depth within the 227 KB per CTA
+    static constexpr int kStages = NT == 1 ? 4 : (NT == 2 ? 3 : 2);  // ring depth within 227 KB
+    static constexpr int kCtasPerSm = 1;
+    static constexpr int kRedBytes = kRowWarps * 32 * 2 * NT * 4 * 4;  // partial sums of the second warp half
     static constexpr int kXaBytes = 32 * MP * 16 * 2;  // [G*4+i = 32][MP][16] bf16
     static constexpr int kGsBytes = MP * 8 * 4;        // [MP][8] fp32
-    static constexpr int kStageBytes = ((2 * kCodeTileBytes + kXaBytes + kGsBytes) + 1023) & ~1023;
-    static constexpr int kTotal = kStages * kStageBytes + 1024;  // + alignment slack
+    static constexpr int kScBytes = 2 * 128 * 8 * 4;   // [2 halves][128 rows][8 groups] fp32 scales
+    static constexpr int kStageBytes = ((2 * kCodeTileBytes + kXaBytes + kGsBytes + kScBytes) + 1023) & ~1023;
+    static constexpr int kTotal = kStages * kStageBytes + kRedBytes + 1024;  // + alignment slack
     static_assert(kTotal + 64 <= 227 * 1024, "shared memory per CTA");
-    static constexpr uint32_t kTxBytes = 2 * kCodeTileBytes + kXaBytes + kGsBytes;
+    static constexpr uint32_t kTxBytes = 2 * kCodeTileBytes + kXaBytes + kGsBytes;  // + kScBytes with TMA scales
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -79,17 +83,26 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
     return d;
 }
+// (a & m) | e in one three-input logic op
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t e) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(m), "r"(e));
+    return d;
+}
 
 struct RowDecode {
-    uint64_t ab;    // {alpha, alpha}
-    uint64_t bb;    // {beta, beta}
+    uint64_t ab;    // {alpha, alpha}: code scale of the row
+    uint64_t bb;    // {beta, beta}: code zero-point of the row
 };
 
-// The constants of the decode, held in registers so the compiler keeps the integer multiply.
+// The constants of the decode, held in registers: the integer multiply stays a multiply and the
+// window mask/exponent pair feeds one three-input logic op.
 struct DecodeConsts {
     uint64_t neg_magic;  // {-2^23, -2^23}: byte value from its 0x4B0000bb bit pattern
-    uint64_t round_mag;  // {1.5*2^23, 1.5*2^23 - 0x4B40}
+    uint64_t round_mag;  // {1.5*2^23, 1.5*2^23 - 0x4B40}: round to integer; second byte pre-cancels
     uint32_t mul16;      // 65536
+    uint32_t wmask;      // 0x003F003F: one 6-bit state window per 16-bit half
+    uint32_t wexp;       // 0x43004300: BF16 exponent of 128 in both halves
 };
 
 // Decode one 32-bit word (4 consecutive bytes of one row) into the eight BF16x2 registers
@@ -99,11 +112,11 @@ __device__ __forceinline__ void decode_word(uint32_t w, const RowDecode &rd, con
     const uint32_t magic = 0x4B000000u;
     uint64_t c01 = u2_pack(prmt(w, magic, 0x7650u), prmt(w, magic, 0x7651u));
     uint64_t c23 = u2_pack(prmt(w, magic, 0x7652u), prmt(w, magic, 0x7653u));
-    c01 = f2_add(c01, k.neg_magic);
+    c01 = f2_add(c01, k.neg_magic);                       // the bytes, exact
     c23 = f2_add(c23, k.neg_magic);
-    uint64_t t01 = f2_fma(c01, rd.ab, rd.bb);
+    uint64_t t01 = f2_fma(c01, rd.ab, rd.bb);             // q*alpha + beta, one fp32 rounding
     uint64_t t23 = f2_fma(c23, rd.ab, rd.bb);
-    t01 = f2_add(t01, k.round_mag);
+    t01 = f2_add(t01, k.round_mag);                       // round half to even to an integer
     t23 = f2_add(t23, k.round_mag);
     uint32_t r0, r1, r2, r3;
     u2_unpack(t01, r0, r1);
@@ -111,15 +124,14 @@ __device__ __forceinline__ void decode_word(uint32_t w, const RowDecode &rd, con
     uint32_t X01, X23;
     asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(X01) : "r"(r1), "r"(k.mul16), "r"(r0));
     asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(X23) : "r"(r3), "r"(k.mul16), "r"(r2));
-    const uint32_t M = 0x003F003Fu, E = 0x43004300u;
-    R[0] = ((X01 >> 9) & M) | E;
-    R[1] = ((X23 >> 9) & M) | E;
-    R[2] = ((X01 >> 6) & M) | E;
-    R[3] = ((X23 >> 6) & M) | E;
-    R[4] = ((X01 >> 3) & M) | E;
-    R[5] = ((X23 >> 3) & M) | E;
-    R[6] = (X01 & M) | E;
-    R[7] = (X23 & M) | E;
+    R[0] = and_or(X01 >> 9, k.wmask, k.wexp);
+    R[1] = and_or(X23 >> 9, k.wmask, k.wexp);
+    R[2] = and_or(X01 >> 6, k.wmask, k.wexp);
+    R[3] = and_or(X23 >> 6, k.wmask, k.wexp);
+    R[4] = and_or(X01 >> 3, k.wmask, k.wexp);
+    R[5] = and_or(X23 >> 3, k.wmask, k.wexp);
+    R[6] = and_or(X01, k.wmask, k.wexp);
+    R[7] = and_or(X23, k.wmask, k.wexp);
 }
 
 __device__ __forceinline__ void mma_bf16(float *c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -131,18 +143,77 @@ __device__ __forceinline__ void mma_bf16(float *c, uint32_t a0, uint32_t a1, uin
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// d = a*b + c with c given separately (the group's starting value)
+__device__ __forceinline__ void mma_bf16_c(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                           uint32_t b1, float c0, float c1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%10,%11};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
+}
+
+// fp32 value of bf16_rn(x): one conversion, the BF16 bits land in the high half
+__device__ __forceinline__ float round_bf16(float x) { return __uint_as_float(pack_bf16x2(0.0f, x)); }
+
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
+// One 64-column group of one stage for this thread: 4 code words (rows g, g+8 of both halves),
+// decode, 4 x NT x 2 mma, per-group rescale.  All shared-memory offsets are compile-time
+// constants once G is unrolled.
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ void group_step(const int G, const uint8_t *codes, uint32_t cbase, uint32_t cswz,
+                                           const uint8_t *xa, const uint8_t *gsb, const float sc[4],
+                                           const RowDecode rd[4], const DecodeConsts &kc, float (&acc)[2][NT][4]) {
+    constexpr int MP = 8 * NT;
+    const uint32_t coff = cbase + (((uint32_t)G << 4) ^ cswz);
+    const uint32_t w0 = *reinterpret_cast<const uint32_t *>(codes + coff);
+    const uint32_t w1 = *reinterpret_cast<const uint32_t *>(codes + coff + 1024);
+    const uint32_t w2 = *reinterpret_cast<const uint32_t *>(codes + kCodeTileBytes + coff);
+    const uint32_t w3 = *reinterpret_cast<const uint32_t *>(codes + kCodeTileBytes + coff + 1024);
+    uint32_t RA0[8], RA1[8], RB0[8], RB1[8];
+    decode_word(w0, rd[0], kc, RA0);
+    decode_word(w1, rd[1], kc, RA1);
+    decode_word(w2, rd[2], kc, RB0);
+    decode_word(w3, rd[3], kc, RB1);
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const float gs0 = *reinterpret_cast<const float *>(gsb + n * 256 + G * 4);
+        const float gs1 = *reinterpret_cast<const float *>(gsb + n * 256 + 32 + G * 4);
+        float cA[4], cB[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint2 b = *reinterpret_cast<const uint2 *>(xa + ((G * 4 + i) * MP + n * 8) * 32);
+            if (i == 0) {
+                mma_bf16_c(cA, RA0[0], RA1[0], RA0[1], RA1[1], b.x, b.y, gs0, gs1);
+                mma_bf16_c(cB, RB0[0], RB1[0], RB0[1], RB1[1], b.x, b.y, gs0, gs1);
+            } else {
+                mma_bf16(cA, RA0[2 * i], RA1[2 * i], RA0[2 * i + 1], RA1[2 * i + 1], b.x, b.y);
+                mma_bf16(cB, RB0[2 * i], RB1[2 * i], RB0[2 * i + 1], RB1[2 * i + 1], b.x, b.y);
+            }
+        }
+        acc[0][n][0] = fmaf(sc[0], cA[0], acc[0][n][0]);
+        acc[0][n][1] = fmaf(sc[0], cA[1], acc[0][n][1]);
+        acc[0][n][2] = fmaf(sc[1], cA[2], acc[0][n][2]);
+        acc[0][n][3] = fmaf(sc[1], cA[3], acc[0][n][3]);
+        acc[1][n][0] = fmaf(sc[2], cB[0], acc[1][n][0]);
+        acc[1][n][1] = fmaf(sc[2], cB[1], acc[1][n][1]);
+        acc[1][n][2] = fmaf(sc[3], cB[2], acc[1][n][2]);
+        acc[1][n][3] = fmaf(sc[3], cB[3], acc[1][n][3]);
+    }
+}
+
+template <int NT, bool TMA_SC>
+__global__ void __launch_bounds__(kThreads, Smem<NT>::kCtasPerSm)
 decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_xa,
-                      const __grid_constant__ CUtensorMap tm_gs, const DecodeGemmParams p) {
+                      const __grid_constant__ CUtensorMap tm_gs, const __grid_constant__ CUtensorMap tm_sc,
+                      const DecodeGemmParams p) {
     using S = Smem<NT>;
     constexpr int MP = S::MP;
     constexpr int kStages = S::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t full_bar[kStages], empty_bar[kStages];
+    __shared__ uint64_t full_bar[kStages], empty_bar[kStages], red_full, red_empty;
 
     const int e = blockIdx.z;
     const int rb = blockIdx.x;
@@ -161,46 +232,46 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
     const int ngroups = p.K / 64;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
+    const bool producer = threadIdx.x == 0;
+    if (producer) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full_bar[i], 1);
             mbar_init(&empty_bar[i], kConsumerWarps);
         }
+        mbar_init(&red_full, kRowWarps);
+        mbar_init(&red_empty, kRowWarps);
         fence_mbar_init();
+        prefetch_tensormap(&tm_codes);
+        prefetch_tensormap(&tm_xa);
+        prefetch_tensormap(&tm_gs);
+        if (TMA_SC) prefetch_tensormap(&tm_sc);
     }
     __syncthreads();
 
-    if (warp == kConsumerWarps) {
-        // ---------------- producer ----------------
-        if (lane == 0) {
-            prefetch_tensormap(&tm_codes);
-            prefetch_tensormap(&tm_xa);
-            prefetch_tensormap(&tm_gs);
-            bool ok = true;
-            for (int it = 0; it < total_iters && ok; ++it) {
-                const int slot = it % kStages;
-                if (it >= kStages) ok = mbar_wait(&empty_bar[slot], ((it / kStages) - 1) & 1, p.err);
-                if (!ok) break;
-                const int c = it / nst, st = s_begin + it % nst;
-                uint8_t *base = smem + slot * S::kStageBytes;
-                mbar_arrive_expect_tx(&full_bar[slot], S::kTxBytes);
-                tma_load_2d(base, &tm_codes, &full_bar[slot], st * 128, rowA);
-                tma_load_2d(base + kCodeTileBytes, &tm_codes, &full_bar[slot], st * 128, rowB);
-                tma_load_3d(base + 2 * kCodeTileBytes, &tm_xa, &full_bar[slot], 0, seg0 + c * MP, st * 32);
-                tma_load_2d(base + 2 * kCodeTileBytes + S::kXaBytes, &tm_gs, &full_bar[slot], st * 8,
-                            seg0 + c * MP);
-            }
-            // every issued copy must land before the CTA may exit
-            const int issued = ok ? total_iters : 0;
-            for (int it = max(0, issued - kStages); it < issued && ok; ++it)
-                ok = mbar_wait(&full_bar[it % kStages], (it / kStages) & 1, p.err);
+    // TMA loads of iteration `it` (token chunk, 512-column stage) into its ring slot
+    auto issue = [&](int it) {
+        const int slot = it % kStages;
+        const int c = it / nst, st = s_begin + it % nst;
+        uint8_t *base = smem + slot * S::kStageBytes;
+        mbar_arrive_expect_tx(&full_bar[slot], S::kTxBytes + (TMA_SC ? S::kScBytes : 0));
+        if (TMA_SC) {
+            uint8_t *sc = base + 2 * kCodeTileBytes + S::kXaBytes + S::kGsBytes;
+            tma_load_2d(sc, &tm_sc, &full_bar[slot], st * 8, rowA);
+            tma_load_2d(sc + S::kScBytes / 2, &tm_sc, &full_bar[slot], st * 8, rowB);
         }
-        return;
-    }
+        tma_load_2d(base, &tm_codes, &full_bar[slot], st * 128, rowA);
+        tma_load_2d(base + kCodeTileBytes, &tm_codes, &full_bar[slot], st * 128, rowB);
+        tma_load_3d(base + 2 * kCodeTileBytes, &tm_xa, &full_bar[slot], 0, seg0 + c * MP, st * 32);
+        tma_load_2d(base + 2 * kCodeTileBytes + S::kXaBytes, &tm_gs, &full_bar[slot], st * 8, seg0 + c * MP);
+    };
+    if (producer)
+        for (int it = 0; it < min(kStages - 1, total_iters); ++it) issue(it);
 
     // ---------------- consumers ----------------
     const int g = lane >> 2, tig = lane & 3;
-    const int wrow = warp * 16;  // this warp's 16 rows inside each 128-row half
+    const int wslot = warp & (kRowWarps - 1);  // row slot: 16 rows inside each 128-row half
+    const int khalf = warp / kRowWarps;        // 0: groups 0-3 of every stage, 1: groups 4-7
+    const int wrow = wslot * 16;
     // local rows (within the expert) of the four rows this thread decodes
     int lrow[4] = {localA + wrow + g, localA + wrow + g + 8, localB + wrow + g, localB + wrow + g + 8};
     RowDecode rd[4];
@@ -214,9 +285,12 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
         rd[r].bb = f2_pack(b, b);
     }
     DecodeConsts kc;
+    const uint32_t opaque = (uint32_t)(p.K >> 30);  // == 0; keeps the constants in registers
     kc.neg_magic = f2_pack(-8388608.0f, -8388608.0f);
     kc.round_mag = f2_pack(12582912.0f, 12582912.0f - 19264.0f);
-    kc.mul16 = 65536u + (uint32_t)(p.K >> 30);  // == 65536; kept opaque so it stays a multiply
+    kc.mul16 = 65536u + opaque;
+    kc.wmask = 0x003F003Fu ^ opaque;
+    kc.wexp = 0x43004300u ^ opaque;
 
     float acc[2][NT][4];
 #pragma unroll
@@ -226,70 +300,64 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc[t][n][q] = 0.0f;
 
-    const uint32_t swz = (uint32_t)g;  // row & 7 for rows wrow+g and wrow+g+8
+    // per-thread shared-memory offsets inside a stage
+    const uint32_t cbase = (uint32_t)(wrow + g) * 128u + 4u * (uint32_t)tig;  // code word of row wrow+g (unswizzled)
+    const uint32_t cswz = (uint32_t)g << 4;         // 128B swizzle of rows wrow+g and wrow+g+8
+    const uint32_t xa_thr = (uint32_t)g * 32u + (uint32_t)tig * 8u;  // B fragment of token g, lane tig
+    const uint32_t gs_thr = (uint32_t)(2 * tig) * 32u;               // group sums of token 2*tig
+    const uint32_t sc_thr = (uint32_t)(wrow + g) * 32u;              // scales of row wrow+g
 
+    bool ok = true;
+    int consumed = 0;  // iterations whose loads this thread has seen land
     for (int it = 0; it < total_iters; ++it) {
         const int slot = it % kStages;
         const int c = it / nst, st = s_begin + it % nst;
-        if (!mbar_wait(&full_bar[slot], (it / kStages) & 1, p.err)) break;
+        if (producer && it + kStages - 1 < total_iters) {
+            // refill the slot every warp released at iteration it-1 (kStages-1 stages of lookahead)
+            const int nx = it + kStages - 1;
+            if (nx >= kStages) ok = mbar_wait(&empty_bar[nx % kStages], ((nx / kStages) - 1) & 1, p.err);
+            if (ok) issue(nx);
+        }
+        if (!ok || !mbar_wait(&full_bar[slot], (it / kStages) & 1, p.err)) {
+            ok = false;
+            break;
+        }
+        consumed = it + 1;
         const uint8_t *base = smem + slot * S::kStageBytes;
-        const uint8_t *codesA = base, *codesB = base + kCodeTileBytes;
-        const uint8_t *xa = base + 2 * kCodeTileBytes;
-        const float *gs = reinterpret_cast<const float *>(base + 2 * kCodeTileBytes + S::kXaBytes);
-        const int g_lim = min(8, ngroups - st * 8);
+        const uint8_t *xa = base + 2 * kCodeTileBytes + xa_thr;
+        const uint8_t *gsb = base + 2 * kCodeTileBytes + S::kXaBytes + gs_thr;
+        if (TMA_SC) {
+            // full stage: groups beyond K read TMA zero fill (scale 0, activations 0) and add nothing
+            const uint8_t *scb = base + 2 * kCodeTileBytes + S::kXaBytes + S::kGsBytes + sc_thr;
+            {
+                // this warp's four groups of the stage: offsets are immediates
+                const int Gh = 4 * khalf;
+                const uint8_t *xah = xa + Gh * 4 * MP * 32;
+                const uint8_t *gsh = gsb + Gh * 4;
+                const uint8_t *sch = scb + Gh * 4;
+                const uint32_t cswz_h = cswz ^ ((uint32_t)Gh << 4);
+#pragma unroll
+                for (int G = 0; G < 4; ++G) {
+                    float sc[4];
+                    sc[0] = round_bf16(*reinterpret_cast<const float *>(sch + G * 4));
+                    sc[1] = round_bf16(*reinterpret_cast<const float *>(sch + 256 + G * 4));
+                    sc[2] = round_bf16(*reinterpret_cast<const float *>(sch + 4096 + G * 4));
+                    sc[3] = round_bf16(*reinterpret_cast<const float *>(sch + 4096 + 256 + G * 4));
+                    group_step<NT>(G, base, cbase, cswz_h, xah, gsh, sc, rd, kc, acc);
+                }
+            }
+        } else {
+            const int g_lim = min(8, ngroups - st * 8);
 #pragma unroll 1
-        for (int G = 0; G < g_lim; ++G) {
-            const int gg = st * 8 + G;
-            float sc[4];
+            for (int G = 4 * khalf; G < min(g_lim, 4 * khalf + 4); ++G) {
+                const int gg = st * 8 + G;
+                float sc[4];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int grow = e * p.N + (rvalid[r] ? lrow[r] : 0);
-                sc[r] = bf16_bits_to_float(float_to_bf16_bits(__ldg(p.scales + (size_t)grow * ngroups + gg)));
-            }
-            const uint32_t off0 = (uint32_t)(wrow + g) * 128u + ((((uint32_t)G) ^ swz) << 4) + 4u * tig;
-            const uint32_t off1 = off0 + 8u * 128u;
-            const uint32_t w0 = *reinterpret_cast<const uint32_t *>(codesA + off0);
-            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(codesA + off1);
-            const uint32_t w2 = *reinterpret_cast<const uint32_t *>(codesB + off0);
-            const uint32_t w3 = *reinterpret_cast<const uint32_t *>(codesB + off1);
-            uint32_t RA0[8], RA1[8], RB0[8], RB1[8];
-            decode_word(w0, rd[0], kc, RA0);
-            decode_word(w1, rd[1], kc, RA1);
-            decode_word(w2, rd[2], kc, RB0);
-            decode_word(w3, rd[3], kc, RB1);
-            float cg[2][NT][4];
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const float gs0 = gs[(n * 8 + 2 * tig) * 8 + G];
-                const float gs1 = gs[(n * 8 + 2 * tig + 1) * 8 + G];
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    cg[t][n][0] = gs0;
-                    cg[t][n][1] = gs1;
-                    cg[t][n][2] = gs0;
-                    cg[t][n][3] = gs1;
+                for (int r = 0; r < 4; ++r) {
+                    const int grow = e * p.N + (rvalid[r] ? lrow[r] : 0);
+                    sc[r] = round_bf16(__ldg(p.scales + (size_t)grow * ngroups + gg));
                 }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    const uint2 b = *reinterpret_cast<const uint2 *>(
-                        xa + ((size_t)((G * 4 + i) * MP + n * 8 + g) * 16 + tig * 4) * 2);
-                    mma_bf16(cg[0][n], RA0[2 * i], RA1[2 * i], RA0[2 * i + 1], RA1[2 * i + 1], b.x, b.y);
-                    mma_bf16(cg[1][n], RB0[2 * i], RB1[2 * i], RB0[2 * i + 1], RB1[2 * i + 1], b.x, b.y);
-                }
-            }
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                acc[0][n][0] = fmaf(sc[0], cg[0][n][0], acc[0][n][0]);
-                acc[0][n][1] = fmaf(sc[0], cg[0][n][1], acc[0][n][1]);
-                acc[0][n][2] = fmaf(sc[1], cg[0][n][2], acc[0][n][2]);
-                acc[0][n][3] = fmaf(sc[1], cg[0][n][3], acc[0][n][3]);
-                acc[1][n][0] = fmaf(sc[2], cg[1][n][0], acc[1][n][0]);
-                acc[1][n][1] = fmaf(sc[2], cg[1][n][1], acc[1][n][1]);
-                acc[1][n][2] = fmaf(sc[3], cg[1][n][2], acc[1][n][2]);
-                acc[1][n][3] = fmaf(sc[3], cg[1][n][3], acc[1][n][3]);
+                group_step<NT>(G, base, cbase, cswz, xa, gsb, sc, rd, kc, acc);
             }
         }
         __syncwarp();
@@ -297,8 +365,31 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
 
         if (st == s_end - 1) {
             // ---------------- epilogue for token chunk c ----------------
+            // the second warp of each row slot hands its partial sums to the first (bounded waits)
+            float *red = reinterpret_cast<float *>(smem + kStages * S::kStageBytes) + (wslot * 32 + lane) * (2 * NT * 4);
+            if (khalf == 1) {
+                if (c > 0 && !mbar_wait(&red_empty, (c - 1) & 1, p.err)) break;
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int n = 0; n < NT; ++n)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) red[(t * NT + n) * 4 + q] = acc[t][n][q];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&red_full);
+            } else {
+                if (!mbar_wait(&red_full, c & 1, p.err)) break;
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int n = 0; n < NT; ++n)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) acc[t][n][q] += red[(t * NT + n) * 4 + q];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&red_empty);
+            }
+#pragma unroll
+            for (int n = 0; n < NT && khalf == 0; ++n) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int tok = c * MP + n * 8 + 2 * tig + (q & 1);
@@ -337,29 +428,36 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
                     for (int q = 0; q < 4; ++q) acc[t][n][q] = 0.0f;
         }
     }
+    if (producer && !ok) {
+        // after a failed wait: let the copies already issued land before the CTA exits (bounded)
+        const int issued = min(total_iters, consumed + kStages - 1);
+        for (int it = consumed; it < issued; ++it)
+            if (!mbar_wait(&full_bar[it % kStages], (it / kStages) & 1, p.err)) break;
+    }
 }
 
 template <int NT>
 cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUtensorMap &b,
-                      const CUtensorMap &c, int row_blocks, int ksplit, int experts, cudaStream_t s) {
-    auto kern = decode_gemm_w2_kernel<NT>;
+                      const CUtensorMap &c, const CUtensorMap &d, int row_blocks, int ksplit, int experts,
+                      cudaStream_t s) {
+    auto kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true> : decode_gemm_w2_kernel<NT, false>;
     const int smem = Smem<NT>::kTotal;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     dim3 grid(row_blocks, ksplit, experts);
-    kern<<<grid, kThreads, smem, s>>>(a, b, c, p);
+    kern<<<grid, kThreads, smem, s>>>(a, b, c, d, p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_decode_gemm_w2(const DecodeGemmParams &p, const CUtensorMap &tm_codes,
-                                  const CUtensorMap &tm_xa, const CUtensorMap &tm_gs, int row_blocks,
-                                  int ksplit, int experts, int nt, cudaStream_t s) {
+                                  const CUtensorMap &tm_xa, const CUtensorMap &tm_gs, const CUtensorMap &tm_sc,
+                                  int row_blocks, int ksplit, int experts, int nt, cudaStream_t s) {
     switch (nt) {
-        case 1: return launch_nt<1>(p, tm_codes, tm_xa, tm_gs, row_blocks, ksplit, experts, s);
-        case 2: return launch_nt<2>(p, tm_codes, tm_xa, tm_gs, row_blocks, ksplit, experts, s);
-        case 4: return launch_nt<4>(p, tm_codes, tm_xa, tm_gs, row_blocks, ksplit, experts, s);
+        case 1: return launch_nt<1>(p, tm_codes, tm_xa, tm_gs, tm_sc, row_blocks, ksplit, experts, s);
+        case 2: return launch_nt<2>(p, tm_codes, tm_xa, tm_gs, tm_sc, row_blocks, ksplit, experts, s);
+        case 4: return launch_nt<4>(p, tm_codes, tm_xa, tm_gs, tm_sc, row_blocks, ksplit, experts, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -48,12 +48,43 @@ struct DecodeGemmParams {
     const float *rw;      // EPI_DOWN: routing weight per operand row
     int h_P;              // EPI_GATEUP: rows of the H operand (== P)
     int I;                // EPI_GATEUP: gate rows per expert
+    int tma_scales;       // 1: scales staged by TMA with the codes (row pitch a multiple of 16 B)
     uint32_t *err;
 };
 
 cudaError_t launch_decode_gemm_w2(const DecodeGemmParams &p, const CUtensorMap &tm_codes,
-                                  const CUtensorMap &tm_xa, const CUtensorMap &tm_gs, int row_blocks,
-                                  int ksplit, int experts, int nt, cudaStream_t s);
+                                  const CUtensorMap &tm_xa, const CUtensorMap &tm_gs, const CUtensorMap &tm_sc,
+                                  int row_blocks, int ksplit, int experts, int nt, cudaStream_t s);
+
+// Prefill-sized tcgen05 kernel.
+struct TcGemmParams {
+    const float *scales;   // [rows_total][K/64]
+    const float *alpha;    // [rows_total]
+    const float *beta;     // [rows_total]
+    int N;                 // rows per expert
+    int K;
+    int row_block_stride;  // local row of row tile nt = nt * row_block_stride
+    int half_stride;       // second 128-row half of a tile starts half_stride rows later
+    int n_tiles;           // row tiles per expert
+    const int2 *tile_list; // (expert, token tile) entries; NULL: (0, i) for i < static_tiles
+    const int *tile_count; // device count of tile_list entries; NULL: static_tiles
+    int static_tiles;
+    int m_tile;            // tokens per token tile (128 * MT)
+    const int *seg_off;    // [E+1] operand row segments; NULL: one segment of M rows
+    int M;
+    int mode;              // EPI_GATEUP, EPI_DOWN or EPI_BF16
+    void *out;
+    int out_ld;
+    const float *rw;       // EPI_DOWN: routing weight per operand row
+    int I;                 // EPI_GATEUP: gate rows per expert
+    uint32_t *err;
+};
+
+cudaError_t launch_tc_gemm_w2(const TcGemmParams &p, const CUtensorMap &tm_a, const CUtensorMap &tm_codes, int mt,
+                              int grid, cudaStream_t s);
+cudaError_t launch_build_tiles(const int *seg_off, int E, int m_tile, int2 *list, int *count, cudaStream_t s);
+// rows gathered by tok_of (or identity), each 16-column block in the decoders' window-major order
+cudaError_t launch_pack_xt(const uint16_t *x, const int *tok_of, int P_valid, int K, uint16_t *xt, cudaStream_t s);
 
 cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, const float *alpha,
                            const float *beta, int rows, int K, uint16_t *out, cudaStream_t s);

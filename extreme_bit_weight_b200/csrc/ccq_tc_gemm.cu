@@ -1,0 +1,484 @@
+// Prefill-sized CCQ W2A16 grouped matmul on the 5th-generation tensor cores (tcgen05 + TMEM),
+// sm_100a.  The grouped GEMM of the CCQ paper's Table 5 at prefill batch sizes, and the dense
+// large-M shape.
+//
+// Tile: 128*MT tokens x 256 weight rows (two 128-row halves of the weight) x K in steps of one
+// 64-column group.  Persistent CTAs walk a device-built list of (expert, token-tile) entries
+// crossed with the weight's row tiles.  Warp roles:
+//   warp 0      TMA producer: activation tiles ([128 tok][64] BF16, 128B swizzle) and code tiles
+//               ([128 rows][64 B], 64B swizzle, 4 groups per load)
+//   warp 1      TMEM allocation and the single MMA-issuing thread (tcgen05.mma kind::f16,
+//               M=128, N=256, K=16, fp32 accumulators in TMEM)
+//   warps 2-9   decoders: each thread owns one weight row of the tile, decodes its 16 code bytes of
+//               the group (CCQ §3.3 Eq. 1 inverted / §3.5 Algorithm 3: fp32 FMA, ties-to-even
+//               rounding, Table 1 shifts) to BF16 w = bf16((u - 32) * bf16(scale)) and stores them
+//               as the MMA B operand in the canonical K-major 128B-swizzled shared-memory layout
+//   warps 10-13 epilogue: tcgen05.ld of the accumulators; SiLU(gate)*up, routing-weight scaling or
+//               BF16 conversion; stores to global memory
+// Column order: within every 16-column block the decoders emit the 16 weights of one 4-byte word
+// window-major (position 4i + j holds state window i of byte j, i.e. column 4j + i), so the
+// activation operand is stored with the same permutation (see pack_xt).  Every column is then
+// multiplied by its own weight; only the order of the k sum inside a block differs.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ccq_device.cuh"
+#include "ccq_kernels.cuh"
+
+namespace ccq {
+namespace {
+
+constexpr int kDecWarps = 8;
+constexpr int kEpiWarps = 4;
+constexpr int kTcThreads = (2 + kDecWarps + kEpiWarps) * 32;  // 448
+constexpr int kSA = 3;   // activation stages
+constexpr int kSB = 2;   // decoded-weight stages
+constexpr int kSC = 2;   // code stages (4 groups each)
+constexpr int kATile = 128 * 64 * 2;   // 16 KB per 128-token sub-tile
+constexpr int kBTile = 256 * 64 * 2;   // 32 KB
+constexpr int kCTile = 2 * 128 * 64;   // 16 KB: two 128-row halves x 64 code bytes
+
+template <int MT>
+struct TcSmem {
+    static constexpr int kA = kSA * MT * kATile;
+    static constexpr int kB = kSB * kBTile;
+    static constexpr int kC = kSC * kCTile;
+    static constexpr int kTotal = kA + kB + kC + 1024;
+    static_assert(kTotal + 512 <= 227 * 1024, "shared memory per CTA");
+};
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;             // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset: one 8-row x 128 B swizzle atom
+    d |= (uint64_t)1 << 46;             // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;             // 128-byte swizzle
+    return d;
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, BF16 A and B, both K-major, M=128, N=256.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+__device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// One 4-byte word of a row -> 16 BF16 weights (u - 32) * s in window-major order, as 8 registers:
+// out[2i], out[2i+1] = window i of bytes (0,1) and (2,3).
+__device__ __forceinline__ void decode_word_bf16(uint32_t w, float alpha, float beta, uint32_t s2, uint32_t out[8]) {
+    const uint32_t magic = 0x4B000000u;
+    float c[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) c[b] = __uint_as_float(prmt(w, magic, 0x7650u + b)) - 8388608.0f;
+    uint32_t r[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const float t = __fmaf_rn(c[b], alpha, beta);
+        r[b] = __float_as_uint(__fadd_rn(t, (b & 1) ? 12563648.0f : 12582912.0f));
+    }
+    const uint32_t X01 = r[1] * 65536u + r[0];
+    const uint32_t X23 = r[3] * 65536u + r[2];
+    const uint32_t M = 0x003F003Fu, E = 0x43004300u, Z = 0x43204320u;  // Z = bf16x2(160, 160)
+    out[0] = bmul2(bsub2(((X01 >> 9) & M) | E, Z), s2);
+    out[1] = bmul2(bsub2(((X23 >> 9) & M) | E, Z), s2);
+    out[2] = bmul2(bsub2(((X01 >> 6) & M) | E, Z), s2);
+    out[3] = bmul2(bsub2(((X23 >> 6) & M) | E, Z), s2);
+    out[4] = bmul2(bsub2(((X01 >> 3) & M) | E, Z), s2);
+    out[5] = bmul2(bsub2(((X23 >> 3) & M) | E, Z), s2);
+    out[6] = bmul2(bsub2((X01 & M) | E, Z), s2);
+    out[7] = bmul2(bsub2((X23 & M) | E, Z), s2);
+}
+
+__device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
+
+// position p of a 16-column block holds column 4*(p%4) + p/4 (and the map is its own inverse)
+__device__ __forceinline__ int perm16(int p) { return ((p & 3) << 2) | (p >> 2); }
+
+struct TileInfo {
+    int e, m0, seg0, Me, nt;
+};
+
+__device__ __forceinline__ bool tile_of(const TcGemmParams &p, int w, TileInfo &t) {
+    const int li = w / p.n_tiles;
+    t.nt = w - li * p.n_tiles;
+    const int2 ent = p.tile_list ? p.tile_list[li] : make_int2(0, li);
+    t.e = ent.x;
+    t.seg0 = p.seg_off ? p.seg_off[t.e] : 0;
+    t.Me = p.seg_off ? p.seg_off[t.e + 1] - t.seg0 : p.M;
+    t.m0 = ent.y * p.m_tile;
+    return true;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kTcThreads, 1)
+tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_codes,
+                  const TcGemmParams p) {
+    using S = TcSmem<MT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + S::kA;
+    uint8_t *sC = smem + S::kA + S::kB;
+    __shared__ uint64_t a_full[kSA], a_empty[kSA], b_full[kSB], b_empty[kSB], c_full[kSC], c_empty[kSC];
+    __shared__ uint64_t acc_full, acc_empty;
+    __shared__ uint32_t tmem_base_slot;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int total_work = (p.tile_count ? *p.tile_count : p.static_tiles) * p.n_tiles;
+    const int nk = p.K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kSA; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < kSB; ++i) { mbar_init(&b_full[i], kDecWarps); mbar_init(&b_empty[i], 1); }
+        for (int i = 0; i < kSC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], kDecWarps); }
+        mbar_init(&acc_full, 1);
+        mbar_init(&acc_empty, kEpiWarps);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_slot)),
+                     "r"(MT * 256));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_slot;
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            prefetch_tensormap(&tm_a);
+            prefetch_tensormap(&tm_codes);
+            uint32_t ai = 0, ci = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < total_work && ok; w += gridDim.x) {
+                TileInfo t;
+                tile_of(p, w, t);
+                const int localA = t.nt * p.row_block_stride;
+                const int rowA = t.e * p.N + localA, rowB = rowA + p.half_stride;
+                for (int ks = 0; ks < nk && ok; ++ks) {
+                    if ((ks & 3) == 0) {
+                        const int s = ci % kSC;
+                        if (ci >= kSC) ok = mbar_wait(&c_empty[s], ((ci / kSC) - 1) & 1, p.err);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(&c_full[s], kCTile);
+                        tma_load_2d(sC + s * kCTile, &tm_codes, &c_full[s], (ks >> 2) * 64, rowA);
+                        tma_load_2d(sC + s * kCTile + kCTile / 2, &tm_codes, &c_full[s], (ks >> 2) * 64, rowB);
+                        ++ci;
+                    }
+                    const int s = ai % kSA;
+                    if (ai >= kSA) ok = mbar_wait(&a_empty[s], ((ai / kSA) - 1) & 1, p.err);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&a_full[s], MT * kATile);
+#pragma unroll
+                    for (int j = 0; j < MT; ++j)
+                        tma_load_2d(sA + (s * MT + j) * kATile, &tm_a, &a_full[s], ks * 64, t.seg0 + t.m0 + j * 128);
+                    ++ai;
+                }
+            }
+            // drain: the last copies must land before exit
+            for (uint32_t i = (ai > kSA ? ai - kSA : 0); i < ai && ok; ++i)
+                ok = mbar_wait(&a_full[i % kSA], (i / kSA) & 1, p.err);
+            for (uint32_t i = (ci > kSC ? ci - kSC : 0); i < ci && ok; ++i)
+                ok = mbar_wait(&c_full[i % kSC], (i / kSC) & 1, p.err);
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            uint32_t ai = 0, bi = 0, ti = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < total_work && ok; w += gridDim.x, ++ti) {
+                if (ti > 0) ok = mbar_wait(&acc_empty, (ti - 1) & 1, p.err);
+                if (!ok) break;
+                tc_fence_after();
+                for (int ks = 0; ks < nk && ok; ++ks) {
+                    const int sa = ai % kSA, sb = bi % kSB;
+                    ok = mbar_wait(&a_full[sa], (ai / kSA) & 1, p.err) && mbar_wait(&b_full[sb], (bi / kSB) & 1, p.err);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int j = 0; j < MT; ++j) {
+                        const uint32_t abase = smem_u32(sA + (sa * MT + j) * kATile);
+                        const uint32_t bbase = smem_u32(sB + sb * kBTile);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16_ss(tmem + j * 256, smem_desc_sw128(abase + kk * 32), smem_desc_sw128(bbase + kk * 32),
+                                        (ks > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&a_empty[sa]);
+                    mma_commit(&b_empty[sb]);
+                    ++ai;
+                    ++bi;
+                }
+                if (ok) mma_commit(&acc_full);
+            }
+            // the last MMAs must be complete before TMEM is freed
+            if (ok && ti > 0) ok = mbar_wait(&acc_full, (ti - 1) & 1, p.err);
+            (void)ok;
+        }
+    } else if (warp < 2 + kDecWarps) {
+        // ------------------------------ decoders ------------------------------
+        const int r = threadIdx.x - 64;  // weight row within the tile, 0..255
+        const int half = r >> 7, rr = r & 127;
+        uint32_t bi = 0, ci = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < total_work && ok; w += gridDim.x) {
+            TileInfo t;
+            tile_of(p, w, t);
+            const int local = t.nt * p.row_block_stride + half * p.half_stride + rr;
+            const bool valid = local < p.N;
+            const size_t grow = (size_t)t.e * p.N + (valid ? local : 0);
+            const float alpha = __ldg(p.alpha + grow), beta = __ldg(p.beta + grow);
+            const float *srow = p.scales + grow * nk;
+            for (int ks = 0; ks < nk && ok; ++ks) {
+                const int cs = ci % kSC;
+                if ((ks & 3) == 0) {
+                    ok = mbar_wait(&c_full[cs], (ci / kSC) & 1, p.err);
+                    if (!ok) break;
+                }
+                // this row's 16 code bytes of group ks (64-byte rows, 64B swizzle)
+                const uint8_t *crow = sC + cs * kCTile + half * (kCTile / 2) + rr * 64;
+                const uint32_t chunk = (uint32_t)(ks & 3) ^ (((uint32_t)rr >> 1) & 3u);
+                const uint4 q = *reinterpret_cast<const uint4 *>(crow + (chunk << 4));
+                if ((ks & 3) == 3 || ks == nk - 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&c_empty[cs]);
+                    ++ci;
+                }
+                const float sc = bf16_bits_to_float(float_to_bf16_bits(__ldg(srow + ks)));
+                const uint32_t s2 = pack_bf16x2(sc, sc);
+                uint32_t o[4][8];
+                decode_word_bf16(q.x, alpha, beta, s2, o[0]);
+                decode_word_bf16(q.y, alpha, beta, s2, o[1]);
+                decode_word_bf16(q.z, alpha, beta, s2, o[2]);
+                decode_word_bf16(q.w, alpha, beta, s2, o[3]);
+                const int sb = bi % kSB;
+                if (bi >= kSB) ok = mbar_wait(&b_empty[sb], ((bi / kSB) - 1) & 1, p.err);
+                if (!ok) break;
+                uint8_t *brow = sB + sb * kBTile + r * 128;
+#pragma unroll
+                for (int wd = 0; wd < 4; ++wd) {
+                    const uint32_t c0 = (uint32_t)(2 * wd) ^ ((uint32_t)r & 7u);
+                    const uint32_t c1 = (uint32_t)(2 * wd + 1) ^ ((uint32_t)r & 7u);
+                    *reinterpret_cast<uint4 *>(brow + (c0 << 4)) = make_uint4(o[wd][0], o[wd][1], o[wd][2], o[wd][3]);
+                    *reinterpret_cast<uint4 *>(brow + (c1 << 4)) = make_uint4(o[wd][4], o[wd][5], o[wd][6], o[wd][7]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&b_full[sb]);
+                ++bi;
+            }
+        }
+    } else {
+        // ------------------------------ epilogue ------------------------------
+        const int q = warp & 3;        // TMEM lane quarter this warp may access
+        const int m = q * 32 + lane;   // accumulator row = token within the 128-token sub-tile
+        uint32_t ti = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < total_work && ok; w += gridDim.x, ++ti) {
+            TileInfo t;
+            tile_of(p, w, t);
+            ok = mbar_wait(&acc_full, ti & 1, p.err);
+            if (!ok) break;
+            tc_fence_after();
+            const int localA = t.nt * p.row_block_stride;
+#pragma unroll 1
+            for (int j = 0; j < MT; ++j) {
+                const int tok = t.m0 + j * 128 + m;
+                const bool live = tok < t.Me;
+                const size_t prow = (size_t)(t.seg0 + tok);
+                const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(j * 256);
+                if (p.mode == EPI_GATEUP) {
+#pragma unroll 1
+                    for (int c = 0; c < 128; c += 32) {
+                        uint32_t g[32], u[32];
+                        tmem_ld32(tbase + c, g);
+                        tmem_ld32(tbase + 128 + c, u);
+                        tmem_ld_wait();
+                        if (!live || localA + c >= p.I) continue;
+                        uint32_t h[16];
+#pragma unroll
+                        for (int b = 0; b < 2; ++b)
+#pragma unroll
+                            for (int pp = 0; pp < 16; pp += 2) {
+                                const int c0 = 16 * b + perm16(pp), c1 = 16 * b + perm16(pp + 1);
+                                const float h0 = silu(__uint_as_float(g[c0])) * __uint_as_float(u[c0]);
+                                const float h1 = silu(__uint_as_float(g[c1])) * __uint_as_float(u[c1]);
+                                h[8 * b + pp / 2] = pack_bf16x2(h0, h1);
+                            }
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + prow * p.out_ld + localA + c);
+                        dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
+                        dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+                        dst[2] = make_uint4(h[8], h[9], h[10], h[11]);
+                        dst[3] = make_uint4(h[12], h[13], h[14], h[15]);
+                    }
+                } else {
+                    const float rwv = (p.mode == EPI_DOWN && live) ? __ldg(p.rw + prow) : 1.0f;
+#pragma unroll 1
+                    for (int c = 0; c < 256; c += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(tbase + c, v);
+                        tmem_ld_wait();
+                        const int lr = localA + (c >= 128 ? p.half_stride - 128 : 0) + c;  // local row of column c
+                        if (!live || lr >= p.N) continue;
+                        if (p.mode == EPI_DOWN && lr + 32 > p.N) {  // partial chunk of rows
+                            float *dst = static_cast<float *>(p.out) + prow * p.out_ld + lr;
+#pragma unroll
+                            for (int z = 0; z < 32; ++z)
+                                if (lr + z < p.N) dst[z] = rwv * __uint_as_float(v[z]);
+                        } else if (p.mode == EPI_DOWN) {
+                            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + prow * p.out_ld + lr);
+#pragma unroll
+                            for (int z = 0; z < 8; ++z)
+                                dst[z] = make_float4(rwv * __uint_as_float(v[4 * z]), rwv * __uint_as_float(v[4 * z + 1]),
+                                                     rwv * __uint_as_float(v[4 * z + 2]), rwv * __uint_as_float(v[4 * z + 3]));
+                        } else if (lr + 32 <= p.N) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + prow * p.out_ld + lr);
+#pragma unroll
+                            for (int z = 0; z < 4; ++z)
+                                dst[z] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * z]), __uint_as_float(v[8 * z + 1])),
+                                                    pack_bf16x2(__uint_as_float(v[8 * z + 2]), __uint_as_float(v[8 * z + 3])),
+                                                    pack_bf16x2(__uint_as_float(v[8 * z + 4]), __uint_as_float(v[8 * z + 5])),
+                                                    pack_bf16x2(__uint_as_float(v[8 * z + 6]), __uint_as_float(v[8 * z + 7])));
+                        } else {  // last, partial chunk of rows (N is a multiple of 16, not of 32)
+                            uint16_t *dst = static_cast<uint16_t *>(p.out) + prow * p.out_ld + lr;
+#pragma unroll
+                            for (int z = 0; z < 32; ++z)
+                                if (lr + z < p.N) dst[z] = float_to_bf16_bits(__uint_as_float(v[z]));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(MT * 256));
+    }
+}
+
+// Tile list: one entry (expert, token tile) per 128*MT tokens of each expert's segment.
+__global__ void build_tiles_kernel(const int *__restrict__ seg_off, int E, int m_tile, int2 *__restrict__ list,
+                                   int *__restrict__ count) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    int n = 0;
+    for (int e = 0; e < E; ++e) {
+        const int Me = seg_off[e + 1] - seg_off[e];
+        for (int m = 0; m * m_tile < Me; ++m) list[n++] = make_int2(e, m);
+    }
+    *count = n;
+}
+
+// Prefill activation operand: rows gathered by tok_of (or identity), each 16-column block stored in
+// the decoders' window-major order (position p <- column perm16(p)).
+__global__ void pack_xt_kernel(const uint16_t *__restrict__ x, const int *__restrict__ tok_of, int P_valid, int K,
+                               uint16_t *__restrict__ xt) {
+    const int nb = K / 16;
+    const size_t total = (size_t)P_valid * nb;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int pr = (int)(idx / nb), b = (int)(idx % nb);
+        const int src = tok_of ? __ldg(tok_of + pr) : pr;
+        const uint4 *s = reinterpret_cast<const uint4 *>(x + (size_t)src * K + (size_t)b * 16);
+        const uint4 v0 = __ldg(s), v1 = __ldg(s + 1);
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        uint16_t in[16], o[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            in[2 * i] = (uint16_t)(w[i] & 0xFFFFu);
+            in[2 * i + 1] = (uint16_t)(w[i] >> 16);
+        }
+#pragma unroll
+        for (int pp = 0; pp < 16; ++pp) o[pp] = in[perm16(pp)];
+        uint4 *d = reinterpret_cast<uint4 *>(xt + (size_t)pr * K + (size_t)b * 16);
+        d[0] = make_uint4((uint32_t)o[0] | ((uint32_t)o[1] << 16), (uint32_t)o[2] | ((uint32_t)o[3] << 16),
+                          (uint32_t)o[4] | ((uint32_t)o[5] << 16), (uint32_t)o[6] | ((uint32_t)o[7] << 16));
+        d[1] = make_uint4((uint32_t)o[8] | ((uint32_t)o[9] << 16), (uint32_t)o[10] | ((uint32_t)o[11] << 16),
+                          (uint32_t)o[12] | ((uint32_t)o[13] << 16), (uint32_t)o[14] | ((uint32_t)o[15] << 16));
+    }
+}
+
+template <int MT>
+cudaError_t launch_tc_mt(const TcGemmParams &p, const CUtensorMap &ta, const CUtensorMap &tc, int grid, cudaStream_t s) {
+    auto kern = tc_gemm_w2_kernel<MT>;
+    const int smem = TcSmem<MT>::kTotal;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, kTcThreads, smem, s>>>(ta, tc, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_gemm_w2(const TcGemmParams &p, const CUtensorMap &tm_a, const CUtensorMap &tm_codes, int mt,
+                              int grid, cudaStream_t s) {
+    if (mt == 1) return launch_tc_mt<1>(p, tm_a, tm_codes, grid, s);
+    if (mt == 2) return launch_tc_mt<2>(p, tm_a, tm_codes, grid, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_build_tiles(const int *seg_off, int E, int m_tile, int2 *list, int *count, cudaStream_t s) {
+    build_tiles_kernel<<<1, 32, 0, s>>>(seg_off, E, m_tile, list, count);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_xt(const uint16_t *x, const int *tok_of, int P_valid, int K, uint16_t *xt, cudaStream_t s) {
+    if (P_valid <= 0) return cudaSuccess;
+    size_t work = (size_t)P_valid * (K / 16);
+    size_t b = (work + 255) / 256;
+    if (b > 148 * 32) b = 148 * 32;
+    pack_xt_kernel<<<(int)b, 256, 0, s>>>(x, tok_of, P_valid, K, xt);
+    return cudaGetLastError();
+}
+
+}  // namespace ccq

@@ -84,13 +84,25 @@ def test_dequant_w4_bitexact(ccq):
 # ----------------------------------------------------------------------------------------------
 # decode-sized matmul
 # ----------------------------------------------------------------------------------------------
-def test_gemm_one_hot_identity(ccq):
-    # x = I_K: y[m][n] = w[n][m], so every weight the fused kernel decodes is observed exactly
+def test_gemm_one_hot_identity_small_m(ccq):
+    # x = rows of I_K, 16 at a time (the register-decode mma.sync kernel): y[m][n] = w[n][m], so
+    # every weight the fused kernel decodes is observed exactly
     n, k = 272, 320
     codes, scales, alpha, beta = synth.w2_format_random(n, k, 1400)
     W = w2_weight(ccq, codes, scales, alpha, beta)
-    x = synth.one_hot_rows(k).cuda()
-    y = ccq.ccq_w2a16_gemm(W, x).float().cpu().numpy()
+    eye = synth.one_hot_rows(k).cuda()
+    ref = oracle.bf16_to_f64(oracle.dequant_w2(codes, scales, alpha, beta)).T
+    for j in range(0, k, 16):
+        y = ccq.ccq_w2a16_gemm(W, eye[j:j + 16].contiguous()).float().cpu().numpy()
+        assert np.array_equal(y, ref[j:j + 16].astype(np.float32)), j
+
+
+def test_gemm_one_hot_identity_tcgen05(ccq):
+    # x = I_K with K >= 48 rows runs the tcgen05 kernel: decoded BF16 weights in shared memory
+    n, k = 528, 576
+    codes, scales, alpha, beta = synth.w2_format_random(n, k, 1401)
+    W = w2_weight(ccq, codes, scales, alpha, beta)
+    y = ccq.ccq_w2a16_gemm(W, synth.one_hot_rows(k).cuda()).float().cpu().numpy()
     ref = oracle.bf16_to_f64(oracle.dequant_w2(codes, scales, alpha, beta)).T
     assert np.array_equal(y, ref.astype(np.float32))
 
@@ -108,7 +120,8 @@ def test_gemm_small_linear(ccq):
 
 
 @pytest.mark.parametrize("m,n,k", [(1, 16, 64), (3, 48, 192), (8, 256, 512), (9, 272, 576), (17, 128, 1088),
-                                   (33, 256, 1024), (1, 8192, 8192), (16, 8192, 8192)])
+                                   (33, 256, 1024), (1, 8192, 8192), (16, 8192, 8192),
+                                   (48, 256, 256), (130, 272, 576), (300, 512, 1088), (128, 8192, 8192)])
 def test_gemm_shapes(ccq, m, n, k):
     codes, scales, alpha, beta = synth.w2_format_random(n, k, 1500 + m + n + k)
     W = w2_weight(ccq, codes, scales, alpha, beta)
@@ -232,6 +245,47 @@ def test_moe_decode_layer_full_size_sampled(ccq):
                                 a13[e * 2 * I:(e + 1) * 2 * I], b13[e * 2 * I:(e + 1) * 2 * I])
         d2 = oracle.dequant_w2(c2[e * H:(e + 1) * H], s2[e * H:(e + 1) * H], a2[e * H:(e + 1) * H],
                                b2[e * H:(e + 1) * H])
+        for si, t in enumerate(sample):
+            for j in range(topk):
+                if ids[t, j] == e:
+                    ref[si] += float(rw[t, j]) * oracle.expert_ffn_f64(xb[t:t + 1], d13, d2, round_h=True)[0]
+    assert rel_err(y[sample], ref) <= TOL
+
+
+@pytest.mark.parametrize("T,E,topk,H,I,zipf", [(256, 8, 2, 256, 128, False), (512, 16, 4, 1024, 512, True),
+                                               (700, 4, 1, 576, 192, False)])
+def test_moe_prefill_full(ccq, T, E, topk, H, I, zipf):
+    # prefill-sized (>= 48 rows per expert on average): tcgen05 grouped GEMMs
+    W13, W2, d13, d2 = moe_weights(ccq, E, H, I, 2400 + T)
+    x = synth.activations(T, H, 2401 + T, outlier_frac=0.01)
+    ids, rw = (synth.routing_zipf(T, E, topk, 2402 + T) if zipf else synth.routing_uniform(T, E, topk, 2402 + T))
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    xb = synth.bf16_bits(x)
+    ref = oracle.moe_f64(xb, d13, d2, ids, rw, round_h=True)
+    assert rel_err(y, ref) <= TOL
+    assert rel_err(y, oracle.moe_f64(xb, d13, d2, ids, rw, round_h=False)) <= TOL
+
+
+def test_moe_prefill_layer_full_size_sampled(ccq):
+    # the prefill-sized MoE layer: 4096 tokens, hidden 8192, 64 experts, top-8 with Zipf(1.1) expert
+    # popularity, activations N(0,1) with 1% of channels x20; checked on sampled tokens
+    T, H, I, E, topk = 4096, 8192, 3584, 64, 8
+    c13, s13, a13, b13 = synth.w2_format_random(E * 2 * I, H, 3100)
+    c2, s2, a2, b2 = synth.w2_format_random(E * H, I, 3101)
+    W13 = ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, 2 * I, H, c13, s13, a13, b13, experts=E)
+    W2 = ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, H, I, c2, s2, a2, b2, experts=E)
+    x = synth.activations(T, H, 3102, outlier_frac=0.01, outlier_scale=20.0)
+    ids, rw = synth.routing_zipf(T, E, topk, 3103, s=1.1)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    xb = synth.bf16_bits(x)
+    sample = [0, 1, 2047, 4095]
+    ref = np.zeros((len(sample), H))
+    for e in sorted({int(ids[t, j]) for t in sample for j in range(topk)}):
+        sl13, sl2 = slice(e * 2 * I, (e + 1) * 2 * I), slice(e * H, (e + 1) * H)
+        d13 = oracle.dequant_w2(c13[sl13], s13[sl13], a13[sl13], b13[sl13])
+        d2 = oracle.dequant_w2(c2[sl2], s2[sl2], a2[sl2], b2[sl2])
         for si, t in enumerate(sample):
             for j in range(topk):
                 if ids[t, j] == e:
