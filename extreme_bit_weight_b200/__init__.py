@@ -73,6 +73,8 @@ _lib.ccq_moe_w2a16_forward.argtypes = [ctypes.POINTER(ccq_weight), ctypes.POINTE
 _lib.ccq_moe_w2a16_forward_traced.argtypes = [ctypes.POINTER(ccq_weight), ctypes.POINTER(ccq_weight), _I, _P, _I,
                                               _P, _P, _I, _P, _P, ctypes.c_size_t, _P, _P]
 _lib.ccq_check_device_error.argtypes = [_P, _P]
+_lib.ccq_w2a16_gemm_noalloc.argtypes = [ctypes.POINTER(ccq_weight), _P, _I, _P, _P]
+_lib.ccq_w2a16_gemm_noalloc_max_scratch.restype = ctypes.c_size_t
 CCQ_MOE_TRACE_POINTS = 7
 
 
@@ -201,6 +203,20 @@ def ccq_w2a16_gemm(w: CcqWeight, x: torch.Tensor, y: torch.Tensor = None, ws: to
     _check(_lib.ccq_w2a16_gemm(ctypes.byref(s), _dptr(x), m, _dptr(y), _dptr(ws), ws.numel(), _stream(stream)),
            "ccq_w2a16_gemm")
     return y
+
+
+def ccq_w2a16_gemm_noalloc(w: CcqWeight, x: torch.Tensor, y: torch.Tensor, stream=None) -> torch.Tensor:
+    """y = x W^T without a caller workspace: for code that cannot allocate device memory, the
+    library uses its own fixed per-device scratch array (see ccq_w2a16_gemm_noalloc in ccq.h).
+    `y` must be supplied by the caller; nothing here allocates."""
+    s = w.struct()
+    _check(_lib.ccq_w2a16_gemm_noalloc(ctypes.byref(s), _dptr(x), x.shape[0], _dptr(y), _stream(stream)),
+           "ccq_w2a16_gemm_noalloc")
+    return y
+
+
+def ccq_w2a16_gemm_noalloc_max_scratch() -> int:
+    return int(_lib.ccq_w2a16_gemm_noalloc_max_scratch())
 
 
 def ccq_moe_workspace_size(T: int, topk: int, H: int, I: int, num_experts: int) -> int:

@@ -129,6 +129,25 @@ size_t ccq_gemm_workspace_size(const ccq_weight *w, int32_t m);
 ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, void *y_bf16, void *ws,
                           size_t ws_bytes, ccq_stream_t stream);
 
+/* ccq_w2a16_gemm_noalloc - ccq_w2a16_gemm for callers that cannot allocate device memory.
+ * No counterpart in the paper: it exists for host code that is handed only input and output
+ * pointers (e.g. a plugin whose host framework owns and pre-plans all device memory) or that must
+ * not call cudaMalloc/cudaFree (which can synchronize the device) on its critical path.  It
+ * computes the same result as ccq_w2a16_gemm with the same arguments, but takes its scratch from
+ * a fixed array inside the library (ccq_w2a16_gemm_noalloc_max_scratch() bytes per device, held
+ * by every GPU that loads the library until the process exits) and calls no allocator.
+ *   - Shapes whose workspace (ccq_gemm_workspace_size) exceeds that size return
+ *     CCQ_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on each device looks up the array's device address (with that device
+ *     current) and caches it; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents (every byte a call
+ *     reads it writes first).  Calls that may overlap on the GPU (different streams, or several
+ *     threads) race on it: serialize them. */
+ccq_status ccq_w2a16_gemm_noalloc(const ccq_weight *w, const void *x_bf16, int32_t m, void *y_bf16,
+                                  ccq_stream_t stream);
+/* ccq_w2a16_gemm_noalloc_max_scratch - bytes of the fixed scratch array (per device). */
+size_t ccq_w2a16_gemm_noalloc_max_scratch(void);
+
 /* ccq_moe_workspace_size - workspace bytes of ccq_moe_w2a16_forward for these sizes. */
 size_t ccq_moe_workspace_size(int32_t T, int32_t topk, int32_t H, int32_t I, int32_t num_experts);
 
