@@ -61,7 +61,7 @@ __global__ void dequant_w4_kernel(const uint8_t *__restrict__ codes, const float
 // ------------------------------------------------------------------------------------------------
 // Activation operand packing.  One thread per (operand row p, 64-column group G): reads the
 // group's 64 BF16 values of source row tok_of[p] (or p), writes them in the XA order and the
-// group sum -160 * sum (fp32, summed in column order).
+// group sum (fp32, summed in column order).
 // ------------------------------------------------------------------------------------------------
 __global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__restrict__ tok_of, int P_valid,
                                int P, int K, uint16_t *__restrict__ xa, float *__restrict__ gsum) {
@@ -86,7 +86,9 @@ __global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__rest
         float sum = 0.0f;
 #pragma unroll
         for (int k = 0; k < 64; ++k) sum += bf16_bits_to_float(v[k]);
-        gsum[(size_t)pr * ld + G] = -160.0f * sum;
+        gsum[(size_t)pr * ld + G] = sum;
+        if (G == ng - 1)  // the row's padding groups read as zero activations
+            for (int Gp = ng; Gp < ld; ++Gp) gsum[(size_t)pr * ld + Gp] = 0.0f;
         // 16 runs of 4 values: (i, tig) -> j = 0..3 contiguous
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -110,7 +112,9 @@ __global__ void gsum_from_xa_kernel(const uint16_t *__restrict__ xa, int P_valid
         float sum = 0.0f;
         for (int k = 0; k < 64; ++k)
             sum += bf16_bits_to_float(xa[xa_index((size_t)pr, (size_t)G * 64 + k, (size_t)P)]);
-        gsum[(size_t)pr * ld + G] = -160.0f * sum;
+        gsum[(size_t)pr * ld + G] = sum;
+        if (G == ng - 1)
+            for (int Gp = ng; Gp < ld; ++Gp) gsum[(size_t)pr * ld + Gp] = 0.0f;
     }
 }
 

@@ -62,9 +62,9 @@ ccq_status check_weight(const ccq_weight *w, int experts) {
 }
 
 // --- decode-sized path ----------------------------------------------------------------------
-int pick_nt(double rows_per_expert) {
+int pick_nt(double rows_per_expert, int fmt = CCQ_FMT_W2_CCQ_G64) {
     if (rows_per_expert <= 8.0) return 1;
-    if (rows_per_expert <= 16.0) return 2;
+    if (rows_per_expert <= 16.0 || fmt == CCQ_FMT_W4_PER_CHANNEL) return 2;  // W4 code tiles are twice as wide
     return 4;
 }
 
@@ -76,10 +76,12 @@ struct DecodeMaps {
 bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t *xa, const float *gs, int P,
                  int nt) {
     const int K = w->k;
+    const bool w4 = w->fmt == CCQ_FMT_W4_PER_CHANNEL;
     const cuuint64_t rows = (cuuint64_t)experts * w->n;
+    const cuuint64_t row_bytes = (cuuint64_t)(w4 ? K / 2 : K / 4);
     {
-        cuuint64_t dims[2] = {(cuuint64_t)(K / 4), rows};
-        cuuint64_t str[1] = {(cuuint64_t)(K / 4)};
+        cuuint64_t dims[2] = {row_bytes, rows};
+        cuuint64_t str[1] = {row_bytes};
         cuuint32_t box[2] = {128, 128};
         if (!make_map(&m.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w->codes, dims, str, box,
                       CU_TENSOR_MAP_SWIZZLE_128B))
@@ -101,7 +103,7 @@ bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t
             return false;
     }
     // group scales [rows][K/64] fp32: staged by TMA when the row pitch is a multiple of 16 bytes
-    m.tma_scales = (K / 64) % 4 == 0;
+    m.tma_scales = !w4 && (K / 64) % 4 == 0;
     if (m.tma_scales) {
         cuuint64_t dims[2] = {(cuuint64_t)(K / 64), rows};
         cuuint64_t str[1] = {(cuuint64_t)(K / 64) * 4};
@@ -135,7 +137,7 @@ GemmWs gemm_layout(const ccq_weight *w, int m) {
         return L;
     }
     L.P = (m + 3) & ~3;
-    L.nt = pick_nt((double)m);
+    L.nt = pick_nt((double)m, w->fmt);
     const int K = w->k, N = w->n;
     const int nst = ceil_div(K, 512);
     L.row_blocks = ceil_div(N, 256);
@@ -196,8 +198,9 @@ bool tc_maps(CUtensorMap &ta, CUtensorMap &tcodes, const ccq_weight *w, int expe
             return false;
     }
     {
-        cuuint64_t dims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)experts * w->n};
-        cuuint64_t str[1] = {(cuuint64_t)(K / 4)};
+        const cuuint64_t row_bytes = (cuuint64_t)(w->fmt == CCQ_FMT_W4_PER_CHANNEL ? K / 2 : K / 4);
+        cuuint64_t dims[2] = {row_bytes, (cuuint64_t)experts * w->n};
+        cuuint64_t str[1] = {row_bytes};
         cuuint32_t box[2] = {64, 128};
         if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w->codes, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
             return false;
@@ -263,7 +266,6 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
     if (m < 0) return CCQ_ERR_INVALID_ARG;
     if (m == 0) return CCQ_OK;
     if (!x_bf16 || !y_bf16 || !aligned16(x_bf16) || !aligned16(y_bf16)) return CCQ_ERR_INVALID_ARG;
-    if (w->fmt != CCQ_FMT_W2_CCQ_G64) return CCQ_ERR_UNSUPPORTED;
     const GemmWs L = gemm_layout(w, m);
     if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return CCQ_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
@@ -289,6 +291,7 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
         p.mode = EPI_BF16;
         p.out = y_bf16;
         p.out_ld = w->n;
+        p.w4 = w->fmt == CCQ_FMT_W4_PER_CHANNEL;
         const int grid = std::min(sm_count(), p.static_tiles * p.n_tiles);
         return cuda_status(launch_tc_gemm_w2(p, ta, tcodes, kTcMT, grid, s));
     }
@@ -322,6 +325,7 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
         p.out = y_bf16;
     }
     p.tma_scales = maps.tma_scales;
+    p.w4 = w->fmt == CCQ_FMT_W4_PER_CHANNEL;
     e = launch_decode_gemm_w2(p, maps.codes, maps.xa, maps.gs, maps.sc, L.row_blocks, L.ksplit, 1, L.nt, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     if (L.ksplit > 1) {
@@ -360,7 +364,6 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     if (!x_bf16 || !y_bf16 || !expert_ids || !routing_w || !aligned16(x_bf16) || !aligned16(y_bf16))
         return CCQ_ERR_INVALID_ARG;
     if (x_bf16 == y_bf16) return CCQ_ERR_INVALID_ARG;
-    if (w13->fmt != CCQ_FMT_W2_CCQ_G64 || w2->fmt != CCQ_FMT_W2_CCQ_G64) return CCQ_ERR_UNSUPPORTED;
     const MoeWs L = moe_layout(T, topk, H, I, num_experts);
     if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return CCQ_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
@@ -415,6 +418,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q1.out_ld = I;
         q1.I = I;
         q1.err = err;
+        q1.w4 = w13->fmt == CCQ_FMT_W4_PER_CHANNEL;
         e = launch_tc_gemm_w2(q1, ta1, tc1, kTcMT, std::min(sm_count(), L.max_tiles * q1.n_tiles), s);
         if (e == cudaSuccess) e = trace(events, 3, s);
         if (e == cudaSuccess) e = trace(events, 4, s);
@@ -432,6 +436,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q2.out_ld = H;
         q2.rw = rwp;
         q2.I = 0;
+        q2.w4 = w2->fmt == CCQ_FMT_W4_PER_CHANNEL;
         if (e == cudaSuccess) e = launch_tc_gemm_w2(q2, ta2, tc2, kTcMT, std::min(sm_count(), L.max_tiles * q2.n_tiles), s);
         if (e == cudaSuccess) e = trace(events, 5, s);
         if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
@@ -441,11 +446,12 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), tok, pairs, L.P, H, xa_x, gs_x, s);
     if (e == cudaSuccess) e = trace(events, 2, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
-    const int nt = pick_nt((double)pairs / num_experts);
+    const int nt1 = pick_nt((double)pairs / num_experts, w13->fmt);
+    const int nt2 = pick_nt((double)pairs / num_experts, w2->fmt);
 
     // gate/up projection with the SiLU gate fused in its epilogue -> h (activation operand layout)
     DecodeMaps m1;
-    if (!decode_maps(m1, w13, num_experts, xa_x, gs_x, L.P, nt)) return CCQ_ERR_CUDA;
+    if (!decode_maps(m1, w13, num_experts, xa_x, gs_x, L.P, nt1)) return CCQ_ERR_CUDA;
     DecodeGemmParams p1{};
     p1.scales = w13->scales;
     p1.alpha = w13->alpha;
@@ -464,7 +470,8 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p1.I = I;
     p1.err = err;
     p1.tma_scales = m1.tma_scales;
-    e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), 1, num_experts, nt, s);
+    p1.w4 = w13->fmt == CCQ_FMT_W4_PER_CHANNEL;
+    e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), 1, num_experts, nt1, s);
     if (e == cudaSuccess) e = trace(events, 3, s);
     if (e == cudaSuccess) e = launch_gsum_from_xa(xa_h, pairs, L.P, I, gs_h, s);
     if (e == cudaSuccess) e = trace(events, 4, s);
@@ -472,7 +479,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
 
     // down projection, scaled by each pair's routing weight -> fp32 slots
     DecodeMaps m2;
-    if (!decode_maps(m2, w2, num_experts, xa_h, gs_h, L.P, nt)) return CCQ_ERR_CUDA;
+    if (!decode_maps(m2, w2, num_experts, xa_h, gs_h, L.P, nt2)) return CCQ_ERR_CUDA;
     DecodeGemmParams p2{};
     p2.scales = w2->scales;
     p2.alpha = w2->alpha;
@@ -491,7 +498,8 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p2.rw = rwp;
     p2.err = err;
     p2.tma_scales = m2.tma_scales;
-    e = launch_decode_gemm_w2(p2, m2.codes, m2.xa, m2.gs, m2.sc, ceil_div(H, 256), 1, num_experts, nt, s);
+    p2.w4 = w2->fmt == CCQ_FMT_W4_PER_CHANNEL;
+    e = launch_decode_gemm_w2(p2, m2.codes, m2.xa, m2.gs, m2.sc, ceil_div(H, 256), 1, num_experts, nt2, s);
     if (e == cudaSuccess) e = trace(events, 5, s);
     if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
     if (e == cudaSuccess) e = trace(events, 6, s);

@@ -39,19 +39,21 @@ constexpr int kConsumerWarps = 2 * kRowWarps;       // two warps per row slot: g
 constexpr int kThreads = kConsumerWarps * 32;       // lane 0 of warp 0 also issues the TMA loads
 constexpr int kCodeTileBytes = 128 * 128;  // [128 rows][128 B] = 8 groups of 16 bytes
 
-template <int NT>
+template <int NT, bool W4 = false>
 struct Smem {
     static constexpr int MP = 8 * NT;
-    static constexpr int kStages = NT == 1 ? 4 : (NT == 2 ? 3 : 2);  // ring depth within 227 KB
-    static constexpr int kCtasPerSm = 1;
-    static constexpr int kRedBytes = kRowWarps * 32 * 2 * NT * 4 * 4;  // partial sums of the second warp half
+    static constexpr int kCodeBytes = (W4 ? 2 : 1) * 2 * kCodeTileBytes;  // both halves, one stage
     static constexpr int kXaBytes = 32 * MP * 16 * 2;  // [G*4+i = 32][MP][16] bf16
     static constexpr int kGsBytes = MP * 8 * 4;        // [MP][8] fp32
-    static constexpr int kScBytes = 2 * 128 * 8 * 4;   // [2 halves][128 rows][8 groups] fp32 scales
-    static constexpr int kStageBytes = ((2 * kCodeTileBytes + kXaBytes + kGsBytes + kScBytes) + 1023) & ~1023;
+    static constexpr int kScBytes = W4 ? 0 : 2 * 128 * 8 * 4;  // [2 halves][128 rows][8 groups] fp32 scales
+    static constexpr int kStageBytes = ((kCodeBytes + kXaBytes + kGsBytes + kScBytes) + 1023) & ~1023;
+    static constexpr int kRedBytes = kRowWarps * 32 * 2 * NT * 4 * 4;  // partial sums of the second warp half
+    static constexpr int kStages = ((227 * 1024 - 2048 - kRedBytes) / kStageBytes) < 4
+                                       ? ((227 * 1024 - 2048 - kRedBytes) / kStageBytes) : 4;  // ring depth
     static constexpr int kTotal = kStages * kStageBytes + kRedBytes + 1024;  // + alignment slack
     static_assert(kTotal + 64 <= 227 * 1024, "shared memory per CTA");
-    static constexpr uint32_t kTxBytes = 2 * kCodeTileBytes + kXaBytes + kGsBytes;  // + kScBytes with TMA scales
+    static constexpr uint32_t kTxBytes = kCodeBytes + kXaBytes + kGsBytes;  // + kScBytes with TMA scales
+    static_assert(kStages >= 2, "ring depth");
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -134,6 +136,16 @@ __device__ __forceinline__ void decode_word(uint32_t w, const RowDecode &rd, con
     R[7] = and_or(X23, k.wmask, k.wexp);
 }
 
+// W4: one 32-bit word = 8 signed 4-bit codes (first of a pair in the low nibble).  Register i holds
+// codes i and i+4 as BF16 (128 + (q + 8)) -- the sign bit of each nibble flipped, OR-ed into the
+// exponent pattern of 128 -- so one shift and one three-input logic op per register.
+__device__ __forceinline__ void decode_word_w4(uint32_t w, uint32_t m4, uint32_t x4, uint32_t R[4]) {
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[0]) : "r"(w), "r"(m4), "r"(x4));
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[1]) : "r"(w >> 4), "r"(m4), "r"(x4));
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[2]) : "r"(w >> 8), "r"(m4), "r"(x4));
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[3]) : "r"(w >> 12), "r"(m4), "r"(x4));
+}
+
 __device__ __forceinline__ void mma_bf16(float *c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -161,25 +173,58 @@ __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z));
 // One 64-column group of one stage for this thread: 4 code words (rows g, g+8 of both halves),
 // decode, 4 x NT x 2 mma, per-group rescale.  All shared-memory offsets are compile-time
 // constants once G is unrolled.
-template <int NT>
+template <int NT, bool W4>
 __device__ __forceinline__ void group_step(const int G, const uint8_t *codes, uint32_t cbase, uint32_t cswz,
                                            const uint8_t *xa, const uint8_t *gsb, const float sc[4],
                                            const RowDecode rd[4], const DecodeConsts &kc, float (&acc)[2][NT][4]) {
     constexpr int MP = 8 * NT;
-    const uint32_t coff = cbase + (((uint32_t)G << 4) ^ cswz);
-    const uint32_t w0 = *reinterpret_cast<const uint32_t *>(codes + coff);
-    const uint32_t w1 = *reinterpret_cast<const uint32_t *>(codes + coff + 1024);
-    const uint32_t w2 = *reinterpret_cast<const uint32_t *>(codes + kCodeTileBytes + coff);
-    const uint32_t w3 = *reinterpret_cast<const uint32_t *>(codes + kCodeTileBytes + coff + 1024);
+    // A fragments per state window i: RA0/RA1 = rows g / g+8 of half A, RB0/RB1 of half B;
+    // [2i] and [2i+1] are the k-pairs (j=0,1) and (j=2,3) of the window
     uint32_t RA0[8], RA1[8], RB0[8], RB1[8];
-    decode_word(w0, rd[0], kc, RA0);
-    decode_word(w1, rd[1], kc, RA1);
-    decode_word(w2, rd[2], kc, RB0);
-    decode_word(w3, rd[3], kc, RB1);
+    if constexpr (!W4) {
+        const uint32_t coff = cbase + (((uint32_t)G << 4) ^ cswz);
+        const uint32_t w0 = *reinterpret_cast<const uint32_t *>(codes + coff);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(codes + coff + 1024);
+        const uint32_t w2 = *reinterpret_cast<const uint32_t *>(codes + kCodeTileBytes + coff);
+        const uint32_t w3 = *reinterpret_cast<const uint32_t *>(codes + kCodeTileBytes + coff + 1024);
+        decode_word(w0, rd[0], kc, RA0);
+        decode_word(w1, rd[1], kc, RA1);
+        decode_word(w2, rd[2], kc, RB0);
+        decode_word(w3, rd[3], kc, RB1);
+    } else {
+        // 32 bytes per row and group: this thread's 8 bytes sit in 16-byte chunk 2(G%4) + tig/2 of
+        // the 128-byte line (box G/4); cbase holds 8*(tig&1) and the row offset, cswz the row swizzle
+        const int box = (G >> 2) * (2 * kCodeTileBytes);
+        const uint32_t coff = cbase + ((((uint32_t)(2 * (G & 3))) << 4) ^ cswz);
+        const uint2 q0 = *reinterpret_cast<const uint2 *>(codes + box + coff);
+        const uint2 q1 = *reinterpret_cast<const uint2 *>(codes + box + coff + 1024);
+        const uint2 q2 = *reinterpret_cast<const uint2 *>(codes + box + kCodeTileBytes + coff);
+        const uint2 q3 = *reinterpret_cast<const uint2 *>(codes + box + kCodeTileBytes + coff + 1024);
+        uint32_t t[4];
+        decode_word_w4(q0.x, kc.wmask, kc.wexp, t);
+        RA0[0] = t[0]; RA0[2] = t[1]; RA0[4] = t[2]; RA0[6] = t[3];
+        decode_word_w4(q0.y, kc.wmask, kc.wexp, t);
+        RA0[1] = t[0]; RA0[3] = t[1]; RA0[5] = t[2]; RA0[7] = t[3];
+        decode_word_w4(q1.x, kc.wmask, kc.wexp, t);
+        RA1[0] = t[0]; RA1[2] = t[1]; RA1[4] = t[2]; RA1[6] = t[3];
+        decode_word_w4(q1.y, kc.wmask, kc.wexp, t);
+        RA1[1] = t[0]; RA1[3] = t[1]; RA1[5] = t[2]; RA1[7] = t[3];
+        decode_word_w4(q2.x, kc.wmask, kc.wexp, t);
+        RB0[0] = t[0]; RB0[2] = t[1]; RB0[4] = t[2]; RB0[6] = t[3];
+        decode_word_w4(q2.y, kc.wmask, kc.wexp, t);
+        RB0[1] = t[0]; RB0[3] = t[1]; RB0[5] = t[2]; RB0[7] = t[3];
+        decode_word_w4(q3.x, kc.wmask, kc.wexp, t);
+        RB1[0] = t[0]; RB1[2] = t[1]; RB1[4] = t[2]; RB1[6] = t[3];
+        decode_word_w4(q3.y, kc.wmask, kc.wexp, t);
+        RB1[1] = t[0]; RB1[3] = t[1]; RB1[5] = t[2]; RB1[7] = t[3];
+    }
+    // group sums of the activations times the format's level offset (160 for W2, 136 for W4)
+    const float off = W4 ? -136.0f : -160.0f;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-        const float gs0 = *reinterpret_cast<const float *>(gsb + n * 256 + G * 4);
-        const float gs1 = *reinterpret_cast<const float *>(gsb + n * 256 + 32 + G * 4);
+        // the group's starting value: the activation sum times the level offset
+        const float gs0 = off * *reinterpret_cast<const float *>(gsb + n * 256 + G * 4);
+        const float gs1 = off * *reinterpret_cast<const float *>(gsb + n * 256 + 32 + G * 4);
         float cA[4], cB[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -203,14 +248,18 @@ __device__ __forceinline__ void group_step(const int G, const uint8_t *codes, ui
     }
 }
 
-template <int NT, bool TMA_SC>
-__global__ void __launch_bounds__(kThreads, Smem<NT>::kCtasPerSm)
+template <int NT, bool TMA_SC, bool W4>
+__global__ void __launch_bounds__(kThreads, 1)
 decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_xa,
                       const __grid_constant__ CUtensorMap tm_gs, const __grid_constant__ CUtensorMap tm_sc,
                       const DecodeGemmParams p) {
-    using S = Smem<NT>;
+    using S = Smem<NT, W4>;
     constexpr int MP = S::MP;
     constexpr int kStages = S::kStages;
+    constexpr int kCodeOff = 0;                       // code tiles of the stage
+    constexpr int kXaOff = S::kCodeBytes;             // activation operand slice
+    constexpr int kGsOff = S::kCodeBytes + S::kXaBytes;
+    constexpr int kScOff = kGsOff + S::kGsBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full_bar[kStages], empty_bar[kStages], red_full, red_empty;
@@ -253,16 +302,21 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
         const int slot = it % kStages;
         const int c = it / nst, st = s_begin + it % nst;
         uint8_t *base = smem + slot * S::kStageBytes;
-        mbar_arrive_expect_tx(&full_bar[slot], S::kTxBytes + (TMA_SC ? S::kScBytes : 0));
-        if (TMA_SC) {
-            uint8_t *sc = base + 2 * kCodeTileBytes + S::kXaBytes + S::kGsBytes;
+        mbar_arrive_expect_tx(&full_bar[slot], S::kTxBytes + ((TMA_SC && !W4) ? S::kScBytes : 0));
+        if (TMA_SC && !W4) {
+            uint8_t *sc = base + kScOff;
             tma_load_2d(sc, &tm_sc, &full_bar[slot], st * 8, rowA);
             tma_load_2d(sc + S::kScBytes / 2, &tm_sc, &full_bar[slot], st * 8, rowB);
         }
-        tma_load_2d(base, &tm_codes, &full_bar[slot], st * 128, rowA);
-        tma_load_2d(base + kCodeTileBytes, &tm_codes, &full_bar[slot], st * 128, rowB);
-        tma_load_3d(base + 2 * kCodeTileBytes, &tm_xa, &full_bar[slot], 0, seg0 + c * MP, st * 32);
-        tma_load_2d(base + 2 * kCodeTileBytes + S::kXaBytes, &tm_gs, &full_bar[slot], st * 8, seg0 + c * MP);
+        // W2: 128 code bytes per row per stage; W4: 256, as two 128-byte boxes
+#pragma unroll
+        for (int bx = 0; bx < (W4 ? 2 : 1); ++bx) {
+            const int x = st * (W4 ? 256 : 128) + bx * 128;
+            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes, &tm_codes, &full_bar[slot], x, rowA);
+            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes + kCodeTileBytes, &tm_codes, &full_bar[slot], x, rowB);
+        }
+        tma_load_3d(base + kXaOff, &tm_xa, &full_bar[slot], 0, seg0 + c * MP, st * 32);
+        tma_load_2d(base + kGsOff, &tm_gs, &full_bar[slot], st * 8, seg0 + c * MP);
     };
     if (producer)
         for (int it = 0; it < min(kStages - 1, total_iters); ++it) issue(it);
@@ -276,21 +330,28 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
     int lrow[4] = {localA + wrow + g, localA + wrow + g + 8, localB + wrow + g, localB + wrow + g + 8};
     RowDecode rd[4];
     bool rvalid[4];
+    float sc_row[4];  // W4: per-channel scales, bf16-rounded
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         rvalid[r] = lrow[r] < p.N;
         const int grow = e * p.N + (rvalid[r] ? lrow[r] : 0);
-        const float a = __ldg(p.alpha + grow), b = __ldg(p.beta + grow);
-        rd[r].ab = f2_pack(a, a);
-        rd[r].bb = f2_pack(b, b);
+        if constexpr (!W4) {
+            const float a = __ldg(p.alpha + grow), b = __ldg(p.beta + grow);
+            rd[r].ab = f2_pack(a, a);
+            rd[r].bb = f2_pack(b, b);
+            sc_row[r] = 0.0f;
+        } else {
+            rd[r].ab = rd[r].bb = 0;
+            sc_row[r] = round_bf16(__ldg(p.scales + grow));
+        }
     }
     DecodeConsts kc;
     const uint32_t opaque = (uint32_t)(p.K >> 30);  // == 0; keeps the constants in registers
     kc.neg_magic = f2_pack(-8388608.0f, -8388608.0f);
     kc.round_mag = f2_pack(12582912.0f, 12582912.0f - 19264.0f);
     kc.mul16 = 65536u + opaque;
-    kc.wmask = 0x003F003Fu ^ opaque;
-    kc.wexp = 0x43004300u ^ opaque;
+    kc.wmask = (W4 ? 0x000F000Fu : 0x003F003Fu) ^ opaque;  // one state window / one nibble per half
+    kc.wexp = (W4 ? 0x43084308u : 0x43004300u) ^ opaque;   // BF16 128 (W4: and the nibble sign flip)
 
     float acc[2][NT][4];
 #pragma unroll
@@ -301,8 +362,9 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
             for (int q = 0; q < 4; ++q) acc[t][n][q] = 0.0f;
 
     // per-thread shared-memory offsets inside a stage
-    const uint32_t cbase = (uint32_t)(wrow + g) * 128u + 4u * (uint32_t)tig;  // code word of row wrow+g (unswizzled)
-    const uint32_t cswz = (uint32_t)g << 4;         // 128B swizzle of rows wrow+g and wrow+g+8
+    const uint32_t cbase = (uint32_t)(wrow + g) * 128u +
+                           (W4 ? 8u * ((uint32_t)tig & 1u) : 4u * (uint32_t)tig);  // code word of row wrow+g
+    const uint32_t cswz = ((uint32_t)g << 4) ^ (W4 ? (((uint32_t)tig >> 1) << 4) : 0u);  // 128B swizzle (+ W4 chunk)
     const uint32_t xa_thr = (uint32_t)g * 32u + (uint32_t)tig * 8u;  // B fragment of token g, lane tig
     const uint32_t gs_thr = (uint32_t)(2 * tig) * 32u;               // group sums of token 2*tig
     const uint32_t sc_thr = (uint32_t)(wrow + g) * 32u;              // scales of row wrow+g
@@ -324,11 +386,17 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
         }
         consumed = it + 1;
         const uint8_t *base = smem + slot * S::kStageBytes;
-        const uint8_t *xa = base + 2 * kCodeTileBytes + xa_thr;
-        const uint8_t *gsb = base + 2 * kCodeTileBytes + S::kXaBytes + gs_thr;
-        if (TMA_SC) {
+        const uint8_t *xa = base + kXaOff + xa_thr;
+        const uint8_t *gsb = base + kGsOff + gs_thr;
+        if (W4) {
+            // per-channel scales; groups beyond K read TMA zero fill (activations 0) and add nothing
+            const int Gh = 4 * khalf;
+#pragma unroll
+            for (int G = 0; G < 4; ++G)
+                group_step<NT, W4>(Gh + G, base, cbase, cswz, xa, gsb, sc_row, rd, kc, acc);
+        } else if (TMA_SC) {
             // full stage: groups beyond K read TMA zero fill (scale 0, activations 0) and add nothing
-            const uint8_t *scb = base + 2 * kCodeTileBytes + S::kXaBytes + S::kGsBytes + sc_thr;
+            const uint8_t *scb = base + kScOff + sc_thr;
             {
                 // this warp's four groups of the stage: offsets are immediates
                 const int Gh = 4 * khalf;
@@ -343,7 +411,7 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
                     sc[1] = round_bf16(*reinterpret_cast<const float *>(sch + 256 + G * 4));
                     sc[2] = round_bf16(*reinterpret_cast<const float *>(sch + 4096 + G * 4));
                     sc[3] = round_bf16(*reinterpret_cast<const float *>(sch + 4096 + 256 + G * 4));
-                    group_step<NT>(G, base, cbase, cswz_h, xah, gsh, sc, rd, kc, acc);
+                    group_step<NT, W4>(G, base, cbase, cswz_h, xah, gsh, sc, rd, kc, acc);
                 }
             }
         } else {
@@ -357,7 +425,7 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
                     const int grow = e * p.N + (rvalid[r] ? lrow[r] : 0);
                     sc[r] = round_bf16(__ldg(p.scales + (size_t)grow * ngroups + gg));
                 }
-                group_step<NT>(G, base, cbase, cswz, xa, gsb, sc, rd, kc, acc);
+                group_step<NT, W4>(G, base, cbase, cswz, xa, gsb, sc, rd, kc, acc);
             }
         }
         __syncwarp();
@@ -440,8 +508,19 @@ template <int NT>
 cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUtensorMap &b,
                       const CUtensorMap &c, const CUtensorMap &d, int row_blocks, int ksplit, int experts,
                       cudaStream_t s) {
-    auto kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true> : decode_gemm_w2_kernel<NT, false>;
-    const int smem = Smem<NT>::kTotal;
+    void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, DecodeGemmParams) = nullptr;
+    int smem = 0;
+    if constexpr (NT <= 2) {  // W4 keeps at most 16 tokens per chunk (its code tiles are twice as wide)
+        if (p.w4) {
+            kern = decode_gemm_w2_kernel<NT, false, true>;
+            smem = Smem<NT, true>::kTotal;
+        }
+    }
+    if (!p.w4) {
+        kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false> : decode_gemm_w2_kernel<NT, false, false>;
+        smem = Smem<NT, false>::kTotal;
+    }
+    if (!kern) return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     dim3 grid(row_blocks, ksplit, experts);
@@ -454,6 +533,7 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
 cudaError_t launch_decode_gemm_w2(const DecodeGemmParams &p, const CUtensorMap &tm_codes,
                                   const CUtensorMap &tm_xa, const CUtensorMap &tm_gs, const CUtensorMap &tm_sc,
                                   int row_blocks, int ksplit, int experts, int nt, cudaStream_t s) {
+    if (p.w4 && nt > 2) return cudaErrorInvalidValue;  // W4 tiles hold at most 16 tokens per chunk
     switch (nt) {
         case 1: return launch_nt<1>(p, tm_codes, tm_xa, tm_gs, tm_sc, row_blocks, ksplit, experts, s);
         case 2: return launch_nt<2>(p, tm_codes, tm_xa, tm_gs, tm_sc, row_blocks, ksplit, experts, s);

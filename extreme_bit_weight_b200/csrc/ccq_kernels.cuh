@@ -19,7 +19,7 @@ enum EpiMode : int {
 // sits at  ((((G*4 + i)*P + p)*4 + tig)*4 + j).  Rows of one 16-column block are thus grouped by
 // the state window i they meet in the decoded weights, which makes every mma B fragment one
 // contiguous, bank-conflict-free 8-byte shared-memory read.  Alongside it, gsum[p][G] holds
-// -160 * sum_{k in group G} x[p][k] (fp32, row pitch gsum_ld = round_up(K/64, 4)).
+// sum_{k in group G} x[p][k] (fp32, summed in column order; row pitch gsum_ld = round_up(K/64, 4)).
 __host__ __device__ inline size_t xa_index(size_t p, size_t k, size_t P) {
     size_t G = k >> 6, r = k & 63, tig = r >> 4, j = (r >> 2) & 3, i = r & 3;
     return ((((G * 4 + i) * P + p) * 4 + tig) * 4 + j);
@@ -49,6 +49,7 @@ struct DecodeGemmParams {
     int h_P;              // EPI_GATEUP: rows of the H operand (== P)
     int I;                // EPI_GATEUP: gate rows per expert
     int tma_scales;       // 1: scales staged by TMA with the codes (row pitch a multiple of 16 B)
+    int w4;               // 1: W4 per-channel codes (two per byte), scales[row]
     uint32_t *err;
 };
 
@@ -77,6 +78,7 @@ struct TcGemmParams {
     int out_ld;
     const float *rw;       // EPI_DOWN: routing weight per operand row
     int I;                 // EPI_GATEUP: gate rows per expert
+    int w4;                // 1: W4 per-channel codes (two per byte), scales[row]
     uint32_t *err;
 };
 

@@ -132,6 +132,18 @@ __device__ __forceinline__ void decode_word_bf16(uint32_t w, float alpha, float 
     out[7] = bmul2(bsub2((X23 & M) | E, Z), s2);
 }
 
+// W4: one word = 8 signed 4-bit codes (low nibble first).  out[i] = BF16 (q_i * s, q_{i+4} * s):
+// nibble i and i+4 land in the two halves as 128 + (q + 8), minus 136 exactly, times s once.
+__device__ __forceinline__ void decode_word_w4_bf16(uint32_t w, uint32_t s2, uint32_t out[4]) {
+    const uint32_t M4 = 0x000F000Fu, X4 = 0x43084308u, Z = 0x43084308u;  // Z = bf16x2(136, 136)
+    uint32_t r;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(r) : "r"(w >> (4 * i)), "r"(M4), "r"(X4));
+        out[i] = bmul2(bsub2(r, Z), s2);
+    }
+}
+
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
 // position p of a 16-column block holds column 4*(p%4) + p/4 (and the map is its own inverse)
@@ -152,7 +164,7 @@ __device__ __forceinline__ bool tile_of(const TcGemmParams &p, int w, TileInfo &
     return true;
 }
 
-template <int MT>
+template <int MT, bool W4>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_codes,
                   const TcGemmParams p) {
@@ -169,6 +181,8 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int total_work = (p.tile_count ? *p.tile_count : p.static_tiles) * p.n_tiles;
     const int nk = p.K / 64;
+    // one code stage holds 64 bytes of every row: 4 groups of W2 codes or 2 groups of W4 codes
+    constexpr int kKsPerCode = W4 ? 2 : 4;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kSA; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
@@ -201,13 +215,13 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 const int localA = t.nt * p.row_block_stride;
                 const int rowA = t.e * p.N + localA, rowB = rowA + p.half_stride;
                 for (int ks = 0; ks < nk && ok; ++ks) {
-                    if ((ks & 3) == 0) {
+                    if (ks % kKsPerCode == 0) {
                         const int s = ci % kSC;
                         if (ci >= kSC) ok = mbar_wait(&c_empty[s], ((ci / kSC) - 1) & 1, p.err);
                         if (!ok) break;
                         mbar_arrive_expect_tx(&c_full[s], kCTile);
-                        tma_load_2d(sC + s * kCTile, &tm_codes, &c_full[s], (ks >> 2) * 64, rowA);
-                        tma_load_2d(sC + s * kCTile + kCTile / 2, &tm_codes, &c_full[s], (ks >> 2) * 64, rowB);
+                        tma_load_2d(sC + s * kCTile, &tm_codes, &c_full[s], (ks / kKsPerCode) * 64, rowA);
+                        tma_load_2d(sC + s * kCTile + kCTile / 2, &tm_codes, &c_full[s], (ks / kKsPerCode) * 64, rowB);
                         ++ci;
                     }
                     const int s = ai % kSA;
@@ -272,30 +286,53 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             const int local = t.nt * p.row_block_stride + half * p.half_stride + rr;
             const bool valid = local < p.N;
             const size_t grow = (size_t)t.e * p.N + (valid ? local : 0);
-            const float alpha = __ldg(p.alpha + grow), beta = __ldg(p.beta + grow);
-            const float *srow = p.scales + grow * nk;
+            const float alpha = W4 ? 0.0f : __ldg(p.alpha + grow), beta = W4 ? 0.0f : __ldg(p.beta + grow);
+            const float *srow = p.scales + grow * (W4 ? 1 : nk);
+            const float sc_row = W4 ? bf16_bits_to_float(float_to_bf16_bits(__ldg(srow))) : 0.0f;
             for (int ks = 0; ks < nk && ok; ++ks) {
                 const int cs = ci % kSC;
-                if ((ks & 3) == 0) {
+                if (ks % kKsPerCode == 0) {
                     ok = mbar_wait(&c_full[cs], (ci / kSC) & 1, p.err);
                     if (!ok) break;
                 }
-                // this row's 16 code bytes of group ks (64-byte rows, 64B swizzle)
+                // this row's code bytes of group ks (64-byte rows, 64B swizzle): 16 (W2) or 32 (W4)
                 const uint8_t *crow = sC + cs * kCTile + half * (kCTile / 2) + rr * 64;
-                const uint32_t chunk = (uint32_t)(ks & 3) ^ (((uint32_t)rr >> 1) & 3u);
-                const uint4 q = *reinterpret_cast<const uint4 *>(crow + (chunk << 4));
-                if ((ks & 3) == 3 || ks == nk - 1) {
+                const uint32_t swz = ((uint32_t)rr >> 1) & 3u;
+                uint4 q, q2 = make_uint4(0, 0, 0, 0);
+                if (!W4) {
+                    q = *reinterpret_cast<const uint4 *>(crow + ((((uint32_t)(ks & 3)) ^ swz) << 4));
+                } else {
+                    const uint32_t c0 = 2u * (uint32_t)(ks & 1);
+                    q = *reinterpret_cast<const uint4 *>(crow + ((c0 ^ swz) << 4));
+                    q2 = *reinterpret_cast<const uint4 *>(crow + (((c0 + 1u) ^ swz) << 4));
+                }
+                if (ks % kKsPerCode == kKsPerCode - 1 || ks == nk - 1) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&c_empty[cs]);
                     ++ci;
                 }
-                const float sc = bf16_bits_to_float(float_to_bf16_bits(__ldg(srow + ks)));
-                const uint32_t s2 = pack_bf16x2(sc, sc);
                 uint32_t o[4][8];
-                decode_word_bf16(q.x, alpha, beta, s2, o[0]);
-                decode_word_bf16(q.y, alpha, beta, s2, o[1]);
-                decode_word_bf16(q.z, alpha, beta, s2, o[2]);
-                decode_word_bf16(q.w, alpha, beta, s2, o[3]);
+                if (!W4) {
+                    const float sc = bf16_bits_to_float(float_to_bf16_bits(__ldg(srow + ks)));
+                    const uint32_t s2 = pack_bf16x2(sc, sc);
+                    decode_word_bf16(q.x, alpha, beta, s2, o[0]);
+                    decode_word_bf16(q.y, alpha, beta, s2, o[1]);
+                    decode_word_bf16(q.z, alpha, beta, s2, o[2]);
+                    decode_word_bf16(q.w, alpha, beta, s2, o[3]);
+                } else {
+                    // block b of 16 columns = words 2b, 2b+1; emit the same window-major order as W2:
+                    // positions (4i, 4i+1) <- codes (i, i+4) of word 2b, (4i+2, 4i+3) <- of word 2b+1
+                    const uint32_t s2 = pack_bf16x2(sc_row, sc_row);
+                    const uint32_t wds[8] = {q.x, q.y, q.z, q.w, q2.x, q2.y, q2.z, q2.w};
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        uint32_t r0[4], r1[4];
+                        decode_word_w4_bf16(wds[2 * b], s2, r0);
+                        decode_word_w4_bf16(wds[2 * b + 1], s2, r1);
+                        o[b][0] = r0[0]; o[b][1] = r1[0]; o[b][2] = r0[1]; o[b][3] = r1[1];
+                        o[b][4] = r0[2]; o[b][5] = r1[2]; o[b][6] = r0[3]; o[b][7] = r1[3];
+                    }
+                }
                 const int sb = bi % kSB;
                 if (bi >= kSB) ok = mbar_wait(&b_empty[sb], ((bi / kSB) - 1) & 1, p.err);
                 if (!ok) break;
@@ -450,7 +487,7 @@ __global__ void pack_xt_kernel(const uint16_t *__restrict__ x, const int *__rest
 
 template <int MT>
 cudaError_t launch_tc_mt(const TcGemmParams &p, const CUtensorMap &ta, const CUtensorMap &tc, int grid, cudaStream_t s) {
-    auto kern = tc_gemm_w2_kernel<MT>;
+    auto kern = p.w4 ? tc_gemm_w2_kernel<MT, true> : tc_gemm_w2_kernel<MT, false>;
     const int smem = TcSmem<MT>::kTotal;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;

@@ -119,7 +119,7 @@ size_t ccq_gemm_workspace_size(const ccq_weight *w, int32_t m);
 /* ccq_w2a16_gemm - y[m][n] = x[m][k] * W^T with W decoded on the fly (never stored), fp32
  * accumulation, BF16 output.  The GEMV / small-M shapes of CCQ's "Inference Performance"
  * section (Table 4) and the dense prefill shape.
- *   w      single layer (num_experts = 1)
+ *   w      single layer (num_experts = 1), CCQ_FMT_W2_CCQ_G64 or CCQ_FMT_W4_PER_CHANNEL
  *   x_bf16 (device) BF16 [m][k], 16-byte aligned;  m >= 0 (m == 0 is a no-op)
  *   y_bf16 (device) BF16 [m][n], 16-byte aligned
  *   ws     (device) workspace of ccq_gemm_workspace_size(w, m) bytes (may be NULL if that is 0)

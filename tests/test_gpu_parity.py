@@ -291,3 +291,88 @@ def test_moe_prefill_layer_full_size_sampled(ccq):
                 if ids[t, j] == e:
                     ref[si] += float(rw[t, j]) * oracle.expert_ffn_f64(xb[t:t + 1], d13, d2, round_h=True)[0]
     assert rel_err(y[sample], ref) <= TOL
+
+
+# ----------------------------------------------------------------------------------------------
+# W4 per-channel (the mixed W4/W2 expert stack: WINT2 page's quantization_config)
+# ----------------------------------------------------------------------------------------------
+def w4_weight(ccq, codes, scales, experts=1):
+    n = codes.shape[0] // experts
+    return ccq.CcqWeight(ccq.CCQ_FMT_W4_PER_CHANNEL, n, codes.shape[1] * 2, codes, scales, experts=experts)
+
+
+def test_gemm_w4_one_hot_identity_both_paths(ccq):
+    n, k = 272, 576
+    codes, scales = synth.w4_format_random(n, k, 5000)
+    W = w4_weight(ccq, codes, scales)
+    ref = oracle.bf16_to_f64(oracle.dequant_w4(codes, scales)).T.astype(np.float32)
+    eye = synth.one_hot_rows(k).cuda()
+    for j in range(0, 64, 16):  # register-decode mma.sync kernel
+        y = ccq.ccq_w2a16_gemm(W, eye[j:j + 16].contiguous()).float().cpu().numpy()
+        assert np.array_equal(y, ref[j:j + 16]), j
+    y = ccq.ccq_w2a16_gemm(W, eye).float().cpu().numpy()  # tcgen05 kernel
+    assert np.array_equal(y, ref)
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 256, 512), (9, 272, 576), (16, 1024, 2048), (33, 256, 1024),
+                                   (64, 512, 1024), (300, 272, 576), (1, 8192, 8192)])
+def test_gemm_w4_shapes(ccq, m, n, k):
+    codes, scales = synth.w4_format_random(n, k, 5100 + m + n)
+    W = w4_weight(ccq, codes, scales)
+    x = synth.activations(m, k, 5101 + m)
+    y = ccq.ccq_w2a16_gemm(W, x.cuda()).float().cpu().numpy()
+    ref = oracle.gemm_f64(synth.bf16_bits(x), oracle.dequant_w4(codes, scales))
+    e = rel_err(y, ref)
+    assert e <= TOL
+    assert e <= 4e-3
+
+
+def moe_weights_fmt(ccq, E, H, I, seed, fmt13, fmt2):
+    def make(rows, k, s, fmt):
+        if fmt == 4:
+            c, sc = synth.w4_format_random(rows, k, s)
+            return (ccq.CcqWeight(ccq.CCQ_FMT_W4_PER_CHANNEL, rows // E, k, c, sc, experts=E),
+                    oracle.dequant_w4(c, sc))
+        c, sc, a, b = synth.w2_format_random(rows, k, s)
+        return (ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, rows // E, k, c, sc, a, b, experts=E),
+                oracle.dequant_w2(c, sc, a, b))
+    W13, d13 = make(E * 2 * I, H, seed, fmt13)
+    W2, d2 = make(E * H, I, seed + 1, fmt2)
+    return W13, W2, d13.reshape(E, 2 * I, H), d2.reshape(E, H, I)
+
+
+@pytest.mark.parametrize("fmts", [(4, 2), (2, 4), (4, 4)])
+@pytest.mark.parametrize("T", [6, 300])
+def test_moe_mixed_formats(ccq, fmts, T):
+    E, H, I, topk = 8, 512, 256, 2
+    W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 5200 + T + 10 * fmts[0], *fmts)
+    x = synth.activations(T, H, 5201 + T)
+    ids, rw = synth.routing_uniform(T, E, topk, 5202 + T)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    ref = oracle.moe_f64(synth.bf16_bits(x), d13, d2, ids, rw, round_h=True)
+    assert rel_err(y, ref) <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 8, 64, 300])
+def test_mixed_stack_layer_by_layer(ccq, M):
+    # 8 MoE layers: the first 2 with W4 per-channel experts, the last 6 with CCQ W2 g64 (scaled-down
+    # shapes); fresh uniform routing per layer; x_{l+1} = RMSnorm(MoE_l(x_l)) -- random weights grow
+    # the activations by 10-1000x per layer, so without the norm a model keeps between layers the
+    # stack overflows bf16 by the last layer; every layer checked against the oracle on the GPU's own
+    # input to that layer
+    E, H, I, topk = 8, 512, 256, 4
+    x = synth.activations(M, H, 5300 + M).cuda()
+    for layer in range(8):
+        fmt = 4 if layer < 2 else 2
+        W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 5400 + 100 * layer, fmt, fmt)
+        ids, rw = synth.routing_uniform(M, E, topk, 5500 + 100 * layer + M)
+        ids_t = torch.from_numpy(ids).cuda()
+        rw_t = torch.from_numpy(rw).cuda()
+        ws = ccq.workspace(ccq.ccq_moe_workspace_size(M, topk, H, I, E))
+        y = ccq.ccq_moe_w2a16_forward(W13, W2, x, ids_t, rw_t, ws=ws)
+        assert ccq.ccq_check_device_error(ws) == ccq.CCQ_OK
+        ref = oracle.moe_f64(bits_of(x), d13, d2, ids, rw, round_h=True)
+        assert rel_err(y.float().cpu().numpy(), ref) <= TOL, layer
+        yf = y.float()
+        x = (yf * torch.rsqrt(yf.pow(2).mean(dim=1, keepdim=True) + 1e-12)).to(torch.bfloat16)
