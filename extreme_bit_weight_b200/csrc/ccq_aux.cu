@@ -61,10 +61,31 @@ __global__ void dequant_w4_kernel(const uint8_t *__restrict__ codes, const float
 // ------------------------------------------------------------------------------------------------
 // Activation operand packing.  One thread per (operand row p, 64-column group G): reads the
 // group's 64 BF16 values of source row tok_of[p] (or p), writes them in the XA order and the
-// group sum (fp32, summed in column order).
+// group sum S(p, G) (fp32, summed in column order) into the gsq table.
+//
+// gsq[p][G] = {L*S(p,G), L*S(p+1,G), L*S(p,G), L*S(p+1,G)} (float4, row pitch gsum_ld(K) groups,
+// S = 0 past row P_valid - 1): L is the weight format's level offset, and the float4 is exactly the
+// accumulator start of one mma C fragment (tokens p, p+1 for both of its rows), so the matmul
+// kernel fills it with one 16-byte shared-memory read.  Padding groups [K/64, gsum_ld) are never
+// read (the tensor map stops at K/64).
 // ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void store_gsq(float *gsq, int pr, int G, int ld, int P_valid, float v) {
+    float *mine = gsq + ((size_t)pr * ld + G) * 4;
+    mine[0] = v;
+    mine[2] = v;
+    if (pr + 1 == P_valid) {  // no next row: its half of this entry reads zero
+        mine[1] = 0.0f;
+        mine[3] = 0.0f;
+    }
+    if (pr > 0) {  // the previous row's entry holds this row as its second token
+        float *prev = gsq + ((size_t)(pr - 1) * ld + G) * 4;
+        prev[1] = v;
+        prev[3] = v;
+    }
+}
+
 __global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__restrict__ tok_of, int P_valid,
-                               int P, int K, uint16_t *__restrict__ xa, float *__restrict__ gsum) {
+                               int P, int K, float level, uint16_t *__restrict__ xa, float *__restrict__ gsq) {
     const int ng = K / 64, ld = gsum_ld(K);
     const size_t total = (size_t)P_valid * ng;
     for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
@@ -86,9 +107,7 @@ __global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__rest
         float sum = 0.0f;
 #pragma unroll
         for (int k = 0; k < 64; ++k) sum += bf16_bits_to_float(v[k]);
-        gsum[(size_t)pr * ld + G] = sum;
-        if (G == ng - 1)  // the row's padding groups read as zero activations
-            for (int Gp = ng; Gp < ld; ++Gp) gsum[(size_t)pr * ld + Gp] = 0.0f;
+        store_gsq(gsq, pr, G, ld, P_valid, level * sum);
         // 16 runs of 4 values: (i, tig) -> j = 0..3 contiguous
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -102,8 +121,8 @@ __global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__rest
     }
 }
 
-__global__ void gsum_from_xa_kernel(const uint16_t *__restrict__ xa, int P_valid, int P, int K,
-                                    float *__restrict__ gsum) {
+__global__ void gsum_from_xa_kernel(const uint16_t *__restrict__ xa, int P_valid, int P, int K, float level,
+                                    float *__restrict__ gsq) {
     const int ng = K / 64, ld = gsum_ld(K);
     const size_t total = (size_t)P_valid * ng;
     for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
@@ -112,9 +131,7 @@ __global__ void gsum_from_xa_kernel(const uint16_t *__restrict__ xa, int P_valid
         float sum = 0.0f;
         for (int k = 0; k < 64; ++k)
             sum += bf16_bits_to_float(xa[xa_index((size_t)pr, (size_t)G * 64 + k, (size_t)P)]);
-        gsum[(size_t)pr * ld + G] = sum;
-        if (G == ng - 1)
-            for (int Gp = ng; Gp < ld; ++Gp) gsum[(size_t)pr * ld + Gp] = 0.0f;
+        store_gsq(gsq, pr, G, ld, P_valid, level * sum);
     }
 }
 
@@ -230,16 +247,17 @@ cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, c
     return cudaGetLastError();
 }
 
-cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, uint16_t *xa,
-                           float *gsum, cudaStream_t s) {
+cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,
+                           uint16_t *xa, float *gsq, cudaStream_t s) {
     if (P_valid <= 0) return cudaSuccess;
-    pack_xa_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(x, tok_of, P_valid, P, K, xa, gsum);
+    pack_xa_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(x, tok_of, P_valid, P, K, level, xa, gsq);
     return cudaGetLastError();
 }
 
-cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float *gsum, cudaStream_t s) {
+cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float level, float *gsq,
+                                cudaStream_t s) {
     if (P_valid <= 0) return cudaSuccess;
-    gsum_from_xa_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(xa, P_valid, P, K, gsum);
+    gsum_from_xa_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(xa, P_valid, P, K, level, gsq);
     return cudaGetLastError();
 }
 

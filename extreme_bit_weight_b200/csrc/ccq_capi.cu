@@ -95,10 +95,12 @@ bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t
             return false;
     }
     {
+        // gsq table: [P][gsum_ld(K)] float4 entries; the map stops at K/64 groups so that a stage
+        // running past the last group reads zeros
         const int ld = gsum_ld(K);
-        cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)P};
-        cuuint64_t str[1] = {(cuuint64_t)ld * 4};
-        cuuint32_t box[2] = {8, (cuuint32_t)(8 * nt)};
+        cuuint64_t dims[2] = {(cuuint64_t)(4 * (K / 64)), (cuuint64_t)P};
+        cuuint64_t str[1] = {(cuuint64_t)ld * 16};
+        cuuint32_t box[2] = {32, (cuuint32_t)(8 * nt)};
         if (!make_map(&m.gs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, gs, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return false;
     }
@@ -149,7 +151,7 @@ GemmWs gemm_layout(const ccq_weight *w, int m) {
     L.xa = off;
     off = up256(off + (size_t)L.P * K * 2);
     L.gs = off;
-    off = up256(off + (size_t)L.P * gsum_ld(K) * 4);
+    off = up256(off + (size_t)L.P * gsum_ld(K) * 16);
     L.partial = off;
     if (L.ksplit > 1) off = up256(off + (size_t)L.ksplit * m * N * 4);
     L.total = off;
@@ -178,9 +180,9 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     // activation operand of the first projection and of the second (XA + group sums for the
     // decode-sized kernel, the plain permuted-column layout for the tcgen05 kernel)
     L.xa_x = off; off = up256(off + (size_t)L.P * H * 2);
-    L.gs_x = off; if (!L.tc) off = up256(off + (size_t)L.P * gsum_ld(H) * 4);
+    L.gs_x = off; if (!L.tc) off = up256(off + (size_t)L.P * gsum_ld(H) * 16);
     L.xa_h = off; off = up256(off + (size_t)L.P * I * 2);
-    L.gs_h = off; if (!L.tc) off = up256(off + (size_t)L.P * gsum_ld(I) * 4);
+    L.gs_h = off; if (!L.tc) off = up256(off + (size_t)L.P * gsum_ld(I) * 16);
     L.tiles = off; if (L.tc) off = up256(off + sizeof(int2) * (size_t)L.max_tiles);
     L.tcount = off; if (L.tc) off = up256(off + 16);
     L.slot = off; off = up256(off + (size_t)L.P * H * 4);
@@ -297,7 +299,8 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
     }
     uint16_t *xa = reinterpret_cast<uint16_t *>(base + L.xa);
     float *gs = reinterpret_cast<float *>(base + L.gs);
-    cudaError_t e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), nullptr, m, L.P, w->k, xa, gs, s);
+    cudaError_t e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), nullptr, m, L.P, w->k,
+                                   gsq_level(w->fmt == CCQ_FMT_W4_PER_CHANNEL), xa, gs, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     DecodeMaps maps;
     if (!decode_maps(maps, w, 1, xa, gs, L.P, L.nt)) return CCQ_ERR_CUDA;
@@ -443,7 +446,8 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         if (e == cudaSuccess) e = trace(events, 6, s);
         return cuda_status(e);
     }
-    e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), tok, pairs, L.P, H, xa_x, gs_x, s);
+    e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), tok, pairs, L.P, H,
+                           gsq_level(w13->fmt == CCQ_FMT_W4_PER_CHANNEL), xa_x, gs_x, s);
     if (e == cudaSuccess) e = trace(events, 2, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     const int nt1 = pick_nt((double)pairs / num_experts, w13->fmt);
@@ -473,7 +477,8 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p1.w4 = w13->fmt == CCQ_FMT_W4_PER_CHANNEL;
     e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), 1, num_experts, nt1, s);
     if (e == cudaSuccess) e = trace(events, 3, s);
-    if (e == cudaSuccess) e = launch_gsum_from_xa(xa_h, pairs, L.P, I, gs_h, s);
+    if (e == cudaSuccess)
+        e = launch_gsum_from_xa(xa_h, pairs, L.P, I, gsq_level(w2->fmt == CCQ_FMT_W4_PER_CHANNEL), gs_h, s);
     if (e == cudaSuccess) e = trace(events, 4, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
 

@@ -1,13 +1,18 @@
 // Decode-sized CCQ W2A16 grouped matmul (the GEMV / small-M shapes of the CCQ paper's Table 4 and
 // the small-M grouped GEMM of Table 5), sm_100a.
 //
-// One CTA = one expert x two 128-row halves of its weight x one k range (split-K) x all of the
-// expert's tokens (in chunks of 8*NT).  A producer warp streams, per 512-column stage:
+// Work unit = one expert x two 128-row halves of its weight x one k range (split-K) x all of the
+// expert's tokens (in chunks of 8*NT).  The kernel is persistent: CTA b takes units b,
+// b + gridDim.x, ... and one producer thread streams every 512-column stage of all of them through
+// one shared-memory ring (so the next unit's first stages load while the current unit finishes):
 //   * the two halves' code bytes, [128 rows][128 B] each, by TMA with the 128-byte swizzle;
-//   * the activation operand slice in the XA layout (see ccq_kernels.cuh) and its group sums.
-// Eight consumer warps decode the bytes in registers and feed them straight into
+//   * their group scales, the activation operand slice in the XA layout (see ccq_kernels.cuh)
+//     and its gsq group-sum table;
+//   * with a unit's first stage, the unit's per-row alpha/beta (or W4 channel scales).
+// Sixteen consumer warps decode the bytes in registers and feed them straight into
 // mma.sync.m16n8k16 (BF16 in, fp32 accumulate) as the A operand -- weights on the M side, tokens
-// on the N side -- so no decoded weight is ever written to memory.
+// on the N side -- so no decoded weight is ever written to memory.  The producer warpgroup gives
+// its registers to the consumer warpgroups (setmaxnreg), so the issue work never slows a consumer.
 //
 // Decode (CCQ §3.3 Eq. 1 inverted and §3.5 Algorithm 3, Table 1 row (6,4,3)):
 //   code  C = round_half_even(fma(q, alpha, beta))   fp32 FMA; the rounding is an add of
@@ -28,6 +33,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "ccq_device.cuh"
 #include "ccq_kernels.cuh"
 
@@ -36,7 +43,16 @@ namespace {
 
 constexpr int kRowWarps = 8;                       // warps per 16-row slot set (256 rows per CTA)
 constexpr int kConsumerWarps = 2 * kRowWarps;       // two warps per row slot: groups 0-3 / 4-7 of a stage
-constexpr int kThreads = kConsumerWarps * 32;       // lane 0 of warp 0 also issues the TMA loads
+constexpr int kProducerWarps = 4;                   // one warpgroup; lane 0 of its first warp issues the loads
+constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
+// Register split: the CTA launches with kLaunchRegs per thread (the most 640 threads can have), the
+// producer warpgroup hands registers back and the consumer warpgroups take them.  The split must
+// fit in the launch allocation, or the consumers' increase would wait for registers forever; the
+// launcher also checks that the compiled kernel really launches with kLaunchRegs.
+constexpr int kLaunchRegs = 96, kProducerRegs = 24, kConsumerRegs = 112;
+static_assert(kProducerWarps * 32 * kProducerRegs + kConsumerWarps * 32 * kConsumerRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+static_assert(65536 / kThreads >= kLaunchRegs, "launch registers");
 constexpr int kCodeTileBytes = 128 * 128;  // [128 rows][128 B] = 8 groups of 16 bytes
 
 template <int NT, bool W4 = false>
@@ -44,9 +60,10 @@ struct Smem {
     static constexpr int MP = 8 * NT;
     static constexpr int kCodeBytes = (W4 ? 2 : 1) * 2 * kCodeTileBytes;  // both halves, one stage
     static constexpr int kXaBytes = 32 * MP * 16 * 2;  // [G*4+i = 32][MP][16] bf16
-    static constexpr int kGsBytes = MP * 8 * 4;        // [MP][8] fp32
+    static constexpr int kGsBytes = MP * 8 * 16;       // [MP][8] gsq float4 entries
     static constexpr int kScBytes = W4 ? 0 : 2 * 128 * 8 * 4;  // [2 halves][128 rows][8 groups] fp32 scales
-    static constexpr int kStageBytes = ((kCodeBytes + kXaBytes + kGsBytes + kScBytes) + 1023) & ~1023;
+    static constexpr int kRowsBytes = 2048;  // [4][128] fp32: alpha A, alpha B, beta A, beta B (W4: scales A, B)
+    static constexpr int kStageBytes = ((kCodeBytes + kXaBytes + kGsBytes + kScBytes + kRowsBytes) + 1023) & ~1023;
     static constexpr int kRedBytes = kRowWarps * 32 * 2 * NT * 4 * 4;  // partial sums of the second warp half
     static constexpr int kStages = ((227 * 1024 - 2048 - kRedBytes) / kStageBytes) < 4
                                        ? ((227 * 1024 - 2048 - kRedBytes) / kStageBytes) : 4;  // ring depth
@@ -146,6 +163,23 @@ __device__ __forceinline__ void decode_word_w4(uint32_t w, uint32_t m4, uint32_t
     asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[3]) : "r"(w >> 12), "r"(m4), "r"(x4));
 }
 
+// shared-memory reads through 32-bit shared-window addresses
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float4 lds128f(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+    return v;
+}
+
 __device__ __forceinline__ void mma_bf16(float *c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -155,14 +189,14 @@ __device__ __forceinline__ void mma_bf16(float *c, uint32_t a0, uint32_t a1, uin
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// d = a*b + c with c given separately (the group's starting value)
-__device__ __forceinline__ void mma_bf16_c(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                           uint32_t b1, float c0, float c1) {
+// d = a*b + q: q is the group's starting value, read as one float4 from the gsq table
+__device__ __forceinline__ void mma_bf16_q(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                           uint32_t b1, const float4 &q) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%11,%10,%11};"
+        "{%10,%11,%12,%13};"
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(q.x), "f"(q.y), "f"(q.z), "f"(q.w));
 }
 
 // fp32 value of bf16_rn(x): one conversion, the BF16 bits land in the high half
@@ -170,68 +204,25 @@ __device__ __forceinline__ float round_bf16(float x) { return __uint_as_float(pa
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
-// One 64-column group of one stage for this thread: 4 code words (rows g, g+8 of both halves),
-// decode, 4 x NT x 2 mma, per-group rescale.  All shared-memory offsets are compile-time
-// constants once G is unrolled.
-template <int NT, bool W4>
-__device__ __forceinline__ void group_step(const int G, const uint8_t *codes, uint32_t cbase, uint32_t cswz,
-                                           const uint8_t *xa, const uint8_t *gsb, const float sc[4],
-                                           const RowDecode rd[4], const DecodeConsts &kc, float (&acc)[2][NT][4]) {
+// The mma part of one 64-column group: 4 state windows x NT token tiles x 2 halves, each token
+// tile's accumulators starting from its gsq entry, then the per-group rescale into acc.
+//   xb: shared address of the (window 0, tile 0) B fragment of this thread for the group
+//   gq: shared address of the gsq entry (tile 0) of this thread's token pair for the group
+template <int NT>
+__device__ __forceinline__ void group_mma(const uint32_t (&RA0)[8], const uint32_t (&RA1)[8], const uint32_t (&RB0)[8],
+                                          const uint32_t (&RB1)[8], uint32_t xb, uint32_t gq, const float sc[4],
+                                          float (&acc)[2][NT][4]) {
     constexpr int MP = 8 * NT;
-    // A fragments per state window i: RA0/RA1 = rows g / g+8 of half A, RB0/RB1 of half B;
-    // [2i] and [2i+1] are the k-pairs (j=0,1) and (j=2,3) of the window
-    uint32_t RA0[8], RA1[8], RB0[8], RB1[8];
-    if constexpr (!W4) {
-        const uint32_t coff = cbase + (((uint32_t)G << 4) ^ cswz);
-        const uint32_t w0 = *reinterpret_cast<const uint32_t *>(codes + coff);
-        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(codes + coff + 1024);
-        const uint32_t w2 = *reinterpret_cast<const uint32_t *>(codes + kCodeTileBytes + coff);
-        const uint32_t w3 = *reinterpret_cast<const uint32_t *>(codes + kCodeTileBytes + coff + 1024);
-        decode_word(w0, rd[0], kc, RA0);
-        decode_word(w1, rd[1], kc, RA1);
-        decode_word(w2, rd[2], kc, RB0);
-        decode_word(w3, rd[3], kc, RB1);
-    } else {
-        // 32 bytes per row and group: this thread's 8 bytes sit in 16-byte chunk 2(G%4) + tig/2 of
-        // the 128-byte line (box G/4); cbase holds 8*(tig&1) and the row offset, cswz the row swizzle
-        const int box = (G >> 2) * (2 * kCodeTileBytes);
-        const uint32_t coff = cbase + ((((uint32_t)(2 * (G & 3))) << 4) ^ cswz);
-        const uint2 q0 = *reinterpret_cast<const uint2 *>(codes + box + coff);
-        const uint2 q1 = *reinterpret_cast<const uint2 *>(codes + box + coff + 1024);
-        const uint2 q2 = *reinterpret_cast<const uint2 *>(codes + box + kCodeTileBytes + coff);
-        const uint2 q3 = *reinterpret_cast<const uint2 *>(codes + box + kCodeTileBytes + coff + 1024);
-        uint32_t t[4];
-        decode_word_w4(q0.x, kc.wmask, kc.wexp, t);
-        RA0[0] = t[0]; RA0[2] = t[1]; RA0[4] = t[2]; RA0[6] = t[3];
-        decode_word_w4(q0.y, kc.wmask, kc.wexp, t);
-        RA0[1] = t[0]; RA0[3] = t[1]; RA0[5] = t[2]; RA0[7] = t[3];
-        decode_word_w4(q1.x, kc.wmask, kc.wexp, t);
-        RA1[0] = t[0]; RA1[2] = t[1]; RA1[4] = t[2]; RA1[6] = t[3];
-        decode_word_w4(q1.y, kc.wmask, kc.wexp, t);
-        RA1[1] = t[0]; RA1[3] = t[1]; RA1[5] = t[2]; RA1[7] = t[3];
-        decode_word_w4(q2.x, kc.wmask, kc.wexp, t);
-        RB0[0] = t[0]; RB0[2] = t[1]; RB0[4] = t[2]; RB0[6] = t[3];
-        decode_word_w4(q2.y, kc.wmask, kc.wexp, t);
-        RB0[1] = t[0]; RB0[3] = t[1]; RB0[5] = t[2]; RB0[7] = t[3];
-        decode_word_w4(q3.x, kc.wmask, kc.wexp, t);
-        RB1[0] = t[0]; RB1[2] = t[1]; RB1[4] = t[2]; RB1[6] = t[3];
-        decode_word_w4(q3.y, kc.wmask, kc.wexp, t);
-        RB1[1] = t[0]; RB1[3] = t[1]; RB1[5] = t[2]; RB1[7] = t[3];
-    }
-    // group sums of the activations times the format's level offset (160 for W2, 136 for W4)
-    const float off = W4 ? -136.0f : -160.0f;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-        // the group's starting value: the activation sum times the level offset
-        const float gs0 = off * *reinterpret_cast<const float *>(gsb + n * 256 + G * 4);
-        const float gs1 = off * *reinterpret_cast<const float *>(gsb + n * 256 + 32 + G * 4);
+        const float4 q = lds128f(gq + n * 8 * 128);
         float cA[4], cB[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint2 b = *reinterpret_cast<const uint2 *>(xa + ((G * 4 + i) * MP + n * 8) * 32);
+            const uint2 b = lds64(xb + (i * MP + n * 8) * 32);
             if (i == 0) {
-                mma_bf16_c(cA, RA0[0], RA1[0], RA0[1], RA1[1], b.x, b.y, gs0, gs1);
-                mma_bf16_c(cB, RB0[0], RB1[0], RB0[1], RB1[1], b.x, b.y, gs0, gs1);
+                mma_bf16_q(cA, RA0[0], RA1[0], RA0[1], RA1[1], b.x, b.y, q);
+                mma_bf16_q(cB, RB0[0], RB1[0], RB0[1], RB1[1], b.x, b.y, q);
             } else {
                 mma_bf16(cA, RA0[2 * i], RA1[2 * i], RA0[2 * i + 1], RA1[2 * i + 1], b.x, b.y);
                 mma_bf16(cB, RB0[2 * i], RB1[2 * i], RB0[2 * i + 1], RB1[2 * i + 1], b.x, b.y);
@@ -248,6 +239,81 @@ __device__ __forceinline__ void group_step(const int G, const uint8_t *codes, ui
     }
 }
 
+// One W2 group: the four code words of this thread (rows g, g+8 of both halves) at ca, ca+1024,
+// and one code tile further.
+template <int NT>
+__device__ __forceinline__ void group_w2(uint32_t ca, uint32_t xb, uint32_t gq, const float sc[4],
+                                         const RowDecode rd[4], const DecodeConsts &kc, float (&acc)[2][NT][4]) {
+    uint32_t RA0[8], RA1[8], RB0[8], RB1[8];
+    decode_word(lds32(ca), rd[0], kc, RA0);
+    decode_word(lds32(ca + 1024), rd[1], kc, RA1);
+    decode_word(lds32(ca + kCodeTileBytes), rd[2], kc, RB0);
+    decode_word(lds32(ca + kCodeTileBytes + 1024), rd[3], kc, RB1);
+    group_mma<NT>(RA0, RA1, RB0, RB1, xb, gq, sc, acc);
+}
+
+// One W4 group: 8 bytes per row (16 nibbles), same row arrangement as W2.
+template <int NT>
+__device__ __forceinline__ void group_w4(uint32_t ca, uint32_t xb, uint32_t gq, const float sc[4],
+                                         const DecodeConsts &kc, float (&acc)[2][NT][4]) {
+    uint32_t R[4][8];
+    const uint32_t off[4] = {0u, 1024u, (uint32_t)kCodeTileBytes, (uint32_t)kCodeTileBytes + 1024u};
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const uint2 q = lds64(ca + off[r]);
+        uint32_t t[4];
+        decode_word_w4(q.x, kc.wmask, kc.wexp, t);
+        R[r][0] = t[0]; R[r][2] = t[1]; R[r][4] = t[2]; R[r][6] = t[3];
+        decode_word_w4(q.y, kc.wmask, kc.wexp, t);
+        R[r][1] = t[0]; R[r][3] = t[1]; R[r][5] = t[2]; R[r][7] = t[3];
+    }
+    group_mma<NT>(R[0], R[1], R[2], R[3], xb, gq, sc, acc);
+}
+
+// One work unit of the persistent kernel: expert e, 256-row block rb (two 128-row halves), k split ks.
+// A unit walks its stages starting at s_begin + rot (wrapping): units that run at the same time
+// then read different 128-byte column slabs of their rows, which spreads the loads over the DRAM
+// channels instead of having every CTA hit the same address interleave.
+struct Unit {
+    int e, ks, seg0, Me, s_begin, s_end, nchunks, localA, localB, nA, nB, rot;
+};
+
+// Fills U for unit u; false when the unit has no work (an expert without tokens).
+template <int MP>
+__device__ __forceinline__ bool load_unit(const DecodeGemmParams &p, int u, Unit &U) {
+    const int rb = u % p.row_blocks, t = u / p.row_blocks;
+    U.ks = t % p.ksplit;
+    U.e = t / p.ksplit;
+    U.seg0 = p.seg_off ? __ldg(p.seg_off + U.e) : 0;
+    U.Me = p.seg_off ? __ldg(p.seg_off + U.e + 1) - U.seg0 : p.M;
+    U.s_begin = U.ks * p.stages_per_split;
+    U.s_end = min(p.num_stages, U.s_begin + p.stages_per_split);
+    if (U.Me <= 0 || U.s_begin >= U.s_end) return false;
+    U.nchunks = (U.Me + MP - 1) / MP;
+    U.localA = rb * p.row_block_stride;
+    U.localB = U.localA + p.half_stride;
+    U.nA = max(0, min(128, p.N - U.localA));
+    U.nB = max(0, min(128, p.N - U.localB));
+    U.rot = u % (U.s_end - U.s_begin);
+    return true;
+}
+
+// 1D bulk copy global -> shared completing on an mbarrier (16-byte aligned, size a multiple of 16)
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
+}
+
+// Persistent: CTA b walks units b, b + gridDim.x, ...; its producer streams every stage of every
+// unit through one ring, so the next unit's first stages load while this unit finishes.
 template <int NT, bool TMA_SC, bool W4>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_xa,
@@ -260,29 +326,16 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
     constexpr int kXaOff = S::kCodeBytes;             // activation operand slice
     constexpr int kGsOff = S::kCodeBytes + S::kXaBytes;
     constexpr int kScOff = kGsOff + S::kGsBytes;
+    constexpr int kRowsOff = kScOff + S::kScBytes;    // per-row constants of the unit (its first stage)
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned start (the 128-byte swizzle repeats every 1024 bytes)
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ uint64_t full_bar[kStages], empty_bar[kStages], red_full, red_empty;
 
-    const int e = blockIdx.z;
-    const int rb = blockIdx.x;
-    const int ks = blockIdx.y;
-    const int seg0 = p.seg_off ? __ldg(p.seg_off + e) : 0;
-    const int Me = p.seg_off ? __ldg(p.seg_off + e + 1) - seg0 : p.M;
-    const int s_begin = ks * p.stages_per_split;
-    const int s_end = min(p.num_stages, s_begin + p.stages_per_split);
-    if (Me <= 0 || s_begin >= s_end) return;
-    const int nchunks = (Me + MP - 1) / MP;
-    const int nst = s_end - s_begin;
-    const int total_iters = nchunks * nst;
-    const int localA = rb * p.row_block_stride;       // first local row of half A
-    const int localB = localA + p.half_stride;        // first local row of half B
-    const int rowA = e * p.N + localA, rowB = e * p.N + localB;
+    const int units = p.units;
     const int ngroups = p.K / 64;
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool producer = threadIdx.x == 0;
-    if (producer) {
+    if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full_bar[i], 1);
             mbar_init(&empty_bar[i], kConsumerWarps);
@@ -297,54 +350,124 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
     }
     __syncthreads();
 
-    // TMA loads of iteration `it` (token chunk, 512-column stage) into its ring slot
-    auto issue = [&](int it) {
-        const int slot = it % kStages;
-        const int c = it / nst, st = s_begin + it % nst;
+    // ---------------- producer (lane 0 of the first producer warp) ----------------
+    // Its state lives in shared memory (only thread 0 touches it), so that the consumers' register
+    // budget does not pay for it.  pi = next iteration to load (over all of this CTA's units); it
+    // goes to ring slot `slot` in ring round `round` and covers token chunk c, 512-column stage st
+    // of unit U.
+    struct Producer {
+        Unit U;
+        int u, pi, slot, round, c, i, st;  // i: position of stage st within the chunk's walk
+        bool done;
+    };
+    __shared__ Producer P_;
+    Producer &P = P_;
+    // Unit descriptors, by unit ordinal modulo kUnitRing, written by the producer before the unit's
+    // first load and read by the consumers after that load lands.  The producer runs at most
+    // kStages iterations (so at most kStages units) ahead of the slowest consumer, whose unit --
+    // epilogue included -- therefore keeps its entry.
+    constexpr int kUnitRing = kStages + 2;
+    __shared__ Unit udesc[kUnitRing];
+    __shared__ int p_ord;  // producer: ordinal of unit P.U
+    auto p_seek = [&]() {  // first unit with work at or after P.u
+        int u = P.u;
+        Unit U;
+        while (u < units && !load_unit<MP>(p, u, U)) u += gridDim.x;
+        P.u = u;
+        P.U = U;
+        P.done = u >= units;
+        if (!P.done) udesc[p_ord++ % kUnitRing] = U;
+        P.c = 0;
+        P.i = 0;
+        P.st = P.done ? 0 : U.s_begin + U.rot;
+    };
+    auto issue_next = [&]() {
+        const Unit U = P.U;
+        const int slot = P.slot, c = P.c, i = P.i, st = P.st;
         uint8_t *base = smem + slot * S::kStageBytes;
-        mbar_arrive_expect_tx(&full_bar[slot], S::kTxBytes + ((TMA_SC && !W4) ? S::kScBytes : 0));
+        uint64_t *bar = &full_bar[slot];
+        const int rowA = U.e * p.N + U.localA, rowB = U.e * p.N + U.localB;
+        const bool first = c == 0 && i == 0;
+        const uint32_t row_bytes = first ? (uint32_t)(U.nA + U.nB) * 4u * (W4 ? 1u : 2u) : 0u;
+        mbar_arrive_expect_tx(bar, S::kTxBytes + ((TMA_SC && !W4) ? S::kScBytes : 0) + row_bytes);
+        if (first) {
+            // the unit's per-row constants: alpha, beta (W2) or the channel scales (W4) of both halves
+            const float *ra = W4 ? p.scales : p.alpha;
+            if (U.nA) bulk_g2s(base + kRowsOff, ra + rowA, U.nA * 4u, bar);
+            if (U.nB) bulk_g2s(base + kRowsOff + 512, ra + rowB, U.nB * 4u, bar);
+            if (!W4) {
+                if (U.nA) bulk_g2s(base + kRowsOff + 1024, p.beta + rowA, U.nA * 4u, bar);
+                if (U.nB) bulk_g2s(base + kRowsOff + 1536, p.beta + rowB, U.nB * 4u, bar);
+            }
+        }
         if (TMA_SC && !W4) {
             uint8_t *sc = base + kScOff;
-            tma_load_2d(sc, &tm_sc, &full_bar[slot], st * 8, rowA);
-            tma_load_2d(sc + S::kScBytes / 2, &tm_sc, &full_bar[slot], st * 8, rowB);
+            tma_load_2d(sc, &tm_sc, bar, st * 8, rowA);
+            tma_load_2d(sc + S::kScBytes / 2, &tm_sc, bar, st * 8, rowB);
         }
         // W2: 128 code bytes per row per stage; W4: 256, as two 128-byte boxes
 #pragma unroll
         for (int bx = 0; bx < (W4 ? 2 : 1); ++bx) {
             const int x = st * (W4 ? 256 : 128) + bx * 128;
-            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes, &tm_codes, &full_bar[slot], x, rowA);
-            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes + kCodeTileBytes, &tm_codes, &full_bar[slot], x, rowB);
+            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes, &tm_codes, bar, x, rowA);
+            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes + kCodeTileBytes, &tm_codes, bar, x, rowB);
         }
-        tma_load_3d(base + kXaOff, &tm_xa, &full_bar[slot], 0, seg0 + c * MP, st * 32);
-        tma_load_2d(base + kGsOff, &tm_gs, &full_bar[slot], st * 8, seg0 + c * MP);
+        tma_load_3d(base + kXaOff, &tm_xa, bar, 0, U.seg0 + c * MP, st * 32);
+        tma_load_2d(base + kGsOff, &tm_gs, bar, st * 32, U.seg0 + c * MP);
+        ++P.pi;
+        if (slot + 1 == kStages) {
+            P.slot = 0;
+            ++P.round;
+        } else {
+            P.slot = slot + 1;
+        }
+        if (i + 1 == U.s_end - U.s_begin) {
+            P.i = 0;
+            P.st = U.s_begin + U.rot;
+            if (c + 1 == U.nchunks) {
+                P.u += gridDim.x;
+                p_seek();
+            } else {
+                P.c = c + 1;
+            }
+        } else {
+            P.i = i + 1;
+            P.st = st + 1 == U.s_end ? U.s_begin : st + 1;
+        }
     };
-    if (producer)
-        for (int it = 0; it < min(kStages - 1, total_iters); ++it) issue(it);
+    if (warp >= kConsumerWarps) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+        if (warp == kConsumerWarps && lane == 0) {
+            P.u = blockIdx.x;
+            P.pi = P.slot = P.round = 0;
+            p_ord = 0;
+            p_seek();
+            bool pok = true;
+            while (!P.done) {
+                // a slot is free once every consumer warp released its last use (ring round - 1)
+                if (P.pi >= kStages && !mbar_wait(&empty_bar[P.slot], (P.round & 1) ^ 1, p.err)) {
+                    pok = false;
+                    break;
+                }
+                issue_next();
+            }
+            if (!pok) {
+                // consumers stopped releasing: let the copies in flight land before exiting (bounded)
+                for (int j = max(0, P.pi - kStages); j < P.pi; ++j)
+                    if (!mbar_wait(&full_bar[j % kStages], (j / kStages) & 1, p.err)) break;
+            }
+        }
+        return;
+    }
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
 
     // ---------------- consumers ----------------
     const int g = lane >> 2, tig = lane & 3;
     const int wslot = warp & (kRowWarps - 1);  // row slot: 16 rows inside each 128-row half
     const int khalf = warp / kRowWarps;        // 0: groups 0-3 of every stage, 1: groups 4-7
+    const int Gh = 4 * khalf;
     const int wrow = wslot * 16;
-    // local rows (within the expert) of the four rows this thread decodes
-    int lrow[4] = {localA + wrow + g, localA + wrow + g + 8, localB + wrow + g, localB + wrow + g + 8};
-    RowDecode rd[4];
-    bool rvalid[4];
-    float sc_row[4];  // W4: per-channel scales, bf16-rounded
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        rvalid[r] = lrow[r] < p.N;
-        const int grow = e * p.N + (rvalid[r] ? lrow[r] : 0);
-        if constexpr (!W4) {
-            const float a = __ldg(p.alpha + grow), b = __ldg(p.beta + grow);
-            rd[r].ab = f2_pack(a, a);
-            rd[r].bb = f2_pack(b, b);
-            sc_row[r] = 0.0f;
-        } else {
-            rd[r].ab = rd[r].bb = 0;
-            sc_row[r] = round_bf16(__ldg(p.scales + grow));
-        }
-    }
+
     DecodeConsts kc;
     const uint32_t opaque = (uint32_t)(p.K >> 30);  // == 0; keeps the constants in registers
     kc.neg_magic = f2_pack(-8388608.0f, -8388608.0f);
@@ -353,6 +476,36 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
     kc.wmask = (W4 ? 0x000F000Fu : 0x003F003Fu) ^ opaque;  // one state window / one nibble per half
     kc.wexp = (W4 ? 0x43084308u : 0x43004300u) ^ opaque;   // BF16 128 (W4: and the nibble sign flip)
 
+    // per-thread shared-memory offsets inside a stage, for this warp's four groups Gh..Gh+3
+    uint32_t coff[4];
+#pragma unroll
+    for (int G = 0; G < 4; ++G) {
+        if constexpr (!W4) {
+            // word tig of row wrow+g in 16-byte chunk (Gh+G) ^ g (128-byte swizzle)
+            coff[G] = kCodeOff + (uint32_t)(wrow + g) * 128u + 4u * (uint32_t)tig + ((uint32_t)((Gh + G) ^ g) << 4);
+        } else {
+            // 32 bytes per row and group: this thread's 8 bytes sit in chunk (2G + tig/2) ^ g of the
+            // 128-byte line of box khalf
+            coff[G] = kCodeOff + (uint32_t)khalf * (2u * kCodeTileBytes) + (uint32_t)(wrow + g) * 128u +
+                      8u * ((uint32_t)tig & 1u) + ((uint32_t)((2 * G + (tig >> 1)) ^ g) << 4);
+        }
+    }
+    const uint32_t xa_thr = kXaOff + (uint32_t)(Gh * 4 * MP * 32) + (uint32_t)g * 32u + (uint32_t)tig * 8u;
+    const uint32_t gs_thr = kGsOff + (uint32_t)(2 * tig) * 128u + (uint32_t)Gh * 16u;  // token pair 2tig, 2tig+1
+    const uint32_t sc_thr = kScOff + (uint32_t)(wrow + g) * 32u + (uint32_t)Gh * 4u;   // row wrow+g, groups Gh..
+    const uint32_t rows_thr = kRowsOff + (uint32_t)(wrow + g) * 4u;                     // row wrow+g of half A
+    const uint32_t sbase = smem_u32(smem);
+
+    bool ok = true;
+    int it = 0, slot = 0, round = 0, cc = 0;  // iteration (over all units), ring slot and round, chunk count
+    // the number of units with work this CTA will process (same walk as the producer's)
+    int n_units = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        Unit t;
+        n_units += load_unit<MP>(p, u, t) ? 1 : 0;
+    }
+    RowDecode rd[4];
+    float sc_row[4];  // W4: per-channel scales, bf16-rounded
     float acc[2][NT][4];
 #pragma unroll
     for (int t = 0; t < 2; ++t)
@@ -360,147 +513,157 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
         for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc[t][n][q] = 0.0f;
-
-    // per-thread shared-memory offsets inside a stage
-    const uint32_t cbase = (uint32_t)(wrow + g) * 128u +
-                           (W4 ? 8u * ((uint32_t)tig & 1u) : 4u * (uint32_t)tig);  // code word of row wrow+g
-    const uint32_t cswz = ((uint32_t)g << 4) ^ (W4 ? (((uint32_t)tig >> 1) << 4) : 0u);  // 128B swizzle (+ W4 chunk)
-    const uint32_t xa_thr = (uint32_t)g * 32u + (uint32_t)tig * 8u;  // B fragment of token g, lane tig
-    const uint32_t gs_thr = (uint32_t)(2 * tig) * 32u;               // group sums of token 2*tig
-    const uint32_t sc_thr = (uint32_t)(wrow + g) * 32u;              // scales of row wrow+g
-
-    bool ok = true;
-    int consumed = 0;  // iterations whose loads this thread has seen land
-    for (int it = 0; it < total_iters; ++it) {
-        const int slot = it % kStages;
-        const int c = it / nst, st = s_begin + it % nst;
-        if (producer && it + kStages - 1 < total_iters) {
-            // refill the slot every warp released at iteration it-1 (kStages-1 stages of lookahead)
-            const int nx = it + kStages - 1;
-            if (nx >= kStages) ok = mbar_wait(&empty_bar[nx % kStages], ((nx / kStages) - 1) & 1, p.err);
-            if (ok) issue(nx);
-        }
-        if (!ok || !mbar_wait(&full_bar[slot], (it / kStages) & 1, p.err)) {
+    // walk: unit ordinal cu, token chunk c, position i of stage st in the chunk's rotated walk
+    int cu = 0, c = 0, i = 0, st = 0;
+    while (cu < n_units) {
+        if (!ok || !mbar_wait(&full_bar[slot], round & 1, p.err)) {
             ok = false;
             break;
         }
-        consumed = it + 1;
-        const uint8_t *base = smem + slot * S::kStageBytes;
-        const uint8_t *xa = base + kXaOff + xa_thr;
-        const uint8_t *gsb = base + kGsOff + gs_thr;
+        const Unit &U = udesc[cu % kUnitRing];  // written before this unit's first load was issued
+        const bool first = c == 0 && i == 0;
+        if (first) st = U.s_begin + U.rot;
+        const uint32_t sb = sbase + (uint32_t)(slot * S::kStageBytes);
+        if (first) {
+            // this unit's per-row constants arrived with its first stage
+            const uint32_t ra = sb + rows_thr;
+            const float r0 = lds_f32(ra), r1 = lds_f32(ra + 32), r2 = lds_f32(ra + 512), r3 = lds_f32(ra + 544);
+            if constexpr (!W4) {
+                const float b0 = lds_f32(ra + 1024), b1 = lds_f32(ra + 1056), b2 = lds_f32(ra + 1536),
+                            b3 = lds_f32(ra + 1568);
+                rd[0].ab = f2_pack(r0, r0); rd[0].bb = f2_pack(b0, b0);
+                rd[1].ab = f2_pack(r1, r1); rd[1].bb = f2_pack(b1, b1);
+                rd[2].ab = f2_pack(r2, r2); rd[2].bb = f2_pack(b2, b2);
+                rd[3].ab = f2_pack(r3, r3); rd[3].bb = f2_pack(b3, b3);
+            } else {
+                sc_row[0] = round_bf16(r0); sc_row[1] = round_bf16(r1);
+                sc_row[2] = round_bf16(r2); sc_row[3] = round_bf16(r3);
+            }
+        }
         if (W4) {
             // per-channel scales; groups beyond K read TMA zero fill (activations 0) and add nothing
-            const int Gh = 4 * khalf;
 #pragma unroll
-            for (int G = 0; G < 4; ++G)
-                group_step<NT, W4>(Gh + G, base, cbase, cswz, xa, gsb, sc_row, rd, kc, acc);
+            for (int G = 0; G < 4; ++G) {
+                group_w4<NT>(sb + coff[G], sb + xa_thr + G * 4 * MP * 32, sb + gs_thr + G * 16, sc_row, kc, acc);
+            }
         } else if (TMA_SC) {
             // full stage: groups beyond K read TMA zero fill (scale 0, activations 0) and add nothing
-            const uint8_t *scb = base + kScOff + sc_thr;
-            {
-                // this warp's four groups of the stage: offsets are immediates
-                const int Gh = 4 * khalf;
-                const uint8_t *xah = xa + Gh * 4 * MP * 32;
-                const uint8_t *gsh = gsb + Gh * 4;
-                const uint8_t *sch = scb + Gh * 4;
-                const uint32_t cswz_h = cswz ^ ((uint32_t)Gh << 4);
+            const float4 s0 = lds128f(sb + sc_thr);
+            const float4 s1 = lds128f(sb + sc_thr + 256);
+            const float4 s2 = lds128f(sb + sc_thr + 4096);
+            const float4 s3 = lds128f(sb + sc_thr + 4096 + 256);
+            const float v0[4] = {s0.x, s0.y, s0.z, s0.w}, v1[4] = {s1.x, s1.y, s1.z, s1.w};
+            const float v2[4] = {s2.x, s2.y, s2.z, s2.w}, v3[4] = {s3.x, s3.y, s3.z, s3.w};
 #pragma unroll
-                for (int G = 0; G < 4; ++G) {
-                    float sc[4];
-                    sc[0] = round_bf16(*reinterpret_cast<const float *>(sch + G * 4));
-                    sc[1] = round_bf16(*reinterpret_cast<const float *>(sch + 256 + G * 4));
-                    sc[2] = round_bf16(*reinterpret_cast<const float *>(sch + 4096 + G * 4));
-                    sc[3] = round_bf16(*reinterpret_cast<const float *>(sch + 4096 + 256 + G * 4));
-                    group_step<NT, W4>(G, base, cbase, cswz_h, xah, gsh, sc, rd, kc, acc);
-                }
+            for (int G = 0; G < 4; ++G) {
+                const float sc[4] = {round_bf16(v0[G]), round_bf16(v1[G]), round_bf16(v2[G]),
+                                     round_bf16(v3[G])};
+                group_w2<NT>(sb + coff[G], sb + xa_thr + G * 4 * MP * 32, sb + gs_thr + G * 16, sc, rd, kc,
+                             acc);
             }
         } else {
-            const int g_lim = min(8, ngroups - st * 8);
+            const int g_lim = min(4, ngroups - st * 8 - Gh);
 #pragma unroll 1
-            for (int G = 4 * khalf; G < min(g_lim, 4 * khalf + 4); ++G) {
-                const int gg = st * 8 + G;
+            for (int G = 0; G < g_lim; ++G) {
+                const int gg = st * 8 + Gh + G;
                 float sc[4];
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                    const int grow = e * p.N + (rvalid[r] ? lrow[r] : 0);
+                    // local row of row r (g, g+8 of half A, then of half B); rows past N read row 0
+                    const int lr = (r < 2 ? U.localA : U.localB) + wrow + g + 8 * (r & 1);
+                    const int grow = U.e * p.N + (lr < p.N ? lr : 0);
                     sc[r] = round_bf16(__ldg(p.scales + (size_t)grow * ngroups + gg));
                 }
-                group_step<NT, W4>(G, base, cbase, cswz, xa, gsb, sc, rd, kc, acc);
+                const uint32_t ca = kCodeOff + (uint32_t)(wrow + g) * 128u + 4u * (uint32_t)tig +
+                                    ((uint32_t)((Gh + G) ^ g) << 4);
+                group_w2<NT>(sb + ca, sb + xa_thr + G * 4 * MP * 32, sb + gs_thr + G * 16, sc, rd, kc, acc);
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[slot]);
+        if (++slot == kStages) { slot = 0; ++round; }
+        ++it;
+        st = st + 1 == U.s_end ? U.s_begin : st + 1;
+        if (++i < U.s_end - U.s_begin) continue;
+        i = 0;
 
-        if (st == s_end - 1) {
-            // ---------------- epilogue for token chunk c ----------------
-            // the second warp of each row slot hands its partial sums to the first (bounded waits)
-            float *red = reinterpret_cast<float *>(smem + kStages * S::kStageBytes) + (wslot * 32 + lane) * (2 * NT * 4);
-            if (khalf == 1) {
-                if (c > 0 && !mbar_wait(&red_empty, (c - 1) & 1, p.err)) break;
-#pragma unroll
-                for (int t = 0; t < 2; ++t)
-#pragma unroll
-                    for (int n = 0; n < NT; ++n)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) red[(t * NT + n) * 4 + q] = acc[t][n][q];
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&red_full);
-            } else {
-                if (!mbar_wait(&red_full, c & 1, p.err)) break;
-#pragma unroll
-                for (int t = 0; t < 2; ++t)
-#pragma unroll
-                    for (int n = 0; n < NT; ++n)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) acc[t][n][q] += red[(t * NT + n) * 4 + q];
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&red_empty);
-            }
-#pragma unroll
-            for (int n = 0; n < NT && khalf == 0; ++n) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int tok = c * MP + n * 8 + 2 * tig + (q & 1);
-                    if (tok >= Me) continue;
-                    const int hr = q >> 1;  // 0: row g, 1: row g+8
-                    if (p.mode == EPI_GATEUP) {
-                        const int r = lrow[hr];  // gate row; its up row is r + half_stride
-                        if (r >= p.I) continue;
-                        const float h = silu(acc[0][n][q]) * acc[1][n][q];
-                        const size_t pr = (size_t)(seg0 + tok);
-                        reinterpret_cast<uint16_t *>(p.out)[xa_index(pr, (size_t)r, (size_t)p.h_P)] =
-                            float_to_bf16_bits(h);
-                        continue;
-                    }
-#pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        const int r = lrow[2 * t + hr];
-                        if (!rvalid[2 * t + hr]) continue;
-                        const float v = acc[t][n][q];
-                        const size_t m = (size_t)(seg0 + tok);
-                        if (p.mode == EPI_PARTIAL_F32) {
-                            reinterpret_cast<float *>(p.out)[(size_t)ks * p.out_split_stride + m * p.out_ld + r] = v;
-                        } else if (p.mode == EPI_BF16) {
-                            reinterpret_cast<uint16_t *>(p.out)[m * p.out_ld + r] = float_to_bf16_bits(v);
-                        } else {  // EPI_DOWN
-                            reinterpret_cast<float *>(p.out)[m * p.out_ld + r] = __ldg(p.rw + m) * v;
-                        }
-                    }
-                }
+        // ---------------- epilogue for token chunk c ----------------
+        // the second warp of each row slot hands its partial sums to the first (bounded waits)
+        float *red = reinterpret_cast<float *>(smem + kStages * S::kStageBytes) + (wslot * 32 + lane) * (2 * NT * 4);
+        if (khalf == 1) {
+            if (cc > 0 && !mbar_wait(&red_empty, (cc - 1) & 1, p.err)) {
+                ok = false;
+                break;
             }
 #pragma unroll
             for (int t = 0; t < 2; ++t)
 #pragma unroll
                 for (int n = 0; n < NT; ++n)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[t][n][q] = 0.0f;
+                    for (int q = 0; q < 4; ++q) red[(t * NT + n) * 4 + q] = acc[t][n][q];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_full);
+        } else {
+            if (!mbar_wait(&red_full, cc & 1, p.err)) {
+                ok = false;
+                break;
+            }
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[t][n][q] += red[(t * NT + n) * 4 + q];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_empty);
         }
-    }
-    if (producer && !ok) {
-        // after a failed wait: let the copies already issued land before the CTA exits (bounded)
-        const int issued = min(total_iters, consumed + kStages - 1);
-        for (int it = consumed; it < issued; ++it)
-            if (!mbar_wait(&full_bar[it % kStages], (it / kStages) & 1, p.err)) break;
+        ++cc;
+        // local rows (within the expert) of the four rows this thread decoded
+        const int lrow[4] = {U.localA + wrow + g, U.localA + wrow + g + 8, U.localB + wrow + g,
+                             U.localB + wrow + g + 8};
+        const bool rvalid[4] = {wrow + g < U.nA, wrow + g + 8 < U.nA, wrow + g < U.nB, wrow + g + 8 < U.nB};
+#pragma unroll
+        for (int n = 0; n < NT && khalf == 0; ++n) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int tok = c * MP + n * 8 + 2 * tig + (q & 1);
+                if (tok >= U.Me) continue;
+                const int hr = q >> 1;  // 0: row g, 1: row g+8
+                if (p.mode == EPI_GATEUP) {
+                    const int r = lrow[hr];  // gate row; its up row is r + half_stride
+                    if (r >= p.I) continue;
+                    const float h = silu(acc[0][n][q]) * acc[1][n][q];
+                    const size_t pr = (size_t)(U.seg0 + tok);
+                    reinterpret_cast<uint16_t *>(p.out)[xa_index(pr, (size_t)r, (size_t)p.h_P)] =
+                        float_to_bf16_bits(h);
+                    continue;
+                }
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const int r = lrow[2 * t + hr];
+                    if (!rvalid[2 * t + hr]) continue;
+                    const float v = acc[t][n][q];
+                    const size_t m = (size_t)(U.seg0 + tok);
+                    if (p.mode == EPI_PARTIAL_F32) {
+                        reinterpret_cast<float *>(p.out)[(size_t)U.ks * p.out_split_stride + m * p.out_ld + r] = v;
+                    } else if (p.mode == EPI_BF16) {
+                        reinterpret_cast<uint16_t *>(p.out)[m * p.out_ld + r] = float_to_bf16_bits(v);
+                    } else {  // EPI_DOWN
+                        reinterpret_cast<float *>(p.out)[m * p.out_ld + r] = __ldg(p.rw + m) * v;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[t][n][q] = 0.0f;
+        if (++c == U.nchunks) {
+            c = 0;
+            ++cu;
+        }
     }
 }
 
@@ -521,10 +684,23 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
         smem = Smem<NT, false>::kTotal;
     }
     if (!kern) return cudaErrorInvalidValue;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // the register split assumes the kernel launches with exactly kLaunchRegs per thread
+    cudaFuncAttributes fa{};
+    cudaError_t err = cudaFuncGetAttributes(&fa, kern);
     if (err != cudaSuccess) return err;
-    dim3 grid(row_blocks, ksplit, experts);
-    kern<<<grid, kThreads, smem, s>>>(a, b, c, d, p);
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    DecodeGemmParams q = p;
+    q.row_blocks = row_blocks;
+    q.ksplit = ksplit;
+    q.units = row_blocks * ksplit * experts;
+    if (q.units <= 0) return cudaSuccess;
+    int dev = 0, sms = 0;
+    err = cudaGetDevice(&dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    kern<<<std::min(q.units, sms), kThreads, smem, s>>>(a, b, c, d, q);
     return cudaGetLastError();
 }
 

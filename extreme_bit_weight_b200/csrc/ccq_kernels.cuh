@@ -18,13 +18,18 @@ enum EpiMode : int {
 // K columns (K % 64 == 0), element (p, k) with G = k/64, r = k%64, tig = r/16, j = (r/4)%4, i = r%4
 // sits at  ((((G*4 + i)*P + p)*4 + tig)*4 + j).  Rows of one 16-column block are thus grouped by
 // the state window i they meet in the decoded weights, which makes every mma B fragment one
-// contiguous, bank-conflict-free 8-byte shared-memory read.  Alongside it, gsum[p][G] holds
-// sum_{k in group G} x[p][k] (fp32, summed in column order; row pitch gsum_ld = round_up(K/64, 4)).
+// contiguous, bank-conflict-free 8-byte shared-memory read.  Alongside it the group-sum table
+// gsq[p][G] (float4, row pitch gsum_ld(K) entries) holds {L*S(p,G), L*S(p+1,G), L*S(p,G),
+// L*S(p+1,G)}: S(p,G) = sum of x[p][k] over group G (fp32, column order; 0 past the last valid row)
+// and L the weight format's level offset (gsq_level).
 __host__ __device__ inline size_t xa_index(size_t p, size_t k, size_t P) {
     size_t G = k >> 6, r = k & 63, tig = r >> 4, j = (r >> 2) & 3, i = r & 3;
     return ((((G * 4 + i) * P + p) * 4 + tig) * 4 + j);
 }
 __host__ __device__ inline int gsum_ld(int K) { return ((K / 64) + 3) & ~3; }
+// The decoders hand the tensor core BF16 (128 + u) for W2 state u (weight level u - 32) and
+// (128 + q + 8) for W4 nibble q: the per-group accumulator starts at L * S with L = -160 / -136.
+__host__ __device__ inline float gsq_level(bool w4) { return w4 ? -136.0f : -160.0f; }
 
 struct DecodeGemmParams {
     const float *scales;  // [rows_total][K/64]
@@ -51,6 +56,8 @@ struct DecodeGemmParams {
     int tma_scales;       // 1: scales staged by TMA with the codes (row pitch a multiple of 16 B)
     int w4;               // 1: W4 per-channel codes (two per byte), scales[row]
     uint32_t *err;
+    // work units (set by the launcher): unit u = (expert, k split, row block), row block fastest
+    int row_blocks, ksplit, units;
 };
 
 cudaError_t launch_decode_gemm_w2(const DecodeGemmParams &p, const CUtensorMap &tm_codes,
@@ -92,10 +99,11 @@ cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, c
                            const float *beta, int rows, int K, uint16_t *out, cudaStream_t s);
 
 // x (BF16 [rows][K], row r taken from x[tok_of ? tok_of[p] : p]) -> XA operand + group sums.
-cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, uint16_t *xa,
-                           float *gsum, cudaStream_t s);
-// group sums of an operand already in XA layout (rows [0, P_valid))
-cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float *gsum, cudaStream_t s);
+cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,
+                           uint16_t *xa, float *gsq, cudaStream_t s);
+// group-sum table of an operand already in XA layout (rows [0, P_valid))
+cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float level, float *gsq,
+                                cudaStream_t s);
 
 cudaError_t launch_splitk_reduce(const float *partial, int ksplit, size_t split_stride, int M, int N,
                                  uint16_t *y, cudaStream_t s);
