@@ -34,6 +34,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "ccq_device.cuh"
 #include "ccq_kernels.cuh"
@@ -163,22 +164,6 @@ __device__ __forceinline__ void decode_word_w4(uint32_t w, uint32_t m4, uint32_t
     asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[3]) : "r"(w >> 12), "r"(m4), "r"(x4));
 }
 
-// shared-memory reads through 32-bit shared-window addresses
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-    uint2 v;
-    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ float4 lds128f(uint32_t a) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
-    return v;
-}
 
 __device__ __forceinline__ void mma_bf16(float *c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -204,30 +189,63 @@ __device__ __forceinline__ float round_bf16(float x) { return __uint_as_float(pa
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
-// The mma part of one 64-column group: 4 state windows x NT token tiles x 2 halves, each token
+// Shared-memory reads at a base address plus a compile-time offset, written as one instruction
+// with an immediate offset (no address arithmetic per read).
+template <int OFF>
+__device__ __forceinline__ uint32_t lds32_at(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ uint2 lds64_at(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ float4 lds128f_at(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(a), "n"(OFF));
+    return v;
+}
+
+// f(std::integral_constant<int, 0>{}), ..., f(std::integral_constant<int, N-1>{})
+template <class F, int... Is>
+__device__ __forceinline__ void static_for_impl(F &&f, std::integer_sequence<int, Is...>) {
+    (f(std::integral_constant<int, Is>{}), ...);
+}
+template <int N, class F>
+__device__ __forceinline__ void static_for(F &&f) {
+    static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+// The mma part of one 64-column group G: 4 state windows x NT token tiles x 2 halves, each token
 // tile's accumulators starting from its gsq entry, then the per-group rescale into acc.
-//   xb: shared address of the (window 0, tile 0) B fragment of this thread for the group
-//   gq: shared address of the gsq entry (tile 0) of this thread's token pair for the group
-template <int NT>
+//   xs: shared address of this thread's B fragments in the stage (group 0, window 0, tile 0)
+//   gs: shared address of this thread's gsq entries in the stage (group 0, tile 0)
+template <int NT, int G>
 __device__ __forceinline__ void group_mma(const uint32_t (&RA0)[8], const uint32_t (&RA1)[8], const uint32_t (&RB0)[8],
-                                          const uint32_t (&RB1)[8], uint32_t xb, uint32_t gq, const float sc[4],
+                                          const uint32_t (&RB1)[8], uint32_t xs, uint32_t gs, const float sc[4],
                                           float (&acc)[2][NT][4]) {
     constexpr int MP = 8 * NT;
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        const float4 q = lds128f(gq + n * 8 * 128);
+    static_for<NT>([&](auto nc) {
+        constexpr int n = decltype(nc)::value;
+        const float4 q = lds128f_at<G * 16 + n * 8 * 128>(gs);
         float cA[4], cB[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint2 b = lds64(xb + (i * MP + n * 8) * 32);
-            if (i == 0) {
+        static_for<4>([&](auto ic) {
+            constexpr int i = decltype(ic)::value;
+            const uint2 b = lds64_at<((G * 4 + i) * MP + n * 8) * 32>(xs);
+            if constexpr (i == 0) {
                 mma_bf16_q(cA, RA0[0], RA1[0], RA0[1], RA1[1], b.x, b.y, q);
                 mma_bf16_q(cB, RB0[0], RB1[0], RB0[1], RB1[1], b.x, b.y, q);
             } else {
                 mma_bf16(cA, RA0[2 * i], RA1[2 * i], RA0[2 * i + 1], RA1[2 * i + 1], b.x, b.y);
                 mma_bf16(cB, RB0[2 * i], RB1[2 * i], RB0[2 * i + 1], RB1[2 * i + 1], b.x, b.y);
             }
-        }
+        });
         acc[0][n][0] = fmaf(sc[0], cA[0], acc[0][n][0]);
         acc[0][n][1] = fmaf(sc[0], cA[1], acc[0][n][1]);
         acc[0][n][2] = fmaf(sc[1], cA[2], acc[0][n][2]);
@@ -236,38 +254,38 @@ __device__ __forceinline__ void group_mma(const uint32_t (&RA0)[8], const uint32
         acc[1][n][1] = fmaf(sc[2], cB[1], acc[1][n][1]);
         acc[1][n][2] = fmaf(sc[3], cB[2], acc[1][n][2]);
         acc[1][n][3] = fmaf(sc[3], cB[3], acc[1][n][3]);
-    }
+    });
 }
 
 // One W2 group: the four code words of this thread (rows g, g+8 of both halves) at ca, ca+1024,
 // and one code tile further.
-template <int NT>
-__device__ __forceinline__ void group_w2(uint32_t ca, uint32_t xb, uint32_t gq, const float sc[4],
+template <int NT, int G>
+__device__ __forceinline__ void group_w2(uint32_t ca, uint32_t xs, uint32_t gs, const float sc[4],
                                          const RowDecode rd[4], const DecodeConsts &kc, float (&acc)[2][NT][4]) {
     uint32_t RA0[8], RA1[8], RB0[8], RB1[8];
-    decode_word(lds32(ca), rd[0], kc, RA0);
-    decode_word(lds32(ca + 1024), rd[1], kc, RA1);
-    decode_word(lds32(ca + kCodeTileBytes), rd[2], kc, RB0);
-    decode_word(lds32(ca + kCodeTileBytes + 1024), rd[3], kc, RB1);
-    group_mma<NT>(RA0, RA1, RB0, RB1, xb, gq, sc, acc);
+    decode_word(lds32_at<0>(ca), rd[0], kc, RA0);
+    decode_word(lds32_at<1024>(ca), rd[1], kc, RA1);
+    decode_word(lds32_at<kCodeTileBytes>(ca), rd[2], kc, RB0);
+    decode_word(lds32_at<kCodeTileBytes + 1024>(ca), rd[3], kc, RB1);
+    group_mma<NT, G>(RA0, RA1, RB0, RB1, xs, gs, sc, acc);
 }
 
 // One W4 group: 8 bytes per row (16 nibbles), same row arrangement as W2.
-template <int NT>
-__device__ __forceinline__ void group_w4(uint32_t ca, uint32_t xb, uint32_t gq, const float sc[4],
+template <int NT, int G>
+__device__ __forceinline__ void group_w4(uint32_t ca, uint32_t xs, uint32_t gs, const float sc[4],
                                          const DecodeConsts &kc, float (&acc)[2][NT][4]) {
     uint32_t R[4][8];
-    const uint32_t off[4] = {0u, 1024u, (uint32_t)kCodeTileBytes, (uint32_t)kCodeTileBytes + 1024u};
+    const uint2 q[4] = {lds64_at<0>(ca), lds64_at<1024>(ca), lds64_at<kCodeTileBytes>(ca),
+                        lds64_at<kCodeTileBytes + 1024>(ca)};
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const uint2 q = lds64(ca + off[r]);
         uint32_t t[4];
-        decode_word_w4(q.x, kc.wmask, kc.wexp, t);
+        decode_word_w4(q[r].x, kc.wmask, kc.wexp, t);
         R[r][0] = t[0]; R[r][2] = t[1]; R[r][4] = t[2]; R[r][6] = t[3];
-        decode_word_w4(q.y, kc.wmask, kc.wexp, t);
+        decode_word_w4(q[r].y, kc.wmask, kc.wexp, t);
         R[r][1] = t[0]; R[r][3] = t[1]; R[r][5] = t[2]; R[r][7] = t[3];
     }
-    group_mma<NT>(R[0], R[1], R[2], R[3], xb, gq, sc, acc);
+    group_mma<NT, G>(R[0], R[1], R[2], R[3], xs, gs, sc, acc);
 }
 
 // One work unit of the persistent kernel: expert e, 256-row block rb (two 128-row halves), k split ks.
@@ -542,25 +560,26 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
         }
         if (W4) {
             // per-channel scales; groups beyond K read TMA zero fill (activations 0) and add nothing
-#pragma unroll
-            for (int G = 0; G < 4; ++G) {
-                group_w4<NT>(sb + coff[G], sb + xa_thr + G * 4 * MP * 32, sb + gs_thr + G * 16, sc_row, kc, acc);
-            }
+            const uint32_t xs = sb + xa_thr, gs = sb + gs_thr;
+            static_for<4>([&](auto Gc) {
+                constexpr int G = decltype(Gc)::value;
+                group_w4<NT, G>(sb + coff[G], xs, gs, sc_row, kc, acc);
+            });
         } else if (TMA_SC) {
             // full stage: groups beyond K read TMA zero fill (scale 0, activations 0) and add nothing
-            const float4 s0 = lds128f(sb + sc_thr);
-            const float4 s1 = lds128f(sb + sc_thr + 256);
-            const float4 s2 = lds128f(sb + sc_thr + 4096);
-            const float4 s3 = lds128f(sb + sc_thr + 4096 + 256);
+            const uint32_t sa = sb + sc_thr;
+            const float4 s0 = lds128f_at<0>(sa);
+            const float4 s1 = lds128f_at<256>(sa);
+            const float4 s2 = lds128f_at<4096>(sa);
+            const float4 s3 = lds128f_at<4096 + 256>(sa);
             const float v0[4] = {s0.x, s0.y, s0.z, s0.w}, v1[4] = {s1.x, s1.y, s1.z, s1.w};
             const float v2[4] = {s2.x, s2.y, s2.z, s2.w}, v3[4] = {s3.x, s3.y, s3.z, s3.w};
-#pragma unroll
-            for (int G = 0; G < 4; ++G) {
-                const float sc[4] = {round_bf16(v0[G]), round_bf16(v1[G]), round_bf16(v2[G]),
-                                     round_bf16(v3[G])};
-                group_w2<NT>(sb + coff[G], sb + xa_thr + G * 4 * MP * 32, sb + gs_thr + G * 16, sc, rd, kc,
-                             acc);
-            }
+            const uint32_t xs = sb + xa_thr, gs = sb + gs_thr;
+            static_for<4>([&](auto Gc) {
+                constexpr int G = decltype(Gc)::value;
+                const float sc[4] = {round_bf16(v0[G]), round_bf16(v1[G]), round_bf16(v2[G]), round_bf16(v3[G])};
+                group_w2<NT, G>(sb + coff[G], xs, gs, sc, rd, kc, acc);
+            });
         } else {
             const int g_lim = min(4, ngroups - st * 8 - Gh);
 #pragma unroll 1
@@ -576,7 +595,7 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
                 }
                 const uint32_t ca = kCodeOff + (uint32_t)(wrow + g) * 128u + 4u * (uint32_t)tig +
                                     ((uint32_t)((Gh + G) ^ g) << 4);
-                group_w2<NT>(sb + ca, sb + xa_thr + G * 4 * MP * 32, sb + gs_thr + G * 16, sc, rd, kc, acc);
+                group_w2<NT, 0>(sb + ca, sb + xa_thr + G * 4 * MP * 32, sb + gs_thr + G * 16, sc, rd, kc, acc);
             }
         }
         __syncwarp();
