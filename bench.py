@@ -76,8 +76,10 @@ def tensor_peak():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["bf16_tflops"]), "measured bf16_tflops (burst)"
-    return 1590.0, "fallback"
+        # the timed region is seconds of back-to-back steps under the power cap: the sustained
+        # figure is the matching denominator (the burst one is reported beside it)
+        return float(d["bf16_tflops_sustained"]), "measured bf16_tflops_sustained", float(d["bf16_tflops"])
+    return 1400.0, "fallback (sustained)", 1590.0
 
 
 def config_dict():
@@ -397,10 +399,12 @@ def run_ours(args, rank, world, local):
     flops2 = 2.0 * valid_pairs * H * I
     roofline_tensor = None
     if prefill:
-        tf, tsrc = tensor_peak()
+        tf, tsrc, tf_burst = tensor_peak()
+        ach_tf = flops13 / (gemm1_ms * 1e-3) / 1e12
         roofline_tensor = {"bound": "tensor", "kernel": "tc_gemm_w2_kernel (gate/up, SiLU epilogue)",
-                           "achieved": flops13 / (gemm1_ms * 1e-3) / 1e12, "peak": tf, "peak_source": tsrc,
-                           "unit": "TFLOP/s", "frac": flops13 / (gemm1_ms * 1e-3) / 1e12 / tf, "traffic": None,
+                           "achieved": ach_tf, "peak": tf, "peak_source": tsrc,
+                           "unit": "TFLOP/s", "frac": ach_tf / tf, "frac_of_burst": ach_tf / tf_burst,
+                           "traffic": None,
                            "launch_ms": gemm1_ms, "algorithmic_flops_per_launch": flops13,
                            "down_kernel": {"achieved": flops2 / (gemm2_ms * 1e-3) / 1e12, "launch_ms": gemm2_ms,
                                            "algorithmic_flops_per_launch": flops2},

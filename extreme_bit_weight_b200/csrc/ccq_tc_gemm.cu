@@ -170,7 +170,9 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                   const TcGemmParams p) {
     using S = TcSmem<MT>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned start, kept as an offset from the shared array so that loads and stores
+    // through it stay shared-memory instructions
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *sA = smem;
     uint8_t *sB = smem + S::kA;
     uint8_t *sC = smem + S::kA + S::kB;
@@ -289,7 +291,20 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             const float alpha = W4 ? 0.0f : __ldg(p.alpha + grow), beta = W4 ? 0.0f : __ldg(p.beta + grow);
             const float *srow = p.scales + grow * (W4 ? 1 : nk);
             const float sc_row = W4 ? bf16_bits_to_float(float_to_bf16_bits(__ldg(srow))) : 0.0f;
+            // W2 group scales, four groups (one code stage) at a time and one stage ahead, so the
+            // global read is off the decode's critical path
+            auto load_sc4 = [&](int g0) -> float4 {
+                if (W4 || g0 >= nk) return make_float4(0.f, 0.f, 0.f, 0.f);
+                if ((nk & 3) == 0) return __ldg(reinterpret_cast<const float4 *>(srow + g0));
+                return make_float4(__ldg(srow + g0), g0 + 1 < nk ? __ldg(srow + g0 + 1) : 0.f,
+                                   g0 + 2 < nk ? __ldg(srow + g0 + 2) : 0.f, g0 + 3 < nk ? __ldg(srow + g0 + 3) : 0.f);
+            };
+            float4 sc_cur = make_float4(0.f, 0.f, 0.f, 0.f), sc_next = load_sc4(0);
             for (int ks = 0; ks < nk && ok; ++ks) {
+                if (!W4 && (ks & 3) == 0) {
+                    sc_cur = sc_next;
+                    sc_next = load_sc4(ks + 4);
+                }
                 const int cs = ci % kSC;
                 if (ks % kKsPerCode == 0) {
                     ok = mbar_wait(&c_full[cs], (ci / kSC) & 1, p.err);
@@ -313,7 +328,9 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 }
                 uint32_t o[4][8];
                 if (!W4) {
-                    const float sc = bf16_bits_to_float(float_to_bf16_bits(__ldg(srow + ks)));
+                    const int gi = ks & 3;
+                    const float sraw = gi == 0 ? sc_cur.x : gi == 1 ? sc_cur.y : gi == 2 ? sc_cur.z : sc_cur.w;
+                    const float sc = bf16_bits_to_float(float_to_bf16_bits(sraw));
                     const uint32_t s2 = pack_bf16x2(sc, sc);
                     decode_word_bf16(q.x, alpha, beta, s2, o[0]);
                     decode_word_bf16(q.y, alpha, beta, s2, o[1]);
