@@ -350,6 +350,9 @@ def run_ours(args, rank, world, local):
     total_ms = start.elapsed_time(stop)
     gemm1_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     gemm2_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in evs)
+    # the decode path may run both projections as one launch: then events 3, 4, 5 are recorded
+    # back to back and the "down" interval is only event overhead
+    fused = (not prefill) and gemm2_ms < 0.02 * gemm1_ms
     if pg:
         t = torch.tensor([total_ms], device=device)
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
@@ -415,16 +418,22 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(),
         "packed_weight_gbs": layer_gbs, "packed_weight_pct_of_8tbs": 100.0 * layer_gbs / NOMINAL_HBM_GBS,
         "touched_experts": ne,
-        "roofline": roofline_tensor or {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (gate/up, SiLU epilogue)",
-                     "achieved": ach13, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "unit": "GB/s",
-                     "frac": ach13 / hbm, "traffic": None, "launch_ms": gemm1_ms,
-                     "algorithmic_bytes_per_launch": b13,
-                     "down_kernel": {"achieved": b2 / (gemm2_ms * 1e-3) / 1e9, "launch_ms": gemm2_ms,
-                                     "algorithmic_bytes_per_launch": b2}},
+        "roofline": roofline_tensor or (
+            {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (fused MoE: gate/up + SiLU, then down)",
+             "achieved": (b13 + b2) / (gemm1_ms * 1e-3) / 1e9, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)",
+             "unit": "GB/s", "frac": (b13 + b2) / (gemm1_ms * 1e-3) / 1e9 / hbm, "traffic": None,
+             "launch_ms": gemm1_ms, "algorithmic_bytes_per_launch": b13 + b2} if fused else
+            {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (gate/up, SiLU epilogue)",
+             "achieved": ach13, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "unit": "GB/s",
+             "frac": ach13 / hbm, "traffic": None, "launch_ms": gemm1_ms,
+             "algorithmic_bytes_per_launch": b13,
+             "down_kernel": {"achieved": b2 / (gemm2_ms * 1e-3) / 1e9, "launch_ms": gemm2_ms,
+                             "algorithmic_bytes_per_launch": b2}}),
         "cpu_baseline": cpu,
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 6 * K,
+        # our kernels per step: route, pack, matmul(s), [group sums], combine
+        "gpu_launches": (4 if fused else 6) * K,
         "clocks": clk,
     }
     if rank == 0:

@@ -156,11 +156,14 @@ __global__ void splitk_reduce_kernel(const float *__restrict__ partial, int kspl
 __global__ void moe_route_kernel(const int *__restrict__ ids, const float *__restrict__ rw, int T, int topk,
                                  int E, int *__restrict__ seg_off, int *__restrict__ cursor,
                                  int *__restrict__ tok_of, float *__restrict__ rw_perm, int *__restrict__ inv,
-                                 uint32_t *err) {
+                                 int *__restrict__ dep, uint32_t *err) {
     extern __shared__ int sh[];
     int *cnt = sh;          // [E]
     int *off = sh + E;      // [E+1]
-    for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        cnt[i] = 0;
+        if (dep) dep[i] = 0;  // per-expert completion counters of the fused matmul launch
+    }
     __syncthreads();
     const int npairs = T * topk;
     for (int q = threadIdx.x; q < npairs; q += blockDim.x) {
@@ -269,13 +272,13 @@ cudaError_t launch_splitk_reduce(const float *partial, int ksplit, size_t split_
 }
 
 cudaError_t launch_moe_route(const int *ids, const float *rw, int T, int topk, int E, int *seg_off, int *cursor,
-                             int *tok_of, float *rw_perm, int *inv, uint32_t *err, cudaStream_t s) {
+                             int *tok_of, float *rw_perm, int *inv, int *dep, uint32_t *err, cudaStream_t s) {
     const size_t sh = sizeof(int) * (2 * (size_t)E + 1);
     if (sh > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
         if (e != cudaSuccess) return e;
     }
-    moe_route_kernel<<<1, 1024, sh, s>>>(ids, rw, T, topk, E, seg_off, cursor, tok_of, rw_perm, inv, err);
+    moe_route_kernel<<<1, 1024, sh, s>>>(ids, rw, T, topk, E, seg_off, cursor, tok_of, rw_perm, inv, dep, err);
     return cudaGetLastError();
 }
 

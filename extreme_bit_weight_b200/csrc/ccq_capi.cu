@@ -159,7 +159,7 @@ GemmWs gemm_layout(const ccq_weight *w, int m) {
 }
 
 struct MoeWs {
-    size_t err, seg, cursor, tok, rwp, inv, xa_x, gs_x, xa_h, gs_h, tiles, tcount, slot, total;
+    size_t err, seg, cursor, dep, tok, rwp, inv, xa_x, gs_x, xa_h, gs_h, tiles, tcount, slot, total;
     int P, max_tiles;
     bool tc;
 };
@@ -174,6 +174,7 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     L.err = off; off = up256(off + 16);
     L.seg = off; off = up256(off + sizeof(int) * (size_t)(E + 1));
     L.cursor = off; off = up256(off + sizeof(int) * (size_t)E);
+    L.dep = off; off = up256(off + sizeof(int) * (size_t)E);  // per-expert counters of the fused launch
     L.tok = off; off = up256(off + sizeof(int) * (size_t)L.P);
     L.rwp = off; off = up256(off + sizeof(float) * (size_t)L.P);
     L.inv = off; off = up256(off + sizeof(int) * (size_t)pairs);
@@ -374,6 +375,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     uint32_t *err = reinterpret_cast<uint32_t *>(base + L.err);
     int *seg = reinterpret_cast<int *>(base + L.seg);
     int *cursor = reinterpret_cast<int *>(base + L.cursor);
+    int *dep = reinterpret_cast<int *>(base + L.dep);
     int *tok = reinterpret_cast<int *>(base + L.tok);
     float *rwp = reinterpret_cast<float *>(base + L.rwp);
     int *inv = reinterpret_cast<int *>(base + L.inv);
@@ -389,7 +391,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     if (e == cudaSuccess) e = cudaMemsetAsync(base + L.tok, 0, sizeof(int) * (size_t)L.P, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(base + L.rwp, 0, sizeof(float) * (size_t)L.P, s);
     if (e == cudaSuccess)
-        e = launch_moe_route(expert_ids, routing_w, T, topk, num_experts, seg, cursor, tok, rwp, inv, err, s);
+        e = launch_moe_route(expert_ids, routing_w, T, topk, num_experts, seg, cursor, tok, rwp, inv, dep, err, s);
     if (e == cudaSuccess) e = trace(events, 1, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     if (L.tc) {
@@ -475,12 +477,6 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p1.err = err;
     p1.tma_scales = m1.tma_scales;
     p1.w4 = w13->fmt == CCQ_FMT_W4_PER_CHANNEL;
-    e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), 1, num_experts, nt1, s);
-    if (e == cudaSuccess) e = trace(events, 3, s);
-    if (e == cudaSuccess)
-        e = launch_gsum_from_xa(xa_h, pairs, L.P, I, gsq_level(w2->fmt == CCQ_FMT_W4_PER_CHANNEL), gs_h, s);
-    if (e == cudaSuccess) e = trace(events, 4, s);
-    if (e != cudaSuccess) return CCQ_ERR_CUDA;
 
     // down projection, scaled by each pair's routing weight -> fp32 slots
     DecodeMaps m2;
@@ -504,8 +500,41 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p2.err = err;
     p2.tma_scales = m2.tma_scales;
     p2.w4 = w2->fmt == CCQ_FMT_W4_PER_CHANNEL;
-    e = launch_decode_gemm_w2(p2, m2.codes, m2.xa, m2.gs, m2.sc, ceil_div(H, 256), 1, num_experts, nt2, s);
-    if (e == cudaSuccess) e = trace(events, 5, s);
+
+    // Both projections W2 with TMA-staged scales and the same token tiling: one fused launch, in
+    // which the gate/up epilogue also writes h's group-sum table and each down unit starts once
+    // its expert's gate/up units are done.  Otherwise (or if the device refuses the cooperative
+    // launch) two launches with the group sums computed in between.
+    bool fused = !p1.w4 && !p2.w4 && p1.tma_scales && p2.tma_scales && nt1 == nt2;
+    if (fused) {
+        p1.dep = dep;
+        p1.fuse_gsq = gs_h;
+        p1.fuse_gsq_ld = gsum_ld(I);
+        p1.fuse_level = gsq_level(false);
+        p2.dep = dep;
+        e = launch_decode_moe_fused(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), p2, m2.codes, m2.xa, m2.gs,
+                                    m2.sc, ceil_div(H, 256), num_experts, nt1, s);
+        if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorNotSupported) {
+            (void)cudaGetLastError();  // not launched: take the two-launch path
+            fused = false;
+        } else {
+            if (e == cudaSuccess) e = trace(events, 3, s);
+            if (e == cudaSuccess) e = trace(events, 4, s);
+            if (e == cudaSuccess) e = trace(events, 5, s);
+        }
+    }
+    if (!fused) {
+        p1.dep = p2.dep = nullptr;
+        p1.fuse_gsq = nullptr;
+        e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), 1, num_experts, nt1, s);
+        if (e == cudaSuccess) e = trace(events, 3, s);
+        if (e == cudaSuccess)
+            e = launch_gsum_from_xa(xa_h, pairs, L.P, I, gsq_level(w2->fmt == CCQ_FMT_W4_PER_CHANNEL), gs_h, s);
+        if (e == cudaSuccess) e = trace(events, 4, s);
+        if (e == cudaSuccess)
+            e = launch_decode_gemm_w2(p2, m2.codes, m2.xa, m2.gs, m2.sc, ceil_div(H, 256), 1, num_experts, nt2, s);
+        if (e == cudaSuccess) e = trace(events, 5, s);
+    }
     if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
     if (e == cudaSuccess) e = trace(events, 6, s);
     return cuda_status(e);

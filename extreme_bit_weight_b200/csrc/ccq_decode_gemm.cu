@@ -294,6 +294,12 @@ __device__ __forceinline__ void group_w4(uint32_t ca, uint32_t xs, uint32_t gs, 
 // channels instead of having every CTA hit the same address interleave.
 struct Unit {
     int e, ks, seg0, Me, s_begin, s_end, nchunks, localA, localB, nA, nB, rot;
+    int phase;  // fused launch: 0 gate/up, 1 down (always 0 otherwise)
+};
+
+// The four tensor maps of one matmul: codes, activation operand, gsq table, group scales.
+struct MapSet {
+    CUtensorMap codes, xa, gs, sc;
 };
 
 // Fills U for unit u; false when the unit has no work (an expert without tokens).
@@ -313,7 +319,42 @@ __device__ __forceinline__ bool load_unit(const DecodeGemmParams &p, int u, Unit
     U.nA = max(0, min(128, p.N - U.localA));
     U.nB = max(0, min(128, p.N - U.localB));
     U.rot = u % (U.s_end - U.s_begin);
+    U.phase = 0;
     return true;
+}
+
+// Unit u of the whole launch: fused launches number the gate/up units first, then the down units.
+template <int MP, bool FUSED>
+__device__ __forceinline__ bool load_unit_any(const DecodeGemmParams &p, const DecodeGemmParams &p2, int u, Unit &U) {
+    if (!FUSED || u < p.units) return load_unit<MP>(p, u, U);
+    const bool ok = load_unit<MP>(p2, u - p.units, U);
+    U.phase = 1;
+    return ok;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *ptr) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int *ptr, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until *ctr >= need (another CTA's release); false after kWaitLimitNs.
+__device__ __forceinline__ bool wait_counter(const int *ctr, int need, uint32_t *err) {
+    if (ld_acquire_gpu(ctr) >= need) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        __nanosleep(200);
+        if (ld_acquire_gpu(ctr) >= need) return true;
+        if (global_ns() - t0 > kWaitLimitNs) break;
+    }
+    record_error(err, DEV_ERR_TIMEOUT, 0xFFFFFFFEu);
+    return false;
 }
 
 // 1D bulk copy global -> shared completing on an mbarrier (16-byte aligned, size a multiple of 16)
@@ -332,11 +373,11 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
 
 // Persistent: CTA b walks units b, b + gridDim.x, ...; its producer streams every stage of every
 // unit through one ring, so the next unit's first stages load while this unit finishes.
-template <int NT, bool TMA_SC, bool W4>
+// FUSED: the launch holds the MoE gate/up units (p, m1) followed by the down units (p2, m2).
+template <int NT, bool TMA_SC, bool W4, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
-decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_xa,
-                      const __grid_constant__ CUtensorMap tm_gs, const __grid_constant__ CUtensorMap tm_sc,
-                      const DecodeGemmParams p) {
+decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__ MapSet m2,
+                      const __grid_constant__ DecodeGemmParams p, const __grid_constant__ DecodeGemmParams p2) {
     using S = Smem<NT, W4>;
     constexpr int MP = S::MP;
     constexpr int kStages = S::kStages;
@@ -349,9 +390,10 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
     // 1024-byte aligned start (the 128-byte swizzle repeats every 1024 bytes)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ uint64_t full_bar[kStages], empty_bar[kStages], red_full, red_empty;
+    __shared__ float epi_gs[FUSED ? kRowWarps : 1][FUSED ? MP : 1];  // fused gate/up epilogue sums
+    __shared__ uint64_t epi_bar[2];  // fused gate/up epilogue: the 8 first-half warps meet twice per chunk
 
-    const int units = p.units;
-    const int ngroups = p.K / 64;
+    const int units = p.units + (FUSED ? p2.units : 0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -360,11 +402,19 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
         }
         mbar_init(&red_full, kRowWarps);
         mbar_init(&red_empty, kRowWarps);
+        mbar_init(&epi_bar[0], kRowWarps);
+        mbar_init(&epi_bar[1], kRowWarps);
         fence_mbar_init();
-        prefetch_tensormap(&tm_codes);
-        prefetch_tensormap(&tm_xa);
-        prefetch_tensormap(&tm_gs);
-        if (TMA_SC) prefetch_tensormap(&tm_sc);
+        prefetch_tensormap(&m1.codes);
+        prefetch_tensormap(&m1.xa);
+        prefetch_tensormap(&m1.gs);
+        if (TMA_SC) prefetch_tensormap(&m1.sc);
+        if (FUSED) {
+            prefetch_tensormap(&m2.codes);
+            prefetch_tensormap(&m2.xa);
+            prefetch_tensormap(&m2.gs);
+            prefetch_tensormap(&m2.sc);
+        }
     }
     __syncthreads();
 
@@ -390,7 +440,7 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
     auto p_seek = [&]() {  // first unit with work at or after P.u
         int u = P.u;
         Unit U;
-        while (u < units && !load_unit<MP>(p, u, U)) u += gridDim.x;
+        while (u < units && !load_unit_any<MP, FUSED>(p, p2, u, U)) u += gridDim.x;
         P.u = u;
         P.U = U;
         P.done = u >= units;
@@ -402,36 +452,46 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
     auto issue_next = [&]() {
         const Unit U = P.U;
         const int slot = P.slot, c = P.c, i = P.i, st = P.st;
+        const DecodeGemmParams &q = (FUSED && U.phase) ? p2 : p;
+        const MapSet &m = (FUSED && U.phase) ? m2 : m1;
         uint8_t *base = smem + slot * S::kStageBytes;
         uint64_t *bar = &full_bar[slot];
-        const int rowA = U.e * p.N + U.localA, rowB = U.e * p.N + U.localB;
+        const int rowA = U.e * q.N + U.localA, rowB = U.e * q.N + U.localB;
         const bool first = c == 0 && i == 0;
+        if (FUSED && U.phase == 1 && first) {
+            // the down unit reads h and its gsq table: every gate/up unit of the expert must be done
+            if (!wait_counter(q.dep + U.e, q.dep_need, q.err)) {
+                P.done = true;  // consumers time out on this stage and stop
+                return;
+            }
+            fence_proxy_async_global();  // the generic-proxy writes of h are visible to TMA from here
+        }
         const uint32_t row_bytes = first ? (uint32_t)(U.nA + U.nB) * 4u * (W4 ? 1u : 2u) : 0u;
         mbar_arrive_expect_tx(bar, S::kTxBytes + ((TMA_SC && !W4) ? S::kScBytes : 0) + row_bytes);
         if (first) {
             // the unit's per-row constants: alpha, beta (W2) or the channel scales (W4) of both halves
-            const float *ra = W4 ? p.scales : p.alpha;
+            const float *ra = W4 ? q.scales : q.alpha;
             if (U.nA) bulk_g2s(base + kRowsOff, ra + rowA, U.nA * 4u, bar);
             if (U.nB) bulk_g2s(base + kRowsOff + 512, ra + rowB, U.nB * 4u, bar);
             if (!W4) {
-                if (U.nA) bulk_g2s(base + kRowsOff + 1024, p.beta + rowA, U.nA * 4u, bar);
-                if (U.nB) bulk_g2s(base + kRowsOff + 1536, p.beta + rowB, U.nB * 4u, bar);
+                if (U.nA) bulk_g2s(base + kRowsOff + 1024, q.beta + rowA, U.nA * 4u, bar);
+                if (U.nB) bulk_g2s(base + kRowsOff + 1536, q.beta + rowB, U.nB * 4u, bar);
             }
         }
         if (TMA_SC && !W4) {
             uint8_t *sc = base + kScOff;
-            tma_load_2d(sc, &tm_sc, bar, st * 8, rowA);
-            tma_load_2d(sc + S::kScBytes / 2, &tm_sc, bar, st * 8, rowB);
+            tma_load_2d(sc, &m.sc, bar, st * 8, rowA);
+            tma_load_2d(sc + S::kScBytes / 2, &m.sc, bar, st * 8, rowB);
         }
         // W2: 128 code bytes per row per stage; W4: 256, as two 128-byte boxes
 #pragma unroll
         for (int bx = 0; bx < (W4 ? 2 : 1); ++bx) {
             const int x = st * (W4 ? 256 : 128) + bx * 128;
-            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes, &tm_codes, bar, x, rowA);
-            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes + kCodeTileBytes, &tm_codes, bar, x, rowB);
+            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes, &m.codes, bar, x, rowA);
+            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes + kCodeTileBytes, &m.codes, bar, x, rowB);
         }
-        tma_load_3d(base + kXaOff, &tm_xa, bar, 0, U.seg0 + c * MP, st * 32);
-        tma_load_2d(base + kGsOff, &tm_gs, bar, st * 32, U.seg0 + c * MP);
+        tma_load_3d(base + kXaOff, &m.xa, bar, 0, U.seg0 + c * MP, st * 32);
+        tma_load_2d(base + kGsOff, &m.gs, bar, st * 32, U.seg0 + c * MP);
         ++P.pi;
         if (slot + 1 == kStages) {
             P.slot = 0;
@@ -516,11 +576,12 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
 
     bool ok = true;
     int it = 0, slot = 0, round = 0, cc = 0;  // iteration (over all units), ring slot and round, chunk count
+    int ec = 0;                               // fused gate/up chunks done (epilogue meeting parity)
     // the number of units with work this CTA will process (same walk as the producer's)
     int n_units = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
         Unit t;
-        n_units += load_unit<MP>(p, u, t) ? 1 : 0;
+        n_units += load_unit_any<MP, FUSED>(p, p2, u, t) ? 1 : 0;
     }
     RowDecode rd[4];
     float sc_row[4];  // W4: per-channel scales, bf16-rounded
@@ -539,6 +600,7 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
             break;
         }
         const Unit &U = udesc[cu % kUnitRing];  // written before this unit's first load was issued
+        const DecodeGemmParams &pq = (FUSED && U.phase) ? p2 : p;
         const bool first = c == 0 && i == 0;
         if (first) st = U.s_begin + U.rot;
         const uint32_t sb = sbase + (uint32_t)(slot * S::kStageBytes);
@@ -581,6 +643,7 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
                 group_w2<NT, G>(sb + coff[G], xs, gs, sc, rd, kc, acc);
             });
         } else {
+            const int ngroups = pq.K / 64;
             const int g_lim = min(4, ngroups - st * 8 - Gh);
 #pragma unroll 1
             for (int G = 0; G < g_lim; ++G) {
@@ -590,8 +653,8 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
                 for (int r = 0; r < 4; ++r) {
                     // local row of row r (g, g+8 of half A, then of half B); rows past N read row 0
                     const int lr = (r < 2 ? U.localA : U.localB) + wrow + g + 8 * (r & 1);
-                    const int grow = U.e * p.N + (lr < p.N ? lr : 0);
-                    sc[r] = round_bf16(__ldg(p.scales + (size_t)grow * ngroups + gg));
+                    const int grow = U.e * pq.N + (lr < pq.N ? lr : 0);
+                    sc[r] = round_bf16(__ldg(pq.scales + (size_t)grow * ngroups + gg));
                 }
                 const uint32_t ca = kCodeOff + (uint32_t)(wrow + g) * 128u + 4u * (uint32_t)tig +
                                     ((uint32_t)((Gh + G) ^ g) << 4);
@@ -641,6 +704,9 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
         const int lrow[4] = {U.localA + wrow + g, U.localA + wrow + g + 8, U.localB + wrow + g,
                              U.localB + wrow + g + 8};
         const bool rvalid[4] = {wrow + g < U.nA, wrow + g + 8 < U.nA, wrow + g < U.nB, wrow + g + 8 < U.nB};
+        float hsum[NT][2];  // fused gate/up: sums of the stored BF16 h over this thread's two rows
+#pragma unroll
+        for (int n = 0; n < NT; ++n) hsum[n][0] = hsum[n][1] = 0.0f;
 #pragma unroll
         for (int n = 0; n < NT && khalf == 0; ++n) {
 #pragma unroll
@@ -648,13 +714,14 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
                 const int tok = c * MP + n * 8 + 2 * tig + (q & 1);
                 if (tok >= U.Me) continue;
                 const int hr = q >> 1;  // 0: row g, 1: row g+8
-                if (p.mode == EPI_GATEUP) {
+                if (pq.mode == EPI_GATEUP) {
                     const int r = lrow[hr];  // gate row; its up row is r + half_stride
-                    if (r >= p.I) continue;
+                    if (r >= pq.I) continue;
                     const float h = silu(acc[0][n][q]) * acc[1][n][q];
                     const size_t pr = (size_t)(U.seg0 + tok);
-                    reinterpret_cast<uint16_t *>(p.out)[xa_index(pr, (size_t)r, (size_t)p.h_P)] =
-                        float_to_bf16_bits(h);
+                    const uint16_t hb = float_to_bf16_bits(h);
+                    reinterpret_cast<uint16_t *>(pq.out)[xa_index(pr, (size_t)r, (size_t)pq.h_P)] = hb;
+                    if constexpr (FUSED) hsum[n][q & 1] += bf16_bits_to_float(hb);
                     continue;
                 }
 #pragma unroll
@@ -663,13 +730,68 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
                     if (!rvalid[2 * t + hr]) continue;
                     const float v = acc[t][n][q];
                     const size_t m = (size_t)(U.seg0 + tok);
-                    if (p.mode == EPI_PARTIAL_F32) {
-                        reinterpret_cast<float *>(p.out)[(size_t)U.ks * p.out_split_stride + m * p.out_ld + r] = v;
-                    } else if (p.mode == EPI_BF16) {
-                        reinterpret_cast<uint16_t *>(p.out)[m * p.out_ld + r] = float_to_bf16_bits(v);
+                    if (pq.mode == EPI_PARTIAL_F32) {
+                        reinterpret_cast<float *>(pq.out)[(size_t)U.ks * pq.out_split_stride + m * pq.out_ld + r] = v;
+                    } else if (pq.mode == EPI_BF16) {
+                        reinterpret_cast<uint16_t *>(pq.out)[m * pq.out_ld + r] = float_to_bf16_bits(v);
                     } else {  // EPI_DOWN
-                        reinterpret_cast<float *>(p.out)[m * p.out_ld + r] = __ldg(p.rw + m) * v;
+                        reinterpret_cast<float *>(pq.out)[m * pq.out_ld + r] = __ldg(pq.rw + m) * v;
                     }
+                }
+            }
+        }
+        if constexpr (FUSED) {
+            if (U.phase == 0 && khalf == 0) {
+                // The down operand's gsq table for this chunk's tokens over the unit's two 64-column
+                // groups of h (row slots 0-3 and 4-7): per warp, sum the 16 rows over g in a fixed
+                // shuffle order; then the four row slots of a group, in slot order.
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        float v = hsum[n][j];
+                        v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+                        v += __shfl_xor_sync(0xFFFFFFFFu, v, 8);
+                        v += __shfl_xor_sync(0xFFFFFFFFu, v, 16);
+                        if (g == 0) epi_gs[wslot][n * 8 + 2 * tig + j] = v;
+                    }
+                // bounded meeting points (a plain barrier could wait forever for a warp that left
+                // after a timed-out wait)
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&epi_bar[0]);
+                if (!mbar_wait(&epi_bar[0], ec & 1, p.err)) {
+                    ok = false;
+                    break;
+                }
+                if ((wslot & 3) == 0 && lane < MP / 2) {
+                    const int t0 = c * MP + 2 * lane;  // token pair (t0, t0 + 1) of the expert
+                    if (t0 < U.Me) {
+                        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            s0 += epi_gs[wslot + w][2 * lane];
+                            s1 += epi_gs[wslot + w][2 * lane + 1];
+                        }
+                        if (t0 + 1 >= U.Me) s1 = 0.0f;
+                        const int G = U.localA / 64 + (wslot >> 2);
+                        const float L = pq.fuse_level;
+                        reinterpret_cast<float4 *>(pq.fuse_gsq)[(size_t)(U.seg0 + t0) * pq.fuse_gsq_ld + G] =
+                            make_float4(L * s0, L * s1, L * s0, L * s1);
+                    }
+                }
+                // epi_gs reusable, and every store of the chunk issued before the publication below
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&epi_bar[1]);
+                if (!mbar_wait(&epi_bar[1], ec & 1, p.err)) {
+                    ok = false;
+                    break;
+                }
+                ++ec;
+                if (c + 1 == U.nchunks && warp == 0 && lane == 0) {
+                    // publish the finished unit: its h and gsq writes, ordered by the barrier above
+                    __threadfence();
+                    fence_proxy_async_global();
+                    red_release_gpu_add(pq.dep + U.e, 1);
                 }
             }
         }
@@ -686,40 +808,86 @@ decode_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid
     }
 }
 
-template <int NT>
-cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUtensorMap &b,
-                      const CUtensorMap &c, const CUtensorMap &d, int row_blocks, int ksplit, int experts,
-                      cudaStream_t s) {
-    void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, DecodeGemmParams) = nullptr;
-    int smem = 0;
-    if constexpr (NT <= 2) {  // W4 keeps at most 16 tokens per chunk (its code tiles are twice as wide)
-        if (p.w4) {
-            kern = decode_gemm_w2_kernel<NT, false, true>;
-            smem = Smem<NT, true>::kTotal;
-        }
-    }
-    if (!p.w4) {
-        kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false> : decode_gemm_w2_kernel<NT, false, false>;
-        smem = Smem<NT, false>::kTotal;
-    }
-    if (!kern) return cudaErrorInvalidValue;
-    // the register split assumes the kernel launches with exactly kLaunchRegs per thread
+using DecodeKernel = void (*)(MapSet, MapSet, DecodeGemmParams, DecodeGemmParams);
+
+// Checks the kernel's launch register count (the register split assumes kLaunchRegs) and sets its
+// dynamic shared memory.
+cudaError_t prepare_kernel(DecodeKernel kern, int smem) {
     cudaFuncAttributes fa{};
     cudaError_t err = cudaFuncGetAttributes(&fa, kern);
     if (err != cudaSuccess) return err;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}
+
+int device_sms(cudaError_t &err) {
+    int dev = 0, sms = 0;
+    err = cudaGetDevice(&dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+template <int NT>
+cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUtensorMap &b,
+                      const CUtensorMap &c, const CUtensorMap &d, int row_blocks, int ksplit, int experts,
+                      cudaStream_t s) {
+    DecodeKernel kern = nullptr;
+    int smem = 0;
+    if constexpr (NT <= 2) {  // W4 keeps at most 16 tokens per chunk (its code tiles are twice as wide)
+        if (p.w4) {
+            kern = decode_gemm_w2_kernel<NT, false, true, false>;
+            smem = Smem<NT, true>::kTotal;
+        }
+    }
+    if (!p.w4) {
+        kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false, false>
+                            : decode_gemm_w2_kernel<NT, false, false, false>;
+        smem = Smem<NT, false>::kTotal;
+    }
+    if (!kern) return cudaErrorInvalidValue;
+    cudaError_t err = prepare_kernel(kern, smem);
     if (err != cudaSuccess) return err;
     DecodeGemmParams q = p;
     q.row_blocks = row_blocks;
     q.ksplit = ksplit;
     q.units = row_blocks * ksplit * experts;
     if (q.units <= 0) return cudaSuccess;
-    int dev = 0, sms = 0;
-    err = cudaGetDevice(&dev);
-    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sms(err);
     if (err != cudaSuccess) return err;
-    kern<<<std::min(q.units, sms), kThreads, smem, s>>>(a, b, c, d, q);
+    MapSet m{a, b, c, d};
+    kern<<<std::min(q.units, sms), kThreads, smem, s>>>(m, m, q, q);
+    return cudaGetLastError();
+}
+
+template <int NT>
+cudaError_t launch_fused_nt(const DecodeGemmParams &p1, const MapSet &m1, int row_blocks1, const DecodeGemmParams &p2,
+                            const MapSet &m2, int row_blocks2, int experts, cudaStream_t s) {
+    DecodeKernel kern = decode_gemm_w2_kernel<NT, true, false, true>;
+    const int smem = Smem<NT, false>::kTotal;
+    cudaError_t err = prepare_kernel(kern, smem);
+    if (err != cudaSuccess) return err;
+    DecodeGemmParams q1 = p1, q2 = p2;
+    q1.row_blocks = row_blocks1;
+    q1.ksplit = 1;
+    q1.units = row_blocks1 * experts;
+    q2.row_blocks = row_blocks2;
+    q2.ksplit = 1;
+    q2.units = row_blocks2 * experts;
+    q2.dep_need = row_blocks1;
+    if (q1.units + q2.units <= 0) return cudaSuccess;
+    // down units wait for other CTAs' gate/up units: every CTA must be resident at once, which a
+    // cooperative launch guarantees (or refuses)
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+    const int sms = device_sms(err);
+    if (err != cudaSuccess) return err;
+    const int grid = std::min(q1.units + q2.units, sms * per_sm);
+    MapSet a = m1, b = m2;
+    void *args[] = {&a, &b, &q1, &q2};
+    err = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), dim3(grid), dim3(kThreads), args, smem, s);
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 
@@ -733,6 +901,23 @@ cudaError_t launch_decode_gemm_w2(const DecodeGemmParams &p, const CUtensorMap &
         case 1: return launch_nt<1>(p, tm_codes, tm_xa, tm_gs, tm_sc, row_blocks, ksplit, experts, s);
         case 2: return launch_nt<2>(p, tm_codes, tm_xa, tm_gs, tm_sc, row_blocks, ksplit, experts, s);
         case 4: return launch_nt<4>(p, tm_codes, tm_xa, tm_gs, tm_sc, row_blocks, ksplit, experts, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_decode_moe_fused(const DecodeGemmParams &p1, const CUtensorMap &a1, const CUtensorMap &b1,
+                                    const CUtensorMap &c1, const CUtensorMap &d1, int row_blocks1,
+                                    const DecodeGemmParams &p2, const CUtensorMap &a2, const CUtensorMap &b2,
+                                    const CUtensorMap &c2, const CUtensorMap &d2, int row_blocks2, int experts,
+                                    int nt, cudaStream_t s) {
+    if (p1.w4 || p2.w4 || !p1.tma_scales || !p2.tma_scales || p1.mode != EPI_GATEUP || p2.mode != EPI_DOWN ||
+        !p1.dep || !p2.dep || !p1.fuse_gsq)
+        return cudaErrorInvalidValue;
+    const MapSet m1{a1, b1, c1, d1}, m2{a2, b2, c2, d2};
+    switch (nt) {
+        case 1: return launch_fused_nt<1>(p1, m1, row_blocks1, p2, m2, row_blocks2, experts, s);
+        case 2: return launch_fused_nt<2>(p1, m1, row_blocks1, p2, m2, row_blocks2, experts, s);
+        case 4: return launch_fused_nt<4>(p1, m1, row_blocks1, p2, m2, row_blocks2, experts, s);
         default: return cudaErrorInvalidValue;
     }
 }

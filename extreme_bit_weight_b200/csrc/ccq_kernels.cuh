@@ -58,7 +58,23 @@ struct DecodeGemmParams {
     uint32_t *err;
     // work units (set by the launcher): unit u = (expert, k split, row block), row block fastest
     int row_blocks, ksplit, units;
+    // fused MoE launch (gate/up and down in one kernel): the gate/up epilogue also writes the down
+    // operand's gsq table and counts finished units per expert in dep[]; a down unit of expert e
+    // loads only after dep[e] reaches dep_need
+    int *dep;
+    float *fuse_gsq;     // gate/up: gsq table of h (row pitch fuse_gsq_ld entries)
+    int fuse_gsq_ld;
+    float fuse_level;    // level offset of the down weight's format
+    int dep_need;        // down: gate/up units per expert
 };
+
+// Fused MoE decode: gate/up (p1, maps a1..d1) then down (p2, maps a2..d2) in one cooperative
+// persistent launch.  Both must be W2 with TMA-staged scales and the same token tile count nt.
+cudaError_t launch_decode_moe_fused(const DecodeGemmParams &p1, const CUtensorMap &a1, const CUtensorMap &b1,
+                                    const CUtensorMap &c1, const CUtensorMap &d1, int row_blocks1,
+                                    const DecodeGemmParams &p2, const CUtensorMap &a2, const CUtensorMap &b2,
+                                    const CUtensorMap &c2, const CUtensorMap &d2, int row_blocks2, int experts,
+                                    int nt, cudaStream_t s);
 
 cudaError_t launch_decode_gemm_w2(const DecodeGemmParams &p, const CUtensorMap &tm_codes,
                                   const CUtensorMap &tm_xa, const CUtensorMap &tm_gs, const CUtensorMap &tm_sc,
@@ -108,9 +124,9 @@ cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, f
 cudaError_t launch_splitk_reduce(const float *partial, int ksplit, size_t split_stride, int M, int N,
                                  uint16_t *y, cudaStream_t s);
 
-// MoE routing: counts, offsets, placement, inverse map; validates ids.
+// MoE routing: counts, offsets, placement, inverse map; validates ids; zeroes dep[E] (if given).
 cudaError_t launch_moe_route(const int *ids, const float *rw, int T, int topk, int E, int *seg_off,
-                             int *cursor, int *tok_of, float *rw_perm, int *inv, uint32_t *err,
+                             int *cursor, int *tok_of, float *rw_perm, int *inv, int *dep, uint32_t *err,
                              cudaStream_t s);
 cudaError_t launch_moe_combine(const float *slot, const int *inv, int T, int topk, int H, uint16_t *y,
                                cudaStream_t s);

@@ -171,9 +171,11 @@ ccq_status ccq_moe_w2a16_forward(const ccq_weight *w13, const ccq_weight *w2, in
 /* ccq_moe_w2a16_forward_traced - ccq_moe_w2a16_forward that also records CUDA events on `stream`
  * between its steps, for per-kernel timing: events[0] before routing, [1] after routing,
  * [2] after activation packing, [3] after the gate/up kernel, [4] after the group-sum kernel,
- * [5] after the down kernel, [6] after the combine.  `events` (host) holds CCQ_MOE_TRACE_POINTS
- * cudaEvent_t handles created by the caller (NULL: no events).  No paper counterpart: a
- * measurement hook. */
+ * [5] after the down kernel, [6] after the combine.  When the decode-sized path runs both
+ * projections as one fused launch (W2 weights on both, group-scale rows a multiple of 16 bytes),
+ * [3], [4] and [5] are all recorded after that launch.  `events` (host) holds
+ * CCQ_MOE_TRACE_POINTS cudaEvent_t handles created by the caller (NULL: no events).  No paper
+ * counterpart: a measurement hook. */
 enum { CCQ_MOE_TRACE_POINTS = 7 };
 ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight *w2, int32_t num_experts,
                                         const void *x_bf16, int32_t T, const int32_t *expert_ids,
