@@ -82,6 +82,14 @@ def tensor_peak():
     return 1400.0, "fallback (sustained)", 1590.0
 
 
+# DRAM bytes (read + write) per touched expert of the fused decode launch, from the ncu capture of
+# the same kernel on the 16-expert small case (profiles/decode_gemm_w2_moe_decode_T8_E16_full.md:
+# 458.3 MB over 16 experts); each expert's weights cost the same bytes at any expert count, so the
+# full workload's traffic is this times the touched experts.  Retake the capture (and update this
+# figure) whenever the kernel changes.
+FUSED_DECODE_DRAM_BYTES_PER_EXPERT = 458_330_000 / 16
+
+
 def config_dict():
     prefill = WORKLOAD.startswith("moe_ffn_prefill")
     return {
@@ -421,7 +429,9 @@ def run_ours(args, rank, world, local):
         "roofline": roofline_tensor or (
             {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (fused MoE: gate/up + SiLU, then down)",
              "achieved": (b13 + b2) / (gemm1_ms * 1e-3) / 1e9, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)",
-             "unit": "GB/s", "frac": (b13 + b2) / (gemm1_ms * 1e-3) / 1e9 / hbm, "traffic": None,
+             "unit": "GB/s", "frac": (b13 + b2) / (gemm1_ms * 1e-3) / 1e9 / hbm,
+             "traffic": FUSED_DECODE_DRAM_BYTES_PER_EXPERT * ne,
+             "traffic_source": "ncu dram__bytes_read+write of the 16-expert capture, scaled by touched experts",
              "launch_ms": gemm1_ms, "algorithmic_bytes_per_launch": b13 + b2} if fused else
             {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (gate/up, SiLU epilogue)",
              "achieved": ach13, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "unit": "GB/s",
