@@ -42,9 +42,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-small", action="store_true",
                     help="8 tokens over 16 experts (same tokens per expert, 442 MB of weights): for ncu captures")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "gemm", "stack"],
                     help="decode: 32 tokens, uniform routing (the headline line); prefill: 4096 tokens, "
-                         "Zipf(1.1) routing, 1%% of channels x20 (tcgen05 path, tensor roofline)")
+                         "Zipf(1.1) routing, 1%% of channels x20 (tcgen05 path, tensor roofline); gemm: one "
+                         "dense 8192x8192 W2 linear at --m tokens; stack: 8 MoE layers (2 W4 + 6 W2) at --m tokens")
+    ap.add_argument("--m", type=int, default=0, help="tokens for --workload gemm (default 1) / stack (default 32)")
     args = ap.parse_args()
     global T, E, WORKLOAD
     if args.workload == "prefill":
@@ -452,10 +454,182 @@ def run_ours(args, rank, world, local):
         pg.destroy_process_group()
 
 
+# ------------------------------------------------------------------------------------------------
+# side workloads: the dense linear and the mixed W4/W2 layer stack (reported per M, not headline)
+# ------------------------------------------------------------------------------------------------
+def _timed(torch, device, stream, step, K, W):
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(K):
+        step(W + i)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    return a.elapsed_time(b) / K, clocks.stop()
+
+
+def run_gemm(args, rank, world, local):
+    """y = x W^T, K = N = 8192, CCQ W2 g64, at M tokens.  The weight (21.04 MB) is smaller than L2,
+    so the timed calls rotate over enough device copies to exceed twice the L2 size."""
+    import torch
+
+    import extreme_bit_weight_b200 as ccq
+    import synth
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    M, KD, ND = (args.m or 1), 8192, 8192
+    w = synth.weights_normal(ND, KD, 4100)
+    c, sc, al, be, _ = ccq.ccq_encode_host(w, 64, 0, 0)
+    per_copy = c.nbytes + sc.nbytes + al.nbytes + be.nbytes
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    R = max(2, -(-2 * l2 // per_copy))
+    Ws = [ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, ND, KD, c, sc, al, be, device=device) for _ in range(R)]
+    x = synth.activations(M, KD, 4101).to(device)
+    y = torch.empty((M, ND), dtype=torch.bfloat16, device=device)
+    ws = ccq.workspace(max(ccq.ccq_gemm_workspace_size(Ws[0], M), 256), device)
+    stream = torch.cuda.current_stream(device)
+    ms, clk = _timed(torch, device, stream, lambda i: ccq.ccq_w2a16_gemm(Ws[i % R], x, y=y, ws=ws, stream=stream),
+                     args.steps, args.warmup)
+    # end to end: pinned host x in, y out, every call
+    xp = x.cpu().pin_memory()
+    yp = torch.empty((M, ND), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(x)
+
+    def e2e(i):
+        xd.copy_(xp, non_blocking=True)
+        ccq.ccq_w2a16_gemm(Ws[i % R], xd, y=y, ws=ws, stream=stream)
+        yp.copy_(y, non_blocking=True)
+
+    e2e_ms, _ = _timed(torch, device, stream, e2e, max(1, args.steps // 4), 3)
+    hbm, src = peaks()
+    tf, tsrc, tf_burst = tensor_peak()
+    flops = 2.0 * M * ND * KD
+    tensor = M >= 48
+    gbs = per_copy / (ms * 1e-3) / 1e9
+    roof = ({"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": tf, "peak_source": tsrc,
+             "unit": "TFLOP/s", "frac": flops / (ms * 1e-3) / 1e12 / tf} if tensor else
+            {"bound": "hbm", "achieved": gbs, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "unit": "GB/s",
+             "frac": gbs / hbm})
+    roof.update({"kernel": "whole ccq_w2a16_gemm call (" + ("tcgen05 kernel" if tensor else
+                 "activation packing, decode kernel, split-K reduce") + ")", "traffic": None,
+                 "algorithmic_bytes_per_call": per_copy, "algorithmic_flops_per_call": flops})
+    line = {"metric": "W2A16 dense linear tokens/s (K=N=8192)", "value": M / (ms * 1e-3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "us_per_call": 1000.0 * ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"dense_gemm_M{M}_K8192_N8192_ccq_w2_g64", "m": M, "k": KD, "n": ND,
+                       "weights": "N(0,0.02) encoded by ccq_encode_host",
+                       "l2": f"{R} rotating weight copies ({R * per_copy / 1e6:.0f} MB) vs {l2 / 1e6:.0f} MB L2"},
+            "packed_weight_gbs": gbs, "roofline": roof,
+            "e2e": {"value": M / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * 2,
+                    "d2h_bytes_per_step": y.numel() * 2},
+            "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_stack(args, rank, world, local):
+    """Eight MoE layers of the decode layer's shape: layers 0-1 with W4 per-channel experts, 2-7 with
+    CCQ W2 g64; fresh uniform top-8 routing per layer; x_{l+1} = MoE_l(x_l).  A step is the whole
+    stack at M tokens."""
+    import torch
+
+    import extreme_bit_weight_b200 as ccq
+    import synth
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    M = args.m or 32
+    parts = {}
+
+    def w4_layer(seed):
+        def q(rows, cols, sd):
+            c, s = ccq.ccq_quantize_w4_host(synth.weights_normal(rows, cols, sd))
+            return torch.from_numpy(c).to(device), torch.from_numpy(s).to(device)
+
+        if "w4" not in parts:
+            parts["w4"] = ([q(2 * I, H, seed + e) for e in range(DISTINCT)], [q(H, I, seed + 50 + e) for e in range(DISTINCT)])
+        p13, p2 = parts["w4"]
+
+        def stack(pp, n, k):
+            codes = torch.empty((E * n, k // 2), dtype=torch.uint8, device=device)
+            scales = torch.empty((E * n,), dtype=torch.float32, device=device)
+            for e in range(E):
+                codes[e * n:(e + 1) * n].copy_(pp[e % len(pp)][0])
+                scales[e * n:(e + 1) * n].copy_(pp[e % len(pp)][1])
+            return ccq.CcqWeight(ccq.CCQ_FMT_W4_PER_CHANNEL, n, k, codes, scales, experts=E, device=device)
+
+        return stack(p13, 2 * I, H), stack(p2, H, I)
+
+    def clone(w):  # a layer of its own memory with the same contents
+        cp = lambda t: None if t is None else t.clone()
+        return ccq.CcqWeight(w.fmt, w.n, w.k, cp(w.codes), cp(w.scales), cp(w.alpha), cp(w.beta),
+                             experts=w.experts, device=device)
+
+    w2_first = make_layer(ccq, torch, device)
+    layers = ([w4_layer(4200) for _ in range(2)] + [w2_first] +
+              [(clone(w2_first[0]), clone(w2_first[1])) for _ in range(5)])
+    routes = []
+    for l in range(8):
+        ids_np, rw_np = synth.routing_uniform(M, E, TOPK, 4300 + l)
+        routes.append((ids_np, torch.from_numpy(ids_np).to(device), torch.from_numpy(rw_np).to(device)))
+    xs = [synth.activations(M, H, 4400).to(device)] + [torch.empty((M, H), dtype=torch.bfloat16, device=device)
+                                                       for _ in range(8)]
+    ws = ccq.workspace(ccq.ccq_moe_workspace_size(M, TOPK, H, I, E), device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(_):
+        for l, (w13, w2) in enumerate(layers):
+            ccq.ccq_moe_w2a16_forward(w13, w2, xs[l], routes[l][1], routes[l][2], y=xs[l + 1], ws=ws, stream=stream)
+
+    ms, clk = _timed(torch, device, stream, step, args.steps, args.warmup)
+    assert ccq.ccq_check_device_error(ws, stream) == ccq.CCQ_OK
+    # algorithmic bytes and flops of one step (touched experts of every layer)
+    per_w4 = 2 * I * (H // 2) + 2 * I * 4 + H * (I // 2) + H * 4
+    per_w2 = sum(touched_bytes(np.zeros((1, 1), dtype=np.int32))[:2])
+    nbytes = 0
+    for l in range(8):
+        ne = len(set(int(v) for v in routes[l][0].ravel()))
+        nbytes += ne * (per_w4 if l < 2 else per_w2)
+    flops = 8 * 6.0 * M * TOPK * H * I
+    hbm, src = peaks()
+    tf, tsrc, _ = tensor_peak()
+    tensor = M * TOPK / E >= 48
+    roof = ({"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": tf, "peak_source": tsrc,
+             "unit": "TFLOP/s", "frac": flops / (ms * 1e-3) / 1e12 / tf} if tensor else
+            {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)",
+             "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / hbm})
+    roof.update({"kernel": "whole 8-layer stack", "traffic": None, "algorithmic_bytes_per_step": nbytes,
+                 "algorithmic_flops_per_step": flops})
+    line = {"metric": "W2A16/W4A16 8-layer MoE stack tokens/s", "value": M / (ms * 1e-3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"moe_stack_8layers_M{M}_H8192_I3584_E64_top8_w4x2_w2x6", "m": M,
+                       "weights": f"W4: N(0,0.02) quantized by ccq_quantize_w4_host; W2: ccq_encode_host; "
+                                  f"{DISTINCT} distinct experts per layer copied to all {E}",
+                       "l2": f"{nbytes / 1e9:.2f} GB of packed weights touched per step vs 126 MB L2"},
+            "roofline": roof, "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
-    if args.impl == "reference":
+    if args.workload in ("gemm", "stack"):
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the oracle on the "
+                                  "decode MoE layer only"}), flush=True)
+            return
+        (run_gemm if args.workload == "gemm" else run_stack)(args, rank, world, local)
+    elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
         run_ours(args, rank, world, local)
