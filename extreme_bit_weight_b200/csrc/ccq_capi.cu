@@ -121,7 +121,10 @@ bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t
 // Token counts above these run on the tcgen05 kernel (dense GEMM: m; MoE: mean rows per expert).
 constexpr int kTcMinM = 48;
 constexpr double kTcMinRowsPerExpert = 48.0;
-constexpr int kTcMT = 2;  // 128-token sub-tiles per tcgen05 tile
+// 128-token sub-tiles per tcgen05 tile: 1 while experts average at most 96 rows (a half-empty
+// 256-token tile would double the MMA time, which bounds the kernel there, and few experts spill
+// into a second 128-token tile), else 2 (a second tile would decode the weights again)
+int tc_mt(double rows_per_expert) { return rows_per_expert > 96.0 ? 2 : 1; }
 
 struct GemmWs {
     size_t xa, gs, partial, xt, total;
@@ -129,13 +132,38 @@ struct GemmWs {
     bool tc;
 };
 
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            n = 148;
+    }
+    return n;
+}
+
 GemmWs gemm_layout(const ccq_weight *w, int m) {
     GemmWs L{};
     if (m >= kTcMinM) {
         L.tc = true;
         L.P = m;
         L.xt = 0;
-        L.total = up256((size_t)m * w->k * 2);
+        size_t off = up256((size_t)m * w->k * 2);
+        // split-K when the (token tile, row tile) items cannot fill the SMs: ranges of kg groups
+        // (a multiple of 4, one code stage), as many ranges as keep every item on its own SM
+        const int nk = w->k / 64;
+        const int items = ceil_div(m, 128 * tc_mt((double)m)) * ceil_div(w->n, 256);
+        const int sms = sm_count();
+        L.ksplit = 1;
+        L.spp = nk;
+        if (2 * items <= sms && nk >= 8) {
+            const int want = std::max(1, std::min(sms / items, nk / 4));
+            L.spp = ((ceil_div(nk, want) + 3) / 4) * 4;  // groups per split
+            L.ksplit = ceil_div(nk, L.spp);
+        }
+        L.partial = off;
+        if (L.ksplit > 1) off = up256(off + (size_t)L.ksplit * m * w->n * 4);
+        L.total = off;
         return L;
     }
     L.P = (m + 3) & ~3;
@@ -169,7 +197,7 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     const int pairs = T * topk;
     L.P = (pairs + 3) & ~3;
     L.tc = (double)pairs / E >= kTcMinRowsPerExpert;
-    L.max_tiles = L.P / (128 * kTcMT) + E + 1;
+    L.max_tiles = L.P / 128 + E + 1;  // enough for 128-token tiles
     size_t off = 0;
     L.err = off; off = up256(off + 16);
     L.seg = off; off = up256(off + sizeof(int) * (size_t)(E + 1));
@@ -209,16 +237,6 @@ bool tc_maps(CUtensorMap &ta, CUtensorMap &tcodes, const ccq_weight *w, int expe
             return false;
     }
     return true;
-}
-
-int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            n = 148;
-    }
-    return n;
 }
 
 inline ccq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CCQ_OK : CCQ_ERR_CUDA; }
@@ -288,15 +306,28 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
         p.row_block_stride = 256;
         p.half_stride = 128;
         p.n_tiles = ceil_div(w->n, 256);
-        p.m_tile = 128 * kTcMT;
+        const int mt = tc_mt((double)m);
+        p.m_tile = 128 * mt;
         p.static_tiles = ceil_div(m, p.m_tile);
         p.M = m;
-        p.mode = EPI_BF16;
-        p.out = y_bf16;
         p.out_ld = w->n;
         p.w4 = w->fmt == CCQ_FMT_W4_PER_CHANNEL;
-        const int grid = std::min(sm_count(), p.static_tiles * p.n_tiles);
-        return cuda_status(launch_tc_gemm_w2(p, ta, tcodes, kTcMT, grid, s));
+        p.ksplit = L.ksplit;
+        p.kg = L.spp;
+        if (L.ksplit > 1) {
+            p.mode = EPI_PARTIAL_F32;
+            p.out = base + L.partial;
+            p.out_split_stride = (size_t)m * w->n;
+        } else {
+            p.mode = EPI_BF16;
+            p.out = y_bf16;
+        }
+        const int grid = std::min(sm_count(), p.static_tiles * p.n_tiles * L.ksplit);
+        e = launch_tc_gemm_w2(p, ta, tcodes, mt, grid, s);
+        if (e == cudaSuccess && L.ksplit > 1)
+            e = launch_splitk_reduce(reinterpret_cast<const float *>(base + L.partial), L.ksplit, (size_t)m * w->n, m,
+                                     w->n, static_cast<uint16_t *>(y_bf16), s);
+        return cuda_status(e);
     }
     uint16_t *xa = reinterpret_cast<uint16_t *>(base + L.xa);
     float *gs = reinterpret_cast<float *>(base + L.gs);
@@ -398,8 +429,9 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         // prefill-sized: tcgen05 grouped GEMMs over (expert, 256-token tile) entries
         int2 *tiles = reinterpret_cast<int2 *>(base + L.tiles);
         int *tcount = reinterpret_cast<int *>(base + L.tcount);
+        const int mt = tc_mt((double)pairs / num_experts);
         e = launch_pack_xt(static_cast<const uint16_t *>(x_bf16), tok, pairs, H, xa_x, s);
-        if (e == cudaSuccess) e = launch_build_tiles(seg, num_experts, 128 * kTcMT, tiles, tcount, s);
+        if (e == cudaSuccess) e = launch_build_tiles(seg, num_experts, 128 * mt, tiles, tcount, s);
         if (e == cudaSuccess) e = trace(events, 2, s);
         if (e != cudaSuccess) return CCQ_ERR_CUDA;
         CUtensorMap ta1, tc1, ta2, tc2;
@@ -416,7 +448,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q1.n_tiles = ceil_div(I, 128);
         q1.tile_list = tiles;
         q1.tile_count = tcount;
-        q1.m_tile = 128 * kTcMT;
+        q1.m_tile = 128 * mt;
         q1.seg_off = seg;
         q1.mode = EPI_GATEUP;
         q1.out = xa_h;
@@ -424,7 +456,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q1.I = I;
         q1.err = err;
         q1.w4 = w13->fmt == CCQ_FMT_W4_PER_CHANNEL;
-        e = launch_tc_gemm_w2(q1, ta1, tc1, kTcMT, std::min(sm_count(), L.max_tiles * q1.n_tiles), s);
+        e = launch_tc_gemm_w2(q1, ta1, tc1, mt, std::min(sm_count(), L.max_tiles * q1.n_tiles), s);
         if (e == cudaSuccess) e = trace(events, 3, s);
         if (e == cudaSuccess) e = trace(events, 4, s);
         TcGemmParams q2 = q1;
@@ -442,7 +474,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q2.rw = rwp;
         q2.I = 0;
         q2.w4 = w2->fmt == CCQ_FMT_W4_PER_CHANNEL;
-        if (e == cudaSuccess) e = launch_tc_gemm_w2(q2, ta2, tc2, kTcMT, std::min(sm_count(), L.max_tiles * q2.n_tiles), s);
+        if (e == cudaSuccess) e = launch_tc_gemm_w2(q2, ta2, tc2, mt, std::min(sm_count(), L.max_tiles * q2.n_tiles), s);
         if (e == cudaSuccess) e = trace(events, 5, s);
         if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
         if (e == cudaSuccess) e = trace(events, 6, s);

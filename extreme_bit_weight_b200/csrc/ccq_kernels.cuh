@@ -103,6 +103,10 @@ struct TcGemmParams {
     int I;                 // EPI_GATEUP: gate rows per expert
     int w4;                // 1: W4 per-channel codes (two per byte), scales[row]
     uint32_t *err;
+    // split-K (dense matmul with few tiles): ksplit > 1 splits the 64-column groups into ranges of
+    // kg groups (a multiple of 4); each range writes EPI_PARTIAL_F32 sums at out + ks*out_split_stride
+    int ksplit, kg;
+    size_t out_split_stride;
 };
 
 cudaError_t launch_tc_gemm_w2(const TcGemmParams &p, const CUtensorMap &tm_a, const CUtensorMap &tm_codes, int mt,

@@ -9,11 +9,12 @@
 //               ([128 rows][64 B], 64B swizzle, 4 groups per load)
 //   warp 1      TMEM allocation and the single MMA-issuing thread (tcgen05.mma kind::f16,
 //               M=128, N=256, K=16, fp32 accumulators in TMEM)
-//   warps 2-9   decoders: each thread owns one weight row of the tile, decodes its 16 code bytes of
-//               the group (CCQ §3.3 Eq. 1 inverted / §3.5 Algorithm 3: fp32 FMA, ties-to-even
-//               rounding, Table 1 shifts) to BF16 w = bf16((u - 32) * bf16(scale)) and stores them
-//               as the MMA B operand in the canonical K-major 128B-swizzled shared-memory layout
-//   warps 10-13 epilogue: tcgen05.ld of the accumulators; SiLU(gate)*up, routing-weight scaling or
+//   warps 2-17  decoders: two threads per weight row of the tile; each decodes its half of the
+//               row's code bytes of the group (CCQ §3.3 Eq. 1 inverted / §3.5 Algorithm 3: fp32
+//               FMA, ties-to-even rounding, Table 1 shifts) to BF16 w = bf16((u - 32) * bf16(scale))
+//               and stores them as the MMA B operand in the canonical K-major 128B-swizzled
+//               shared-memory layout
+//   warps 18-21 epilogue: tcgen05.ld of the accumulators; SiLU(gate)*up, routing-weight scaling or
 //               BF16 conversion; stores to global memory
 // Column order: within every 16-column block the decoders emit the 16 weights of one 4-byte word
 // window-major (position 4i + j holds state window i of byte j, i.e. column 4j + i), so the
@@ -30,11 +31,14 @@
 namespace ccq {
 namespace {
 
-constexpr int kDecWarps = 8;
+constexpr int kDecWarps = 16;  // two threads per weight row of the 256-row tile
 constexpr int kEpiWarps = 4;
-constexpr int kTcThreads = (2 + kDecWarps + kEpiWarps) * 32;  // 448
+constexpr int kTcThreads = (2 + kDecWarps + kEpiWarps) * 32;  // 704
 constexpr int kSA = 3;   // activation stages
-constexpr int kSB = 2;   // decoded-weight stages
+// decoded-weight stages: 3 with 128-token tiles (the MMA of a stage is short, so the decoders need
+// more room ahead), 2 with 256-token tiles (shared memory)
+template <int MT>
+constexpr int kSBof = MT == 1 ? 3 : 2;
 constexpr int kSC = 2;   // code stages (4 groups each)
 constexpr int kATile = 128 * 64 * 2;   // 16 KB per 128-token sub-tile
 constexpr int kBTile = 256 * 64 * 2;   // 32 KB
@@ -43,7 +47,7 @@ constexpr int kCTile = 2 * 128 * 64;   // 16 KB: two 128-row halves x 64 code by
 template <int MT>
 struct TcSmem {
     static constexpr int kA = kSA * MT * kATile;
-    static constexpr int kB = kSB * kBTile;
+    static constexpr int kB = kSBof<MT> * kBTile;
     static constexpr int kC = kSC * kCTile;
     static constexpr int kTotal = kA + kB + kC + 1024;
     static_assert(kTotal + 512 <= 227 * 1024, "shared memory per CTA");
@@ -88,6 +92,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -106,21 +117,48 @@ __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
     return d;
 }
 
+__device__ __forceinline__ uint64_t pk2(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, uint32_t &lo, uint32_t &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fpk2(float lo, float hi) { return pk2(__float_as_uint(lo), __float_as_uint(hi)); }
+
+// Per-row and per-thread constants of the W2 decode, held in registers.
+struct RowCodeParams {
+    uint64_t ab, bb;         // {alpha, alpha}, {beta, beta}
+    uint64_t neg, rnd;       // {-2^23, -2^23}; {1.5*2^23, 1.5*2^23 - 0x4B40} (second byte pre-cancels)
+};
+
 // One 4-byte word of a row -> 16 BF16 weights (u - 32) * s in window-major order, as 8 registers:
-// out[2i], out[2i+1] = window i of bytes (0,1) and (2,3).
-__device__ __forceinline__ void decode_word_bf16(uint32_t w, float alpha, float beta, uint32_t s2, uint32_t out[8]) {
+// out[2i], out[2i+1] = window i of bytes (0,1) and (2,3).  Byte value, q*alpha + beta (one fp32
+// rounding) and the half-to-even rounding to an integer run two bytes per f32x2 instruction.
+__device__ __forceinline__ void decode_word_bf16(uint32_t w, const RowCodeParams &rp, uint32_t s2, uint32_t out[8]) {
     const uint32_t magic = 0x4B000000u;
-    float c[4];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) c[b] = __uint_as_float(prmt(w, magic, 0x7650u + b)) - 8388608.0f;
-    uint32_t r[4];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        const float t = __fmaf_rn(c[b], alpha, beta);
-        r[b] = __float_as_uint(__fadd_rn(t, (b & 1) ? 12563648.0f : 12582912.0f));
-    }
-    const uint32_t X01 = r[1] * 65536u + r[0];
-    const uint32_t X23 = r[3] * 65536u + r[2];
+    uint64_t c01 = pk2(prmt(w, magic, 0x7650u), prmt(w, magic, 0x7651u));
+    uint64_t c23 = pk2(prmt(w, magic, 0x7652u), prmt(w, magic, 0x7653u));
+    c01 = fadd2(c01, rp.neg);
+    c23 = fadd2(c23, rp.neg);
+    c01 = fadd2(ffma2(c01, rp.ab, rp.bb), rp.rnd);
+    c23 = fadd2(ffma2(c23, rp.ab, rp.bb), rp.rnd);
+    uint32_t r0, r1, r2, r3;
+    upk2(c01, r0, r1);
+    upk2(c23, r2, r3);
+    const uint32_t X01 = r1 * 65536u + r0;
+    const uint32_t X23 = r3 * 65536u + r2;
     const uint32_t M = 0x003F003Fu, E = 0x43004300u, Z = 0x43204320u;  // Z = bf16x2(160, 160)
     out[0] = bmul2(bsub2(((X01 >> 9) & M) | E, Z), s2);
     out[1] = bmul2(bsub2(((X23 >> 9) & M) | E, Z), s2);
@@ -149,11 +187,33 @@ __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z));
 // position p of a 16-column block holds column 4*(p%4) + p/4 (and the map is its own inverse)
 __device__ __forceinline__ int perm16(int p) { return ((p & 3) << 2) | (p >> 2); }
 
-struct TileInfo {
-    int e, m0, seg0, Me, nt;
+// Position in a ring of N shared-memory stages: slot and the parity of the current round (no
+// division by N in the loops).
+template <int N>
+struct Ring {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void advance() {
+        if (++slot == N) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
 };
 
+struct TileInfo {
+    int e, m0, seg0, Me, nt;
+    int ks, g0, g1;  // k split and its 64-column groups [g0, g1)
+};
+
+// work item w = ((token tile * n_tiles + row tile) * ksplit + k split)
 __device__ __forceinline__ bool tile_of(const TcGemmParams &p, int w, TileInfo &t) {
+    const int ksn = p.ksplit > 1 ? p.ksplit : 1;
+    const int nk = p.K / 64;
+    t.ks = w % ksn;
+    w /= ksn;
+    t.g0 = ksn > 1 ? t.ks * p.kg : 0;
+    t.g1 = ksn > 1 ? min(nk, t.g0 + p.kg) : nk;
     const int li = w / p.n_tiles;
     t.nt = w - li * p.n_tiles;
     const int2 ent = p.tile_list ? p.tile_list[li] : make_int2(0, li);
@@ -169,6 +229,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_codes,
                   const TcGemmParams p) {
     using S = TcSmem<MT>;
+    constexpr int kSB = kSBof<MT>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned start, kept as an offset from the shared array so that loads and stores
     // through it stay shared-memory instructions
@@ -181,7 +242,7 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     __shared__ uint32_t tmem_base_slot;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int total_work = (p.tile_count ? *p.tile_count : p.static_tiles) * p.n_tiles;
+    const int total_work = (p.tile_count ? *p.tile_count : p.static_tiles) * p.n_tiles * (p.ksplit > 1 ? p.ksplit : 1);
     const int nk = p.K / 64;
     // one code stage holds 64 bytes of every row: 4 groups of W2 codes or 2 groups of W4 codes
     constexpr int kKsPerCode = W4 ? 2 : 4;
@@ -210,30 +271,34 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             prefetch_tensormap(&tm_a);
             prefetch_tensormap(&tm_codes);
             uint32_t ai = 0, ci = 0;
+            Ring<kSA> ra;
+            Ring<kSC> rc;
             bool ok = true;
             for (int w = blockIdx.x; w < total_work && ok; w += gridDim.x) {
                 TileInfo t;
                 tile_of(p, w, t);
                 const int localA = t.nt * p.row_block_stride;
                 const int rowA = t.e * p.N + localA, rowB = rowA + p.half_stride;
-                for (int ks = 0; ks < nk && ok; ++ks) {
+                for (int ks = t.g0; ks < t.g1 && ok; ++ks) {
                     if (ks % kKsPerCode == 0) {
-                        const int s = ci % kSC;
-                        if (ci >= kSC) ok = mbar_wait(&c_empty[s], ((ci / kSC) - 1) & 1, p.err);
+                        const int s = rc.slot;
+                        if (ci >= kSC) ok = mbar_wait(&c_empty[s], rc.phase ^ 1u, p.err);
                         if (!ok) break;
                         mbar_arrive_expect_tx(&c_full[s], kCTile);
                         tma_load_2d(sC + s * kCTile, &tm_codes, &c_full[s], (ks / kKsPerCode) * 64, rowA);
                         tma_load_2d(sC + s * kCTile + kCTile / 2, &tm_codes, &c_full[s], (ks / kKsPerCode) * 64, rowB);
                         ++ci;
+                        rc.advance();
                     }
-                    const int s = ai % kSA;
-                    if (ai >= kSA) ok = mbar_wait(&a_empty[s], ((ai / kSA) - 1) & 1, p.err);
+                    const int s = ra.slot;
+                    if (ai >= kSA) ok = mbar_wait(&a_empty[s], ra.phase ^ 1u, p.err);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&a_full[s], MT * kATile);
 #pragma unroll
                     for (int j = 0; j < MT; ++j)
                         tma_load_2d(sA + (s * MT + j) * kATile, &tm_a, &a_full[s], ks * 64, t.seg0 + t.m0 + j * 128);
                     ++ai;
+                    ra.advance();
                 }
             }
             // drain: the last copies must land before exit
@@ -245,15 +310,19 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     } else if (warp == 1) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
-            uint32_t ai = 0, bi = 0, ti = 0;
+            uint32_t ti = 0;
+            Ring<kSA> ra;
+            Ring<kSB> rb;
             bool ok = true;
             for (int w = blockIdx.x; w < total_work && ok; w += gridDim.x, ++ti) {
+                TileInfo t;
+                tile_of(p, w, t);
                 if (ti > 0) ok = mbar_wait(&acc_empty, (ti - 1) & 1, p.err);
                 if (!ok) break;
                 tc_fence_after();
-                for (int ks = 0; ks < nk && ok; ++ks) {
-                    const int sa = ai % kSA, sb = bi % kSB;
-                    ok = mbar_wait(&a_full[sa], (ai / kSA) & 1, p.err) && mbar_wait(&b_full[sb], (bi / kSB) & 1, p.err);
+                for (int ks = t.g0; ks < t.g1 && ok; ++ks) {
+                    const int sa = ra.slot, sb = rb.slot;
+                    ok = mbar_wait(&a_full[sa], ra.phase, p.err) && mbar_wait(&b_full[sb], rb.phase, p.err);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
@@ -263,12 +332,12 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             mma_bf16_ss(tmem + j * 256, smem_desc_sw128(abase + kk * 32), smem_desc_sw128(bbase + kk * 32),
-                                        (ks > 0 || kk > 0) ? 1u : 0u);
+                                        (ks > t.g0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(&a_empty[sa]);
                     mma_commit(&b_empty[sb]);
-                    ++ai;
-                    ++bi;
+                    ra.advance();
+                    rb.advance();
                 }
                 if (ok) mma_commit(&acc_full);
             }
@@ -278,10 +347,18 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         }
     } else if (warp < 2 + kDecWarps) {
         // ------------------------------ decoders ------------------------------
-        const int r = threadIdx.x - 64;  // weight row within the tile, 0..255
+        // two threads per weight row: thread part pt decodes words 2pt, 2pt+1 (W2: bytes 8pt..8pt+7 of
+        // the row's 16 bytes of the group; W4: the second 16-byte chunk of the row's 32 bytes)
+        const int d = threadIdx.x - 64;
+        const int r = d >> 1, pt = d & 1;  // weight row within the tile, 0..255; part
         const int half = r >> 7, rr = r & 127;
-        uint32_t bi = 0, ci = 0;
+        uint32_t bi = 0;
+        Ring<kSB> rb;
+        Ring<kSC> rc;
         bool ok = true;
+        RowCodeParams rp;
+        rp.neg = fpk2(-8388608.0f, -8388608.0f);
+        rp.rnd = fpk2(12582912.0f, 12582912.0f - 19264.0f);
         for (int w = blockIdx.x; w < total_work && ok; w += gridDim.x) {
             TileInfo t;
             tile_of(p, w, t);
@@ -289,6 +366,8 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             const bool valid = local < p.N;
             const size_t grow = (size_t)t.e * p.N + (valid ? local : 0);
             const float alpha = W4 ? 0.0f : __ldg(p.alpha + grow), beta = W4 ? 0.0f : __ldg(p.beta + grow);
+            rp.ab = fpk2(alpha, alpha);
+            rp.bb = fpk2(beta, beta);
             const float *srow = p.scales + grow * (W4 ? 1 : nk);
             const float sc_row = W4 ? bf16_bits_to_float(float_to_bf16_bits(__ldg(srow))) : 0.0f;
             // W2 group scales, four groups (one code stage) at a time and one stage ahead, so the
@@ -299,50 +378,48 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 return make_float4(__ldg(srow + g0), g0 + 1 < nk ? __ldg(srow + g0 + 1) : 0.f,
                                    g0 + 2 < nk ? __ldg(srow + g0 + 2) : 0.f, g0 + 3 < nk ? __ldg(srow + g0 + 3) : 0.f);
             };
-            float4 sc_cur = make_float4(0.f, 0.f, 0.f, 0.f), sc_next = load_sc4(0);
-            for (int ks = 0; ks < nk && ok; ++ks) {
+            float4 sc_cur = make_float4(0.f, 0.f, 0.f, 0.f), sc_next = load_sc4(t.g0);
+            for (int ks = t.g0; ks < t.g1 && ok; ++ks) {
                 if (!W4 && (ks & 3) == 0) {
                     sc_cur = sc_next;
                     sc_next = load_sc4(ks + 4);
                 }
-                const int cs = ci % kSC;
+                const int cs = rc.slot;
                 if (ks % kKsPerCode == 0) {
-                    ok = mbar_wait(&c_full[cs], (ci / kSC) & 1, p.err);
+                    ok = mbar_wait(&c_full[cs], rc.phase, p.err);
                     if (!ok) break;
                 }
-                // this row's code bytes of group ks (64-byte rows, 64B swizzle): 16 (W2) or 32 (W4)
+                // this thread's code bytes of group ks (64-byte rows, 64B swizzle)
                 const uint8_t *crow = sC + cs * kCTile + half * (kCTile / 2) + rr * 64;
                 const uint32_t swz = ((uint32_t)rr >> 1) & 3u;
-                uint4 q, q2 = make_uint4(0, 0, 0, 0);
+                uint2 q2w = make_uint2(0, 0);
+                uint4 q4w = make_uint4(0, 0, 0, 0);
                 if (!W4) {
-                    q = *reinterpret_cast<const uint4 *>(crow + ((((uint32_t)(ks & 3)) ^ swz) << 4));
+                    q2w = *reinterpret_cast<const uint2 *>(crow + ((((uint32_t)(ks & 3)) ^ swz) << 4) + 8 * pt);
                 } else {
-                    const uint32_t c0 = 2u * (uint32_t)(ks & 1);
-                    q = *reinterpret_cast<const uint4 *>(crow + ((c0 ^ swz) << 4));
-                    q2 = *reinterpret_cast<const uint4 *>(crow + (((c0 + 1u) ^ swz) << 4));
+                    const uint32_t c0 = 2u * (uint32_t)(ks & 1) + (uint32_t)pt;
+                    q4w = *reinterpret_cast<const uint4 *>(crow + ((c0 ^ swz) << 4));
                 }
-                if (ks % kKsPerCode == kKsPerCode - 1 || ks == nk - 1) {
+                if (ks % kKsPerCode == kKsPerCode - 1 || ks == t.g1 - 1) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&c_empty[cs]);
-                    ++ci;
+                    rc.advance();
                 }
-                uint32_t o[4][8];
+                uint32_t o[2][8];
                 if (!W4) {
                     const int gi = ks & 3;
                     const float sraw = gi == 0 ? sc_cur.x : gi == 1 ? sc_cur.y : gi == 2 ? sc_cur.z : sc_cur.w;
                     const float sc = bf16_bits_to_float(float_to_bf16_bits(sraw));
                     const uint32_t s2 = pack_bf16x2(sc, sc);
-                    decode_word_bf16(q.x, alpha, beta, s2, o[0]);
-                    decode_word_bf16(q.y, alpha, beta, s2, o[1]);
-                    decode_word_bf16(q.z, alpha, beta, s2, o[2]);
-                    decode_word_bf16(q.w, alpha, beta, s2, o[3]);
+                    decode_word_bf16(q2w.x, rp, s2, o[0]);
+                    decode_word_bf16(q2w.y, rp, s2, o[1]);
                 } else {
                     // block b of 16 columns = words 2b, 2b+1; emit the same window-major order as W2:
                     // positions (4i, 4i+1) <- codes (i, i+4) of word 2b, (4i+2, 4i+3) <- of word 2b+1
                     const uint32_t s2 = pack_bf16x2(sc_row, sc_row);
-                    const uint32_t wds[8] = {q.x, q.y, q.z, q.w, q2.x, q2.y, q2.z, q2.w};
+                    const uint32_t wds[4] = {q4w.x, q4w.y, q4w.z, q4w.w};
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) {
+                    for (int b = 0; b < 2; ++b) {
                         uint32_t r0[4], r1[4];
                         decode_word_w4_bf16(wds[2 * b], s2, r0);
                         decode_word_w4_bf16(wds[2 * b + 1], s2, r1);
@@ -350,21 +427,23 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                         o[b][4] = r0[2]; o[b][5] = r1[2]; o[b][6] = r0[3]; o[b][7] = r1[3];
                     }
                 }
-                const int sb = bi % kSB;
-                if (bi >= kSB) ok = mbar_wait(&b_empty[sb], ((bi / kSB) - 1) & 1, p.err);
+                const int sb = rb.slot;
+                if (bi >= kSB) ok = mbar_wait(&b_empty[sb], rb.phase ^ 1u, p.err);
                 if (!ok) break;
                 uint8_t *brow = sB + sb * kBTile + r * 128;
 #pragma unroll
-                for (int wd = 0; wd < 4; ++wd) {
+                for (int j = 0; j < 2; ++j) {
+                    const int wd = 2 * pt + j;  // 16-column block of the group
                     const uint32_t c0 = (uint32_t)(2 * wd) ^ ((uint32_t)r & 7u);
                     const uint32_t c1 = (uint32_t)(2 * wd + 1) ^ ((uint32_t)r & 7u);
-                    *reinterpret_cast<uint4 *>(brow + (c0 << 4)) = make_uint4(o[wd][0], o[wd][1], o[wd][2], o[wd][3]);
-                    *reinterpret_cast<uint4 *>(brow + (c1 << 4)) = make_uint4(o[wd][4], o[wd][5], o[wd][6], o[wd][7]);
+                    *reinterpret_cast<uint4 *>(brow + (c0 << 4)) = make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]);
+                    *reinterpret_cast<uint4 *>(brow + (c1 << 4)) = make_uint4(o[j][4], o[j][5], o[j][6], o[j][7]);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&b_full[sb]);
                 ++bi;
+                rb.advance();
             }
         }
     } else {
@@ -388,30 +467,30 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(j * 256);
                 if (p.mode == EPI_GATEUP) {
 #pragma unroll 1
-                    for (int c = 0; c < 128; c += 32) {
-                        uint32_t g[32], u[32];
-                        tmem_ld32(tbase + c, g);
-                        tmem_ld32(tbase + 128 + c, u);
+                    for (int c = 0; c < 128; c += 16) {  // one 16-column block at a time
+                        uint32_t g[16], u[16];
+                        tmem_ld16(tbase + c, g);
+                        tmem_ld16(tbase + 128 + c, u);
                         tmem_ld_wait();
                         if (!live || localA + c >= p.I) continue;
-                        uint32_t h[16];
+                        uint32_t h[8];
 #pragma unroll
-                        for (int b = 0; b < 2; ++b)
-#pragma unroll
-                            for (int pp = 0; pp < 16; pp += 2) {
-                                const int c0 = 16 * b + perm16(pp), c1 = 16 * b + perm16(pp + 1);
-                                const float h0 = silu(__uint_as_float(g[c0])) * __uint_as_float(u[c0]);
-                                const float h1 = silu(__uint_as_float(g[c1])) * __uint_as_float(u[c1]);
-                                h[8 * b + pp / 2] = pack_bf16x2(h0, h1);
-                            }
+                        for (int pp = 0; pp < 16; pp += 2) {
+                            const int c0 = perm16(pp), c1 = perm16(pp + 1);
+                            const float h0 = silu(__uint_as_float(g[c0])) * __uint_as_float(u[c0]);
+                            const float h1 = silu(__uint_as_float(g[c1])) * __uint_as_float(u[c1]);
+                            h[pp / 2] = pack_bf16x2(h0, h1);
+                        }
                         uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + prow * p.out_ld + localA + c);
                         dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
                         dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
-                        dst[2] = make_uint4(h[8], h[9], h[10], h[11]);
-                        dst[3] = make_uint4(h[12], h[13], h[14], h[15]);
                     }
                 } else {
                     const float rwv = (p.mode == EPI_DOWN && live) ? __ldg(p.rw + prow) : 1.0f;
+                    // fp32 outputs: routing-weighted slots, or this k split's partial sums
+                    const bool f32 = p.mode == EPI_DOWN || p.mode == EPI_PARTIAL_F32;
+                    float *fout = static_cast<float *>(p.out) +
+                                  (p.mode == EPI_PARTIAL_F32 ? (size_t)t.ks * p.out_split_stride : 0);
 #pragma unroll 1
                     for (int c = 0; c < 256; c += 32) {
                         uint32_t v[32];
@@ -419,13 +498,13 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                         tmem_ld_wait();
                         const int lr = localA + (c >= 128 ? p.half_stride - 128 : 0) + c;  // local row of column c
                         if (!live || lr >= p.N) continue;
-                        if (p.mode == EPI_DOWN && lr + 32 > p.N) {  // partial chunk of rows
-                            float *dst = static_cast<float *>(p.out) + prow * p.out_ld + lr;
+                        if (f32 && lr + 32 > p.N) {  // partial chunk of rows
+                            float *dst = fout + prow * p.out_ld + lr;
 #pragma unroll
                             for (int z = 0; z < 32; ++z)
                                 if (lr + z < p.N) dst[z] = rwv * __uint_as_float(v[z]);
-                        } else if (p.mode == EPI_DOWN) {
-                            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + prow * p.out_ld + lr);
+                        } else if (f32) {
+                            float4 *dst = reinterpret_cast<float4 *>(fout + prow * p.out_ld + lr);
 #pragma unroll
                             for (int z = 0; z < 8; ++z)
                                 dst[z] = make_float4(rwv * __uint_as_float(v[4 * z]), rwv * __uint_as_float(v[4 * z + 1]),
