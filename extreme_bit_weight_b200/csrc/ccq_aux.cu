@@ -84,40 +84,45 @@ __device__ __forceinline__ void store_gsq(float *gsq, int pr, int G, int ld, int
     }
 }
 
+// Four threads per (operand row p, group G): thread tig handles columns 16*tig .. 16*tig+15 of the
+// group (one 16-column block of the XA order) and the four lanes sum the group in a fixed order.
 __global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__restrict__ tok_of, int P_valid,
                                int P, int K, float level, uint16_t *__restrict__ xa, float *__restrict__ gsq) {
     const int ng = K / 64, ld = gsum_ld(K);
-    const size_t total = (size_t)P_valid * ng;
-    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+    const size_t total = (size_t)P_valid * ng * 4;  // a multiple of 4: the lanes of one group stay together
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < ((total + 31) & ~size_t(31));
          idx += (size_t)gridDim.x * blockDim.x) {
-        const int pr = (int)(idx / ng), G = (int)(idx % ng);
+        const bool live = idx < total;
+        const size_t q = live ? idx : 0;
+        const int tig = (int)(q & 3);
+        const int pr = (int)((q >> 2) / ng), G = (int)((q >> 2) % ng);
         const int src = tok_of ? __ldg(tok_of + pr) : pr;
-        const uint4 *row = reinterpret_cast<const uint4 *>(x + (size_t)src * K + (size_t)G * 64);
-        uint16_t v[64];
+        const uint4 *blk = reinterpret_cast<const uint4 *>(x + (size_t)src * K + (size_t)G * 64 + 16 * tig);
+        const uint4 w0 = __ldg(blk), w1 = __ldg(blk + 1);
+        const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint16_t v[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            uint4 w = __ldg(row + q);
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                v[q * 8 + 2 * h] = (uint16_t)(ws[h] & 0xFFFFu);
-                v[q * 8 + 2 * h + 1] = (uint16_t)(ws[h] >> 16);
-            }
+        for (int h = 0; h < 8; ++h) {
+            v[2 * h] = (uint16_t)(ws[h] & 0xFFFFu);
+            v[2 * h + 1] = (uint16_t)(ws[h] >> 16);
         }
         float sum = 0.0f;
 #pragma unroll
-        for (int k = 0; k < 64; ++k) sum += bf16_bits_to_float(v[k]);
-        store_gsq(gsq, pr, G, ld, P_valid, level * sum);
-        // 16 runs of 4 values: (i, tig) -> j = 0..3 contiguous
+        for (int k = 0; k < 16; ++k) sum += bf16_bits_to_float(v[k]);
+        // group sum over the four 16-column blocks, in block order
+        const float s1 = __shfl_down_sync(0xFFFFFFFFu, sum, 1, 4);
+        const float s2 = __shfl_down_sync(0xFFFFFFFFu, sum, 2, 4);
+        const float s3 = __shfl_down_sync(0xFFFFFFFFu, sum, 3, 4);
+        if (!live) continue;
+        if (tig == 0) store_gsq(gsq, pr, G, ld, P_valid, level * (((sum + s1) + s2) + s3));
+        // this block's 4 runs of 4 values: (i) -> j = 0..3 contiguous
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int tig = 0; tig < 4; ++tig) {
-                uint2 o;
-                o.x = (uint32_t)v[16 * tig + 0 + i] | ((uint32_t)v[16 * tig + 4 + i] << 16);
-                o.y = (uint32_t)v[16 * tig + 8 + i] | ((uint32_t)v[16 * tig + 12 + i] << 16);
-                *reinterpret_cast<uint2 *>(xa + xa_index((size_t)pr, (size_t)G * 64 + 16 * tig + i, (size_t)P)) = o;
-            }
+        for (int i = 0; i < 4; ++i) {
+            uint2 o;
+            o.x = (uint32_t)v[0 + i] | ((uint32_t)v[4 + i] << 16);
+            o.y = (uint32_t)v[8 + i] | ((uint32_t)v[12 + i] << 16);
+            *reinterpret_cast<uint2 *>(xa + xa_index((size_t)pr, (size_t)G * 64 + 16 * tig + i, (size_t)P)) = o;
+        }
     }
 }
 
@@ -253,7 +258,7 @@ cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, c
 cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,
                            uint16_t *xa, float *gsq, cudaStream_t s) {
     if (P_valid <= 0) return cudaSuccess;
-    pack_xa_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(x, tok_of, P_valid, P, K, level, xa, gsq);
+    pack_xa_kernel<<<grid_for((size_t)P_valid * (K / 64) * 4, 128), 128, 0, s>>>(x, tok_of, P_valid, P, K, level, xa, gsq);
     return cudaGetLastError();
 }
 
