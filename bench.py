@@ -64,6 +64,27 @@ def dist_env():
     return rank, world, local
 
 
+def replica_seed(base: int, rank: int) -> int:
+    """Seed of a rank's replica inputs (every rank times its own copy of the layer)."""
+    return base + 17 * rank
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's time: the job's time for replicas that run concurrently."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's step time."""
+    return world * tokens / (ms_per_step * 1e-3)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -316,11 +337,11 @@ def run_ours(args, rank, world, local):
 
     W13, W2 = make_layer(ccq, torch, device)
     prefill = args.workload == "prefill"
-    x_host = synth.activations(T, H, 3002 + 17 * rank, outlier_frac=0.01 if prefill else 0.0)
+    x_host = synth.activations(T, H, replica_seed(3002, rank), outlier_frac=0.01 if prefill else 0.0)
     if prefill:
-        ids_np, rw_np = synth.routing_zipf(T, E, TOPK, 3003 + 17 * rank, s=1.1)
+        ids_np, rw_np = synth.routing_zipf(T, E, TOPK, replica_seed(3003, rank), s=1.1)
     else:
-        ids_np, rw_np = synth.routing_uniform(T, E, TOPK, 3003 + 17 * rank)
+        ids_np, rw_np = synth.routing_uniform(T, E, TOPK, replica_seed(3003, rank))
     x = x_host.to(device)
     ids = torch.from_numpy(ids_np).to(device)
     rw = torch.from_numpy(rw_np).to(device)
@@ -363,12 +384,9 @@ def run_ours(args, rank, world, local):
     # the decode path may run both projections as one launch: then events 3, 4, 5 are recorded
     # back to back and the "down" interval is only event overhead
     fused = (not prefill) and gemm2_ms < 0.02 * gemm1_ms
-    if pg:
-        t = torch.tensor([total_ms], device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, pg, device)
     ms_per_step = total_ms / K
-    value = world * T / (ms_per_step * 1e-3)
+    value = job_tokens_per_s(world, T, ms_per_step)
 
     # ---- end to end: pinned host inputs in, result out, through the same public call ----
     xp = x_host.pin_memory()
@@ -396,10 +414,7 @@ def run_ours(args, rank, world, local):
     b.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = a.elapsed_time(b) / K2
-    if pg:
-        t = torch.tensor([e2e_ms], device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, pg, device)
     h2d = xp.numel() * 2 + idp.numel() * 4 + rwp.numel() * 4
     d2h = yp.numel() * 2
 
