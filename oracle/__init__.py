@@ -57,6 +57,8 @@ def lib():
         L.oracle_cluster_code.restype = ctypes.c_int32
         L.oracle_dequant_w2.argtypes = [P, P, P, P, i, i, i, P]
         L.oracle_dequant_w4.argtypes = [P, P, i, i, P]
+        L.oracle_dequant_w2q4.argtypes = [P, P, P, P, P, i, i, i, P]
+        L.oracle_encode_w2q4.argtypes = [P, i, i, i, ctypes.c_uint32, P, P, P, P, P]
         L.oracle_gemm_bf16_f64.argtypes = [P, P, i, i, i, P]
         L.oracle_gemm_bf16_f64.restype = None
         L.oracle_expert_ffn_f64.argtypes = [P, i, i, i, P, P, i, P]
@@ -128,6 +130,25 @@ def dequant_w2(codes, scales, alpha, beta, group: int = 64) -> np.ndarray:
     rc = lib().oracle_dequant_w2(_p(codes), _p(scales), _p(alpha), _p(beta), n, k, group, _p(out))
     if rc != 0:
         raise ValueError("dequant_w2: bad shape")
+    return out
+
+
+def dequant_w2q4(codes, scale_q4, super_scale, alpha, beta, group: int = 64) -> np.ndarray:
+    """W2 CCQ decode with 4-bit group scales ([CCQ] §3.4 Scale Compression, Algorithm 3):
+    s = q4 * super_scale, two q4 per byte (even group in the low nibble) -> BF16 bits [n][k]."""
+    codes = _c(codes, np.uint8)
+    n, kb = codes.shape
+    k = kb * 4
+    nb = (k // group + 1) // 2
+    scale_q4 = _c(scale_q4, np.uint8).reshape(n, nb)
+    super_scale = _c(super_scale, np.float32).reshape(n)
+    alpha = _c(alpha, np.float32).reshape(n)
+    beta = _c(beta, np.float32).reshape(n)
+    out = np.zeros((n, k), dtype=np.uint16)
+    rc = lib().oracle_dequant_w2q4(_p(codes), _p(scale_q4), _p(super_scale), _p(alpha), _p(beta), n, k, group,
+                                   _p(out))
+    if rc != 0:
+        raise ValueError("dequant_w2q4: bad shape")
     return out
 
 
@@ -210,6 +231,29 @@ def encode_w2(w, group: int = 64, flags: int = 0):
     if rc != 0:
         raise ValueError("encode_w2: bad shape")
     return codes, scales, alpha, beta
+
+
+def encode_w2q4(w, group: int = 64, flags: int = 0):
+    """CCQ encode for the 4-bit scale format -> (codes, scale_q4 [n][ceil(k/g/2)] u8, super [n], alpha, beta)."""
+    w = _c(w, np.float32)
+    n, k = w.shape
+    nb = (k // group + 1) // 2
+    codes = np.zeros((n, k // 4), dtype=np.uint8)
+    sq = np.zeros((n, nb), dtype=np.uint8)
+    sup = np.zeros(n, dtype=np.float32)
+    alpha = np.zeros(n, dtype=np.float32)
+    beta = np.zeros(n, dtype=np.float32)
+    rc = lib().oracle_encode_w2q4(_p(w), n, k, group, flags, _p(codes), _p(sq), _p(sup), _p(alpha), _p(beta))
+    if rc != 0:
+        raise ValueError("encode_w2q4: bad shape or flags")
+    return codes, sq, sup, alpha, beta
+
+
+def q4_unpack(scale_q4, ng: int) -> np.ndarray:
+    """The 4-bit group scales as integers [n][ng] (even group in the low nibble)."""
+    b = np.asarray(scale_q4, dtype=np.uint8)
+    lo, hi = b & 0xF, b >> 4
+    return np.stack([lo, hi], axis=-1).reshape(b.shape[0], -1)[:, :ng]
 
 
 def w2_sq_error(w, codes, scales, alpha, beta, group: int = 64) -> float:

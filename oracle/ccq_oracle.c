@@ -164,6 +164,41 @@ int oracle_dequant_w2(const uint8_t *codes, const float *scales, const float *co
 }
 
 /* ------------------------------------------------------------------------------------------
+ * 4-bit group scales, [CCQ] §3.4 "Scale Compression" and §3.5 Algorithm 3 (first line):
+ * s = ((s_q >> s_shift) & s_mask) * s_super, s_mask = 0xF for (6,4,3) (Table 1), one fp32 super
+ * scale per output channel.  Storage (the pages fix only the formula; reading): two 4-bit group
+ * scales per byte, scale_q4[n][ceil(k/g / 2)], group G in byte G/2, the low nibble holding the even
+ * group (s_shift = 4 * (G mod 2)).  The group scale is the fp32 product q4 * s_super; the weight
+ * rule is then the one above, w = bf16((u - 32) * bf16(s)).
+ * ------------------------------------------------------------------------------------------ */
+static float q4_group_scale(const uint8_t *sq_row, float super, int G)
+{
+    int q = (sq_row[G >> 1] >> (4 * (G & 1))) & 0xF;
+    return (float)q * super; /* one fp32 multiply (the file is built without contraction) */
+}
+
+int oracle_dequant_w2q4(const uint8_t *codes, const uint8_t *scale_q4, const float *super,
+                        const float *code_scale, const float *code_zero, int n, int k, int group,
+                        uint16_t *out)
+{
+    const int32_t *cb = codebook_643();
+    if (!cb || n < 0 || k < 0 || group <= 0 || k % 4 || k % group) return -1;
+    int ng = k / group, nb = (ng + 1) / 2;
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < n; ++r) {
+        for (int kk = 0; kk < k; ++kk) {
+            uint8_t q = codes[(size_t)r * (k / 4) + kk / 4];
+            int32_t C = oracle_cluster_code(q, code_scale[r], code_zero[r]);
+            uint32_t idx = ((uint32_t)C) & 0x7FFFu;
+            int32_t u = cb[(size_t)idx * 4 + (kk % 4)];
+            float s = q4_group_scale(scale_q4 + (size_t)r * nb, super[r], kk / group);
+            out[(size_t)r * k + kk] = dequant_state(u, s);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------
  * W4 per-channel dequantization ([WINT2] quantization_config "wint4", "per_channel"; [GPTQ]
  * Part 2 pack_int4/unpack_int4): codes[n][k/2], two signed 4-bit codes per byte, the first code
  * of a pair in the low nibble; the code is sign-extended; w = bf16(q * bf16(scale[n])).
@@ -298,6 +333,11 @@ int oracle_moe_f64(const uint16_t *x /* [T][H] */, int T, int H, int I, int E,
  * ------------------------------------------------------------------------------------------ */
 #define ORACLE_ENC_LITERAL_EQ1 1u
 #define ORACLE_ENC_REFIT_SCALE 2u
+/* 4-bit group scales (§3.4 "Scale Compression"; reading of the unstated quantizer): the raw group
+ * scales s_g = absmax_g / 31 (fp32) give the channel's super scale s_super = max_g s_g / 15 (fp32)
+ * and q4_g = round-half-even(s_g / s_super) in 0..15; the search then uses s_g' = q4_g * s_super.
+ * The Eq. 4 refit does not apply (the scale is no longer free). */
+#define ORACLE_ENC_Q4_SCALE 4u
 
 static double vec_err(const float *v, const int32_t *st, const double *D)
 {
@@ -328,17 +368,48 @@ static uint8_t best_byte(const float *v, const double *D, const int32_t *cb, flo
 }
 
 static void encode_row(const float *wr, int k, int group, uint32_t flags, const int32_t *cb,
-                       int32_t *C, uint8_t *codes, float *scales, float *alpha, float *beta)
+                       int32_t *C, uint8_t *codes, float *scales, float *alpha, float *beta,
+                       uint8_t *q4 /* [ng], Q4 only */, float *super /* Q4 only */)
 {
     int ng = k / group, nv = k / 4;
+    /* 1 (Q4): raw group scales, the channel's super scale and the 4-bit scale of each group */
+    if (flags & ORACLE_ENC_Q4_SCALE) {
+        double smax = 0.0;
+        for (int g = 0; g < ng; ++g) {
+            double amax = 0.0;
+            for (int i = 0; i < group; ++i) {
+                double a = fabs((double)wr[g * group + i]);
+                if (a > amax) amax = a;
+            }
+            scales[g] = (float)(amax / 31.0);
+            if ((double)scales[g] > smax) smax = (double)scales[g];
+        }
+        float sup = (float)(smax / 15.0);
+        *super = sup;
+        int old = fegetround();
+        fesetround(FE_TONEAREST);
+        for (int g = 0; g < ng; ++g) {
+            double qq = sup > 0.0f ? nearbyint((double)scales[g] / (double)sup) : 0.0;
+            if (qq < 0.0) qq = 0.0;
+            if (qq > 15.0) qq = 15.0;
+            q4[g] = (uint8_t)qq;
+            scales[g] = (float)q4[g] * sup;
+        }
+        fesetround(old);
+    }
     /* 1-2: group scale, then codebook search for every 4-vector */
     for (int g = 0; g < ng; ++g) {
-        double amax = 0.0;
-        for (int i = 0; i < group; ++i) {
-            double a = fabs((double)wr[g * group + i]);
-            if (a > amax) amax = a;
+        float s;
+        if (flags & ORACLE_ENC_Q4_SCALE) {
+            s = scales[g];
+        } else {
+            double amax = 0.0;
+            for (int i = 0; i < group; ++i) {
+                double a = fabs((double)wr[g * group + i]);
+                if (a > amax) amax = a;
+            }
+            s = oracle_bf16_to_float(oracle_bf16_bits((float)(amax / 31.0)));
         }
-        float s = oracle_bf16_to_float(oracle_bf16_bits((float)(amax / 31.0)));
         scales[g] = s;
         double D[64];
         level_table(s, D);
@@ -386,7 +457,7 @@ static void encode_row(const float *wr, int k, int group, uint32_t flags, const 
             codes[j] = c;
         }
         /* 5: Eq. 4 refit of this group's scale, then one more byte choice */
-        if (flags & ORACLE_ENC_REFIT_SCALE) {
+        if ((flags & ORACLE_ENC_REFIT_SCALE) && !(flags & ORACLE_ENC_Q4_SCALE)) {
             double num = 0.0, den = 0.0;
             for (int vq = 0; vq < group / 4; ++vq) {
                 int j = g * (group / 4) + vq;
@@ -427,9 +498,37 @@ int oracle_encode_w2(const float *w, int n, int k, int group, uint32_t flags, ui
     for (int r = 0; r < n; ++r) {
         int32_t *C = (int32_t *)malloc(sizeof(int32_t) * (size_t)nv);
         if (!C) { fail = 1; continue; }
-        encode_row(w + (size_t)r * k, k, group, flags, cb, C, codes + (size_t)r * nv,
-                   scales + (size_t)r * ng, alpha + r, beta + r);
+        encode_row(w + (size_t)r * k, k, group, flags & ~ORACLE_ENC_Q4_SCALE, cb, C, codes + (size_t)r * nv,
+                   scales + (size_t)r * ng, alpha + r, beta + r, NULL, NULL);
         free(C);
+    }
+    return fail ? -1 : 0;
+}
+
+/* Encoder for the 4-bit scale format: codes, packed scale_q4[n][ceil(ng/2)] (even group in the
+ * low nibble), super[n], alpha[n], beta[n].  flags: ORACLE_ENC_LITERAL_EQ1 only. */
+int oracle_encode_w2q4(const float *w, int n, int k, int group, uint32_t flags, uint8_t *codes,
+                       uint8_t *scale_q4, float *super, float *alpha, float *beta)
+{
+    const int32_t *cb = codebook_643();
+    if (!cb || n < 0 || k <= 0 || group <= 0 || group % 4 || k % group) return -1;
+    if (flags & ORACLE_ENC_REFIT_SCALE) return -1;
+    int ng = k / group, nv = k / 4, nb = (ng + 1) / 2;
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : fail)
+    for (int r = 0; r < n; ++r) {
+        int32_t *C = (int32_t *)malloc(sizeof(int32_t) * (size_t)nv);
+        float *sc = (float *)malloc(sizeof(float) * (size_t)ng);
+        uint8_t *q4 = (uint8_t *)malloc((size_t)ng);
+        if (!C || !sc || !q4) { fail = 1; free(C); free(sc); free(q4); continue; }
+        encode_row(w + (size_t)r * k, k, group, flags | ORACLE_ENC_Q4_SCALE, cb, C, codes + (size_t)r * nv, sc,
+                   alpha + r, beta + r, q4, super + r);
+        uint8_t *dst = scale_q4 + (size_t)r * nb;
+        for (int b = 0; b < nb; ++b) dst[b] = 0;
+        for (int g = 0; g < ng; ++g) dst[g >> 1] |= (uint8_t)(q4[g] << (4 * (g & 1)));
+        free(C);
+        free(sc);
+        free(q4);
     }
     return fail ? -1 : 0;
 }

@@ -521,3 +521,67 @@ def test_eq4_closed_form():
     h = 1e-6
     assert abs((err(s_star + h) - err(s_star - h)) / (2 * h)) < 1e-6
     assert err(s_star) <= min(err(s_star * 1.01), err(s_star * 0.99))
+
+
+# ----------------------------------------------------------------------------------------------
+# 4-bit group scales: CCQ §3.4 "Scale Compression", Eq. 5 and Algorithm 3's first line
+# ----------------------------------------------------------------------------------------------
+def test_dequant_w2q4_hand_example():
+    # byte 0 with alpha = 1, beta = 12345: C = 12345 = 011000 000 111 001 (15 bits):
+    #   u0 = 24, u1 = (24<<3 | 0) mod 64 = 0, u2 = (0<<3 | 7) = 7, u3 = (7<<3 | 1) = 57
+    # scale byte 0xA3 with super 0.5: group 0 (low nibble) q = 3 -> s = 1.5, group 1 q = 10 -> 5.0
+    #   group 0: (24-32, 0-32, 7-32, 57-32) * 1.5 = -12, -48, -37.5, 37.5
+    #   group 1: the same levels * 5.0 = -40, -160, -125, 125
+    codes = np.zeros((1, 32), dtype=np.uint8)
+    out = oracle.bf16_to_f64(oracle.dequant_w2q4(codes, np.array([[0xA3]], np.uint8), [0.5], [1.0], [12345.0]))
+    assert list(out[0, :4]) == [-12.0, -48.0, -37.5, 37.5]
+    assert list(out[0, 60:64]) == [-12.0, -48.0, -37.5, 37.5]
+    assert list(out[0, 64:68]) == [-40.0, -160.0, -125.0, 125.0]
+    # a zero 4-bit scale decodes its group to (signed) zeros
+    z = oracle.bf16_to_f64(oracle.dequant_w2q4(codes, np.array([[0x30]], np.uint8), [0.5], [1.0], [12345.0]))
+    assert np.all(z[0, :64] == 0.0) and list(z[0, 64:68]) == [-12.0, -48.0, -37.5, 37.5]
+
+
+def test_dequant_w2q4_is_w2_with_product_scales():
+    # the 4-bit format decodes exactly like the fp32-scale format given the fp32 products q4 * super
+    rng = np.random.default_rng(77)
+    n, k = 5, 384
+    codes = rng.integers(0, 256, (n, k // 4), dtype=np.uint8)
+    sq = rng.integers(0, 256, (n, 3), dtype=np.uint8)
+    sup = (rng.random(n) * 1e-3).astype(np.float32)
+    a = (rng.random(n) * 60).astype(np.float32)
+    b = rng.integers(0, 12000, n).astype(np.float32)
+    q = np.stack([sq & 0xF, sq >> 4], axis=-1).reshape(n, 6)
+    sc = (q.astype(np.float32) * sup[:, None]).astype(np.float32)
+    assert np.array_equal(oracle.dequant_w2q4(codes, sq, sup, a, b), oracle.dequant_w2(codes, sc, a, b))
+
+
+def test_encode_w2q4_scale_quantizer():
+    # the channel super scale is the largest raw group scale (absmax/31) over 15; that group gets
+    # q4 = 15 and every group's q4 is its raw scale over the super scale, rounded half to even
+    w = synth.weights_normal(4, 512, 91)
+    codes, sq, sup, a, b = oracle.encode_w2q4(w)
+    q = oracle.q4_unpack(sq, 8)
+    raw = (np.abs(w.reshape(4, 8, 64)).max(axis=2) / 31.0).astype(np.float32)
+    assert np.allclose(sup, (raw.max(axis=1) / 15.0).astype(np.float32), rtol=0, atol=0)
+    assert np.all(q[np.arange(4), raw.argmax(axis=1)] == 15)
+    assert np.array_equal(q, np.clip(np.rint(raw.astype(np.float64) / sup[:, None].astype(np.float64)), 0, 15))
+    # storage: 16 code bytes + half a scale byte per 64 weights = 2.0625 bits per weight (Eq. 5)
+    assert (codes.nbytes + sq.nbytes) * 8 / w.size == pytest.approx(2.0625)
+
+
+def test_encode_w2q4_codes_are_optimal_for_the_quantized_scales():
+    # with the group scales fixed at q4 * super, the bytes are the argmin of the decoded error over
+    # all 256 bytes of the channel (the same re-search as the fp32-scale encoder)
+    w = synth.weights_normal(2, 128, 93)
+    codes, sq, sup, a, b = oracle.encode_w2q4(w)
+    q = oracle.q4_unpack(sq, 2)
+    for r in range(2):
+        table = np.zeros((256, 128), dtype=np.uint16)
+        for c in range(256):
+            table[c] = oracle.dequant_w2q4(np.full((1, 32), c, np.uint8), sq[r:r + 1], sup[r:r + 1],
+                                           a[r:r + 1], b[r:r + 1])[0]
+        dec = oracle.bf16_to_f64(table).reshape(256, 32, 4)
+        err = ((w[r].reshape(32, 4)[None] - dec) ** 2).sum(axis=2)  # [byte][vector]
+        assert np.array_equal(codes[r], np.argmin(err, axis=0).astype(np.uint8))
+        assert q[r].max() == 15
