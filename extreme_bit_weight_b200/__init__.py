@@ -26,6 +26,7 @@ CCQ_ERR_TIMEOUT = 5
 
 CCQ_FMT_W2_CCQ_G64 = 1
 CCQ_FMT_W4_PER_CHANNEL = 2
+CCQ_FMT_W2_CCQ_G64_Q4SCALE = 3
 CCQ_ENC_LITERAL_EQ1 = 1
 CCQ_ENC_REFIT_SCALE = 2
 
@@ -52,6 +53,8 @@ class ccq_weight(ctypes.Structure):
         ("scales", ctypes.c_void_p),
         ("alpha", ctypes.c_void_p),
         ("beta", ctypes.c_void_p),
+        ("scale_q4", ctypes.c_void_p),
+        ("super_scale", ctypes.c_void_p),
     ]
 
 
@@ -62,6 +65,7 @@ _lib.ccq_status_string.restype = ctypes.c_char_p
 _lib.ccq_build_info.restype = ctypes.c_char_p
 _lib.ccq_encode_host.argtypes = [_P, _I, _I, _I, ctypes.c_uint32, _I, _P, _P, _P, _P, _P]
 _lib.ccq_quantize_w4_host.argtypes = [_P, _I, _I, _I, _P, _P]
+_lib.ccq_encode_host_q4.argtypes = [_P, _I, _I, _I, ctypes.c_uint32, _I, _P, _P, _P, _P, _P, _P]
 _lib.ccq_dequant_bf16.argtypes = [ctypes.POINTER(ccq_weight), _I, _P, _P]
 _lib.ccq_gemm_workspace_size.argtypes = [ctypes.POINTER(ccq_weight), _I]
 _lib.ccq_gemm_workspace_size.restype = ctypes.c_size_t
@@ -129,6 +133,23 @@ def ccq_encode_host(w: np.ndarray, group: int = 64, flags: int = 0, threads: int
     return codes, scales, alpha, beta, err.value
 
 
+def ccq_encode_host_q4(w: np.ndarray, group: int = 64, flags: int = 0, threads: int = 0):
+    """CCQ encode with 4-bit group scales (CCQ_FMT_W2_CCQ_G64_Q4SCALE) of fp32 w [n][k]
+    -> (codes, scale_q4 [n][k/128], super_scale [n], alpha, beta, sq_err)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    n, k = w.shape
+    codes = np.zeros((n, k // 4), np.uint8)
+    sq = np.zeros((n, k // (2 * group)), np.uint8)
+    sup = np.zeros(n, np.float32)
+    alpha = np.zeros(n, np.float32)
+    beta = np.zeros(n, np.float32)
+    err = ctypes.c_double(0.0)
+    _check(_lib.ccq_encode_host_q4(_np_ptr(w), n, k, group, flags, threads, _np_ptr(codes), _np_ptr(sq),
+                                   _np_ptr(sup), _np_ptr(alpha), _np_ptr(beta), ctypes.byref(err)),
+           "ccq_encode_host_q4")
+    return codes, sq, sup, alpha, beta, err.value
+
+
 def ccq_quantize_w4_host(w: np.ndarray, threads: int = 0):
     """W4 per-channel RTN of fp32 w [n][k] -> (codes [n][k/2], scales [n])."""
     w = np.ascontiguousarray(w, dtype=np.float32)
@@ -147,7 +168,7 @@ class CcqWeight:
     """Device copy of one (or E stacked) quantized weight(s) [E][n][k] and its ccq_weight view."""
 
     def __init__(self, fmt: int, n: int, k: int, codes, scales, alpha=None, beta=None, experts: int = 1,
-                 device="cuda"):
+                 device="cuda", scale_q4=None, super_scale=None):
         self.fmt, self.n, self.k, self.experts = int(fmt), int(n), int(k), int(experts)
 
         def dev(a, dtype):
@@ -161,14 +182,18 @@ class CcqWeight:
         self.scales = dev(scales, torch.float32)
         self.alpha = dev(alpha, torch.float32)
         self.beta = dev(beta, torch.float32)
+        self.scale_q4 = dev(scale_q4, torch.uint8)
+        self.super_scale = dev(super_scale, torch.float32)
 
     def struct(self) -> ccq_weight:
-        return ccq_weight(self.fmt, self.n, self.k, 64 if self.fmt == CCQ_FMT_W2_CCQ_G64 else 0,
-                          _dptr(self.codes), _dptr(self.scales), _dptr(self.alpha), _dptr(self.beta))
+        return ccq_weight(self.fmt, self.n, self.k, 0 if self.fmt == CCQ_FMT_W4_PER_CHANNEL else 64,
+                          _dptr(self.codes), _dptr(self.scales), _dptr(self.alpha), _dptr(self.beta),
+                          _dptr(self.scale_q4), _dptr(self.super_scale))
 
     @property
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in (self.codes, self.scales, self.alpha, self.beta)
+        return sum(t.numel() * t.element_size()
+                   for t in (self.codes, self.scales, self.alpha, self.beta, self.scale_q4, self.super_scale)
                    if t is not None)
 
 

@@ -18,9 +18,12 @@ namespace {
 // stored byte.  The code is rounded with cvt.rni (round to nearest even, saturating at the int32
 // range, NaN -> 0), so this kernel is exact for any alpha/beta, unlike the fast path.
 // ------------------------------------------------------------------------------------------------
+// scales == NULL: 4-bit group scales, s = fl32(q4 * super[r]) (CCQ §3.4 "Scale Compression"),
+// two per byte of scale_q4[r][K/128], the even group in the low nibble.
 __global__ void dequant_w2_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales,
                                   const float *__restrict__ alpha, const float *__restrict__ beta, int rows,
-                                  int K, uint16_t *__restrict__ out) {
+                                  int K, uint16_t *__restrict__ out, const uint8_t *__restrict__ scale_q4,
+                                  const float *__restrict__ super) {
     const size_t nbytes = (size_t)rows * (K / 4);
     const int kb = K / 4, ng = K / 64;
     for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < nbytes;
@@ -28,7 +31,15 @@ __global__ void dequant_w2_kernel(const uint8_t *__restrict__ codes, const float
         const int r = (int)(idx / kb), j = (int)(idx % kb);
         const float t = __fmaf_rn((float)codes[idx], __ldg(alpha + r), __ldg(beta + r));
         const uint32_t C = (uint32_t)__float2int_rn(t);
-        const float s = bf16_bits_to_float(float_to_bf16_bits(__ldg(scales + (size_t)r * ng + (4 * j) / 64)));
+        const int G = (4 * j) / 64;
+        float sraw;
+        if (scales) {
+            sraw = __ldg(scales + (size_t)r * ng + G);
+        } else {
+            const uint32_t q = (__ldg(scale_q4 + (size_t)r * (K / 128) + G / 2) >> (4 * (G & 1))) & 0xFu;
+            sraw = __fmul_rn((float)q, __ldg(super + r));
+        }
+        const float s = bf16_bits_to_float(float_to_bf16_bits(sraw));
         uint16_t o[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -245,10 +256,13 @@ inline int grid_for(size_t work, int threads) {
 }  // namespace
 
 cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, const float *alpha,
-                           const float *beta, int rows, int K, uint16_t *out, cudaStream_t s) {
+                           const float *beta, int rows, int K, uint16_t *out, cudaStream_t s,
+                           const uint8_t *scale_q4, const float *super) {
     if (rows == 0) return cudaSuccess;
-    if (fmt == CCQ_FMT_W2_CCQ_G64) {
-        dequant_w2_kernel<<<grid_for((size_t)rows * K / 4, 256), 256, 0, s>>>(codes, scales, alpha, beta, rows, K, out);
+    if (fmt == CCQ_FMT_W2_CCQ_G64 || fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE) {
+        const bool q4 = fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
+        dequant_w2_kernel<<<grid_for((size_t)rows * K / 4, 256), 256, 0, s>>>(
+            codes, q4 ? nullptr : scales, alpha, beta, rows, K, out, scale_q4, super);
     } else {
         dequant_w4_kernel<<<grid_for((size_t)rows * K / 2, 256), 256, 0, s>>>(codes, scales, rows, K, out);
     }

@@ -50,9 +50,18 @@ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 ccq_status check_weight(const ccq_weight *w, int experts) {
     if (!w || experts <= 0) return CCQ_ERR_INVALID_ARG;
-    if (w->fmt != CCQ_FMT_W2_CCQ_G64 && w->fmt != CCQ_FMT_W4_PER_CHANNEL) return CCQ_ERR_UNSUPPORTED;
+    if (w->fmt != CCQ_FMT_W2_CCQ_G64 && w->fmt != CCQ_FMT_W4_PER_CHANNEL && w->fmt != CCQ_FMT_W2_CCQ_G64_Q4SCALE)
+        return CCQ_ERR_UNSUPPORTED;
     if (w->n <= 0 || w->k <= 0 || w->n % 16 || w->k % 64) return CCQ_ERR_INVALID_ARG;
-    if (!w->codes || !w->scales || !aligned16(w->codes) || !aligned16(w->scales)) return CCQ_ERR_INVALID_ARG;
+    if (!w->codes || !aligned16(w->codes)) return CCQ_ERR_INVALID_ARG;
+    if (w->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE) {
+        if (w->group != 64) return CCQ_ERR_UNSUPPORTED;
+        if (w->k % 128 || !w->scale_q4 || !w->super_scale || !w->alpha || !w->beta) return CCQ_ERR_INVALID_ARG;
+        if (!aligned16(w->scale_q4) || !aligned16(w->super_scale) || !aligned16(w->alpha) || !aligned16(w->beta))
+            return CCQ_ERR_INVALID_ARG;
+    } else {
+        if (!w->scales || !aligned16(w->scales)) return CCQ_ERR_INVALID_ARG;
+    }
     if (w->fmt == CCQ_FMT_W2_CCQ_G64) {
         if (w->group != 64) return CCQ_ERR_UNSUPPORTED;
         if (!w->alpha || !w->beta) return CCQ_ERR_INVALID_ARG;
@@ -105,7 +114,7 @@ bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t
             return false;
     }
     // group scales [rows][K/64] fp32: staged by TMA when the row pitch is a multiple of 16 bytes
-    m.tma_scales = !w4 && (K / 64) % 4 == 0;
+    m.tma_scales = !w4 && w->fmt != CCQ_FMT_W2_CCQ_G64_Q4SCALE && (K / 64) % 4 == 0;
     if (m.tma_scales) {
         cuuint64_t dims[2] = {(cuuint64_t)(K / 64), rows};
         cuuint64_t str[1] = {(cuuint64_t)(K / 64) * 4};
@@ -272,7 +281,8 @@ ccq_status ccq_dequant_bf16(const ccq_weight *w, int32_t num_experts, void *out_
     if (st != CCQ_OK) return st;
     if (!out_bf16 || !aligned16(out_bf16)) return CCQ_ERR_INVALID_ARG;
     return cuda_status(launch_dequant(w->fmt, w->codes, w->scales, w->alpha, w->beta, num_experts * w->n, w->k,
-                                      static_cast<uint16_t *>(out_bf16), (cudaStream_t)stream));
+                                      static_cast<uint16_t *>(out_bf16), (cudaStream_t)stream, w->scale_q4,
+                                      w->super_scale));
 }
 
 size_t ccq_gemm_workspace_size(const ccq_weight *w, int32_t m) {
@@ -312,6 +322,9 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
         p.M = m;
         p.out_ld = w->n;
         p.w4 = w->fmt == CCQ_FMT_W4_PER_CHANNEL;
+        p.q4 = w->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
+        p.scale_q4 = w->scale_q4;
+        p.super_scale = w->super_scale;
         p.ksplit = L.ksplit;
         p.kg = L.spp;
         if (L.ksplit > 1) {
@@ -361,6 +374,9 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
     }
     p.tma_scales = maps.tma_scales;
     p.w4 = w->fmt == CCQ_FMT_W4_PER_CHANNEL;
+    p.q4 = w->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
+    p.scale_q4 = w->scale_q4;
+    p.super_scale = w->super_scale;
     e = launch_decode_gemm_w2(p, maps.codes, maps.xa, maps.gs, maps.sc, L.row_blocks, L.ksplit, 1, L.nt, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     if (L.ksplit > 1) {
@@ -456,6 +472,9 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q1.I = I;
         q1.err = err;
         q1.w4 = w13->fmt == CCQ_FMT_W4_PER_CHANNEL;
+        q1.q4 = w13->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
+        q1.scale_q4 = w13->scale_q4;
+        q1.super_scale = w13->super_scale;
         e = launch_tc_gemm_w2(q1, ta1, tc1, mt, std::min(sm_count(), L.max_tiles * q1.n_tiles), s);
         if (e == cudaSuccess) e = trace(events, 3, s);
         if (e == cudaSuccess) e = trace(events, 4, s);
@@ -474,6 +493,9 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q2.rw = rwp;
         q2.I = 0;
         q2.w4 = w2->fmt == CCQ_FMT_W4_PER_CHANNEL;
+        q2.q4 = w2->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
+        q2.scale_q4 = w2->scale_q4;
+        q2.super_scale = w2->super_scale;
         if (e == cudaSuccess) e = launch_tc_gemm_w2(q2, ta2, tc2, mt, std::min(sm_count(), L.max_tiles * q2.n_tiles), s);
         if (e == cudaSuccess) e = trace(events, 5, s);
         if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
@@ -509,6 +531,9 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p1.err = err;
     p1.tma_scales = m1.tma_scales;
     p1.w4 = w13->fmt == CCQ_FMT_W4_PER_CHANNEL;
+    p1.q4 = w13->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
+    p1.scale_q4 = w13->scale_q4;
+    p1.super_scale = w13->super_scale;
 
     // down projection, scaled by each pair's routing weight -> fp32 slots
     DecodeMaps m2;
@@ -532,6 +557,9 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p2.err = err;
     p2.tma_scales = m2.tma_scales;
     p2.w4 = w2->fmt == CCQ_FMT_W4_PER_CHANNEL;
+    p2.q4 = w2->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
+    p2.scale_q4 = w2->scale_q4;
+    p2.super_scale = w2->super_scale;
 
     // Both projections W2 with TMA-staged scales and the same token tiling: one fused launch, in
     // which the gate/up epilogue also writes h's group-sum table and each down unit starts once

@@ -56,14 +56,16 @@ static_assert(kProducerWarps * 32 * kProducerRegs + kConsumerWarps * 32 * kConsu
 static_assert(65536 / kThreads >= kLaunchRegs, "launch registers");
 constexpr int kCodeTileBytes = 128 * 128;  // [128 rows][128 B] = 8 groups of 16 bytes
 
-template <int NT, bool W4 = false>
+template <int NT, bool W4 = false, bool Q4 = false>
 struct Smem {
     static constexpr int MP = 8 * NT;
     static constexpr int kCodeBytes = (W4 ? 2 : 1) * 2 * kCodeTileBytes;  // both halves, one stage
     static constexpr int kXaBytes = 32 * MP * 16 * 2;  // [G*4+i = 32][MP][16] bf16
     static constexpr int kGsBytes = MP * 8 * 16;       // [MP][8] gsq float4 entries
-    static constexpr int kScBytes = W4 ? 0 : 2 * 128 * 8 * 4;  // [2 halves][128 rows][8 groups] fp32 scales
-    static constexpr int kRowsBytes = 2048;  // [4][128] fp32: alpha A, alpha B, beta A, beta B (W4: scales A, B)
+    // [2 halves][128 rows][8 groups] fp32 scales (none for W4; 4-bit scales are read from global)
+    static constexpr int kScBytes = (W4 || Q4) ? 0 : 2 * 128 * 8 * 4;
+    // [4][128] fp32: alpha A, alpha B, beta A, beta B (W4: scales A, B); Q4: then super A, super B
+    static constexpr int kRowsBytes = Q4 ? 3072 : 2048;
     static constexpr int kStageBytes = ((kCodeBytes + kXaBytes + kGsBytes + kScBytes + kRowsBytes) + 1023) & ~1023;
     static constexpr int kRedBytes = kRowWarps * 32 * 2 * NT * 4 * 4;  // partial sums of the second warp half
     static constexpr int kStages = ((227 * 1024 - 2048 - kRedBytes) / kStageBytes) < 4
@@ -374,11 +376,11 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
 // Persistent: CTA b walks units b, b + gridDim.x, ...; its producer streams every stage of every
 // unit through one ring, so the next unit's first stages load while this unit finishes.
 // FUSED: the launch holds the MoE gate/up units (p, m1) followed by the down units (p2, m2).
-template <int NT, bool TMA_SC, bool W4, bool FUSED>
+template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__ MapSet m2,
                       const __grid_constant__ DecodeGemmParams p, const __grid_constant__ DecodeGemmParams p2) {
-    using S = Smem<NT, W4>;
+    using S = Smem<NT, W4, Q4>;
     constexpr int MP = S::MP;
     constexpr int kStages = S::kStages;
     constexpr int kCodeOff = 0;                       // code tiles of the stage
@@ -466,7 +468,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             }
             fence_proxy_async_global();  // the generic-proxy writes of h are visible to TMA from here
         }
-        const uint32_t row_bytes = first ? (uint32_t)(U.nA + U.nB) * 4u * (W4 ? 1u : 2u) : 0u;
+        const uint32_t row_bytes = first ? (uint32_t)(U.nA + U.nB) * 4u * (W4 ? 1u : Q4 ? 3u : 2u) : 0u;
         mbar_arrive_expect_tx(bar, S::kTxBytes + ((TMA_SC && !W4) ? S::kScBytes : 0) + row_bytes);
         if (first) {
             // the unit's per-row constants: alpha, beta (W2) or the channel scales (W4) of both halves
@@ -476,6 +478,10 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             if (!W4) {
                 if (U.nA) bulk_g2s(base + kRowsOff + 1024, q.beta + rowA, U.nA * 4u, bar);
                 if (U.nB) bulk_g2s(base + kRowsOff + 1536, q.beta + rowB, U.nB * 4u, bar);
+            }
+            if (Q4) {
+                if (U.nA) bulk_g2s(base + kRowsOff + 2048, q.super_scale + rowA, U.nA * 4u, bar);
+                if (U.nB) bulk_g2s(base + kRowsOff + 2560, q.super_scale + rowB, U.nB * 4u, bar);
             }
         }
         if (TMA_SC && !W4) {
@@ -584,7 +590,8 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
         n_units += load_unit_any<MP, FUSED>(p, p2, u, t) ? 1 : 0;
     }
     RowDecode rd[4];
-    float sc_row[4];  // W4: per-channel scales, bf16-rounded
+    float sc_row[4];  // W4: per-channel scales, bf16-rounded; Q4: the rows' super scales
+    uint32_t q4cur[4] = {0, 0, 0, 0}, q4nxt[4] = {0, 0, 0, 0};  // Q4: this / the next stage's scale nibbles
     float acc[2][NT][4];
 #pragma unroll
     for (int t = 0; t < 2; ++t)
@@ -615,6 +622,10 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                 rd[1].ab = f2_pack(r1, r1); rd[1].bb = f2_pack(b1, b1);
                 rd[2].ab = f2_pack(r2, r2); rd[2].bb = f2_pack(b2, b2);
                 rd[3].ab = f2_pack(r3, r3); rd[3].bb = f2_pack(b3, b3);
+                if constexpr (Q4) {
+                    sc_row[0] = lds_f32(ra + 2048); sc_row[1] = lds_f32(ra + 2080);
+                    sc_row[2] = lds_f32(ra + 2560); sc_row[3] = lds_f32(ra + 2592);
+                }
             } else {
                 sc_row[0] = round_bf16(r0); sc_row[1] = round_bf16(r1);
                 sc_row[2] = round_bf16(r2); sc_row[3] = round_bf16(r3);
@@ -626,6 +637,44 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             static_for<4>([&](auto Gc) {
                 constexpr int G = decltype(Gc)::value;
                 group_w4<NT, G>(sb + coff[G], xs, gs, sc_row, kc, acc);
+            });
+        } else if (Q4) {
+            // 4-bit group scales: this thread's 4 nibbles (groups Gh..Gh+3) of each of its rows, read
+            // from global memory one stage ahead; s = bf16(fl32(q4 * super)).  Groups beyond K
+            // read activations 0 (TMA zero fill) and add nothing.
+            const int nst = U.s_end - U.s_begin;
+            auto q4_load = [&](int stg, uint32_t (&dst)[4]) {
+                const int qpr = pq.K / 128;  // scale bytes per row
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int lr = (r < 2 ? U.localA : U.localB) + wrow + g + 8 * (r & 1);
+                    const int grow = U.e * pq.N + (lr < pq.N ? lr : 0);
+                    // two single bytes: a row's scale bytes need not be 2-byte aligned, and the
+                    // last stage may end inside the row
+                    const int byte = stg * 4 + khalf * 2;
+                    const uint8_t *src = pq.scale_q4 + (size_t)grow * qpr + byte;
+                    const uint32_t lo = byte < qpr ? (uint32_t)__ldg(src) : 0u;
+                    const uint32_t hi = byte + 1 < qpr ? (uint32_t)__ldg(src + 1) : 0u;
+                    dst[r] = lo | (hi << 8);
+                }
+            };
+            if (first) q4_load(st, q4cur);
+            else {
+#pragma unroll
+                for (int r = 0; r < 4; ++r) q4cur[r] = q4nxt[r];
+            }
+            if (i + 1 < nst) q4_load(st + 1 == U.s_end ? U.s_begin : st + 1, q4nxt);
+            const uint32_t xs = sb + xa_thr, gs = sb + gs_thr;
+            static_for<4>([&](auto Gc) {
+                constexpr int G = decltype(Gc)::value;
+                float sc[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    // the nibble as a float: its bits under the exponent of 2^23, minus 2^23
+                    const float qf = __uint_as_float(0x4B000000u | ((q4cur[r] >> (4 * G)) & 0xFu)) - 8388608.0f;
+                    sc[r] = round_bf16(__fmul_rn(qf, sc_row[r]));
+                }
+                group_w2<NT, G>(sb + coff[G], xs, gs, sc, rd, kc, acc);
             });
         } else if (TMA_SC) {
             // full stage: groups beyond K read TMA zero fill (scale 0, activations 0) and add nothing
@@ -839,7 +888,10 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
             smem = Smem<NT, true>::kTotal;
         }
     }
-    if (!p.w4) {
+    if (!p.w4 && p.q4) {
+        kern = decode_gemm_w2_kernel<NT, false, false, false, true>;
+        smem = Smem<NT, false, true>::kTotal;
+    } else if (!p.w4) {
         kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false, false>
                             : decode_gemm_w2_kernel<NT, false, false, false>;
         smem = Smem<NT, false>::kTotal;
@@ -910,7 +962,7 @@ cudaError_t launch_decode_moe_fused(const DecodeGemmParams &p1, const CUtensorMa
                                     const DecodeGemmParams &p2, const CUtensorMap &a2, const CUtensorMap &b2,
                                     const CUtensorMap &c2, const CUtensorMap &d2, int row_blocks2, int experts,
                                     int nt, cudaStream_t s) {
-    if (p1.w4 || p2.w4 || !p1.tma_scales || !p2.tma_scales || p1.mode != EPI_GATEUP || p2.mode != EPI_DOWN ||
+    if (p1.w4 || p2.w4 || p1.q4 || p2.q4 || !p1.tma_scales || !p2.tma_scales || p1.mode != EPI_GATEUP || p2.mode != EPI_DOWN ||
         !p1.dep || !p2.dep || !p1.fuse_gsq)
         return cudaErrorInvalidValue;
     const MapSet m1{a1, b1, c1, d1}, m2{a2, b2, c2, d2};

@@ -117,15 +117,39 @@ inline uint8_t best_byte(const float *v, const double *D, const ByteTable &bt) {
     return uint8_t(arg);
 }
 
+// q4 != nullptr: 4-bit group scales (CCQ §3.4 "Scale Compression"): q4[g] and *super_out are
+// outputs and scales[] holds the group scales fl32(q4 * super) the search uses.
 void encode_row(const float *wr, int k, int group, uint32_t flags, uint8_t *codes, float *scales,
-                float *alpha_out, float *beta_out, double *err_out) {
+                float *alpha_out, float *beta_out, double *err_out, uint8_t *q4 = nullptr,
+                float *super_out = nullptr) {
     const int ng = k / group, nv = k / 4, vpg = group / 4;
     std::vector<int32_t> C(nv);
     std::vector<double> Dall(size_t(ng) * 64);
+    if (q4) {
+        double smax = 0.0;
+        for (int g = 0; g < ng; ++g) {
+            double amax = 0.0;
+            for (int i = 0; i < group; ++i) amax = std::max(amax, std::fabs(double(wr[g * group + i])));
+            scales[g] = float(amax / 31.0);
+            smax = std::max(smax, double(scales[g]));
+        }
+        const float sup = float(smax / 15.0);
+        *super_out = sup;
+        for (int g = 0; g < ng; ++g) {
+            double qq = sup > 0.0f ? std::nearbyint(double(scales[g]) / double(sup)) : 0.0;
+            q4[g] = uint8_t(std::min(15.0, std::max(0.0, qq)));
+            scales[g] = float(q4[g]) * sup;
+        }
+    }
     for (int g = 0; g < ng; ++g) {
-        double amax = 0.0;
-        for (int i = 0; i < group; ++i) amax = std::max(amax, std::fabs(double(wr[g * group + i])));
-        float s = to_bf16(float(amax / 31.0));
+        float s;
+        if (q4) {
+            s = scales[g];
+        } else {
+            double amax = 0.0;
+            for (int i = 0; i < group; ++i) amax = std::max(amax, std::fabs(double(wr[g * group + i])));
+            s = to_bf16(float(amax / 31.0));
+        }
         scales[g] = s;
         double *D = &Dall[size_t(g) * 64];
         levels(s, D);
@@ -151,7 +175,7 @@ void encode_row(const float *wr, int k, int group, uint32_t flags, uint8_t *code
                 codes[j] = best_byte(wr + size_t(j) * 4, D, bt);
             }
         }
-        if (flags & CCQ_ENC_REFIT_SCALE) {
+        if ((flags & CCQ_ENC_REFIT_SCALE) && !q4) {
             double num = 0.0, den = 0.0;
             for (int q = 0; q < vpg; ++q) {
                 int j = g * vpg + q;
@@ -228,6 +252,31 @@ extern "C" ccq_status ccq_encode_host(const float *w, int32_t n, int32_t k, int3
     parallel_rows(n, threads, [&](int r) {
         encode_row(w + size_t(r) * k, k, group, flags, codes + size_t(r) * (k / 4), scales + size_t(r) * ng,
                    alpha + r, beta + r, sq_err ? &errs[r] : nullptr);
+    });
+    if (sq_err) {
+        double e = 0.0;
+        for (double v : errs) e += v;
+        *sq_err = e;
+    }
+    return CCQ_OK;
+}
+
+extern "C" ccq_status ccq_encode_host_q4(const float *w, int32_t n, int32_t k, int32_t group, uint32_t flags,
+                                         int32_t threads, uint8_t *codes, uint8_t *scale_q4, float *super_scale,
+                                         float *alpha, float *beta, double *sq_err) {
+    if (!w || !codes || !scale_q4 || !super_scale || !alpha || !beta) return CCQ_ERR_INVALID_ARG;
+    if (n < 0 || k <= 0 || group <= 0 || group % 4 || k % (2 * group)) return CCQ_ERR_INVALID_ARG;
+    if (flags & ~uint32_t(CCQ_ENC_LITERAL_EQ1)) return CCQ_ERR_INVALID_ARG;
+    if (n == 0) { if (sq_err) *sq_err = 0.0; return CCQ_OK; }
+    std::vector<double> errs(sq_err ? size_t(n) : 0);
+    const int ng = k / group;
+    parallel_rows(n, threads, [&](int r) {
+        std::vector<float> sc(ng);
+        std::vector<uint8_t> q(ng);
+        encode_row(w + size_t(r) * k, k, group, flags, codes + size_t(r) * (k / 4), sc.data(), alpha + r, beta + r,
+                   sq_err ? &errs[r] : nullptr, q.data(), super_scale + r);
+        uint8_t *dst = scale_q4 + size_t(r) * (ng / 2);
+        for (int b = 0; b < ng / 2; ++b) dst[b] = uint8_t(q[2 * b] | (q[2 * b + 1] << 4));
     });
     if (sq_err) {
         double e = 0.0;

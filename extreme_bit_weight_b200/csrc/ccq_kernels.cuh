@@ -55,6 +55,10 @@ struct DecodeGemmParams {
     int I;                // EPI_GATEUP: gate rows per expert
     int tma_scales;       // 1: scales staged by TMA with the codes (row pitch a multiple of 16 B)
     int w4;               // 1: W4 per-channel codes (two per byte), scales[row]
+    // 1: 4-bit group scales s = fl32(q4 * super[row]) (two per byte, even group in the low nibble)
+    int q4;
+    const uint8_t *scale_q4;   // [rows_total][K/128]
+    const float *super_scale;  // [rows_total]
     uint32_t *err;
     // work units (set by the launcher): unit u = (expert, k split, row block), row block fastest
     int row_blocks, ksplit, units;
@@ -102,6 +106,9 @@ struct TcGemmParams {
     const float *rw;       // EPI_DOWN: routing weight per operand row
     int I;                 // EPI_GATEUP: gate rows per expert
     int w4;                // 1: W4 per-channel codes (two per byte), scales[row]
+    int q4;                // 1: 4-bit group scales (see DecodeGemmParams)
+    const uint8_t *scale_q4;
+    const float *super_scale;
     uint32_t *err;
     // split-K (dense matmul with few tiles): ksplit > 1 splits the 64-column groups into ranges of
     // kg groups (a multiple of 4); each range writes EPI_PARTIAL_F32 sums at out + ks*out_split_stride
@@ -116,7 +123,8 @@ cudaError_t launch_build_tiles(const int *seg_off, int E, int m_tile, int2 *list
 cudaError_t launch_pack_xt(const uint16_t *x, const int *tok_of, int P_valid, int K, uint16_t *xt, cudaStream_t s);
 
 cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, const float *alpha,
-                           const float *beta, int rows, int K, uint16_t *out, cudaStream_t s);
+                           const float *beta, int rows, int K, uint16_t *out, cudaStream_t s,
+                           const uint8_t *scale_q4 = nullptr, const float *super = nullptr);
 
 // x (BF16 [rows][K], row r taken from x[tok_of ? tok_of[p] : p]) -> XA operand + group sums.
 cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,

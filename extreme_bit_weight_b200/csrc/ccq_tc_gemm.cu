@@ -224,7 +224,7 @@ __device__ __forceinline__ bool tile_of(const TcGemmParams &p, int w, TileInfo &
     return true;
 }
 
-template <int MT, bool W4>
+template <int MT, bool W4, bool Q4 = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_codes,
                   const TcGemmParams p) {
@@ -372,8 +372,18 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             const float sc_row = W4 ? bf16_bits_to_float(float_to_bf16_bits(__ldg(srow))) : 0.0f;
             // W2 group scales, four groups (one code stage) at a time and one stage ahead, so the
             // global read is off the decode's critical path
+            const float sup_row = Q4 ? __ldg(p.super_scale + grow) : 0.0f;
             auto load_sc4 = [&](int g0) -> float4 {
                 if (W4 || g0 >= nk) return make_float4(0.f, 0.f, 0.f, 0.f);
+                if (Q4) {
+                    // 4-bit group scales: groups g0..g0+3 in two bytes (even group in the low nibble)
+                    const int qpr = p.K / 128;
+                    const uint8_t *qrow = p.scale_q4 + grow * (size_t)qpr;
+                    const uint32_t b0 = g0 / 2 < qpr ? __ldg(qrow + g0 / 2) : 0u;
+                    const uint32_t b1 = g0 / 2 + 1 < qpr ? __ldg(qrow + g0 / 2 + 1) : 0u;
+                    return make_float4(__fmul_rn((float)(b0 & 0xFu), sup_row), __fmul_rn((float)(b0 >> 4), sup_row),
+                                       __fmul_rn((float)(b1 & 0xFu), sup_row), __fmul_rn((float)(b1 >> 4), sup_row));
+                }
                 if ((nk & 3) == 0) return __ldg(reinterpret_cast<const float4 *>(srow + g0));
                 return make_float4(__ldg(srow + g0), g0 + 1 < nk ? __ldg(srow + g0 + 1) : 0.f,
                                    g0 + 2 < nk ? __ldg(srow + g0 + 2) : 0.f, g0 + 3 < nk ? __ldg(srow + g0 + 3) : 0.f);
@@ -583,7 +593,7 @@ __global__ void pack_xt_kernel(const uint16_t *__restrict__ x, const int *__rest
 
 template <int MT>
 cudaError_t launch_tc_mt(const TcGemmParams &p, const CUtensorMap &ta, const CUtensorMap &tc, int grid, cudaStream_t s) {
-    auto kern = p.w4 ? tc_gemm_w2_kernel<MT, true> : tc_gemm_w2_kernel<MT, false>;
+    auto kern = p.w4 ? tc_gemm_w2_kernel<MT, true> : p.q4 ? tc_gemm_w2_kernel<MT, false, true> : tc_gemm_w2_kernel<MT, false>;
     const int smem = TcSmem<MT>::kTotal;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;

@@ -59,12 +59,20 @@ typedef enum {
  *   nibble ("GPTQ and AWQ" lesson, pack_int4 layout); one scale per output row
  *   (WINT2 page, quantization_config "wint4" / "per_channel"):
  *     codes[n][k/2] uint8, scales[n] fp32; w = bf16_rn(sext4(nibble) * bf16_rn(scales[n])).
+ * CCQ_FMT_W2_CCQ_G64_Q4SCALE: the CCQ paper's 2.06-bpw form of CCQ_FMT_W2_CCQ_G64 (§3.4 "Scale
+ *   Compression", Eq. 5, Algorithm 3 first line: s = ((s_q >> s_shift) & 0xF) * s_super).  The
+ *   codes, alpha and beta are as for CCQ_FMT_W2_CCQ_G64; the group scales are 4-bit:
+ *     scale_q4[n][k/128] uint8, group g in byte g/2, the low nibble holding the even group;
+ *     super_scale[n] fp32;
+ *     group scale s = fl32(q4 * super_scale[n]) (one fp32 multiply), then the same weight rule
+ *     w = bf16_rn((u - 32) * bf16_rn(s)).  `scales` is unused (NULL).  k must be a multiple of 128.
  */
-enum { CCQ_FMT_W2_CCQ_G64 = 1, CCQ_FMT_W4_PER_CHANNEL = 2 };
+enum { CCQ_FMT_W2_CCQ_G64 = 1, CCQ_FMT_W4_PER_CHANNEL = 2, CCQ_FMT_W2_CCQ_G64_Q4SCALE = 3 };
 
 /* One linear layer, or `num_experts` layers of the same shape stacked back to back: expert e's
  * arrays start at codes + e*n*(k/4) (W2) or e*n*(k/2) (W4), scales + e*n*(k/64) (W2) or e*n (W4),
- * alpha/beta + e*n.  All device pointers, 16-byte aligned.  y = x W^T: W is [n][k]. */
+ * alpha/beta/super_scale + e*n, scale_q4 + e*n*(k/128).  All device pointers, 16-byte aligned.
+ * y = x W^T: W is [n][k]. */
 typedef struct {
     int32_t fmt;          /* CCQ_FMT_* */
     int32_t n;            /* output features (rows of W), multiple of 16 */
@@ -74,6 +82,8 @@ typedef struct {
     const float *scales;  /* (device) group scales (W2) or channel scales (W4) */
     const float *alpha;   /* (device) W2 code scale per row; NULL for W4 */
     const float *beta;    /* (device) W2 code zero-point per row; NULL for W4 */
+    const uint8_t *scale_q4;   /* (device) Q4SCALE: packed 4-bit group scales; NULL otherwise */
+    const float *super_scale;  /* (device) Q4SCALE: super scale per row; NULL otherwise */
 } ccq_weight;
 
 /* Encoder flags for ccq_encode_host. */
@@ -99,6 +109,19 @@ enum {
 ccq_status ccq_encode_host(const float *w, int32_t n, int32_t k, int32_t group, uint32_t flags,
                            int32_t threads, uint8_t *codes, float *scales, float *alpha, float *beta,
                            double *sq_err);
+
+/* ccq_encode_host_q4 - ccq_encode_host for CCQ_FMT_W2_CCQ_G64_Q4SCALE (CCQ §3.4 "Scale
+ * Compression"; the pages give no quantizer for the 4-bit scales, this is the plain reading):
+ *   raw group scale r_g = max|w_g|/31 (fp32); super_scale[n] = max_g r_g / 15 (fp32);
+ *   q4_g = clip(round_half_even(r_g / super), 0, 15) (in fp64); the codes are then searched and
+ *   clustered exactly as by ccq_encode_host at the group scales fl32(q4_g * super).
+ *   w (host) fp32 [n][k], k % 128 == 0 (group 64); flags: CCQ_ENC_LITERAL_EQ1 only (the Eq. 4
+ *   refit does not apply to a quantized scale); codes (host) out [n][k/4]; scale_q4 (host) out
+ *   [n][k/128]; super_scale, alpha, beta (host) out fp32 [n]; sq_err as for ccq_encode_host.
+ * Returns CCQ_ERR_INVALID_ARG on null pointers, bad shapes or flags. */
+ccq_status ccq_encode_host_q4(const float *w, int32_t n, int32_t k, int32_t group, uint32_t flags,
+                              int32_t threads, uint8_t *codes, uint8_t *scale_q4, float *super_scale,
+                              float *alpha, float *beta, double *sq_err);
 
 /* ccq_quantize_w4_host - W4 per-channel round-to-nearest ("GPTQ and AWQ" Part 2 rtn/pack_int4):
  * s = bf16(max|w_row|/7), q = clip(round_half_even(w/s), -8, 7) (w/s in fp64), two codes per byte,

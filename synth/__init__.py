@@ -96,6 +96,17 @@ def w2_format_random(n: int, k: int, seed: int, group: int = 64, scale_std: floa
     return codes, scales, alpha, beta
 
 
+def w2q4_format_random(n: int, k: int, seed: int, group: int = 64, scale_std: float = 0.02):
+    """Random well-formed parameters of the 4-bit-scale W2 format: codes, alpha and beta as
+    w2_format_random; 4-bit group scales uniform over 0..15 packed two per byte (even group in
+    the low nibble); per-channel super scales of the magnitude a N(0, scale_std^2) row gives."""
+    codes, _, alpha, beta = w2_format_random(n, k, seed, group, scale_std)
+    g = rng(seed + 7)
+    sq = g.integers(0, 256, size=(n, k // (2 * group)), dtype=np.uint8)
+    sup = (np.abs(g.normal(3.0, 0.3, size=n)) * scale_std / 31.0 / 15.0).astype(np.float32)
+    return codes, sq, sup, alpha, beta
+
+
 def w4_format_random(n: int, k: int, seed: int, scale_std: float = 0.02):
     """Random W4 per-channel parameters: codes uniform bytes (two signed nibbles), scales of the
     magnitude a N(0, scale_std^2) row gives."""

@@ -90,6 +90,22 @@ def test_encoder_matches_oracle(ccq):
         assert abs(err - oracle.w2_sq_error(w, c, s, a, b)) <= 1e-12 * max(err, 1e-30)
 
 
+def test_encoder_q4_matches_oracle(ccq):
+    # the 4-bit-scale encoder (CCQ §3.4 Scale Compression) vs the oracle's: identical bytes
+    w = synth.weights_normal(6, 256, 103)
+    w[3, 64:128] = 0.0  # one all-zero group (scale 0)
+    for flags in (0, ccq.CCQ_ENC_LITERAL_EQ1):
+        c, sq, sup, a, b, err = ccq.ccq_encode_host_q4(w, 64, flags, threads=3)
+        oc, osq, osup, oa, ob = oracle.encode_w2q4(w, 64, flags)
+        assert np.array_equal(sup, osup) and np.array_equal(sq, osq)
+        assert np.array_equal(a, oa) and np.array_equal(b, ob)
+        assert np.array_equal(c, oc)
+    with pytest.raises(ccq.CcqError):
+        ccq.ccq_encode_host_q4(w, 64, ccq.CCQ_ENC_REFIT_SCALE)
+    with pytest.raises(ccq.CcqError):
+        ccq.ccq_encode_host_q4(np.zeros((2, 192), np.float32), 64)  # k not a multiple of 128
+
+
 def test_encoder_rejects_bad_args(ccq):
     w = np.zeros((2, 100), np.float32)
     with pytest.raises(ccq.CcqError):

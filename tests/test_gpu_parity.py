@@ -329,6 +329,9 @@ def test_gemm_w4_shapes(ccq, m, n, k):
 
 def moe_weights_fmt(ccq, E, H, I, seed, fmt13, fmt2):
     def make(rows, k, s, fmt):
+        if fmt == 3:  # CCQ W2 with 4-bit group scales
+            c, sq, sup, a, b = synth.w2q4_format_random(rows, k, s)
+            return q4_weight(ccq, c, sq, sup, a, b, experts=E), oracle.dequant_w2q4(c, sq, sup, a, b)
         if fmt == 4:
             c, sc = synth.w4_format_random(rows, k, s)
             return (ccq.CcqWeight(ccq.CCQ_FMT_W4_PER_CHANNEL, rows // E, k, c, sc, experts=E),
@@ -376,3 +379,66 @@ def test_mixed_stack_layer_by_layer(ccq, M):
         assert rel_err(y.float().cpu().numpy(), ref) <= TOL, layer
         yf = y.float()
         x = (yf * torch.rsqrt(yf.pow(2).mean(dim=1, keepdim=True) + 1e-12)).to(torch.bfloat16)
+
+
+# ----------------------------------------------------------------------------------------------
+# CCQ W2 with 4-bit group scales (CCQ §3.4 Scale Compression; 2.06 bpw)
+# ----------------------------------------------------------------------------------------------
+def q4_weight(ccq, codes, sq, sup, alpha, beta, experts=1):
+    n = codes.shape[0] // experts
+    return ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64_Q4SCALE, n, codes.shape[1] * 4, codes, None, alpha, beta,
+                         experts=experts, scale_q4=sq, super_scale=sup)
+
+
+@pytest.mark.parametrize("n,k,E", [(16, 128, 1), (48, 384, 3), (272, 640, 2), (1024, 8192, 1)])
+def test_dequant_q4_bitexact(ccq, n, k, E):
+    codes, sq, sup, a, b = synth.w2q4_format_random(n * E, k, 6000 + n + k)
+    W = q4_weight(ccq, codes, sq, sup, a, b, experts=E)
+    got = bits_of(ccq.ccq_dequant_bf16(W)).reshape(n * E, k)
+    assert np.array_equal(got, oracle.dequant_w2q4(codes, sq, sup, a, b))
+
+
+def test_dequant_q4_encoded_bitexact(ccq):
+    w = synth.weights_normal(64, 512, 6001)
+    codes, sq, sup, a, b, _ = ccq.ccq_encode_host_q4(w, 64)
+    got = bits_of(ccq.ccq_dequant_bf16(q4_weight(ccq, codes, sq, sup, a, b)))[0]
+    assert np.array_equal(got, oracle.dequant_w2q4(codes, sq, sup, a, b))
+
+
+def test_gemm_q4_one_hot_identity_both_paths(ccq):
+    n, k = 272, 640  # 5 scale bytes per row: odd, and a stage that ends inside the row
+    codes, sq, sup, a, b = synth.w2q4_format_random(n, k, 6100)
+    W = q4_weight(ccq, codes, sq, sup, a, b)
+    ref = oracle.bf16_to_f64(oracle.dequant_w2q4(codes, sq, sup, a, b)).T.astype(np.float32)
+    eye = synth.one_hot_rows(k).cuda()
+    for j in range(0, k, 16):  # register-decode mma.sync kernel
+        y = ccq.ccq_w2a16_gemm(W, eye[j:j + 16].contiguous()).float().cpu().numpy()
+        assert np.array_equal(y, ref[j:j + 16]), j
+    y = ccq.ccq_w2a16_gemm(W, eye).float().cpu().numpy()  # tcgen05 kernel
+    assert np.array_equal(y, ref)
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 256, 512), (9, 272, 640), (16, 1024, 2048), (64, 512, 1024),
+                                   (300, 272, 640), (1, 8192, 8192), (128, 8192, 8192)])
+def test_gemm_q4_shapes(ccq, m, n, k):
+    codes, sq, sup, a, b = synth.w2q4_format_random(n, k, 6200 + m + n)
+    W = q4_weight(ccq, codes, sq, sup, a, b)
+    x = synth.activations(m, k, 6201 + m)
+    y = ccq.ccq_w2a16_gemm(W, x.cuda()).float().cpu().numpy()
+    ref = oracle.gemm_f64(synth.bf16_bits(x), oracle.dequant_w2q4(codes, sq, sup, a, b))
+    e = rel_err(y, ref)
+    assert e <= TOL
+    assert e <= 4e-3
+
+
+@pytest.mark.parametrize("fmts", [(3, 3), (3, 2), (2, 3), (4, 3)])
+@pytest.mark.parametrize("T", [6, 300])
+def test_moe_q4_formats(ccq, fmts, T):
+    E, H, I, topk = 8, 512, 256, 2
+    W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 6300 + T + 10 * fmts[0] + fmts[1], *fmts)
+    x = synth.activations(T, H, 6301 + T)
+    ids, rw = synth.routing_uniform(T, E, topk, 6302 + T)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    ref = oracle.moe_f64(synth.bf16_bits(x), d13, d2, ids, rw, round_h=True)
+    assert rel_err(y, ref) <= TOL
