@@ -31,6 +31,7 @@ DISTINCT = 2          # experts encoded from N(0, 0.02) weights; the rest are de
 NOMINAL_HBM_GBS = 8000.0
 METRIC = "W2A16 MoE layer tokens/s; packed-weight HBM GB/s (% of 8 TB/s), 1 B200"
 WORKLOAD = "moe_ffn_decode_T32_H8192_I3584_E64_top8_ccq_w2_g64"
+SCALES = "fp32"       # group scale storage: fp32 (the benchmark format) or q4 (CCQ's 2.06-bpw form)
 
 
 def parse():
@@ -47,13 +48,18 @@ def parse():
                          "Zipf(1.1) routing, 1%% of channels x20 (tcgen05 path, tensor roofline); gemm: one "
                          "dense 8192x8192 W2 linear at --m tokens; stack: 8 MoE layers (2 W4 + 6 W2) at --m tokens")
     ap.add_argument("--m", type=int, default=0, help="tokens for --workload gemm (default 1) / stack (default 32)")
+    ap.add_argument("--scales", default="fp32", choices=["fp32", "q4"],
+                    help="W2 group scales: fp32 (default) or 4-bit x per-channel super scale (2.06 bpw)")
     args = ap.parse_args()
-    global T, E, WORKLOAD
+    global T, E, WORKLOAD, SCALES
+    SCALES = args.scales
     if args.workload == "prefill":
         T = 4096
         WORKLOAD = "moe_ffn_prefill_T4096_zipf1.1_H8192_I3584_E64_top8_ccq_w2_g64"
     if args.profile_small:
         T, E = (8, 16) if args.workload == "decode" else (512, 16)
+    if SCALES == "q4":
+        WORKLOAD = WORKLOAD.replace("ccq_w2_g64", "ccq_w2_g64_q4scale")
     return args
 
 
@@ -118,7 +124,9 @@ def config_dict():
     return {
         "workload": WORKLOAD,
         "tokens": T, "hidden": H, "intermediate": I, "experts": E, "topk": TOPK,
-        "weight_format": "CCQ (6,4,3) code cluster, 4 weights/byte, fp32 group-64 scales",
+        "weight_format": "CCQ (6,4,3) code cluster, 4 weights/byte, " + (
+            "4-bit group-64 scales x fp32 per-channel super scale (2.06 bpw)" if SCALES == "q4" else
+            "fp32 group-64 scales"),
         "routing": ("Zipf(1.1) expert popularity, top-8 by Gumbel-max; " if prefill else "uniform distinct top-8, ")
                    + "softmax of N(0,1) logits",
         "activations": "BF16 N(0,1)" + (", 1% of channels x20" if prefill else ""),
@@ -134,26 +142,38 @@ def config_dict():
 def make_layer(ccq, torch, device):
     import synth
 
+    q4 = SCALES == "q4"
+
     def enc(rows, cols, seed):
         w = synth.weights_normal(rows, cols, seed)
+        if q4:
+            c, sq, sup, a, b, _ = ccq.ccq_encode_host_q4(w, 64, 0, 0)
+            return c, sq, a, b, sup
         c, s, a, b, _ = ccq.ccq_encode_host(w, 64, 0, 0)
-        return c, s, a, b
+        return c, s, a, b, None
 
     parts13 = [enc(2 * I, H, 3100 + e) for e in range(DISTINCT)]
     parts2 = [enc(H, I, 3200 + e) for e in range(DISTINCT)]
 
     def stack(parts, n, k):
         codes = torch.empty((E * n, k // 4), dtype=torch.uint8, device=device)
-        scales = torch.empty((E * n, k // 64), dtype=torch.float32, device=device)
+        scales = (torch.empty((E * n, k // 128), dtype=torch.uint8, device=device) if q4 else
+                  torch.empty((E * n, k // 64), dtype=torch.float32, device=device))
         alpha = torch.empty((E * n,), dtype=torch.float32, device=device)
         beta = torch.empty((E * n,), dtype=torch.float32, device=device)
-        dev = [tuple(torch.from_numpy(a).to(device) for a in p) for p in parts]
+        sup = torch.empty((E * n,), dtype=torch.float32, device=device) if q4 else None
+        dev = [tuple(None if a is None else torch.from_numpy(a).to(device) for a in p) for p in parts]
         for e in range(E):
-            c, s, a, b = dev[e % len(dev)]
+            c, s, a, b, su = dev[e % len(dev)]
             codes[e * n:(e + 1) * n].copy_(c)
             scales[e * n:(e + 1) * n].copy_(s)
             alpha[e * n:(e + 1) * n].copy_(a)
             beta[e * n:(e + 1) * n].copy_(b)
+            if q4:
+                sup[e * n:(e + 1) * n].copy_(su)
+        if q4:
+            return ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64_Q4SCALE, n, k, codes, None, alpha, beta, experts=E,
+                                 device=device, scale_q4=scales, super_scale=sup)
         return ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, n, k, codes, scales, alpha, beta, experts=E, device=device)
 
     W13 = stack(parts13, 2 * I, H)
@@ -162,9 +182,14 @@ def make_layer(ccq, torch, device):
 
 
 def touched_bytes(ids):
-    """Algorithmic packed-weight bytes of one step: codes + scales + alpha/beta of touched experts."""
-    per13 = 2 * I * (H // 4) + 2 * I * (H // 64) * 4 + 2 * I * 8
-    per2 = H * (I // 4) + H * (I // 64) * 4 + H * 8
+    """Algorithmic packed-weight bytes of one step: codes + scales + per-row constants (alpha, beta;
+    q4: and the super scale) of the touched experts."""
+    if SCALES == "q4":
+        per13 = 2 * I * (H // 4) + 2 * I * (H // 128) + 2 * I * 12
+        per2 = H * (I // 4) + H * (I // 128) + H * 12
+    else:
+        per13 = 2 * I * (H // 4) + 2 * I * (H // 64) * 4 + 2 * I * 8
+        per2 = H * (I // 4) + H * (I // 64) * 4 + H * 8
     ne = len(set(int(v) for v in np.asarray(ids).ravel()))
     return ne * per13, ne * per2, ne
 
@@ -447,7 +472,7 @@ def run_ours(args, rank, world, local):
             {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (fused MoE: gate/up + SiLU, then down)",
              "achieved": (b13 + b2) / (gemm1_ms * 1e-3) / 1e9, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)",
              "unit": "GB/s", "frac": (b13 + b2) / (gemm1_ms * 1e-3) / 1e9 / hbm,
-             "traffic": FUSED_DECODE_DRAM_BYTES_PER_EXPERT * ne,
+             "traffic": FUSED_DECODE_DRAM_BYTES_PER_EXPERT * ne if SCALES == "fp32" else None,
              "traffic_source": "ncu dram__bytes_read+write of the 16-expert capture, scaled by touched experts",
              "launch_ms": gemm1_ms, "algorithmic_bytes_per_launch": b13 + b2} if fused else
             {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (gate/up, SiLU epilogue)",
@@ -500,11 +525,18 @@ def run_gemm(args, rank, world, local):
     torch.cuda.set_device(device)
     M, KD, ND = (args.m or 1), 8192, 8192
     w = synth.weights_normal(ND, KD, 4100)
-    c, sc, al, be, _ = ccq.ccq_encode_host(w, 64, 0, 0)
-    per_copy = c.nbytes + sc.nbytes + al.nbytes + be.nbytes
+    if SCALES == "q4":
+        c, sq, sup, al, be, _ = ccq.ccq_encode_host_q4(w, 64, 0, 0)
+        per_copy = c.nbytes + sq.nbytes + sup.nbytes + al.nbytes + be.nbytes
+        mk = lambda: ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64_Q4SCALE, ND, KD, c, None, al, be, device=device,
+                                   scale_q4=sq, super_scale=sup)
+    else:
+        c, sc, al, be, _ = ccq.ccq_encode_host(w, 64, 0, 0)
+        per_copy = c.nbytes + sc.nbytes + al.nbytes + be.nbytes
+        mk = lambda: ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, ND, KD, c, sc, al, be, device=device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     R = max(2, -(-2 * l2 // per_copy))
-    Ws = [ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, ND, KD, c, sc, al, be, device=device) for _ in range(R)]
+    Ws = [mk() for _ in range(R)]
     x = synth.activations(M, KD, 4101).to(device)
     y = torch.empty((M, ND), dtype=torch.bfloat16, device=device)
     ws = ccq.workspace(max(ccq.ccq_gemm_workspace_size(Ws[0], M), 256), device)
@@ -538,7 +570,8 @@ def run_gemm(args, rank, world, local):
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "us_per_call": 1000.0 * ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": f"dense_gemm_M{M}_K8192_N8192_ccq_w2_g64", "m": M, "k": KD, "n": ND,
+            "config": {"workload": f"dense_gemm_M{M}_K8192_N8192_ccq_w2_g64" + ("_q4scale" if SCALES == "q4" else ""),
+                       "m": M, "k": KD, "n": ND,
                        "weights": "N(0,0.02) encoded by ccq_encode_host",
                        "l2": f"{R} rotating weight copies ({R * per_copy / 1e6:.0f} MB) vs {l2 / 1e6:.0f} MB L2"},
             "packed_weight_gbs": gbs, "roofline": roof,
@@ -585,7 +618,8 @@ def run_stack(args, rank, world, local):
     def clone(w):  # a layer of its own memory with the same contents
         cp = lambda t: None if t is None else t.clone()
         return ccq.CcqWeight(w.fmt, w.n, w.k, cp(w.codes), cp(w.scales), cp(w.alpha), cp(w.beta),
-                             experts=w.experts, device=device)
+                             experts=w.experts, device=device, scale_q4=cp(w.scale_q4),
+                             super_scale=cp(w.super_scale))
 
     w2_first = make_layer(ccq, torch, device)
     layers = ([w4_layer(4200) for _ in range(2)] + [w2_first] +

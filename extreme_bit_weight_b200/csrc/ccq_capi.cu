@@ -561,11 +561,13 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p2.scale_q4 = w2->scale_q4;
     p2.super_scale = w2->super_scale;
 
-    // Both projections W2 with TMA-staged scales and the same token tiling: one fused launch, in
+    // Both projections W2 (both with TMA-staged fp32 scales, or both with 4-bit scales) and the same
+    // token tiling: one fused launch, in
     // which the gate/up epilogue also writes h's group-sum table and each down unit starts once
     // its expert's gate/up units are done.  Otherwise (or if the device refuses the cooperative
     // launch) two launches with the group sums computed in between.
-    bool fused = !p1.w4 && !p2.w4 && p1.tma_scales && p2.tma_scales && nt1 == nt2;
+    bool fused = !p1.w4 && !p2.w4 && nt1 == nt2 &&
+                 ((p1.tma_scales && p2.tma_scales && !p1.q4 && !p2.q4) || (p1.q4 && p2.q4));
     if (fused) {
         p1.dep = dep;
         p1.fuse_gsq = gs_h;

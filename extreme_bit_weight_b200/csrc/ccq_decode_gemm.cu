@@ -914,8 +914,9 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
 template <int NT>
 cudaError_t launch_fused_nt(const DecodeGemmParams &p1, const MapSet &m1, int row_blocks1, const DecodeGemmParams &p2,
                             const MapSet &m2, int row_blocks2, int experts, cudaStream_t s) {
-    DecodeKernel kern = decode_gemm_w2_kernel<NT, true, false, true>;
-    const int smem = Smem<NT, false>::kTotal;
+    // fp32 group scales staged by TMA, or 4-bit scales read by the consumers (both projections alike)
+    DecodeKernel kern = p1.q4 ? decode_gemm_w2_kernel<NT, false, false, true, true> : decode_gemm_w2_kernel<NT, true, false, true>;
+    const int smem = p1.q4 ? Smem<NT, false, true>::kTotal : Smem<NT, false>::kTotal;
     cudaError_t err = prepare_kernel(kern, smem);
     if (err != cudaSuccess) return err;
     DecodeGemmParams q1 = p1, q2 = p2;
@@ -962,7 +963,8 @@ cudaError_t launch_decode_moe_fused(const DecodeGemmParams &p1, const CUtensorMa
                                     const DecodeGemmParams &p2, const CUtensorMap &a2, const CUtensorMap &b2,
                                     const CUtensorMap &c2, const CUtensorMap &d2, int row_blocks2, int experts,
                                     int nt, cudaStream_t s) {
-    if (p1.w4 || p2.w4 || p1.q4 || p2.q4 || !p1.tma_scales || !p2.tma_scales || p1.mode != EPI_GATEUP || p2.mode != EPI_DOWN ||
+    const bool fp32_sc = !p1.q4 && !p2.q4 && p1.tma_scales && p2.tma_scales, q4_sc = p1.q4 && p2.q4;
+    if (p1.w4 || p2.w4 || !(fp32_sc || q4_sc) || p1.mode != EPI_GATEUP || p2.mode != EPI_DOWN ||
         !p1.dep || !p2.dep || !p1.fuse_gsq)
         return cudaErrorInvalidValue;
     const MapSet m1{a1, b1, c1, d1}, m2{a2, b2, c2, d2};

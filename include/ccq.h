@@ -195,7 +195,8 @@ ccq_status ccq_moe_w2a16_forward(const ccq_weight *w13, const ccq_weight *w2, in
  * between its steps, for per-kernel timing: events[0] before routing, [1] after routing,
  * [2] after activation packing, [3] after the gate/up kernel, [4] after the group-sum kernel,
  * [5] after the down kernel, [6] after the combine.  When the decode-sized path runs both
- * projections as one fused launch (W2 weights on both, group-scale rows a multiple of 16 bytes),
+ * projections as one fused launch (W2 weights on both, with fp32 group-scale rows a multiple of 16
+ * bytes on both or 4-bit scales on both),
  * [3], [4] and [5] are all recorded after that launch.  `events` (host) holds
  * CCQ_MOE_TRACE_POINTS cudaEvent_t handles created by the caller (NULL: no events).  No paper
  * counterpart: a measurement hook. */
