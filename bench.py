@@ -27,7 +27,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 T, H, I, E, TOPK = 32, 8192, 3584, 64, 8
-DISTINCT = 2          # experts encoded from N(0, 0.02) weights; the rest are device copies of them
+DISTINCT = 2          # 4-bit-scale format: experts encoded on the host, the rest device copies of them
 NOMINAL_HBM_GBS = 8000.0
 METRIC = "W2A16 MoE layer tokens/s; packed-weight HBM GB/s (% of 8 TB/s), 1 B200"
 WORKLOAD = "moe_ffn_decode_T32_H8192_I3584_E64_top8_ccq_w2_g64"
@@ -130,7 +130,8 @@ def config_dict():
         "routing": ("Zipf(1.1) expert popularity, top-8 by Gumbel-max; " if prefill else "uniform distinct top-8, ")
                    + "softmax of N(0,1) logits",
         "activations": "BF16 N(0,1)" + (", 1% of channels x20" if prefill else ""),
-        "weights": f"N(0,0.02) encoded by ccq_encode_host for {DISTINCT} experts, copied to all {E}",
+        "weights": (f"N(0,0.02) encoded by ccq_encode_host_q4 for {DISTINCT} experts, copied to all {E}"
+                    if SCALES == "q4" else f"N(0,0.02) per expert (seeded device RNG), all {E} encoded by ccq_encode_device"),
         "l2": "inputs larger than L2: ~1.74 GB of packed weights touched per step vs 126 MB L2",
         "parallelism": "replicas",
     }
@@ -139,10 +140,34 @@ def config_dict():
 # ------------------------------------------------------------------------------------------------
 # inputs
 # ------------------------------------------------------------------------------------------------
+def make_layer_device(ccq, torch, device, seed_base: int = 3100):
+    """Every expert its own N(0, 0.02) weights (seeded device RNG), encoded by ccq_encode_device."""
+    def stack(n, k, seed):
+        codes = torch.empty((E * n, k // 4), dtype=torch.uint8, device=device)
+        scales = torch.empty((E * n, k // 64), dtype=torch.float32, device=device)
+        alpha = torch.empty((E * n,), dtype=torch.float32, device=device)
+        beta = torch.empty((E * n,), dtype=torch.float32, device=device)
+        ws = ccq.workspace(ccq._lib.ccq_encode_device_workspace_size(n, k), device)
+        g = torch.Generator(device=device)
+        for e in range(E):
+            g.manual_seed(seed + e)
+            w = torch.randn((n, k), generator=g, device=device, dtype=torch.float32) * 0.02
+            c, s, a, b = ccq.ccq_encode_device(w, 64, 0, ws=ws)
+            codes[e * n:(e + 1) * n].copy_(c)
+            scales[e * n:(e + 1) * n].copy_(s)
+            alpha[e * n:(e + 1) * n].copy_(a)
+            beta[e * n:(e + 1) * n].copy_(b)
+        return ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, n, k, codes, scales, alpha, beta, experts=E, device=device)
+
+    return stack(2 * I, H, seed_base), stack(H, I, seed_base + 100)
+
+
 def make_layer(ccq, torch, device):
     import synth
 
     q4 = SCALES == "q4"
+    if not q4:
+        return make_layer_device(ccq, torch, device)
 
     def enc(rows, cols, seed):
         w = synth.weights_normal(rows, cols, seed)
@@ -660,8 +685,9 @@ def run_stack(args, rank, world, local):
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"moe_stack_8layers_M{M}_H8192_I3584_E64_top8_w4x2_w2x6", "m": M,
-                       "weights": f"W4: N(0,0.02) quantized by ccq_quantize_w4_host; W2: ccq_encode_host; "
-                                  f"{DISTINCT} distinct experts per layer copied to all {E}",
+                       "weights": f"W4: N(0,0.02) quantized by ccq_quantize_w4_host for {DISTINCT} experts, copied "
+                                  f"to all {E}; W2: all {E} experts encoded by ccq_encode_device, layers 3-7 "
+                                  f"device copies of layer 2",
                        "l2": f"{nbytes / 1e9:.2f} GB of packed weights touched per step vs 126 MB L2"},
             "roofline": roof, "clocks": clk}
     if rank == 0:

@@ -65,6 +65,9 @@ _lib.ccq_status_string.restype = ctypes.c_char_p
 _lib.ccq_build_info.restype = ctypes.c_char_p
 _lib.ccq_encode_host.argtypes = [_P, _I, _I, _I, ctypes.c_uint32, _I, _P, _P, _P, _P, _P]
 _lib.ccq_quantize_w4_host.argtypes = [_P, _I, _I, _I, _P, _P]
+_lib.ccq_encode_device_workspace_size.argtypes = [_I, _I]
+_lib.ccq_encode_device_workspace_size.restype = ctypes.c_size_t
+_lib.ccq_encode_device.argtypes = [_P, _I, _I, _I, ctypes.c_uint32, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.ccq_encode_host_q4.argtypes = [_P, _I, _I, _I, ctypes.c_uint32, _I, _P, _P, _P, _P, _P, _P]
 _lib.ccq_dequant_bf16.argtypes = [ctypes.POINTER(ccq_weight), _I, _P, _P]
 _lib.ccq_gemm_workspace_size.argtypes = [ctypes.POINTER(ccq_weight), _I]
@@ -148,6 +151,23 @@ def ccq_encode_host_q4(w: np.ndarray, group: int = 64, flags: int = 0, threads: 
                                    _np_ptr(sup), _np_ptr(alpha), _np_ptr(beta), ctypes.byref(err)),
            "ccq_encode_host_q4")
     return codes, sq, sup, alpha, beta, err.value
+
+
+def ccq_encode_device(w: torch.Tensor, group: int = 64, flags: int = 0, ws: torch.Tensor = None, stream=None):
+    """CCQ (6,4,3) code-cluster encode of fp32 w [n][k] on the GPU (the same bytes as
+    ccq_encode_host) -> device tensors (codes, scales, alpha, beta)."""
+    w = w.contiguous()
+    n, k = w.shape
+    dev = w.device
+    codes = torch.empty((n, k // 4), dtype=torch.uint8, device=dev)
+    scales = torch.empty((n, k // group), dtype=torch.float32, device=dev)
+    alpha = torch.empty(n, dtype=torch.float32, device=dev)
+    beta = torch.empty(n, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(max(int(_lib.ccq_encode_device_workspace_size(n, k)), 256), dev)
+    _check(_lib.ccq_encode_device(_dptr(w), n, k, group, flags, _dptr(codes), _dptr(scales), _dptr(alpha),
+                                  _dptr(beta), _dptr(ws), ws.numel(), _stream(stream)), "ccq_encode_device")
+    return codes, scales, alpha, beta
 
 
 def ccq_quantize_w4_host(w: np.ndarray, threads: int = 0):

@@ -8,7 +8,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libccq.so")
-SOURCES = ["ccq_capi.cu", "ccq_decode_gemm.cu", "ccq_tc_gemm.cu", "ccq_aux.cu", "ccq_noalloc.cu", "ccq_encode_host.cpp"]
+SOURCES = ["ccq_capi.cu", "ccq_decode_gemm.cu", "ccq_tc_gemm.cu", "ccq_aux.cu", "ccq_noalloc.cu", "ccq_encode_device.cu",
+           "ccq_encode_host.cpp"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -110,6 +110,20 @@ ccq_status ccq_encode_host(const float *w, int32_t n, int32_t k, int32_t group, 
                            int32_t threads, uint8_t *codes, float *scales, float *alpha, float *beta,
                            double *sq_err);
 
+/* ccq_encode_device - ccq_encode_host on the GPU: the same algorithm (CCQ §3.1 Algorithm 1, §3.3
+ * Eq. 1, §3.4 Eq. 4), the same fp64 arithmetic in the same order and the same tie rules, so the
+ * outputs are identical to ccq_encode_host's for the same input and flags.
+ *   w       (device) fp32 [n][k]; group must be 64 (CCQ_ERR_UNSUPPORTED otherwise), k % 64 == 0
+ *   flags   CCQ_ENC_LITERAL_EQ1 and/or CCQ_ENC_REFIT_SCALE
+ *   codes (device) out [n][k/4]; scales (device) out [n][k/64]; alpha, beta (device) out [n]
+ *   ws      (device) scratch of ccq_encode_device_workspace_size(n, k) bytes
+ * Asynchronous on `stream`; argument errors return before any launch.  No paper counterpart as an
+ * interface: the paper encodes offline and does not say where. */
+size_t ccq_encode_device_workspace_size(int32_t n, int32_t k);
+ccq_status ccq_encode_device(const float *w, int32_t n, int32_t k, int32_t group, uint32_t flags,
+                             uint8_t *codes, float *scales, float *alpha, float *beta, void *ws,
+                             size_t ws_bytes, ccq_stream_t stream);
+
 /* ccq_encode_host_q4 - ccq_encode_host for CCQ_FMT_W2_CCQ_G64_Q4SCALE (CCQ §3.4 "Scale
  * Compression"; the pages give no quantizer for the 4-bit scales, this is the plain reading):
  *   raw group scale r_g = max|w_g|/31 (fp32); super_scale[n] = max_g r_g / 15 (fp32);

@@ -442,3 +442,31 @@ def test_moe_q4_formats(ccq, fmts, T):
     assert st == ccq.CCQ_OK
     ref = oracle.moe_f64(synth.bf16_bits(x), d13, d2, ids, rw, round_h=True)
     assert rel_err(y, ref) <= TOL
+
+
+# ----------------------------------------------------------------------------------------------
+# device encoder: identical bytes to the host encoder and the oracle's brute-force Algorithm 1
+# ----------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("n,k", [(6, 128), (33, 576), (64, 1024)])
+def test_encode_device_matches_oracle(ccq, n, k):
+    w = synth.weights_normal(n, k, 7000 + n + k)
+    w[min(2, n - 1), 64:128] = 0.0  # an all-zero group
+    wd = torch.from_numpy(w).cuda()
+    for flags in (0, ccq.CCQ_ENC_LITERAL_EQ1, ccq.CCQ_ENC_REFIT_SCALE,
+                  ccq.CCQ_ENC_LITERAL_EQ1 | ccq.CCQ_ENC_REFIT_SCALE):
+        c, s, a, b = (t.cpu().numpy() for t in ccq.ccq_encode_device(wd, 64, flags))
+        oc, os_, oa, ob = oracle.encode_w2(w, 64, flags)
+        assert np.array_equal(a, oa) and np.array_equal(b, ob), flags
+        assert np.array_equal(s, os_), flags
+        assert np.array_equal(c, oc), flags
+
+
+def test_encode_device_matches_host_at_size(ccq):
+    # a full-width expert slice (the oracle's brute force is too slow here; the host encoder is
+    # itself checked against the oracle): 256 rows of the decode layer's gate/up weight
+    w = synth.weights_normal(256, 8192, 7100)
+    c, s, a, b = (t.cpu().numpy() for t in ccq.ccq_encode_device(torch.from_numpy(w).cuda(), 64, 0))
+    hc, hs, ha, hb, _ = ccq.ccq_encode_host(w, 64, 0)
+    assert np.array_equal(a, ha) and np.array_equal(b, hb)
+    assert np.array_equal(s, hs)
+    assert np.array_equal(c, hc)
