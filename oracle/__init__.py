@@ -58,6 +58,8 @@ def lib():
         L.oracle_dequant_w2.argtypes = [P, P, P, P, i, i, i, P]
         L.oracle_dequant_w4.argtypes = [P, P, i, i, P]
         L.oracle_dequant_w2q4.argtypes = [P, P, P, P, P, i, i, i, P]
+        L.oracle_dequant_w2std.argtypes = [P, P, i, i, i, P]
+        L.oracle_quantize_w2std.argtypes = [P, i, i, i, P, P]
         L.oracle_encode_w2q4.argtypes = [P, i, i, i, ctypes.c_uint32, P, P, P, P, P]
         L.oracle_gemm_bf16_f64.argtypes = [P, P, i, i, i, P]
         L.oracle_gemm_bf16_f64.restype = None
@@ -150,6 +152,29 @@ def dequant_w2q4(codes, scale_q4, super_scale, alpha, beta, group: int = 64) -> 
     if rc != 0:
         raise ValueError("dequant_w2q4: bad shape")
     return out
+
+
+def dequant_w2std(codes, scales, group: int = 64) -> np.ndarray:
+    """WINT2-Standard decode (plain 2-bit fields, zero-point 2, group scales) -> BF16 bits [n][k]."""
+    codes = _c(codes, np.uint8)
+    n, kb = codes.shape
+    k = kb * 4
+    scales = _c(scales, np.float32).reshape(n, k // group)
+    out = np.zeros((n, k), dtype=np.uint16)
+    if lib().oracle_dequant_w2std(_p(codes), _p(scales), n, k, group, _p(out)) != 0:
+        raise ValueError("dequant_w2std: bad shape")
+    return out
+
+
+def quantize_w2std(w, group: int = 64):
+    """WINT2-Standard round-to-nearest -> (codes [n][k/4] u8, scales [n][k/g] f32)."""
+    w = _c(w, np.float32)
+    n, k = w.shape
+    codes = np.zeros((n, k // 4), dtype=np.uint8)
+    scales = np.zeros((n, k // group), dtype=np.float32)
+    if lib().oracle_quantize_w2std(_p(w), n, k, group, _p(codes), _p(scales)) != 0:
+        raise ValueError("quantize_w2std: bad shape")
+    return codes, scales
 
 
 def dequant_w4(codes, scales) -> np.ndarray:

@@ -199,6 +199,66 @@ int oracle_dequant_w2q4(const uint8_t *codes, const uint8_t *scale_q4, const flo
 }
 
 /* ------------------------------------------------------------------------------------------
+ * "WINT2-Standard": plain 2-bit scalar weights, the comparison format of [CCQ] Table 4 (the pages
+ * compare against it but do not define it; reading): codes[n][k/4], field i of byte j (bits 2i,
+ * 2i+1) is weight 4j+i, level q - 2 (zero-point 2 = 2^(bits-1), as the CCQ format's 32 = 2^(L-1)),
+ * group scales scales[n][k/64] used as bf16: w = bf16((q - 2) * bf16(s)).
+ * Quantizer (round to nearest): s = bf16(max|w_g| / 2), q = clip(round_half_even(w / s) + 2, 0, 3)
+ * in fp64 (q = 2 when s = 0).
+ * ------------------------------------------------------------------------------------------ */
+static uint16_t dequant_std_level(int q, float scale)
+{
+    double s = (double)oracle_bf16_to_float(oracle_bf16_bits(scale));
+    return oracle_bf16_bits((float)((double)(q - 2) * s)); /* exact product, one rounding */
+}
+
+int oracle_dequant_w2std(const uint8_t *codes, const float *scales, int n, int k, int group, uint16_t *out)
+{
+    if (n < 0 || k < 0 || group <= 0 || k % 4 || k % group) return -1;
+    int ng = k / group;
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < n; ++r)
+        for (int kk = 0; kk < k; ++kk) {
+            int q = (codes[(size_t)r * (k / 4) + kk / 4] >> (2 * (kk % 4))) & 3;
+            out[(size_t)r * k + kk] = dequant_std_level(q, scales[(size_t)r * ng + kk / group]);
+        }
+    return 0;
+}
+
+int oracle_quantize_w2std(const float *w, int n, int k, int group, uint8_t *codes, float *scales)
+{
+    if (n < 0 || k <= 0 || group <= 0 || k % 4 || k % group) return -1;
+    int ng = k / group;
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < n; ++r) {
+        int old = fegetround();
+        fesetround(FE_TONEAREST);
+        for (int g = 0; g < ng; ++g) {
+            double amax = 0.0;
+            for (int i = 0; i < group; ++i) {
+                double a = fabs((double)w[(size_t)r * k + g * group + i]);
+                if (a > amax) amax = a;
+            }
+            float s = oracle_bf16_to_float(oracle_bf16_bits((float)(amax / 2.0)));
+            scales[(size_t)r * ng + g] = s;
+            for (int i = 0; i < group; i += 4) {
+                uint8_t byte = 0;
+                for (int t = 0; t < 4; ++t) {
+                    double v = s > 0.0f ? (double)w[(size_t)r * k + g * group + i + t] / (double)s : 0.0;
+                    double q = nearbyint(v) + 2.0;
+                    if (q < 0.0) q = 0.0;
+                    if (q > 3.0) q = 3.0;
+                    byte |= (uint8_t)((int)q << (2 * t));
+                }
+                codes[(size_t)r * (k / 4) + (g * group + i) / 4] = byte;
+            }
+        }
+        fesetround(old);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------
  * W4 per-channel dequantization ([WINT2] quantization_config "wint4", "per_channel"; [GPTQ]
  * Part 2 pack_int4/unpack_int4): codes[n][k/2], two signed 4-bit codes per byte, the first code
  * of a pair in the low nibble; the code is sign-extended; w = bf16(q * bf16(scale[n])).

@@ -585,3 +585,43 @@ def test_encode_w2q4_codes_are_optimal_for_the_quantized_scales():
         err = ((w[r].reshape(32, 4)[None] - dec) ** 2).sum(axis=2)  # [byte][vector]
         assert np.array_equal(codes[r], np.argmin(err, axis=0).astype(np.uint8))
         assert q[r].max() == 15
+
+
+# ----------------------------------------------------------------------------------------------
+# WINT2-Standard, the comparison format of CCQ Table 4 (plain 2-bit fields, reading)
+# ----------------------------------------------------------------------------------------------
+def test_dequant_w2std_hand_example():
+    # byte 0xE4 = 11 10 01 00: fields (low first) 0, 1, 2, 3 -> levels -2, -1, 0, 1; s = 1.5
+    codes = np.zeros((1, 32), dtype=np.uint8)
+    codes[0, 0] = 0xE4
+    codes[0, 17] = 0x1B  # 00 01 10 11 -> fields 3, 2, 1, 0 -> 1, 0, -1, -2; second group s = 0.25
+    out = oracle.bf16_to_f64(oracle.dequant_w2std(codes, np.array([[1.5, 0.25]], np.float32)))
+    assert list(out[0, :4]) == [-3.0, -1.5, 0.0, 1.5]
+    assert list(out[0, 4:8]) == [-3.0, -3.0, -3.0, -3.0]  # byte 0: every field 0
+    assert list(out[0, 68:72]) == [0.25, 0.0, -0.25, -0.5]
+
+
+def test_quantize_w2std_round_to_nearest():
+    w = synth.weights_normal(3, 128, 95)
+    codes, scales = oracle.quantize_w2std(w)
+    amax = np.abs(w.reshape(3, 2, 64)).max(axis=2)
+    assert np.array_equal(scales, oracle.bf16_to_f64(oracle.bf16_bits(amax / 2.0)).astype(np.float32))
+    q = np.stack([(codes >> (2 * i)) & 3 for i in range(4)], axis=-1).reshape(3, 128).astype(np.int64)
+    s = np.repeat(scales.astype(np.float64), 64, axis=1)
+    assert np.array_equal(q, np.clip(np.rint(w.astype(np.float64) / s) + 2, 0, 3))
+    # every weight within half a step of its level, except the clipped positive end
+    lev = (q - 2) * s
+    assert np.all((np.abs(w - lev) <= s / 2 + 1e-12) | (q == 3))
+
+
+def test_quantize_w2std_picks_nearest_level_brute_force():
+    # independent of the rint/clip formula: each weight's level is the closest of the four
+    w = synth.weights_normal(4, 256, 96)
+    codes, scales = oracle.quantize_w2std(w)
+    deq = oracle.bf16_to_f64(oracle.dequant_w2std(codes, scales))
+    s = np.repeat(scales.astype(np.float64), 64, axis=1)
+    levels = np.stack([(lv - 2) * s for lv in range(4)], axis=-1)  # [n][k][4]
+    dist = np.abs(levels - w.astype(np.float64)[..., None])
+    best = dist.min(axis=-1)
+    got = np.abs(deq - w.astype(np.float64))
+    assert np.allclose(got, best, rtol=0, atol=1e-12)
