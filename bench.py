@@ -32,6 +32,7 @@ NOMINAL_HBM_GBS = 8000.0
 METRIC = "W2A16 MoE layer tokens/s; packed-weight HBM GB/s (% of 8 TB/s), 1 B200"
 WORKLOAD = "moe_ffn_decode_T32_H8192_I3584_E64_top8_ccq_w2_g64"
 SCALES = "fp32"       # group scale storage: fp32 (the benchmark format) or q4 (CCQ's 2.06-bpw form)
+CODES = "ccq"         # 2-bit codes: ccq (code cluster) or std (plain WINT2-Standard fields, CCQ Table 4)
 
 
 def parse():
@@ -50,9 +51,18 @@ def parse():
     ap.add_argument("--m", type=int, default=0, help="tokens for --workload gemm (default 1) / stack (default 32)")
     ap.add_argument("--scales", default="fp32", choices=["fp32", "q4"],
                     help="W2 group scales: fp32 (default) or 4-bit x per-channel super scale (2.06 bpw)")
+    ap.add_argument("--codes", default="ccq", choices=["ccq", "std"],
+                    help="2-bit codes: ccq (code cluster, default) or std (plain 2-bit WINT2-Standard fields, "
+                         "the comparison format of CCQ Table 4; fp32 scales only)")
+    ap.add_argument("--shape", default="8192x8192",
+                    help="--workload gemm: input x output size KxN (CCQ Table 4: 4096x4096, 4096x1024, "
+                         "8192x8192, 8192x1024)")
     args = ap.parse_args()
-    global T, E, WORKLOAD, SCALES
+    global T, E, WORKLOAD, SCALES, CODES
     SCALES = args.scales
+    CODES = args.codes
+    if CODES == "std" and SCALES != "fp32":
+        ap.error("--codes std takes fp32 scales only")
     if args.workload == "prefill":
         T = 4096
         WORKLOAD = "moe_ffn_prefill_T4096_zipf1.1_H8192_I3584_E64_top8_ccq_w2_g64"
@@ -60,6 +70,8 @@ def parse():
         T, E = (8, 16) if args.workload == "decode" else (512, 16)
     if SCALES == "q4":
         WORKLOAD = WORKLOAD.replace("ccq_w2_g64", "ccq_w2_g64_q4scale")
+    if CODES == "std":
+        WORKLOAD = WORKLOAD.replace("ccq_w2_g64", "std_w2_g64")
     return args
 
 
@@ -124,14 +136,18 @@ def config_dict():
     return {
         "workload": WORKLOAD,
         "tokens": T, "hidden": H, "intermediate": I, "experts": E, "topk": TOPK,
-        "weight_format": "CCQ (6,4,3) code cluster, 4 weights/byte, " + (
-            "4-bit group-64 scales x fp32 per-channel super scale (2.06 bpw)" if SCALES == "q4" else
-            "fp32 group-64 scales"),
+        "weight_format": ("WINT2-Standard plain 2-bit fields, 4 weights/byte, fp32 group-64 scales"
+                          if CODES == "std" else "CCQ (6,4,3) code cluster, 4 weights/byte, " + (
+                              "4-bit group-64 scales x fp32 per-channel super scale (2.06 bpw)" if SCALES == "q4"
+                              else "fp32 group-64 scales")),
         "routing": ("Zipf(1.1) expert popularity, top-8 by Gumbel-max; " if prefill else "uniform distinct top-8, ")
                    + "softmax of N(0,1) logits",
         "activations": "BF16 N(0,1)" + (", 1% of channels x20" if prefill else ""),
         "weights": (f"N(0,0.02) encoded by ccq_encode_host_q4 for {DISTINCT} experts, copied to all {E}"
-                    if SCALES == "q4" else f"N(0,0.02) per expert (seeded device RNG), all {E} encoded by ccq_encode_device"),
+                    if SCALES == "q4" else
+                    f"N(0,0.02) per expert (seeded device RNG), all {E} quantized by ccq_quantize_std_device"
+                    if CODES == "std" else
+                    f"N(0,0.02) per expert (seeded device RNG), all {E} encoded by ccq_encode_device"),
         "l2": "inputs larger than L2: ~1.74 GB of packed weights touched per step vs 126 MB L2",
         "parallelism": "replicas",
     }
@@ -141,23 +157,30 @@ def config_dict():
 # inputs
 # ------------------------------------------------------------------------------------------------
 def make_layer_device(ccq, torch, device, seed_base: int = 3100):
-    """Every expert its own N(0, 0.02) weights (seeded device RNG), encoded by ccq_encode_device."""
+    """Every expert its own N(0, 0.02) weights (seeded device RNG), encoded by ccq_encode_device
+    (or, for the WINT2-Standard codes, quantized by ccq_quantize_std_device)."""
+    std = CODES == "std"
+
     def stack(n, k, seed):
         codes = torch.empty((E * n, k // 4), dtype=torch.uint8, device=device)
         scales = torch.empty((E * n, k // 64), dtype=torch.float32, device=device)
-        alpha = torch.empty((E * n,), dtype=torch.float32, device=device)
-        beta = torch.empty((E * n,), dtype=torch.float32, device=device)
-        ws = ccq.workspace(ccq._lib.ccq_encode_device_workspace_size(n, k), device)
+        alpha = None if std else torch.empty((E * n,), dtype=torch.float32, device=device)
+        beta = None if std else torch.empty((E * n,), dtype=torch.float32, device=device)
+        ws = None if std else ccq.workspace(ccq._lib.ccq_encode_device_workspace_size(n, k), device)
         g = torch.Generator(device=device)
         for e in range(E):
             g.manual_seed(seed + e)
             w = torch.randn((n, k), generator=g, device=device, dtype=torch.float32) * 0.02
-            c, s, a, b = ccq.ccq_encode_device(w, 64, 0, ws=ws)
+            if std:
+                c, s = ccq.ccq_quantize_std_device(w)
+            else:
+                c, s, a, b = ccq.ccq_encode_device(w, 64, 0, ws=ws)
+                alpha[e * n:(e + 1) * n].copy_(a)
+                beta[e * n:(e + 1) * n].copy_(b)
             codes[e * n:(e + 1) * n].copy_(c)
             scales[e * n:(e + 1) * n].copy_(s)
-            alpha[e * n:(e + 1) * n].copy_(a)
-            beta[e * n:(e + 1) * n].copy_(b)
-        return ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, n, k, codes, scales, alpha, beta, experts=E, device=device)
+        fmt = ccq.CCQ_FMT_W2_STD_G64 if std else ccq.CCQ_FMT_W2_CCQ_G64
+        return ccq.CcqWeight(fmt, n, k, codes, scales, alpha, beta, experts=E, device=device)
 
     return stack(2 * I, H, seed_base), stack(H, I, seed_base + 100)
 
@@ -208,8 +231,11 @@ def make_layer(ccq, torch, device):
 
 def touched_bytes(ids):
     """Algorithmic packed-weight bytes of one step: codes + scales + per-row constants (alpha, beta;
-    q4: and the super scale) of the touched experts."""
-    if SCALES == "q4":
+    q4: and the super scale; std: none) of the touched experts."""
+    if CODES == "std":
+        per13 = 2 * I * (H // 4) + 2 * I * (H // 64) * 4
+        per2 = H * (I // 4) + H * (I // 64) * 4
+    elif SCALES == "q4":
         per13 = 2 * I * (H // 4) + 2 * I * (H // 128) + 2 * I * 12
         per2 = H * (I // 4) + H * (I // 128) + H * 12
     else:
@@ -497,7 +523,7 @@ def run_ours(args, rank, world, local):
             {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (fused MoE: gate/up + SiLU, then down)",
              "achieved": (b13 + b2) / (gemm1_ms * 1e-3) / 1e9, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)",
              "unit": "GB/s", "frac": (b13 + b2) / (gemm1_ms * 1e-3) / 1e9 / hbm,
-             "traffic": FUSED_DECODE_DRAM_BYTES_PER_EXPERT * ne if SCALES == "fp32" else None,
+             "traffic": FUSED_DECODE_DRAM_BYTES_PER_EXPERT * ne if (SCALES, CODES) == ("fp32", "ccq") else None,
              "traffic_source": "ncu dram__bytes_read+write of the 16-expert capture, scaled by touched experts",
              "launch_ms": gemm1_ms, "algorithmic_bytes_per_launch": b13 + b2} if fused else
             {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (gate/up, SiLU epilogue)",
@@ -539,8 +565,9 @@ def _timed(torch, device, stream, step, K, W):
 
 
 def run_gemm(args, rank, world, local):
-    """y = x W^T, K = N = 8192, CCQ W2 g64, at M tokens.  The weight (21.04 MB) is smaller than L2,
-    so the timed calls rotate over enough device copies to exceed twice the L2 size."""
+    """y = x W^T at M tokens, K x N from --shape (default 8192 x 8192), CCQ W2 g64 or the
+    WINT2-Standard codes.  The weight (21.04 MB at 8192 x 8192) is smaller than L2, so the timed
+    calls rotate over enough device copies to exceed twice the L2 size."""
     import torch
 
     import extreme_bit_weight_b200 as ccq
@@ -548,9 +575,14 @@ def run_gemm(args, rank, world, local):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    M, KD, ND = (args.m or 1), 8192, 8192
+    M = args.m or 1
+    KD, ND = (int(v) for v in args.shape.lower().split("x"))
     w = synth.weights_normal(ND, KD, 4100)
-    if SCALES == "q4":
+    if CODES == "std":
+        c, sc = (t.cpu().numpy() for t in ccq.ccq_quantize_std_device(torch.from_numpy(w).to(device)))
+        per_copy = c.nbytes + sc.nbytes
+        mk = lambda: ccq.CcqWeight(ccq.CCQ_FMT_W2_STD_G64, ND, KD, c, sc, device=device)
+    elif SCALES == "q4":
         c, sq, sup, al, be, _ = ccq.ccq_encode_host_q4(w, 64, 0, 0)
         per_copy = c.nbytes + sq.nbytes + sup.nbytes + al.nbytes + be.nbytes
         mk = lambda: ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64_Q4SCALE, ND, KD, c, None, al, be, device=device,
@@ -591,13 +623,15 @@ def run_gemm(args, rank, world, local):
     roof.update({"kernel": "whole ccq_w2a16_gemm call (" + ("tcgen05 kernel" if tensor else
                  "activation packing, decode kernel, split-K reduce") + ")", "traffic": None,
                  "algorithmic_bytes_per_call": per_copy, "algorithmic_flops_per_call": flops})
-    line = {"metric": "W2A16 dense linear tokens/s (K=N=8192)", "value": M / (ms * 1e-3), "unit": "tokens/s",
+    fmt_tag = "std_w2_g64" if CODES == "std" else "ccq_w2_g64" + ("_q4scale" if SCALES == "q4" else "")
+    line = {"metric": f"W2A16 dense linear tokens/s (K={KD}, N={ND})", "value": M / (ms * 1e-3), "unit": "tokens/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "us_per_call": 1000.0 * ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": f"dense_gemm_M{M}_K8192_N8192_ccq_w2_g64" + ("_q4scale" if SCALES == "q4" else ""),
+            "config": {"workload": f"dense_gemm_M{M}_K{KD}_N{ND}_{fmt_tag}",
                        "m": M, "k": KD, "n": ND,
-                       "weights": "N(0,0.02) encoded by ccq_encode_host",
+                       "weights": "N(0,0.02) " + ("quantized by ccq_quantize_std_device" if CODES == "std" else
+                                                  "encoded by ccq_encode_host" + ("_q4" if SCALES == "q4" else "")),
                        "l2": f"{R} rotating weight copies ({R * per_copy / 1e6:.0f} MB) vs {l2 / 1e6:.0f} MB L2"},
             "packed_weight_gbs": gbs, "roofline": roof,
             "e2e": {"value": M / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * 2,

@@ -27,11 +27,12 @@ CCQ_ERR_TIMEOUT = 5
 CCQ_FMT_W2_CCQ_G64 = 1
 CCQ_FMT_W4_PER_CHANNEL = 2
 CCQ_FMT_W2_CCQ_G64_Q4SCALE = 3
+CCQ_FMT_W2_STD_G64 = 4
 CCQ_ENC_LITERAL_EQ1 = 1
 CCQ_ENC_REFIT_SCALE = 2
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libccq.so not built at {LIB_PATH}; run `python -m extreme_bit_weight_b200.build`")
+    raise ImportError(f"libccq.so not built at {LIB_PATH}; run `python extreme_bit_weight_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -69,6 +70,7 @@ _lib.ccq_encode_device_workspace_size.argtypes = [_I, _I]
 _lib.ccq_encode_device_workspace_size.restype = ctypes.c_size_t
 _lib.ccq_encode_device.argtypes = [_P, _I, _I, _I, ctypes.c_uint32, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.ccq_encode_host_q4.argtypes = [_P, _I, _I, _I, ctypes.c_uint32, _I, _P, _P, _P, _P, _P, _P]
+_lib.ccq_quantize_std_device.argtypes = [_P, _I, _I, _P, _P, _P]
 _lib.ccq_dequant_bf16.argtypes = [ctypes.POINTER(ccq_weight), _I, _P, _P]
 _lib.ccq_gemm_workspace_size.argtypes = [ctypes.POINTER(ccq_weight), _I]
 _lib.ccq_gemm_workspace_size.restype = ctypes.c_size_t
@@ -168,6 +170,18 @@ def ccq_encode_device(w: torch.Tensor, group: int = 64, flags: int = 0, ws: torc
     _check(_lib.ccq_encode_device(_dptr(w), n, k, group, flags, _dptr(codes), _dptr(scales), _dptr(alpha),
                                   _dptr(beta), _dptr(ws), ws.numel(), _stream(stream)), "ccq_encode_device")
     return codes, scales, alpha, beta
+
+
+def ccq_quantize_std_device(w: torch.Tensor, stream=None):
+    """WINT2-Standard round-to-nearest of fp32 w [n][k] on the GPU -> device tensors
+    (codes [n][k/4], scales [n][k/64])."""
+    w = w.contiguous()
+    n, k = w.shape
+    codes = torch.empty((n, k // 4), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((n, k // 64), dtype=torch.float32, device=w.device)
+    _check(_lib.ccq_quantize_std_device(_dptr(w), n, k, _dptr(codes), _dptr(scales), _stream(stream)),
+           "ccq_quantize_std_device")
+    return codes, scales
 
 
 def ccq_quantize_w4_host(w: np.ndarray, threads: int = 0):

@@ -69,6 +69,56 @@ __global__ void dequant_w4_kernel(const uint8_t *__restrict__ codes, const float
     }
 }
 
+// WINT2-Standard (CCQ "Inference Performance", Table 4's comparison format): field i of byte j is the
+// level q of weight 4j+i, w = bf16((q - 2) * bf16(s)) (an exact product).  One thread per byte.
+__global__ void dequant_std_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales, int rows,
+                                   int K, uint16_t *__restrict__ out) {
+    const size_t nbytes = (size_t)rows * (K / 4);
+    const int kb = K / 4, ng = K / 64;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < nbytes;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int r = (int)(idx / kb), j = (int)(idx % kb);
+        const uint32_t b = codes[idx];
+        const float s = bf16_bits_to_float(float_to_bf16_bits(__ldg(scales + (size_t)r * ng + (4 * j) / 64)));
+        uint16_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[i] = float_to_bf16_bits(__fmul_rn((float)((int)((b >> (2 * i)) & 3u) - 2), s));
+        uint2 v;
+        v.x = (uint32_t)o[0] | ((uint32_t)o[1] << 16);
+        v.y = (uint32_t)o[2] | ((uint32_t)o[3] << 16);
+        *reinterpret_cast<uint2 *>(out + (size_t)r * K + 4 * j) = v;
+    }
+}
+
+// WINT2-Standard round-to-nearest, one warp per (row, 64-column group); lane l holds columns 2l,
+// 2l+1.  s = bf16(max|w| / 2); the level round_half_even(w / s) clipped to [-2, 1] is decided by
+// comparing w with s/2 and 3s/2, which are exact in fp32 for a BF16 s, so the decision equals the
+// rounding of the exact quotient (ties: -3s/2 -> -2, +-s/2 -> 0, 3s/2 -> 2 clipped to 1).
+__device__ __forceinline__ uint32_t std_field(float w, float s) {
+    if (!(s > 0.0f)) return 2u;
+    const float h = 0.5f * s, t = 1.5f * s;
+    return w <= -t ? 0u : w < -h ? 1u : w <= h ? 2u : 3u;
+}
+
+__global__ void quantize_std_kernel(const float *__restrict__ w, int rows, int K, uint8_t *__restrict__ codes,
+                                    float *__restrict__ scales) {
+    const int ng = K / 64, lane = threadIdx.x & 31;
+    const size_t units = (size_t)rows * ng;
+    const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
+    for (size_t u = blockIdx.x * (size_t)(blockDim.x >> 5) + (threadIdx.x >> 5); u < units; u += warps) {
+        const size_t r = u / ng, g = u % ng;
+        const float2 v = __ldg(reinterpret_cast<const float2 *>(w + r * K + g * 64) + lane);
+        float a = fmaxf(fabsf(v.x), fabsf(v.y));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+        const float s = bf16_bits_to_float(float_to_bf16_bits(a * 0.5f));
+        const uint32_t nib = std_field(v.x, s) | (std_field(v.y, s) << 2);
+        const uint32_t hi = __shfl_down_sync(0xFFFFFFFFu, nib, 1);
+        if ((lane & 1) == 0) codes[r * (K / 4) + g * 16 + lane / 2] = (uint8_t)(nib | (hi << 4));
+        if (lane == 0) scales[r * ng + g] = s;
+    }
+}
+
 // ------------------------------------------------------------------------------------------------
 // Activation operand packing.  One thread per (operand row p, 64-column group G): reads the
 // group's 64 BF16 values of source row tok_of[p] (or p), writes them in the XA order and the
@@ -263,9 +313,17 @@ cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, c
         const bool q4 = fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
         dequant_w2_kernel<<<grid_for((size_t)rows * K / 4, 256), 256, 0, s>>>(
             codes, q4 ? nullptr : scales, alpha, beta, rows, K, out, scale_q4, super);
+    } else if (fmt == CCQ_FMT_W2_STD_G64) {
+        dequant_std_kernel<<<grid_for((size_t)rows * K / 4, 256), 256, 0, s>>>(codes, scales, rows, K, out);
     } else {
         dequant_w4_kernel<<<grid_for((size_t)rows * K / 2, 256), 256, 0, s>>>(codes, scales, rows, K, out);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes, float *scales, cudaStream_t s) {
+    if (rows <= 0) return cudaSuccess;
+    quantize_std_kernel<<<grid_for((size_t)rows * (K / 64) * 32, 256), 256, 0, s>>>(w, rows, K, codes, scales);
     return cudaGetLastError();
 }
 

@@ -50,7 +50,8 @@ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 ccq_status check_weight(const ccq_weight *w, int experts) {
     if (!w || experts <= 0) return CCQ_ERR_INVALID_ARG;
-    if (w->fmt != CCQ_FMT_W2_CCQ_G64 && w->fmt != CCQ_FMT_W4_PER_CHANNEL && w->fmt != CCQ_FMT_W2_CCQ_G64_Q4SCALE)
+    if (w->fmt != CCQ_FMT_W2_CCQ_G64 && w->fmt != CCQ_FMT_W4_PER_CHANNEL && w->fmt != CCQ_FMT_W2_CCQ_G64_Q4SCALE &&
+        w->fmt != CCQ_FMT_W2_STD_G64)
         return CCQ_ERR_UNSUPPORTED;
     if (w->n <= 0 || w->k <= 0 || w->n % 16 || w->k % 64) return CCQ_ERR_INVALID_ARG;
     if (!w->codes || !aligned16(w->codes)) return CCQ_ERR_INVALID_ARG;
@@ -66,8 +67,27 @@ ccq_status check_weight(const ccq_weight *w, int experts) {
         if (w->group != 64) return CCQ_ERR_UNSUPPORTED;
         if (!w->alpha || !w->beta) return CCQ_ERR_INVALID_ARG;
     }
+    if (w->fmt == CCQ_FMT_W2_STD_G64 && w->group != 64) return CCQ_ERR_UNSUPPORTED;
     if ((size_t)experts * w->n > (size_t)INT32_MAX) return CCQ_ERR_INVALID_ARG;
     return CCQ_OK;
+}
+
+// The weight-format fields of a kernel parameter block.
+template <class Params>
+void set_format(Params &p, const ccq_weight *w) {
+    p.scales = w->scales;
+    p.alpha = w->alpha;
+    p.beta = w->beta;
+    p.w4 = w->fmt == CCQ_FMT_W4_PER_CHANNEL;
+    p.q4 = w->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
+    p.std2 = w->fmt == CCQ_FMT_W2_STD_G64;
+    p.scale_q4 = w->scale_q4;
+    p.super_scale = w->super_scale;
+}
+
+// Level offset of the decoders' BF16 values for this format (the gsq table's L).
+float level_of(const ccq_weight *w) {
+    return gsq_level(w->fmt == CCQ_FMT_W4_PER_CHANNEL, w->fmt == CCQ_FMT_W2_STD_G64);
 }
 
 // --- decode-sized path ----------------------------------------------------------------------
@@ -308,9 +328,6 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
         CUtensorMap ta, tcodes;
         if (!tc_maps(ta, tcodes, w, 1, xt, m)) return CCQ_ERR_CUDA;
         TcGemmParams p{};
-        p.scales = w->scales;
-        p.alpha = w->alpha;
-        p.beta = w->beta;
         p.N = w->n;
         p.K = w->k;
         p.row_block_stride = 256;
@@ -321,10 +338,7 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
         p.static_tiles = ceil_div(m, p.m_tile);
         p.M = m;
         p.out_ld = w->n;
-        p.w4 = w->fmt == CCQ_FMT_W4_PER_CHANNEL;
-        p.q4 = w->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
-        p.scale_q4 = w->scale_q4;
-        p.super_scale = w->super_scale;
+        set_format(p, w);
         p.ksplit = L.ksplit;
         p.kg = L.spp;
         if (L.ksplit > 1) {
@@ -345,14 +359,11 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
     uint16_t *xa = reinterpret_cast<uint16_t *>(base + L.xa);
     float *gs = reinterpret_cast<float *>(base + L.gs);
     cudaError_t e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), nullptr, m, L.P, w->k,
-                                   gsq_level(w->fmt == CCQ_FMT_W4_PER_CHANNEL), xa, gs, s);
+                                   level_of(w), xa, gs, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     DecodeMaps maps;
     if (!decode_maps(maps, w, 1, xa, gs, L.P, L.nt)) return CCQ_ERR_CUDA;
     DecodeGemmParams p{};
-    p.scales = w->scales;
-    p.alpha = w->alpha;
-    p.beta = w->beta;
     p.N = w->n;
     p.K = w->k;
     p.row_block_stride = 256;
@@ -373,10 +384,7 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
         p.out = y_bf16;
     }
     p.tma_scales = maps.tma_scales;
-    p.w4 = w->fmt == CCQ_FMT_W4_PER_CHANNEL;
-    p.q4 = w->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
-    p.scale_q4 = w->scale_q4;
-    p.super_scale = w->super_scale;
+    set_format(p, w);
     e = launch_decode_gemm_w2(p, maps.codes, maps.xa, maps.gs, maps.sc, L.row_blocks, L.ksplit, 1, L.nt, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     if (L.ksplit > 1) {
@@ -454,9 +462,6 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         if (!tc_maps(ta1, tc1, w13, num_experts, xa_x, L.P) || !tc_maps(ta2, tc2, w2, num_experts, xa_h, L.P))
             return CCQ_ERR_CUDA;
         TcGemmParams q1{};
-        q1.scales = w13->scales;
-        q1.alpha = w13->alpha;
-        q1.beta = w13->beta;
         q1.N = w13->n;
         q1.K = H;
         q1.row_block_stride = 128;
@@ -471,17 +476,11 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q1.out_ld = I;
         q1.I = I;
         q1.err = err;
-        q1.w4 = w13->fmt == CCQ_FMT_W4_PER_CHANNEL;
-        q1.q4 = w13->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
-        q1.scale_q4 = w13->scale_q4;
-        q1.super_scale = w13->super_scale;
+        set_format(q1, w13);
         e = launch_tc_gemm_w2(q1, ta1, tc1, mt, std::min(sm_count(), L.max_tiles * q1.n_tiles), s);
         if (e == cudaSuccess) e = trace(events, 3, s);
         if (e == cudaSuccess) e = trace(events, 4, s);
         TcGemmParams q2 = q1;
-        q2.scales = w2->scales;
-        q2.alpha = w2->alpha;
-        q2.beta = w2->beta;
         q2.N = H;
         q2.K = I;
         q2.row_block_stride = 256;
@@ -492,10 +491,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q2.out_ld = H;
         q2.rw = rwp;
         q2.I = 0;
-        q2.w4 = w2->fmt == CCQ_FMT_W4_PER_CHANNEL;
-        q2.q4 = w2->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
-        q2.scale_q4 = w2->scale_q4;
-        q2.super_scale = w2->super_scale;
+        set_format(q2, w2);
         if (e == cudaSuccess) e = launch_tc_gemm_w2(q2, ta2, tc2, mt, std::min(sm_count(), L.max_tiles * q2.n_tiles), s);
         if (e == cudaSuccess) e = trace(events, 5, s);
         if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
@@ -503,7 +499,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         return cuda_status(e);
     }
     e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), tok, pairs, L.P, H,
-                           gsq_level(w13->fmt == CCQ_FMT_W4_PER_CHANNEL), xa_x, gs_x, s);
+                           level_of(w13), xa_x, gs_x, s);
     if (e == cudaSuccess) e = trace(events, 2, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     const int nt1 = pick_nt((double)pairs / num_experts, w13->fmt);
@@ -513,9 +509,6 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     DecodeMaps m1;
     if (!decode_maps(m1, w13, num_experts, xa_x, gs_x, L.P, nt1)) return CCQ_ERR_CUDA;
     DecodeGemmParams p1{};
-    p1.scales = w13->scales;
-    p1.alpha = w13->alpha;
-    p1.beta = w13->beta;
     p1.N = w13->n;
     p1.K = H;
     p1.row_block_stride = 128;
@@ -530,18 +523,12 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p1.I = I;
     p1.err = err;
     p1.tma_scales = m1.tma_scales;
-    p1.w4 = w13->fmt == CCQ_FMT_W4_PER_CHANNEL;
-    p1.q4 = w13->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
-    p1.scale_q4 = w13->scale_q4;
-    p1.super_scale = w13->super_scale;
+    set_format(p1, w13);
 
     // down projection, scaled by each pair's routing weight -> fp32 slots
     DecodeMaps m2;
     if (!decode_maps(m2, w2, num_experts, xa_h, gs_h, L.P, nt2)) return CCQ_ERR_CUDA;
     DecodeGemmParams p2{};
-    p2.scales = w2->scales;
-    p2.alpha = w2->alpha;
-    p2.beta = w2->beta;
     p2.N = H;
     p2.K = I;
     p2.row_block_stride = 256;
@@ -556,23 +543,20 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     p2.rw = rwp;
     p2.err = err;
     p2.tma_scales = m2.tma_scales;
-    p2.w4 = w2->fmt == CCQ_FMT_W4_PER_CHANNEL;
-    p2.q4 = w2->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE;
-    p2.scale_q4 = w2->scale_q4;
-    p2.super_scale = w2->super_scale;
+    set_format(p2, w2);
 
-    // Both projections W2 (both with TMA-staged fp32 scales, or both with 4-bit scales) and the same
-    // token tiling: one fused launch, in
-    // which the gate/up epilogue also writes h's group-sum table and each down unit starts once
-    // its expert's gate/up units are done.  Otherwise (or if the device refuses the cooperative
-    // launch) two launches with the group sums computed in between.
-    bool fused = !p1.w4 && !p2.w4 && nt1 == nt2 &&
+    // Both projections in the same 2-bit format (CCQ or STD with TMA-staged fp32 scales, or CCQ
+    // with 4-bit scales) and the same token tiling: one fused launch, in which the gate/up
+    // epilogue also writes h's group-sum table and each down unit starts once its expert's
+    // gate/up units are done.  Otherwise (or if the device refuses the cooperative launch) two
+    // launches with the group sums computed in between.
+    bool fused = !p1.w4 && !p2.w4 && nt1 == nt2 && p1.std2 == p2.std2 &&
                  ((p1.tma_scales && p2.tma_scales && !p1.q4 && !p2.q4) || (p1.q4 && p2.q4));
     if (fused) {
         p1.dep = dep;
         p1.fuse_gsq = gs_h;
         p1.fuse_gsq_ld = gsum_ld(I);
-        p1.fuse_level = gsq_level(false);
+        p1.fuse_level = level_of(w2);
         p2.dep = dep;
         e = launch_decode_moe_fused(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), p2, m2.codes, m2.xa, m2.gs,
                                     m2.sc, ceil_div(H, 256), num_experts, nt1, s);
@@ -591,7 +575,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), 1, num_experts, nt1, s);
         if (e == cudaSuccess) e = trace(events, 3, s);
         if (e == cudaSuccess)
-            e = launch_gsum_from_xa(xa_h, pairs, L.P, I, gsq_level(w2->fmt == CCQ_FMT_W4_PER_CHANNEL), gs_h, s);
+            e = launch_gsum_from_xa(xa_h, pairs, L.P, I, level_of(w2), gs_h, s);
         if (e == cudaSuccess) e = trace(events, 4, s);
         if (e == cudaSuccess)
             e = launch_decode_gemm_w2(p2, m2.codes, m2.xa, m2.gs, m2.sc, ceil_div(H, 256), 1, num_experts, nt2, s);
@@ -600,6 +584,14 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
     if (e == cudaSuccess) e = trace(events, 6, s);
     return cuda_status(e);
+}
+
+ccq_status ccq_quantize_std_device(const float *w, int32_t n, int32_t k, uint8_t *codes, float *scales,
+                                   ccq_stream_t stream) {
+    if (!w || !codes || !scales || n < 0 || k <= 0 || k % 64) return CCQ_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(codes) || !aligned16(scales)) return CCQ_ERR_INVALID_ARG;
+    if ((size_t)n * (k / 64) > (size_t)INT32_MAX * 64) return CCQ_ERR_INVALID_ARG;
+    return cuda_status(launch_quantize_std(w, n, k, codes, scales, (cudaStream_t)stream));
 }
 
 ccq_status ccq_check_device_error(void *ws, ccq_stream_t stream) {

@@ -166,6 +166,20 @@ __device__ __forceinline__ void decode_word_w4(uint32_t w, uint32_t m4, uint32_t
     asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[3]) : "r"(w >> 12), "r"(m4), "r"(x4));
 }
 
+// WINT2-Standard: one 32-bit word = 16 plain 2-bit fields (field i of byte j at bits 2i of the byte),
+// laid out like a CCQ word: R[2i] = (128 + f_i(byte0), 128 + f_i(byte1)), R[2i+1] = (.. byte2, ..
+// byte3).  Bytes 0,1 and 2,3 are first spread into the two 16-bit halves of one register each.
+__device__ __forceinline__ void decode_word_std(uint32_t w, const DecodeConsts &k, uint32_t R[8]) {
+    const uint32_t X01 = prmt(w, 0u, 0x4140u), X23 = prmt(w, 0u, 0x4342u);
+    R[0] = and_or(X01, k.wmask, k.wexp);
+    R[1] = and_or(X23, k.wmask, k.wexp);
+    R[2] = and_or(X01 >> 2, k.wmask, k.wexp);
+    R[3] = and_or(X23 >> 2, k.wmask, k.wexp);
+    R[4] = and_or(X01 >> 4, k.wmask, k.wexp);
+    R[5] = and_or(X23 >> 4, k.wmask, k.wexp);
+    R[6] = and_or(X01 >> 6, k.wmask, k.wexp);
+    R[7] = and_or(X23 >> 6, k.wmask, k.wexp);
+}
 
 __device__ __forceinline__ void mma_bf16(float *c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -259,16 +273,23 @@ __device__ __forceinline__ void group_mma(const uint32_t (&RA0)[8], const uint32
     });
 }
 
-// One W2 group: the four code words of this thread (rows g, g+8 of both halves) at ca, ca+1024,
-// and one code tile further.
-template <int NT, int G>
+// One 2-bit group (CCQ, or STD plain fields): the four code words of this thread (rows g, g+8 of
+// both halves) at ca, ca+1024, and one code tile further.
+template <int NT, int G, bool STD = false>
 __device__ __forceinline__ void group_w2(uint32_t ca, uint32_t xs, uint32_t gs, const float sc[4],
                                          const RowDecode rd[4], const DecodeConsts &kc, float (&acc)[2][NT][4]) {
     uint32_t RA0[8], RA1[8], RB0[8], RB1[8];
-    decode_word(lds32_at<0>(ca), rd[0], kc, RA0);
-    decode_word(lds32_at<1024>(ca), rd[1], kc, RA1);
-    decode_word(lds32_at<kCodeTileBytes>(ca), rd[2], kc, RB0);
-    decode_word(lds32_at<kCodeTileBytes + 1024>(ca), rd[3], kc, RB1);
+    if constexpr (STD) {
+        decode_word_std(lds32_at<0>(ca), kc, RA0);
+        decode_word_std(lds32_at<1024>(ca), kc, RA1);
+        decode_word_std(lds32_at<kCodeTileBytes>(ca), kc, RB0);
+        decode_word_std(lds32_at<kCodeTileBytes + 1024>(ca), kc, RB1);
+    } else {
+        decode_word(lds32_at<0>(ca), rd[0], kc, RA0);
+        decode_word(lds32_at<1024>(ca), rd[1], kc, RA1);
+        decode_word(lds32_at<kCodeTileBytes>(ca), rd[2], kc, RB0);
+        decode_word(lds32_at<kCodeTileBytes + 1024>(ca), rd[3], kc, RB1);
+    }
     group_mma<NT, G>(RA0, RA1, RB0, RB1, xs, gs, sc, acc);
 }
 
@@ -376,7 +397,8 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
 // Persistent: CTA b walks units b, b + gridDim.x, ...; its producer streams every stage of every
 // unit through one ring, so the next unit's first stages load while this unit finishes.
 // FUSED: the launch holds the MoE gate/up units (p, m1) followed by the down units (p2, m2).
-template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false>
+// STD: WINT2-Standard plain 2-bit fields (no per-row constants).
+template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false, bool STD = false>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__ MapSet m2,
                       const __grid_constant__ DecodeGemmParams p, const __grid_constant__ DecodeGemmParams p2) {
@@ -468,9 +490,10 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             }
             fence_proxy_async_global();  // the generic-proxy writes of h are visible to TMA from here
         }
-        const uint32_t row_bytes = first ? (uint32_t)(U.nA + U.nB) * 4u * (W4 ? 1u : Q4 ? 3u : 2u) : 0u;
+        const uint32_t row_bytes =
+            (first && !STD) ? (uint32_t)(U.nA + U.nB) * 4u * (W4 ? 1u : Q4 ? 3u : 2u) : 0u;
         mbar_arrive_expect_tx(bar, S::kTxBytes + ((TMA_SC && !W4) ? S::kScBytes : 0) + row_bytes);
-        if (first) {
+        if (first && !STD) {
             // the unit's per-row constants: alpha, beta (W2) or the channel scales (W4) of both halves
             const float *ra = W4 ? q.scales : q.alpha;
             if (U.nA) bulk_g2s(base + kRowsOff, ra + rowA, U.nA * 4u, bar);
@@ -557,7 +580,8 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     kc.neg_magic = f2_pack(-8388608.0f, -8388608.0f);
     kc.round_mag = f2_pack(12582912.0f, 12582912.0f - 19264.0f);
     kc.mul16 = 65536u + opaque;
-    kc.wmask = (W4 ? 0x000F000Fu : 0x003F003Fu) ^ opaque;  // one state window / one nibble per half
+    // one state window / one nibble / one 2-bit field per half
+    kc.wmask = (W4 ? 0x000F000Fu : STD ? 0x00030003u : 0x003F003Fu) ^ opaque;
     kc.wexp = (W4 ? 0x43084308u : 0x43004300u) ^ opaque;   // BF16 128 (W4: and the nibble sign flip)
 
     // per-thread shared-memory offsets inside a stage, for this warp's four groups Gh..Gh+3
@@ -611,7 +635,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
         const bool first = c == 0 && i == 0;
         if (first) st = U.s_begin + U.rot;
         const uint32_t sb = sbase + (uint32_t)(slot * S::kStageBytes);
-        if (first) {
+        if (first && !STD) {
             // this unit's per-row constants arrived with its first stage
             const uint32_t ra = sb + rows_thr;
             const float r0 = lds_f32(ra), r1 = lds_f32(ra + 32), r2 = lds_f32(ra + 512), r3 = lds_f32(ra + 544);
@@ -674,7 +698,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                     const float qf = __uint_as_float(0x4B000000u | ((q4cur[r] >> (4 * G)) & 0xFu)) - 8388608.0f;
                     sc[r] = round_bf16(__fmul_rn(qf, sc_row[r]));
                 }
-                group_w2<NT, G>(sb + coff[G], xs, gs, sc, rd, kc, acc);
+                group_w2<NT, G, STD>(sb + coff[G], xs, gs, sc, rd, kc, acc);
             });
         } else if (TMA_SC) {
             // full stage: groups beyond K read TMA zero fill (scale 0, activations 0) and add nothing
@@ -689,7 +713,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             static_for<4>([&](auto Gc) {
                 constexpr int G = decltype(Gc)::value;
                 const float sc[4] = {round_bf16(v0[G]), round_bf16(v1[G]), round_bf16(v2[G]), round_bf16(v3[G])};
-                group_w2<NT, G>(sb + coff[G], xs, gs, sc, rd, kc, acc);
+                group_w2<NT, G, STD>(sb + coff[G], xs, gs, sc, rd, kc, acc);
             });
         } else {
             const int ngroups = pq.K / 64;
@@ -707,7 +731,8 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                 }
                 const uint32_t ca = kCodeOff + (uint32_t)(wrow + g) * 128u + 4u * (uint32_t)tig +
                                     ((uint32_t)((Gh + G) ^ g) << 4);
-                group_w2<NT, 0>(sb + ca, sb + xa_thr + G * 4 * MP * 32, sb + gs_thr + G * 16, sc, rd, kc, acc);
+                group_w2<NT, 0, STD>(sb + ca, sb + xa_thr + G * 4 * MP * 32, sb + gs_thr + G * 16, sc, rd, kc,
+                                     acc);
             }
         }
         __syncwarp();
@@ -888,7 +913,11 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
             smem = Smem<NT, true>::kTotal;
         }
     }
-    if (!p.w4 && p.q4) {
+    if (!p.w4 && p.std2) {
+        kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false, false, false, true>
+                            : decode_gemm_w2_kernel<NT, false, false, false, false, true>;
+        smem = Smem<NT, false>::kTotal;
+    } else if (!p.w4 && p.q4) {
         kern = decode_gemm_w2_kernel<NT, false, false, false, true>;
         smem = Smem<NT, false, true>::kTotal;
     } else if (!p.w4) {
@@ -915,7 +944,9 @@ template <int NT>
 cudaError_t launch_fused_nt(const DecodeGemmParams &p1, const MapSet &m1, int row_blocks1, const DecodeGemmParams &p2,
                             const MapSet &m2, int row_blocks2, int experts, cudaStream_t s) {
     // fp32 group scales staged by TMA, or 4-bit scales read by the consumers (both projections alike)
-    DecodeKernel kern = p1.q4 ? decode_gemm_w2_kernel<NT, false, false, true, true> : decode_gemm_w2_kernel<NT, true, false, true>;
+    DecodeKernel kern = p1.q4     ? decode_gemm_w2_kernel<NT, false, false, true, true>
+                        : p1.std2 ? decode_gemm_w2_kernel<NT, true, false, true, false, true>
+                                  : decode_gemm_w2_kernel<NT, true, false, true>;
     const int smem = p1.q4 ? Smem<NT, false, true>::kTotal : Smem<NT, false>::kTotal;
     cudaError_t err = prepare_kernel(kern, smem);
     if (err != cudaSuccess) return err;
@@ -964,7 +995,7 @@ cudaError_t launch_decode_moe_fused(const DecodeGemmParams &p1, const CUtensorMa
                                     const CUtensorMap &c2, const CUtensorMap &d2, int row_blocks2, int experts,
                                     int nt, cudaStream_t s) {
     const bool fp32_sc = !p1.q4 && !p2.q4 && p1.tma_scales && p2.tma_scales, q4_sc = p1.q4 && p2.q4;
-    if (p1.w4 || p2.w4 || !(fp32_sc || q4_sc) || p1.mode != EPI_GATEUP || p2.mode != EPI_DOWN ||
+    if (p1.w4 || p2.w4 || !(fp32_sc || q4_sc) || p1.std2 != p2.std2 || (q4_sc && p1.std2) || p1.mode != EPI_GATEUP || p2.mode != EPI_DOWN ||
         !p1.dep || !p2.dep || !p1.fuse_gsq)
         return cudaErrorInvalidValue;
     const MapSet m1{a1, b1, c1, d1}, m2{a2, b2, c2, d2};

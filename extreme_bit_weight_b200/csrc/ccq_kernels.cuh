@@ -27,9 +27,12 @@ __host__ __device__ inline size_t xa_index(size_t p, size_t k, size_t P) {
     return ((((G * 4 + i) * P + p) * 4 + tig) * 4 + j);
 }
 __host__ __device__ inline int gsum_ld(int K) { return ((K / 64) + 3) & ~3; }
-// The decoders hand the tensor core BF16 (128 + u) for W2 state u (weight level u - 32) and
-// (128 + q + 8) for W4 nibble q: the per-group accumulator starts at L * S with L = -160 / -136.
-__host__ __device__ inline float gsq_level(bool w4) { return w4 ? -136.0f : -160.0f; }
+// The decoders hand the tensor core BF16 (128 + u) for CCQ state u (weight level u - 32),
+// (128 + q + 8) for W4 nibble q and (128 + q) for a STD 2-bit field q (level q - 2): the per-group
+// accumulator starts at L * S with L = -160 / -136 / -130.
+__host__ __device__ inline float gsq_level(bool w4, bool std2 = false) {
+    return w4 ? -136.0f : std2 ? -130.0f : -160.0f;
+}
 
 struct DecodeGemmParams {
     const float *scales;  // [rows_total][K/64]
@@ -59,6 +62,7 @@ struct DecodeGemmParams {
     int q4;
     const uint8_t *scale_q4;   // [rows_total][K/128]
     const float *super_scale;  // [rows_total]
+    int std2;                  // 1: WINT2-Standard plain 2-bit fields (no alpha/beta)
     uint32_t *err;
     // work units (set by the launcher): unit u = (expert, k split, row block), row block fastest
     int row_blocks, ksplit, units;
@@ -73,7 +77,8 @@ struct DecodeGemmParams {
 };
 
 // Fused MoE decode: gate/up (p1, maps a1..d1) then down (p2, maps a2..d2) in one cooperative
-// persistent launch.  Both must be W2 with TMA-staged scales and the same token tile count nt.
+// persistent launch.  Both must be the same 2-bit format (CCQ or STD with TMA-staged fp32 scales,
+// or CCQ with 4-bit scales) with the same token tile count nt.
 cudaError_t launch_decode_moe_fused(const DecodeGemmParams &p1, const CUtensorMap &a1, const CUtensorMap &b1,
                                     const CUtensorMap &c1, const CUtensorMap &d1, int row_blocks1,
                                     const DecodeGemmParams &p2, const CUtensorMap &a2, const CUtensorMap &b2,
@@ -109,6 +114,7 @@ struct TcGemmParams {
     int q4;                // 1: 4-bit group scales (see DecodeGemmParams)
     const uint8_t *scale_q4;
     const float *super_scale;
+    int std2;              // 1: WINT2-Standard plain 2-bit fields (no alpha/beta)
     uint32_t *err;
     // split-K (dense matmul with few tiles): ksplit > 1 splits the 64-column groups into ranges of
     // kg groups (a multiple of 4); each range writes EPI_PARTIAL_F32 sums at out + ks*out_split_stride
@@ -125,6 +131,9 @@ cudaError_t launch_pack_xt(const uint16_t *x, const int *tok_of, int P_valid, in
 cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, const float *alpha,
                            const float *beta, int rows, int K, uint16_t *out, cudaStream_t s,
                            const uint8_t *scale_q4 = nullptr, const float *super = nullptr);
+
+// WINT2-Standard round-to-nearest: w fp32 [rows][K] -> codes [rows][K/4], scales [rows][K/64]
+cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes, float *scales, cudaStream_t s);
 
 // x (BF16 [rows][K], row r taken from x[tok_of ? tok_of[p] : p]) -> XA operand + group sums.
 cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,

@@ -182,6 +182,18 @@ __device__ __forceinline__ void decode_word_w4_bf16(uint32_t w, uint32_t s2, uin
     }
 }
 
+// WINT2-Standard: one word = 16 plain 2-bit fields, in the same window-major order as a CCQ word:
+// out[2i], out[2i+1] = field i of bytes (0,1) and (2,3), each 128 + q minus 130 exactly, times s.
+__device__ __forceinline__ void decode_word_std_bf16(uint32_t w, uint32_t s2, uint32_t out[8]) {
+    const uint32_t X01 = prmt(w, 0u, 0x4140u), X23 = prmt(w, 0u, 0x4342u);
+    const uint32_t M = 0x00030003u, E = 0x43004300u, Z = 0x43024302u;  // Z = bf16x2(130, 130)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        out[2 * i] = bmul2(bsub2(((X01 >> (2 * i)) & M) | E, Z), s2);
+        out[2 * i + 1] = bmul2(bsub2(((X23 >> (2 * i)) & M) | E, Z), s2);
+    }
+}
+
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
 // position p of a 16-column block holds column 4*(p%4) + p/4 (and the map is its own inverse)
@@ -224,7 +236,8 @@ __device__ __forceinline__ bool tile_of(const TcGemmParams &p, int w, TileInfo &
     return true;
 }
 
-template <int MT, bool W4, bool Q4 = false>
+// STD: WINT2-Standard plain 2-bit fields (no per-row constants)
+template <int MT, bool W4, bool Q4 = false, bool STD = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_codes,
                   const TcGemmParams p) {
@@ -365,7 +378,8 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             const int local = t.nt * p.row_block_stride + half * p.half_stride + rr;
             const bool valid = local < p.N;
             const size_t grow = (size_t)t.e * p.N + (valid ? local : 0);
-            const float alpha = W4 ? 0.0f : __ldg(p.alpha + grow), beta = W4 ? 0.0f : __ldg(p.beta + grow);
+            const float alpha = (W4 || STD) ? 0.0f : __ldg(p.alpha + grow);
+            const float beta = (W4 || STD) ? 0.0f : __ldg(p.beta + grow);
             rp.ab = fpk2(alpha, alpha);
             rp.bb = fpk2(beta, beta);
             const float *srow = p.scales + grow * (W4 ? 1 : nk);
@@ -421,8 +435,13 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                     const float sraw = gi == 0 ? sc_cur.x : gi == 1 ? sc_cur.y : gi == 2 ? sc_cur.z : sc_cur.w;
                     const float sc = bf16_bits_to_float(float_to_bf16_bits(sraw));
                     const uint32_t s2 = pack_bf16x2(sc, sc);
-                    decode_word_bf16(q2w.x, rp, s2, o[0]);
-                    decode_word_bf16(q2w.y, rp, s2, o[1]);
+                    if constexpr (STD) {
+                        decode_word_std_bf16(q2w.x, s2, o[0]);
+                        decode_word_std_bf16(q2w.y, s2, o[1]);
+                    } else {
+                        decode_word_bf16(q2w.x, rp, s2, o[0]);
+                        decode_word_bf16(q2w.y, rp, s2, o[1]);
+                    }
                 } else {
                     // block b of 16 columns = words 2b, 2b+1; emit the same window-major order as W2:
                     // positions (4i, 4i+1) <- codes (i, i+4) of word 2b, (4i+2, 4i+3) <- of word 2b+1
@@ -593,7 +612,10 @@ __global__ void pack_xt_kernel(const uint16_t *__restrict__ x, const int *__rest
 
 template <int MT>
 cudaError_t launch_tc_mt(const TcGemmParams &p, const CUtensorMap &ta, const CUtensorMap &tc, int grid, cudaStream_t s) {
-    auto kern = p.w4 ? tc_gemm_w2_kernel<MT, true> : p.q4 ? tc_gemm_w2_kernel<MT, false, true> : tc_gemm_w2_kernel<MT, false>;
+    auto kern = p.w4     ? tc_gemm_w2_kernel<MT, true>
+                : p.q4   ? tc_gemm_w2_kernel<MT, false, true>
+                : p.std2 ? tc_gemm_w2_kernel<MT, false, false, true>
+                         : tc_gemm_w2_kernel<MT, false>;
     const int smem = TcSmem<MT>::kTotal;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;

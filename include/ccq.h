@@ -66,8 +66,19 @@ typedef enum {
  *     super_scale[n] fp32;
  *     group scale s = fl32(q4 * super_scale[n]) (one fp32 multiply), then the same weight rule
  *     w = bf16_rn((u - 32) * bf16_rn(s)).  `scales` is unused (NULL).  k must be a multiple of 128.
+ * CCQ_FMT_W2_STD_G64: "WINT2-Standard", the plain 2-bit scalar format the CCQ paper measures
+ *   against (Inference Performance, Table 4; the paper does not define it, this is the plain
+ *   reading).  Same storage as CCQ_FMT_W2_CCQ_G64 without alpha/beta (NULL):
+ *     codes[n][k/4] uint8, bits 2i..2i+1 of byte j hold the level q of weight k = 4j + i;
+ *     scales[n][k/64] fp32 group scales (used as bf16_rn(scale));
+ *     w = bf16_rn((q - 2) * bf16_rn(scales[n][k/64]))          (levels -2, -1, 0, 1).
  */
-enum { CCQ_FMT_W2_CCQ_G64 = 1, CCQ_FMT_W4_PER_CHANNEL = 2, CCQ_FMT_W2_CCQ_G64_Q4SCALE = 3 };
+enum {
+    CCQ_FMT_W2_CCQ_G64 = 1,
+    CCQ_FMT_W4_PER_CHANNEL = 2,
+    CCQ_FMT_W2_CCQ_G64_Q4SCALE = 3,
+    CCQ_FMT_W2_STD_G64 = 4
+};
 
 /* One linear layer, or `num_experts` layers of the same shape stacked back to back: expert e's
  * arrays start at codes + e*n*(k/4) (W2) or e*n*(k/2) (W4), scales + e*n*(k/64) (W2) or e*n (W4),
@@ -77,11 +88,11 @@ typedef struct {
     int32_t fmt;          /* CCQ_FMT_* */
     int32_t n;            /* output features (rows of W), multiple of 16 */
     int32_t k;            /* input features, multiple of 64 */
-    int32_t group;        /* 64 for CCQ_FMT_W2_CCQ_G64; ignored for W4 */
+    int32_t group;        /* 64 for the W2 formats; ignored for W4 */
     const uint8_t *codes; /* (device) packed code stream */
     const float *scales;  /* (device) group scales (W2) or channel scales (W4) */
-    const float *alpha;   /* (device) W2 code scale per row; NULL for W4 */
-    const float *beta;    /* (device) W2 code zero-point per row; NULL for W4 */
+    const float *alpha;   /* (device) CCQ code scale per row; NULL for W4 and STD */
+    const float *beta;    /* (device) CCQ code zero-point per row; NULL for W4 and STD */
     const uint8_t *scale_q4;   /* (device) Q4SCALE: packed 4-bit group scales; NULL otherwise */
     const float *super_scale;  /* (device) Q4SCALE: super scale per row; NULL otherwise */
 } ccq_weight;
@@ -137,6 +148,17 @@ ccq_status ccq_encode_host_q4(const float *w, int32_t n, int32_t k, int32_t grou
                               int32_t threads, uint8_t *codes, uint8_t *scale_q4, float *super_scale,
                               float *alpha, float *beta, double *sq_err);
 
+/* ccq_quantize_std_device - round-to-nearest quantization to CCQ_FMT_W2_STD_G64 on the GPU (the
+ * pages print no quantizer for WINT2-Standard; this is the plain one):
+ *   per group of 64: s = bf16_rn(max|w| / 2); level q - 2 = clip(round_half_even(w / s), -2, 1),
+ *   q = 2 where s == 0.  Decided by exact fp32 comparisons with s/2 and 3s/2 (both exact for a
+ *   BF16 s), identical to the rounding of the exact quotient.
+ *   w (device) fp32 [n][k], k % 64 == 0; codes (device) out [n][k/4]; scales (device) out
+ *   [n][k/64] (BF16-representable).  Asynchronous on `stream`; argument errors (null pointers,
+ *   bad shapes, misaligned pointers: all three 16-byte aligned) return before any launch. */
+ccq_status ccq_quantize_std_device(const float *w, int32_t n, int32_t k, uint8_t *codes, float *scales,
+                                   ccq_stream_t stream);
+
 /* ccq_quantize_w4_host - W4 per-channel round-to-nearest ("GPTQ and AWQ" Part 2 rtn/pack_int4):
  * s = bf16(max|w_row|/7), q = clip(round_half_even(w/s), -8, 7) (w/s in fp64), two codes per byte,
  * first in the low nibble.  w (host) fp32 [n][k], k even; codes (host) out [n][k/2]; scales (host)
@@ -156,7 +178,7 @@ size_t ccq_gemm_workspace_size(const ccq_weight *w, int32_t m);
 /* ccq_w2a16_gemm - y[m][n] = x[m][k] * W^T with W decoded on the fly (never stored), fp32
  * accumulation, BF16 output.  The GEMV / small-M shapes of CCQ's "Inference Performance"
  * section (Table 4) and the dense prefill shape.
- *   w      single layer (num_experts = 1), CCQ_FMT_W2_CCQ_G64 or CCQ_FMT_W4_PER_CHANNEL
+ *   w      single layer (num_experts = 1), any CCQ_FMT_* format
  *   x_bf16 (device) BF16 [m][k], 16-byte aligned;  m >= 0 (m == 0 is a no-op)
  *   y_bf16 (device) BF16 [m][n], 16-byte aligned
  *   ws     (device) workspace of ccq_gemm_workspace_size(w, m) bytes (may be NULL if that is 0)
@@ -199,7 +221,7 @@ size_t ccq_moe_workspace_size(int32_t T, int32_t topk, int32_t H, int32_t I, int
  *   expert_ids (device) int32 [T][topk], each in [0, E) and distinct within a token
  *   routing_w  (device) fp32 [T][topk], used as given (no renormalisation)
  *   ws         (device) workspace of ccq_moe_workspace_size(...) bytes
- * W2 and W4 formats may be mixed (w13 and w2 need not share a format). */
+ * The formats may be mixed (w13 and w2 need not share a format). */
 ccq_status ccq_moe_w2a16_forward(const ccq_weight *w13, const ccq_weight *w2, int32_t num_experts,
                                  const void *x_bf16, int32_t T, const int32_t *expert_ids,
                                  const float *routing_w, int32_t topk, void *y_bf16, void *ws,
@@ -209,8 +231,8 @@ ccq_status ccq_moe_w2a16_forward(const ccq_weight *w13, const ccq_weight *w2, in
  * between its steps, for per-kernel timing: events[0] before routing, [1] after routing,
  * [2] after activation packing, [3] after the gate/up kernel, [4] after the group-sum kernel,
  * [5] after the down kernel, [6] after the combine.  When the decode-sized path runs both
- * projections as one fused launch (W2 weights on both, with fp32 group-scale rows a multiple of 16
- * bytes on both or 4-bit scales on both),
+ * projections as one fused launch (the same 2-bit format on both: CCQ or STD with fp32 group-scale
+ * rows a multiple of 16 bytes, or CCQ with 4-bit scales),
  * [3], [4] and [5] are all recorded after that launch.  `events` (host) holds
  * CCQ_MOE_TRACE_POINTS cudaEvent_t handles created by the caller (NULL: no events).  No paper
  * counterpart: a measurement hook. */

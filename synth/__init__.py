@@ -114,3 +114,12 @@ def w4_format_random(n: int, k: int, seed: int, scale_std: float = 0.02):
     codes = g.integers(0, 256, size=(n, k // 2), dtype=np.uint8)
     scales = (np.abs(g.normal(4.0, 0.3, size=n)) * scale_std / 7.0).astype(np.float32)
     return codes, scales
+
+
+def std_format_random(n: int, k: int, seed: int, group: int = 64, scale_std: float = 0.02):
+    """Random WINT2-Standard parameters: codes uniform bytes (four 2-bit fields), group scales of the
+    magnitude max|w|/2 of a N(0, scale_std^2) weight group gives."""
+    g = rng(seed)
+    codes = g.integers(0, 256, size=(n, k // 4), dtype=np.uint8)
+    scales = (np.abs(g.normal(2.5, 0.4, size=(n, k // group))) * scale_std / 2.0).astype(np.float32)
+    return codes, scales

@@ -14,10 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 @pytest.fixture(scope="module")
-def ccq():
-    from extreme_bit_weight_b200 import build
-
-    build.build()
+def ccq(built_lib):
     import extreme_bit_weight_b200 as m
 
     return m
@@ -75,6 +72,18 @@ def test_host_validation_returns_before_launch(ccq):
     assert lib.ccq_moe_w2a16_forward(ctypes.byref(w13), ctypes.byref(w2), 4, fake, 0, fake, fake, 2, fake + 512,
                                      None, 0, None) == ccq.CCQ_OK  # T == 0
     assert lib.ccq_check_device_error(None, None) == ccq.CCQ_ERR_INVALID_ARG
+    # WINT2-Standard: no alpha/beta needed (validation passes them and fails on the workspace);
+    # group != 64 unsupported; its quantizer checks shapes, pointers and alignment before launching
+    w = ccq.ccq_weight(ccq.CCQ_FMT_W2_STD_G64, 256, 256, 64, fake, fake, None, None)
+    assert lib.ccq_w2a16_gemm(ctypes.byref(w), fake, 4, fake, fake, 0, None) == ccq.CCQ_ERR_INVALID_ARG
+    assert lib.ccq_w2a16_gemm(ctypes.byref(w), fake, 0, fake, None, 0, None) == ccq.CCQ_OK
+    w = ccq.ccq_weight(ccq.CCQ_FMT_W2_STD_G64, 256, 256, 32, fake, fake, None, None)
+    assert lib.ccq_w2a16_gemm(ctypes.byref(w), fake, 4, fake, fake, 1 << 30, None) == ccq.CCQ_ERR_UNSUPPORTED
+    q = lib.ccq_quantize_std_device
+    assert q(None, 4, 64, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG
+    assert q(fake, 4, 96, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG      # k % 64
+    assert q(fake, -1, 64, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG
+    assert q(fake + 8, 4, 64, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG  # misaligned w
 
 
 def test_encoder_matches_oracle(ccq):

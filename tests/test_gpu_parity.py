@@ -327,15 +327,25 @@ def test_gemm_w4_shapes(ccq, m, n, k):
     assert e <= 4e-3
 
 
+# formats by name: "ccq" (W2 g64, fp32 scales), "q4" (W2 g64, 4-bit scales), "w4" (per channel),
+# "std" (WINT2-Standard); FMT_SEED gives each a number for the seeds
+FMT_SEED = {"ccq": 2, "q4": 3, "w4": 4, "std": 5}
+
+
 def moe_weights_fmt(ccq, E, H, I, seed, fmt13, fmt2):
     def make(rows, k, s, fmt):
-        if fmt == 3:  # CCQ W2 with 4-bit group scales
+        if fmt == "q4":  # CCQ W2 with 4-bit group scales
             c, sq, sup, a, b = synth.w2q4_format_random(rows, k, s)
             return q4_weight(ccq, c, sq, sup, a, b, experts=E), oracle.dequant_w2q4(c, sq, sup, a, b)
-        if fmt == 4:
+        if fmt == "w4":
             c, sc = synth.w4_format_random(rows, k, s)
             return (ccq.CcqWeight(ccq.CCQ_FMT_W4_PER_CHANNEL, rows // E, k, c, sc, experts=E),
                     oracle.dequant_w4(c, sc))
+        if fmt == "std":
+            c, sc = synth.std_format_random(rows, k, s)
+            return (ccq.CcqWeight(ccq.CCQ_FMT_W2_STD_G64, rows // E, k, c, sc, experts=E),
+                    oracle.dequant_w2std(c, sc))
+        assert fmt == "ccq"
         c, sc, a, b = synth.w2_format_random(rows, k, s)
         return (ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, rows // E, k, c, sc, a, b, experts=E),
                 oracle.dequant_w2(c, sc, a, b))
@@ -344,11 +354,11 @@ def moe_weights_fmt(ccq, E, H, I, seed, fmt13, fmt2):
     return W13, W2, d13.reshape(E, 2 * I, H), d2.reshape(E, H, I)
 
 
-@pytest.mark.parametrize("fmts", [(4, 2), (2, 4), (4, 4)])
+@pytest.mark.parametrize("fmts", [("w4", "ccq"), ("ccq", "w4"), ("w4", "w4")])
 @pytest.mark.parametrize("T", [6, 300])
 def test_moe_mixed_formats(ccq, fmts, T):
     E, H, I, topk = 8, 512, 256, 2
-    W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 5200 + T + 10 * fmts[0], *fmts)
+    W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 5200 + T + 10 * FMT_SEED[fmts[0]], *fmts)
     x = synth.activations(T, H, 5201 + T)
     ids, rw = synth.routing_uniform(T, E, topk, 5202 + T)
     y, st = run_moe(ccq, W13, W2, x, ids, rw)
@@ -367,7 +377,7 @@ def test_mixed_stack_layer_by_layer(ccq, M):
     E, H, I, topk = 8, 512, 256, 4
     x = synth.activations(M, H, 5300 + M).cuda()
     for layer in range(8):
-        fmt = 4 if layer < 2 else 2
+        fmt = "w4" if layer < 2 else "ccq"
         W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 5400 + 100 * layer, fmt, fmt)
         ids, rw = synth.routing_uniform(M, E, topk, 5500 + 100 * layer + M)
         ids_t = torch.from_numpy(ids).cuda()
@@ -431,11 +441,11 @@ def test_gemm_q4_shapes(ccq, m, n, k):
     assert e <= 4e-3
 
 
-@pytest.mark.parametrize("fmts", [(3, 3), (3, 2), (2, 3), (4, 3)])
+@pytest.mark.parametrize("fmts", [("q4", "q4"), ("q4", "ccq"), ("ccq", "q4"), ("w4", "q4")])
 @pytest.mark.parametrize("T", [6, 300])
 def test_moe_q4_formats(ccq, fmts, T):
     E, H, I, topk = 8, 512, 256, 2
-    W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 6300 + T + 10 * fmts[0] + fmts[1], *fmts)
+    W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 6300 + T + 10 * FMT_SEED[fmts[0]] + FMT_SEED[fmts[1]], *fmts)
     x = synth.activations(T, H, 6301 + T)
     ids, rw = synth.routing_uniform(T, E, topk, 6302 + T)
     y, st = run_moe(ccq, W13, W2, x, ids, rw)
@@ -470,3 +480,90 @@ def test_encode_device_matches_host_at_size(ccq):
     assert np.array_equal(a, ha) and np.array_equal(b, hb)
     assert np.array_equal(s, hs)
     assert np.array_equal(c, hc)
+
+
+# ----------------------------------------------------------------------------------------------
+# WINT2-Standard, the plain 2-bit comparison format of CCQ "Inference Performance", Table 4
+# ----------------------------------------------------------------------------------------------
+def std_weight(ccq, codes, scales, experts=1):
+    n = codes.shape[0] // experts
+    return ccq.CcqWeight(ccq.CCQ_FMT_W2_STD_G64, n, codes.shape[1] * 4, codes, scales, experts=experts)
+
+
+@pytest.mark.parametrize("n,k,E", [(16, 64, 1), (48, 192, 3), (1024, 8192, 1)])
+def test_dequant_std_bitexact(ccq, n, k, E):
+    codes, scales = synth.std_format_random(n * E, k, 8000 + n + k)
+    got = bits_of(ccq.ccq_dequant_bf16(std_weight(ccq, codes, scales, experts=E))).reshape(n * E, k)
+    assert np.array_equal(got, oracle.dequant_w2std(codes, scales))
+
+
+def test_quantize_std_device_matches_oracle(ccq):
+    w = synth.weights_normal(40, 1088, 8100)
+    # group 0 of row 0: amax 0.5, so s = 0.25, and every rounding tie (+-s/2, +-3s/2) and both clips
+    w[0, :64] = np.resize(np.array([0.5, -0.5, 0.375, -0.375, 0.125, -0.125, 0.0, 0.25, -0.25, 0.4, -0.4],
+                                   np.float32), 64)
+    w[1, 64:128] = 0.0                                   # all-zero group: s = 0, levels 0
+    w[2, 128:192] = np.float32(2.0 ** -149)              # amax/2 rounds to 0: s = 0
+    # subnormal s = 2^-127, quotients k/16: ties at +-1/2 and +-3/2 among them
+    w[3, 192:256] = np.float32(2.0 ** -131) * np.arange(-32, 32, dtype=np.float32)
+    w[4, 256:320] *= 1e4                                 # large values
+    c, sc = (t.cpu().numpy() for t in ccq.ccq_quantize_std_device(torch.from_numpy(w).cuda()))
+    oc, osc = oracle.quantize_w2std(w)
+    assert np.array_equal(sc, osc)
+    assert np.array_equal(c, oc)
+
+
+def test_gemm_std_one_hot_identity_both_paths(ccq):
+    n, k = 272, 576
+    codes, scales = synth.std_format_random(n, k, 8200)
+    W = std_weight(ccq, codes, scales)
+    ref = oracle.bf16_to_f64(oracle.dequant_w2std(codes, scales)).T.astype(np.float32)
+    eye = synth.one_hot_rows(k).cuda()
+    for j in range(0, k, 16):  # register-decode mma.sync kernel
+        y = ccq.ccq_w2a16_gemm(W, eye[j:j + 16].contiguous()).float().cpu().numpy()
+        assert np.array_equal(y, ref[j:j + 16]), j
+    y = ccq.ccq_w2a16_gemm(W, eye).float().cpu().numpy()  # tcgen05 kernel
+    assert np.array_equal(y, ref)
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 256, 512), (4, 1024, 4096), (9, 272, 576), (33, 256, 1088),
+                                   (64, 512, 1024), (300, 272, 576), (1, 8192, 8192), (128, 8192, 8192)])
+def test_gemm_std_shapes(ccq, m, n, k):
+    codes, scales = synth.std_format_random(n, k, 8300 + m + n)
+    W = std_weight(ccq, codes, scales)
+    x = synth.activations(m, k, 8301 + m)
+    y = ccq.ccq_w2a16_gemm(W, x.cuda()).float().cpu().numpy()
+    ref = oracle.gemm_f64(synth.bf16_bits(x), oracle.dequant_w2std(codes, scales))
+    e = rel_err(y, ref)
+    assert e <= TOL
+    assert e <= 4e-3
+
+
+@pytest.mark.parametrize("fmts", [("std", "std"), ("std", "ccq"), ("ccq", "std"), ("w4", "std")])
+@pytest.mark.parametrize("T", [6, 300])
+def test_moe_std_formats(ccq, fmts, T):
+    E, H, I, topk = 8, 512, 256, 2
+    W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 8400 + T + 10 * FMT_SEED[fmts[0]] + FMT_SEED[fmts[1]], *fmts)
+    x = synth.activations(T, H, 8401 + T)
+    ids, rw = synth.routing_uniform(T, E, topk, 8402 + T)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    ref = oracle.moe_f64(synth.bf16_bits(x), d13, d2, ids, rw, round_h=True)
+    assert rel_err(y, ref) <= TOL
+
+
+def test_moe_std_quantized_layer_matches_oracle(ccq):
+    # weights through the device quantizer (not random codes), decode-sized fused path
+    E, H, I, topk, T = 8, 1024, 512, 2, 16
+    def q(rows, k, seed):
+        w = synth.weights_normal(rows, k, seed)
+        c, sc = (t.cpu().numpy() for t in ccq.ccq_quantize_std_device(torch.from_numpy(w).cuda()))
+        return std_weight(ccq, c, sc, experts=E), oracle.dequant_w2std(c, sc)
+    W13, d13 = q(E * 2 * I, H, 8500)
+    W2, d2 = q(E * H, I, 8501)
+    x = synth.activations(T, H, 8502)
+    ids, rw = synth.routing_uniform(T, E, topk, 8503)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    ref = oracle.moe_f64(synth.bf16_bits(x), d13.reshape(E, 2 * I, H), d2.reshape(E, H, I), ids, rw, round_h=True)
+    assert rel_err(y, ref) <= TOL
