@@ -199,7 +199,8 @@ def ccq_quantize_w4_host(w: np.ndarray, threads: int = 0):
 # device weights
 # ------------------------------------------------------------------------------------------------
 class CcqWeight:
-    """Device copy of one (or E stacked) quantized weight(s) [E][n][k] and its ccq_weight view."""
+    """Device copy of one (or E stacked) quantized weight(s) [E][n][k] and its ccq_weight view.
+    The tensors are fixed at construction: the ccq_weight view is built once and reused."""
 
     def __init__(self, fmt: int, n: int, k: int, codes, scales, alpha=None, beta=None, experts: int = 1,
                  device="cuda", scale_q4=None, super_scale=None):
@@ -218,11 +219,13 @@ class CcqWeight:
         self.beta = dev(beta, torch.float32)
         self.scale_q4 = dev(scale_q4, torch.uint8)
         self.super_scale = dev(super_scale, torch.float32)
+        self._struct = ccq_weight(self.fmt, self.n, self.k, 0 if self.fmt == CCQ_FMT_W4_PER_CHANNEL else 64,
+                                  _dptr(self.codes), _dptr(self.scales), _dptr(self.alpha), _dptr(self.beta),
+                                  _dptr(self.scale_q4), _dptr(self.super_scale))
+        self._ref = ctypes.byref(self._struct)
 
     def struct(self) -> ccq_weight:
-        return ccq_weight(self.fmt, self.n, self.k, 0 if self.fmt == CCQ_FMT_W4_PER_CHANNEL else 64,
-                          _dptr(self.codes), _dptr(self.scales), _dptr(self.alpha), _dptr(self.beta),
-                          _dptr(self.scale_q4), _dptr(self.super_scale))
+        return self._struct
 
     @property
     def nbytes(self) -> int:
@@ -255,11 +258,9 @@ def ccq_w2a16_gemm(w: CcqWeight, x: torch.Tensor, y: torch.Tensor = None, ws: to
     m = x.shape[0]
     if y is None:
         y = torch.empty((m, w.n), dtype=torch.bfloat16, device=x.device)
-    need = ccq_gemm_workspace_size(w, m)
-    if ws is None:
-        ws = workspace(need, x.device)
-    s = w.struct()
-    _check(_lib.ccq_w2a16_gemm(ctypes.byref(s), _dptr(x), m, _dptr(y), _dptr(ws), ws.numel(), _stream(stream)),
+    if ws is None:  # (a caller's workspace is size-checked by the library)
+        ws = workspace(ccq_gemm_workspace_size(w, m), x.device)
+    _check(_lib.ccq_w2a16_gemm(w._ref, x.data_ptr(), m, y.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
            "ccq_w2a16_gemm")
     return y
 

@@ -6,11 +6,48 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <vector>
+
 #include "../../include/ccq.h"
 #include "ccq_device.cuh"
 #include "ccq_kernels.cuh"
 
 namespace ccq {
+
+cudaError_t kernel_setup(const void *kern, int smem, int threads, int want_regs, int *per_sm) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    struct Entry {
+        const void *kern;
+        int dev, smem, threads, per_sm;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> done;
+    {
+        std::lock_guard<std::mutex> g(mu);
+        for (const Entry &e : done)
+            if (e.kern == kern && e.dev == dev && e.smem == smem && e.threads == threads) {
+                if (per_sm) *per_sm = e.per_sm;
+                return cudaSuccess;
+            }
+    }
+    cudaFuncAttributes fa{};
+    err = cudaFuncGetAttributes(&fa, kern);
+    if (err != cudaSuccess) return err;
+    if (want_regs && fa.numRegs != want_regs) return cudaErrorInvalidConfiguration;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    int n = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> g(mu);
+    done.push_back({kern, dev, smem, threads, n});
+    if (per_sm) *per_sm = n;
+    return cudaSuccess;
+}
+
 namespace {
 
 // ------------------------------------------------------------------------------------------------
@@ -352,7 +389,7 @@ cudaError_t launch_moe_route(const int *ids, const float *rw, int T, int topk, i
                              int *tok_of, float *rw_perm, int *inv, int *dep, uint32_t *err, cudaStream_t s) {
     const size_t sh = sizeof(int) * (2 * (size_t)E + 1);
     if (sh > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
+        cudaError_t e = kernel_setup(reinterpret_cast<const void *>(moe_route_kernel), (int)sh, 1024, 0, nullptr);
         if (e != cudaSuccess) return e;
     }
     moe_route_kernel<<<1, 1024, sh, s>>>(ids, rw, T, topk, E, seg_off, cursor, tok_of, rw_perm, inv, dep, err);

@@ -884,14 +884,10 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
 
 using DecodeKernel = void (*)(MapSet, MapSet, DecodeGemmParams, DecodeGemmParams);
 
-// Checks the kernel's launch register count (the register split assumes kLaunchRegs) and sets its
-// dynamic shared memory.
-cudaError_t prepare_kernel(DecodeKernel kern, int smem) {
-    cudaFuncAttributes fa{};
-    cudaError_t err = cudaFuncGetAttributes(&fa, kern);
-    if (err != cudaSuccess) return err;
-    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+// Checks the kernel's launch register count (the register split assumes kLaunchRegs), sets its
+// dynamic shared memory and returns the CTAs that fit per SM (once per kernel and device).
+cudaError_t prepare_kernel(DecodeKernel kern, int smem, int *per_sm = nullptr) {
+    return kernel_setup(reinterpret_cast<const void *>(kern), smem, kThreads, kLaunchRegs, per_sm);
 }
 
 int device_sms(cudaError_t &err) {
@@ -948,7 +944,8 @@ cudaError_t launch_fused_nt(const DecodeGemmParams &p1, const MapSet &m1, int ro
                         : p1.std2 ? decode_gemm_w2_kernel<NT, true, false, true, false, true>
                                   : decode_gemm_w2_kernel<NT, true, false, true>;
     const int smem = p1.q4 ? Smem<NT, false, true>::kTotal : Smem<NT, false>::kTotal;
-    cudaError_t err = prepare_kernel(kern, smem);
+    int per_sm = 0;
+    cudaError_t err = prepare_kernel(kern, smem, &per_sm);
     if (err != cudaSuccess) return err;
     DecodeGemmParams q1 = p1, q2 = p2;
     q1.row_blocks = row_blocks1;
@@ -961,9 +958,6 @@ cudaError_t launch_fused_nt(const DecodeGemmParams &p1, const MapSet &m1, int ro
     if (q1.units + q2.units <= 0) return cudaSuccess;
     // down units wait for other CTAs' gate/up units: every CTA must be resident at once, which a
     // cooperative launch guarantees (or refuses)
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
-    if (err != cudaSuccess) return err;
     if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
     const int sms = device_sms(err);
     if (err != cudaSuccess) return err;

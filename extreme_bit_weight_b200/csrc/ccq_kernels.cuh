@@ -6,6 +6,12 @@
 
 namespace ccq {
 
+// Once per (kernel, device, dynamic shared memory size): checks the kernel's launch register count
+// (when want_regs != 0), sets its dynamic shared memory limit and computes how many CTAs of
+// `threads` threads fit on one SM.  Later calls return the cached result without touching the
+// runtime, so a small call's host cost is its launches.  per_sm may be NULL.
+cudaError_t kernel_setup(const void *kern, int smem, int threads, int want_regs, int *per_sm);
+
 // Epilogue modes of the decode-sized grouped kernel.
 enum EpiMode : int {
     EPI_PARTIAL_F32 = 0,  // out_f32[ks][m][n] = partial sum over this CTA's k range

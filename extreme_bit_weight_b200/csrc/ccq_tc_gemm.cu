@@ -617,7 +617,7 @@ cudaError_t launch_tc_mt(const TcGemmParams &p, const CUtensorMap &ta, const CUt
                 : p.std2 ? tc_gemm_w2_kernel<MT, false, false, true>
                          : tc_gemm_w2_kernel<MT, false>;
     const int smem = TcSmem<MT>::kTotal;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t err = kernel_setup(reinterpret_cast<const void *>(kern), smem, kTcThreads, 0, nullptr);
     if (err != cudaSuccess) return err;
     kern<<<grid, kTcThreads, smem, s>>>(ta, tc, p);
     return cudaGetLastError();
