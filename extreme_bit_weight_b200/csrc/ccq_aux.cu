@@ -185,7 +185,9 @@ __device__ __forceinline__ void store_gsq(float *gsq, int pr, int G, int ld, int
 // Four threads per (operand row p, group G): thread tig handles columns 16*tig .. 16*tig+15 of the
 // group (one 16-column block of the XA order) and the four lanes sum the group in a fixed order.
 __global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__restrict__ tok_of, int P_valid,
-                               int P, int K, float level, uint16_t *__restrict__ xa, float *__restrict__ gsq) {
+                               int P, int K, float level, uint16_t *__restrict__ xa, float *__restrict__ gsq,
+                               int *zero_ctr) {
+    if (zero_ctr && blockIdx.x == 0 && threadIdx.x == 0) *zero_ctr = 0;
     const int ng = K / 64, ld = gsum_ld(K);
     const size_t total = (size_t)P_valid * ng * 4;  // a multiple of 4: the lanes of one group stay together
     for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < ((total + 31) & ~size_t(31));
@@ -263,10 +265,9 @@ __global__ void moe_route_kernel(const int *__restrict__ ids, const float *__res
     extern __shared__ int sh[];
     int *cnt = sh;          // [E]
     int *off = sh + E;      // [E+1]
-    for (int i = threadIdx.x; i < E; i += blockDim.x) {
-        cnt[i] = 0;
-        if (dep) dep[i] = 0;  // per-expert completion counters of the fused matmul launch
-    }
+    for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+    // per-expert completion counters of the fused matmul launch, then the matmuls' work counters
+    for (int i = threadIdx.x; dep && i < E + 3; i += blockDim.x) dep[i] = 0;
     __syncthreads();
     const int npairs = T * topk;
     for (int q = threadIdx.x; q < npairs; q += blockDim.x) {
@@ -365,9 +366,10 @@ cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes,
 }
 
 cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,
-                           uint16_t *xa, float *gsq, cudaStream_t s) {
+                           uint16_t *xa, float *gsq, cudaStream_t s, int *zero_ctr) {
     if (P_valid <= 0) return cudaSuccess;
-    pack_xa_kernel<<<grid_for((size_t)P_valid * (K / 64) * 4, 128), 128, 0, s>>>(x, tok_of, P_valid, P, K, level, xa, gsq);
+    pack_xa_kernel<<<grid_for((size_t)P_valid * (K / 64) * 4, 128), 128, 0, s>>>(x, tok_of, P_valid, P, K, level, xa,
+                                                                                 gsq, zero_ctr);
     return cudaGetLastError();
 }
 

@@ -156,7 +156,7 @@ constexpr double kTcMinRowsPerExpert = 48.0;
 int tc_mt(double rows_per_expert) { return rows_per_expert > 96.0 ? 2 : 1; }
 
 struct GemmWs {
-    size_t xa, gs, partial, xt, total;
+    size_t xa, gs, partial, xt, work, total;
     int P, ksplit, spp, row_blocks, nt;
     bool tc;
 };
@@ -205,6 +205,8 @@ GemmWs gemm_layout(const ccq_weight *w, int m) {
     L.spp = ceil_div(nst, want);
     L.ksplit = ceil_div(nst, L.spp);
     size_t off = 0;
+    L.work = off;  // the decode kernel's work counter, zeroed by the activation packing
+    off = up256(off + 16);
     L.xa = off;
     off = up256(off + (size_t)L.P * K * 2);
     L.gs = off;
@@ -231,7 +233,9 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     L.err = off; off = up256(off + 16);
     L.seg = off; off = up256(off + sizeof(int) * (size_t)(E + 1));
     L.cursor = off; off = up256(off + sizeof(int) * (size_t)E);
-    L.dep = off; off = up256(off + sizeof(int) * (size_t)E);  // per-expert counters of the fused launch
+    // per-expert counters of the fused launch, then the work counters of the fused launch and of
+    // the two separate launches
+    L.dep = off; off = up256(off + sizeof(int) * (size_t)(E + 3));
     L.tok = off; off = up256(off + sizeof(int) * (size_t)L.P);
     L.rwp = off; off = up256(off + sizeof(float) * (size_t)L.P);
     L.inv = off; off = up256(off + sizeof(int) * (size_t)pairs);
@@ -358,8 +362,9 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
     }
     uint16_t *xa = reinterpret_cast<uint16_t *>(base + L.xa);
     float *gs = reinterpret_cast<float *>(base + L.gs);
+    int *work = reinterpret_cast<int *>(base + L.work);
     cudaError_t e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), nullptr, m, L.P, w->k,
-                                   level_of(w), xa, gs, s);
+                                   level_of(w), xa, gs, s, work);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     DecodeMaps maps;
     if (!decode_maps(maps, w, 1, xa, gs, L.P, L.nt)) return CCQ_ERR_CUDA;
@@ -385,6 +390,7 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
     }
     p.tma_scales = maps.tma_scales;
     set_format(p, w);
+    p.work = work;
     e = launch_decode_gemm_w2(p, maps.codes, maps.xa, maps.gs, maps.sc, L.row_blocks, L.ksplit, 1, L.nt, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     if (L.ksplit > 1) {
@@ -557,6 +563,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         p1.fuse_gsq = gs_h;
         p1.fuse_gsq_ld = gsum_ld(I);
         p1.fuse_level = level_of(w2);
+        p1.work = dep + num_experts;
         p2.dep = dep;
         e = launch_decode_moe_fused(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), p2, m2.codes, m2.xa, m2.gs,
                                     m2.sc, ceil_div(H, 256), num_experts, nt1, s);
@@ -572,6 +579,8 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     if (!fused) {
         p1.dep = p2.dep = nullptr;
         p1.fuse_gsq = nullptr;
+        p1.work = dep + num_experts + 1;
+        p2.work = dep + num_experts + 2;
         e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), 1, num_experts, nt1, s);
         if (e == cudaSuccess) e = trace(events, 3, s);
         if (e == cudaSuccess)

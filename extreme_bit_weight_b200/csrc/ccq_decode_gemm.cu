@@ -457,15 +457,26 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     // Unit descriptors, by unit ordinal modulo kUnitRing, written by the producer before the unit's
     // first load and read by the consumers after that load lands.  The producer runs at most
     // kStages iterations (so at most kStages units) ahead of the slowest consumer, whose unit --
-    // epilogue included -- therefore keeps its entry.
+    // epilogue included -- therefore keeps its entry.  After the last unit the producer posts an
+    // end marker (e < 0) through one more ring slot that carries no data.
     constexpr int kUnitRing = kStages + 2;
     __shared__ Unit udesc[kUnitRing];
     __shared__ int p_ord;  // producer: ordinal of unit P.U
-    auto p_seek = [&]() {  // first unit with work at or after P.u
-        int u = P.u;
+    // The next unit index.  With a work counter a CTA takes the next unit when it is ready for one,
+    // so units of unequal cost (16-stage gate/up against 7-stage down units, experts with two
+    // token chunks, experts without tokens) even out across CTAs; the counter hands out every
+    // gate/up unit before any down unit, and gate/up units wait on nothing, so the down units'
+    // waits always end.  Without one, CTA b takes units b, b + gridDim.x, ...
+    auto p_next = [&]() -> int {
+        if (p.work) return atomicAdd(p.work, 1);
+        const int u = P.u;
+        P.u += gridDim.x;
+        return u;
+    };
+    auto p_seek = [&]() {  // the next unit with work
         Unit U;
-        while (u < units && !load_unit_any<MP, FUSED>(p, p2, u, U)) u += gridDim.x;
-        P.u = u;
+        int u = p_next();
+        while (u < units && !load_unit_any<MP, FUSED>(p, p2, u, U)) u = p_next();
         P.U = U;
         P.done = u >= units;
         if (!P.done) udesc[p_ord++ % kUnitRing] = U;
@@ -532,7 +543,6 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             P.i = 0;
             P.st = U.s_begin + U.rot;
             if (c + 1 == U.nchunks) {
-                P.u += gridDim.x;
                 p_seek();
             } else {
                 P.c = c + 1;
@@ -557,6 +567,15 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                     break;
                 }
                 issue_next();
+            }
+            if (pok && !(P.pi >= kStages && !mbar_wait(&empty_bar[P.slot], (P.round & 1) ^ 1, p.err))) {
+                // end marker: a ring slot without loads whose descriptor stops the consumers
+                Unit end{};
+                end.e = -1;
+                udesc[p_ord++ % kUnitRing] = end;
+                mbar_arrive(&full_bar[P.slot]);
+            } else {
+                pok = false;
             }
             if (!pok) {
                 // consumers stopped releasing: let the copies in flight land before exiting (bounded)
@@ -607,12 +626,6 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     bool ok = true;
     int it = 0, slot = 0, round = 0, cc = 0;  // iteration (over all units), ring slot and round, chunk count
     int ec = 0;                               // fused gate/up chunks done (epilogue meeting parity)
-    // the number of units with work this CTA will process (same walk as the producer's)
-    int n_units = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
-        Unit t;
-        n_units += load_unit_any<MP, FUSED>(p, p2, u, t) ? 1 : 0;
-    }
     RowDecode rd[4];
     float sc_row[4];  // W4: per-channel scales, bf16-rounded; Q4: the rows' super scales
     uint32_t q4cur[4] = {0, 0, 0, 0}, q4nxt[4] = {0, 0, 0, 0};  // Q4: this / the next stage's scale nibbles
@@ -625,12 +638,13 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             for (int q = 0; q < 4; ++q) acc[t][n][q] = 0.0f;
     // walk: unit ordinal cu, token chunk c, position i of stage st in the chunk's rotated walk
     int cu = 0, c = 0, i = 0, st = 0;
-    while (cu < n_units) {
+    for (;;) {
         if (!ok || !mbar_wait(&full_bar[slot], round & 1, p.err)) {
             ok = false;
             break;
         }
         const Unit &U = udesc[cu % kUnitRing];  // written before this unit's first load was issued
+        if (U.e < 0) break;                     // the producer's end marker
         const DecodeGemmParams &pq = (FUSED && U.phase) ? p2 : p;
         const bool first = c == 0 && i == 0;
         if (first) st = U.s_begin + U.rot;

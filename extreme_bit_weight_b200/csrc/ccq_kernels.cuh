@@ -72,6 +72,9 @@ struct DecodeGemmParams {
     uint32_t *err;
     // work units (set by the launcher): unit u = (expert, k split, row block), row block fastest
     int row_blocks, ksplit, units;
+    // zeroed counter from which CTAs take their next unit (NULL: CTA b takes b, b + grid, ...);
+    // a fused launch uses the gate/up block's
+    int *work;
     // fused MoE launch (gate/up and down in one kernel): the gate/up epilogue also writes the down
     // operand's gsq table and counts finished units per expert in dep[]; a down unit of expert e
     // loads only after dep[e] reaches dep_need
@@ -142,8 +145,9 @@ cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, c
 cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes, float *scales, cudaStream_t s);
 
 // x (BF16 [rows][K], row r taken from x[tok_of ? tok_of[p] : p]) -> XA operand + group sums.
+// zero_ctr (may be NULL): an int the kernel sets to 0 (the following matmul's work counter).
 cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,
-                           uint16_t *xa, float *gsq, cudaStream_t s);
+                           uint16_t *xa, float *gsq, cudaStream_t s, int *zero_ctr = nullptr);
 // group-sum table of an operand already in XA layout (rows [0, P_valid))
 cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float level, float *gsq,
                                 cudaStream_t s);
@@ -151,7 +155,8 @@ cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, f
 cudaError_t launch_splitk_reduce(const float *partial, int ksplit, size_t split_stride, int M, int N,
                                  uint16_t *y, cudaStream_t s);
 
-// MoE routing: counts, offsets, placement, inverse map; validates ids; zeroes dep[E] (if given).
+// MoE routing: counts, offsets, placement, inverse map; validates ids; zeroes dep[0, E + 3) (if
+// given): the fused launch's per-expert counters and three work counters.
 cudaError_t launch_moe_route(const int *ids, const float *rw, int T, int topk, int E, int *seg_off,
                              int *cursor, int *tok_of, float *rw_perm, int *inv, int *dep, uint32_t *err,
                              cudaStream_t s);
