@@ -59,6 +59,8 @@ def lib():
         L.oracle_dequant_w4.argtypes = [P, P, i, i, P]
         L.oracle_dequant_w2q4.argtypes = [P, P, P, P, P, i, i, i, P]
         L.oracle_dequant_w2std.argtypes = [P, P, i, i, i, P]
+        L.oracle_dequant_emb.argtypes = [i, P, P, i, i, P]
+        L.oracle_encode_emb.argtypes = [i, P, i, i, P, P]
         L.oracle_quantize_w2std.argtypes = [P, i, i, i, P, P]
         L.oracle_encode_w2q4.argtypes = [P, i, i, i, ctypes.c_uint32, P, P, P, P, P]
         L.oracle_gemm_bf16_f64.argtypes = [P, P, i, i, i, P]
@@ -175,6 +177,37 @@ def quantize_w2std(w, group: int = 64):
     if lib().oracle_quantize_w2std(_p(w), n, k, group, _p(codes), _p(scales)) != 0:
         raise ValueError("quantize_w2std: bad shape")
     return codes, scales
+
+
+# Formats without code cluster, group scale in the redundant bits (CCQ §3.5 Algorithm 2):
+# kind 1 = (4,3,2) 2.75 bpw, 22 uint8 codes per 64 weights; kind 2 = hybrid (3,3,2)+(3,4,2) 2.5 bpw,
+# 10 uint16 words per 64 weights.  One fp32 super scale per row.
+EMB_KINDS = {1: (np.uint8, 22), 2: (np.uint16, 10)}
+
+
+def dequant_emb(kind: int, codes, super_scale) -> np.ndarray:
+    """Algorithm 2 decode -> BF16 bits [n][k]."""
+    dt, nw = EMB_KINDS[kind]
+    codes = _c(codes, dt)
+    n = codes.shape[0]
+    k = codes.shape[1] // nw * 64
+    sup = _c(super_scale, np.float32).reshape(n)
+    out = np.zeros((n, k), dtype=np.uint16)
+    if lib().oracle_dequant_emb(kind, _p(codes), _p(sup), n, k, _p(out)) != 0:
+        raise ValueError("dequant_emb: bad shape")
+    return out
+
+
+def encode_emb(kind: int, w):
+    """Algorithm 2 format encoder -> (codes [n][k/64*words], super_scale [n])."""
+    dt, nw = EMB_KINDS[kind]
+    w = _c(w, np.float32)
+    n, k = w.shape
+    codes = np.zeros((n, k // 64 * nw), dtype=dt)
+    sup = np.zeros(n, dtype=np.float32)
+    if lib().oracle_encode_emb(kind, _p(w), n, k, _p(codes), _p(sup)) != 0:
+        raise ValueError("encode_emb: bad shape")
+    return codes, sup
 
 
 def dequant_w4(codes, scales) -> np.ndarray:

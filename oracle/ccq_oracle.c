@@ -259,6 +259,188 @@ int oracle_quantize_w2std(const float *w, int n, int k, int group, uint8_t *code
 }
 
 /* ------------------------------------------------------------------------------------------
+ * Formats without code cluster whose group scale sits in the group's redundant bits: [CCQ] §3.2
+ * "Hybrid Encoding", §3.4 "Scale Compression" (redundant bits; Eq. 5, first case), §3.5
+ * Algorithm 2 ("Dequantization without Code Cluster"), Table 1 rows (4,3,2) and (3,3,2)(3,4,2).
+ *
+ * kind 1, (L,N,S) = (4,3,2), 2.75 bpw.  A group of 64 weights is 22 one-byte codes W_q[0..21].
+ *   Code j < 21 covers weights 3j..3j+2 (its 3 states; Table 1 shifts [4,2,0], mask 0xF).  The
+ *   last code covers weight 63 with its first state (its top 4 bits); its low 4 bits, redundant
+ *   for the weights, hold the group's 4-bit scale (s_mask 0xF).  codes[n][k/64 * 22].
+ * kind 2, hybrid (3,3,2)+(3,4,2), 2.5 bpw.  A group is ten 16-bit words W_q[0..9] (uint16,
+ *   codes[n][k/64 * 10]).  Word j < 9 covers weights 7j..7j+6: a (3,3,2) code in its top 7 bits
+ *   (states at shifts 13, 11, 9) then a (3,4,2) code in its low 9 bits (shifts 6, 4, 2, 0); Table
+ *   1 mask 0x7.  The last word covers weight 63 with its top 3 bits and holds a 13-bit scale in
+ *   its low 13 bits (s_mask 0x1FFF).
+ * Decode (Algorithm 2): s = (last code & s_mask) * s_super[n], one fp32 multiply (reading, as for
+ * the code-cluster format's 4-bit scales); w = bf16((u - zp) * bf16(s)) with zp = 2^(L-1), 8 and
+ * 4 (reading, as CCQ's 32).  The states come from the codebooks built by walking the state graph.
+ * ------------------------------------------------------------------------------------------ */
+static int32_t *g_cb432 = NULL, *g_cb332 = NULL, *g_cb342 = NULL;
+
+static int emb_codebooks(void)
+{
+    if (!g_cb432) {
+        int32_t *a = (int32_t *)malloc(sizeof(int32_t) * 256 * 3);
+        int32_t *b = (int32_t *)malloc(sizeof(int32_t) * 128 * 3);
+        int32_t *c = (int32_t *)malloc(sizeof(int32_t) * 512 * 4);
+        if (!a || !b || !c || oracle_codebook(4, 3, 2, a) || oracle_codebook(3, 3, 2, b) ||
+            oracle_codebook(3, 4, 2, c)) {
+            free(a); free(b); free(c);
+            return -1;
+        }
+        g_cb332 = b;
+        g_cb342 = c;
+        g_cb432 = a;
+    }
+    return 0;
+}
+
+/* words per group, scale mask, zero-point, raw-scale divisor 2^(L-1) - 1 */
+static int emb_words(int kind) { return kind == 1 ? 22 : 10; }
+static uint32_t emb_smask(int kind) { return kind == 1 ? 0xFu : 0x1FFFu; }
+static int emb_zp(int kind) { return kind == 1 ? 8 : 4; }
+
+/* state of weight i (0..63) of a group whose codes are W[0..words) */
+static int32_t emb_state(int kind, const uint32_t *W, int i)
+{
+    if (kind == 1) return g_cb432[(size_t)W[i / 3] * 3 + i % 3];
+    uint32_t word = W[i / 7];
+    int t = i % 7;
+    return t < 3 ? g_cb332[(size_t)(word >> 9) * 3 + t] : g_cb342[(size_t)(word & 0x1FFu) * 4 + (t - 3)];
+}
+
+static double emb_level(int32_t u, int zp, float s_bf16)
+{
+    return (double)oracle_bf16_to_float(oracle_bf16_bits((float)((double)(u - zp) * (double)s_bf16)));
+}
+
+static void emb_load_group(int kind, const void *codes, size_t row, int nwords_row, int g, uint32_t *W)
+{
+    int nw = emb_words(kind);
+    for (int j = 0; j < nw; ++j) {
+        size_t at = row * (size_t)nwords_row + (size_t)g * nw + j;
+        W[j] = kind == 1 ? ((const uint8_t *)codes)[at] : ((const uint16_t *)codes)[at];
+    }
+}
+
+int oracle_dequant_emb(int kind, const void *codes, const float *super, int n, int k, uint16_t *out)
+{
+    if ((kind != 1 && kind != 2) || emb_codebooks() || n < 0 || k < 0 || k % 64) return -1;
+    int ng = k / 64, nw = emb_words(kind), zp = emb_zp(kind);
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < n; ++r)
+        for (int g = 0; g < ng; ++g) {
+            uint32_t W[22];
+            emb_load_group(kind, codes, (size_t)r, ng * nw, g, W);
+            float s = (float)(W[nw - 1] & emb_smask(kind)) * super[r];
+            float sb = oracle_bf16_to_float(oracle_bf16_bits(s));
+            for (int i = 0; i < 64; ++i)
+                out[(size_t)r * k + (size_t)g * 64 + i] =
+                    oracle_bf16_bits((float)emb_level(emb_state(kind, W, i), zp, sb));
+        }
+    return 0;
+}
+
+/* Encoder (the pages print none for these formats; plain reading of Algorithm 1 and §3.4):
+ * raw group scale r_g = max|w_g| / (2^(L-1) - 1) (fp32: 7 or 3); s_super = max_g r_g / (2^b - 1)
+ * (fp32; b = 4 or 13 scale bits); q_g = clip(round-half-even(r_g / s_super), 0, 2^b - 1) in fp64
+ * (0 when s_super = 0); the group scale is fl32(q_g * s_super).  Each full code is the one, over all
+ * codes of its width, whose decoded weights have the least squared error to the group's weights
+ * (ties to the smallest code); the last code's weight state is chosen the same way over its 2^L
+ * values, and its low bits are q_g. */
+int oracle_encode_emb(int kind, const float *w, int n, int k, void *codes, float *super)
+{
+    if ((kind != 1 && kind != 2) || emb_codebooks() || n < 0 || k <= 0 || k % 64) return -1;
+    int ng = k / 64, nw = emb_words(kind), zp = emb_zp(kind);
+    int L = kind == 1 ? 4 : 3;
+    double rdiv = kind == 1 ? 7.0 : 3.0, qmax = (double)emb_smask(kind);
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < n; ++r) {
+        const float *wr = w + (size_t)r * k;
+        float *raw = (float *)malloc(sizeof(float) * (size_t)ng);
+        if (!raw) continue;
+        double smax = 0.0;
+        for (int g = 0; g < ng; ++g) {
+            double amax = 0.0;
+            for (int i = 0; i < 64; ++i) {
+                double a = fabs((double)wr[g * 64 + i]);
+                if (a > amax) amax = a;
+            }
+            raw[g] = (float)(amax / rdiv);
+            if ((double)raw[g] > smax) smax = (double)raw[g];
+        }
+        float sup = (float)(smax / qmax);
+        super[r] = sup;
+        int old = fegetround();
+        fesetround(FE_TONEAREST);
+        for (int g = 0; g < ng; ++g) {
+            double qq = sup > 0.0f ? nearbyint((double)raw[g] / (double)sup) : 0.0;
+            if (qq < 0.0) qq = 0.0;
+            if (qq > qmax) qq = qmax;
+            uint32_t q = (uint32_t)qq;
+            float sb = oracle_bf16_to_float(oracle_bf16_bits((float)q * sup));
+            const float *v = wr + g * 64;
+            uint32_t W[22];
+            if (kind == 1) {
+                for (int j = 0; j < 21; ++j) {
+                    double best = INFINITY;
+                    uint32_t bc = 0;
+                    for (uint32_t c = 0; c < 256; ++c) {
+                        double e = 0.0;
+                        for (int t = 0; t < 3; ++t) {
+                            double d = (double)v[3 * j + t] - emb_level(g_cb432[c * 3 + t], zp, sb);
+                            e += d * d;
+                        }
+                        if (e < best) { best = e; bc = c; }
+                    }
+                    W[j] = bc;
+                }
+            } else {
+                for (int j = 0; j < 9; ++j) {
+                    double best = INFINITY;
+                    uint32_t b7 = 0, b9 = 0;
+                    for (uint32_t c = 0; c < 128; ++c) {
+                        double e = 0.0;
+                        for (int t = 0; t < 3; ++t) {
+                            double d = (double)v[7 * j + t] - emb_level(g_cb332[c * 3 + t], zp, sb);
+                            e += d * d;
+                        }
+                        if (e < best) { best = e; b7 = c; }
+                    }
+                    best = INFINITY;
+                    for (uint32_t c = 0; c < 512; ++c) {
+                        double e = 0.0;
+                        for (int t = 0; t < 4; ++t) {
+                            double d = (double)v[7 * j + 3 + t] - emb_level(g_cb342[c * 4 + t], zp, sb);
+                            e += d * d;
+                        }
+                        if (e < best) { best = e; b9 = c; }
+                    }
+                    W[j] = (b7 << 9) | b9;
+                }
+            }
+            /* the last code: weight 63 in its top L bits, the scale in the rest */
+            double best = INFINITY;
+            uint32_t bu = 0;
+            for (uint32_t u = 0; u < (1u << L); ++u) {
+                double d = (double)v[63] - emb_level((int32_t)u, zp, sb);
+                if (d * d < best) { best = d * d; bu = u; }
+            }
+            W[nw - 1] = (bu << (kind == 1 ? 4 : 13)) | q;
+            for (int j = 0; j < nw; ++j) {
+                size_t at = (size_t)r * ng * nw + (size_t)g * nw + j;
+                if (kind == 1) ((uint8_t *)codes)[at] = (uint8_t)W[j];
+                else ((uint16_t *)codes)[at] = (uint16_t)W[j];
+            }
+        }
+        fesetround(old);
+        free(raw);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------
  * W4 per-channel dequantization ([WINT2] quantization_config "wint4", "per_channel"; [GPTQ]
  * Part 2 pack_int4/unpack_int4): codes[n][k/2], two signed 4-bit codes per byte, the first code
  * of a pair in the low nibble; the code is sign-extended; w = bf16(q * bf16(scale[n])).

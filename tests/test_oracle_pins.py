@@ -625,3 +625,138 @@ def test_quantize_w2std_picks_nearest_level_brute_force():
     best = dist.min(axis=-1)
     got = np.abs(deq - w.astype(np.float64))
     assert np.allclose(got, best, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------------------------
+# Formats without code cluster, scale in the redundant bits (CCQ §3.2, §3.4, §3.5 Algorithm 2,
+# Table 1 rows (4,3,2) and (3,3,2)(3,4,2)).  Expected values below come from Table 1's printed
+# shift lists and masks, not from the oracle's codebook walk.
+# ----------------------------------------------------------------------------------------------
+T1_432 = ([4, 2, 0], 0xF)                       # Table 1: weight bit-shift, weight mask
+T1_HYB = ([13, 11, 9, 6, 4, 2, 0], 0x7)
+
+
+def test_dequant_emb_432_hand_example():
+    codes = np.zeros((1, 22), dtype=np.uint8)
+    codes[0, 0] = 0xB6            # states 11, 13, 6 -> levels 3, 5, -2
+    codes[0, 21] = 0x9A           # weight 63: state 9 (level 1); low nibble: scale 10
+    sup = np.array([0.25], np.float32)            # s = 10 * 0.25 = 2.5
+    out = oracle.bf16_to_f64(oracle.dequant_emb(1, codes, sup))[0]
+    sh, m = T1_432
+    assert [((0xB6 >> x) & m) - 8 for x in sh] == [3, 5, -2]
+    assert list(out[:3]) == [7.5, 12.5, -5.0]
+    assert list(out[3:63]) == [-20.0] * 60        # byte 0 -> states 0, 0, 0 -> level -8
+    assert out[63] == 2.5
+
+
+def test_dequant_emb_hybrid_hand_example():
+    c7, c9, u63, q13 = 0b1011100, 0b110011011, 6, 1000
+    word0 = (c7 << 9) | c9
+    codes = np.zeros((1, 10), dtype=np.uint16)
+    codes[0, 0] = word0
+    codes[0, 9] = (u63 << 13) | q13
+    sup = np.array([0.001], np.float32)           # fl32(1000 * 0.001f) = 1.0 exactly
+    assert np.float32(1000) * sup[0] == np.float32(1.0)
+    sh, m = T1_HYB
+    levels = [((word0 >> x) & m) - 4 for x in sh]
+    assert levels == [1, 3, 0, 2, -3, 2, -1]
+    out = oracle.bf16_to_f64(oracle.dequant_emb(2, codes, sup))[0]
+    assert list(out[:7]) == levels
+    assert list(out[7:63]) == [-4.0] * 56         # word 0 -> every state 0 -> level -4
+    assert out[63] == u63 - 4
+
+
+def test_emb_bpw_from_stored_sizes():
+    # Eq. 5, first case: T * ceil(g/N) / g with the scale in the redundant bits (2.75 and 2.5)
+    w = synth.weights_normal(8, 512, 97)
+    for kind, bpw in ((1, 2.75), (2, 2.5)):
+        codes, sup = oracle.encode_emb(kind, w)
+        assert codes.nbytes * 8 / w.size == bpw
+
+
+def test_emb_states_are_convolutional():
+    # consecutive states of one code share L - S bits (§3.1): (4,3,2) shares 2, both hybrid codes 1
+    rng = np.random.default_rng(98)
+    sup = np.full(1, 2.0 ** -4, np.float32)
+    codes = rng.integers(0, 256, size=(1, 22 * 4), dtype=np.uint8)
+    codes[0, 21::22] = (codes[0, 21::22] & 0xF0) | 0x3   # scale 3 * 2^-4 (BF16-exact)
+    u = oracle.bf16_to_f64(oracle.dequant_emb(1, codes, sup))[0] / (3 * 2.0 ** -4) + 8
+    assert np.all(u == np.round(u))
+    u = u.astype(int).reshape(4, 64)[:, :63].reshape(4, 21, 3)
+    assert np.all((u[:, :, 0] & 3) == (u[:, :, 1] >> 2)) and np.all((u[:, :, 1] & 3) == (u[:, :, 2] >> 2))
+    words = rng.integers(0, 1 << 16, size=(1, 10 * 4), dtype=np.uint16)
+    words[0, 9::10] = (words[0, 9::10] & 0xE000) | 0x3
+    u = oracle.bf16_to_f64(oracle.dequant_emb(2, words, sup))[0] / (3 * 2.0 ** -4) + 4
+    u = u.astype(int).reshape(4, 64)[:, :63].reshape(4, 9, 7)
+    for a, b in ((0, 1), (1, 2), (3, 4), (4, 5), (5, 6)):  # within the (3,3,2) and the (3,4,2) code
+        assert np.all((u[:, :, a] & 1) == (u[:, :, b] >> 2))
+
+
+def _viterbi_min_error(v, L, S, level):
+    """Least squared error over all walks of len(v) states of an (L, N, S) code (independent DP)."""
+    nstate = 1 << L
+    cost = np.array([(v[0] - level(s)) ** 2 for s in range(nstate)])
+    for x in v[1:]:
+        nxt = np.full(nstate, np.inf)
+        for s in range(nstate):
+            for b in range(1 << S):
+                t = ((s << S) | b) & (nstate - 1)
+                nxt[t] = min(nxt[t], cost[s] + (x - level(t)) ** 2)
+        cost = nxt
+    return cost.min()
+
+
+def test_encode_emb_codes_are_optimal():
+    w = synth.weights_normal(2, 128, 99)
+    for kind in (1, 2):
+        codes, sup = oracle.encode_emb(kind, w)
+        deq = oracle.bf16_to_f64(oracle.dequant_emb(kind, codes, sup))
+        zp = 8 if kind == 1 else 4
+        for r in range(2):
+            for g in range(2):
+                grp = w[r, 64 * g:64 * g + 64].astype(np.float64)
+                got = deq[r, 64 * g:64 * g + 64]
+                # the group's scale, recovered from a decoded level is not needed: decode level u
+                # as the oracle does, through BF16 of (u - zp) * s with s read back from the codes
+                last = int(codes[r, (g + 1) * (22 if kind == 1 else 10) - 1])
+                s = np.float32(last & (0xF if kind == 1 else 0x1FFF)) * sup[r]
+                sb = oracle.bf16_to_f64(oracle.bf16_bits(np.float32(s)))
+                level = lambda u: float(oracle.bf16_to_f64(oracle.bf16_bits(np.float32((u - zp) * sb))))
+                if kind == 1:
+                    spans = [(3 * j, 3) for j in range(21)]
+                    L, S = 4, 2
+                else:
+                    spans = [(7 * j + o, n) for j in range(9) for (o, n) in ((0, 3), (3, 4))]
+                    L, S = 3, 2
+                for (a, nn) in spans:
+                    best = _viterbi_min_error(grp[a:a + nn], L, S, level)
+                    err = float(((grp[a:a + nn] - got[a:a + nn]) ** 2).sum())
+                    assert abs(err - best) <= 1e-12 * max(1.0, best), (kind, r, g, a)
+                # weight 63: the nearest of the 2^L levels
+                assert (grp[63] - got[63]) ** 2 <= min((grp[63] - level(u)) ** 2 for u in range(1 << L)) + 1e-18
+
+
+def test_encode_emb_scale_quantizer():
+    w = synth.weights_normal(3, 512, 100)
+    w[2] = 0.0                                             # an all-zero row
+    for kind, qmax, rdiv in ((1, 15, 7.0), (2, 8191, 3.0)):
+        codes, sup = oracle.encode_emb(kind, w)
+        nw = 22 if kind == 1 else 10
+        q = codes.reshape(3, 8, nw)[:, :, -1].astype(np.int64) & qmax
+        raw = (np.abs(w.reshape(3, 8, 64)).max(axis=2) / rdiv).astype(np.float32)
+        assert np.array_equal(sup[:2], (raw[:2].max(axis=1) / qmax).astype(np.float32))
+        assert sup[2] == 0.0 and np.all(q[2] == 0)
+        for r in range(2):
+            assert q[r, np.argmax(raw[r])] == qmax          # the largest group takes the top code
+            assert np.all(np.abs(q[r] - raw[r] / sup[r]) <= 0.5 + 1e-6)
+        deq = oracle.bf16_to_f64(oracle.dequant_emb(kind, codes, sup))
+        assert np.all(deq[2] == 0.0)
+
+
+def test_encode_emb_more_bits_less_error():
+    w = synth.weights_normal(16, 1024, 101)
+    err = {}
+    for kind in (1, 2):
+        codes, sup = oracle.encode_emb(kind, w)
+        err[kind] = float(((oracle.bf16_to_f64(oracle.dequant_emb(kind, codes, sup)) - w) ** 2).mean())
+    assert err[1] < err[2] < float((w.astype(np.float64) ** 2).mean())
