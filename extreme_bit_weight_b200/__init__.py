@@ -28,6 +28,9 @@ CCQ_FMT_W2_CCQ_G64 = 1
 CCQ_FMT_W4_PER_CHANNEL = 2
 CCQ_FMT_W2_CCQ_G64_Q4SCALE = 3
 CCQ_FMT_W2_STD_G64 = 4
+CCQ_FMT_W275_432 = 5
+CCQ_FMT_W25_HYBRID = 6
+EMB_GROUP_BYTES = {CCQ_FMT_W275_432: 22, CCQ_FMT_W25_HYBRID: 20}
 CCQ_ENC_LITERAL_EQ1 = 1
 CCQ_ENC_REFIT_SCALE = 2
 
@@ -71,6 +74,7 @@ _lib.ccq_encode_device_workspace_size.restype = ctypes.c_size_t
 _lib.ccq_encode_device.argtypes = [_P, _I, _I, _I, ctypes.c_uint32, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.ccq_encode_host_q4.argtypes = [_P, _I, _I, _I, ctypes.c_uint32, _I, _P, _P, _P, _P, _P, _P]
 _lib.ccq_quantize_std_device.argtypes = [_P, _I, _I, _P, _P, _P]
+_lib.ccq_encode_emb_device.argtypes = [_I, _P, _I, _I, _P, _P, _P]
 _lib.ccq_dequant_bf16.argtypes = [ctypes.POINTER(ccq_weight), _I, _P, _P]
 _lib.ccq_gemm_workspace_size.argtypes = [ctypes.POINTER(ccq_weight), _I]
 _lib.ccq_gemm_workspace_size.restype = ctypes.c_size_t
@@ -182,6 +186,18 @@ def ccq_quantize_std_device(w: torch.Tensor, stream=None):
     _check(_lib.ccq_quantize_std_device(_dptr(w), n, k, _dptr(codes), _dptr(scales), _stream(stream)),
            "ccq_quantize_std_device")
     return codes, scales
+
+
+def ccq_encode_emb_device(fmt: int, w: torch.Tensor, stream=None):
+    """Encode fp32 w [n][k] on the GPU into CCQ_FMT_W275_432 or CCQ_FMT_W25_HYBRID -> device tensors
+    (codes [n][k/64 * 22 or 20] uint8, super_scale [n])."""
+    w = w.contiguous()
+    n, k = w.shape
+    codes = torch.empty((n, k // 64 * EMB_GROUP_BYTES[fmt]), dtype=torch.uint8, device=w.device)
+    sup = torch.empty(n, dtype=torch.float32, device=w.device)
+    _check(_lib.ccq_encode_emb_device(fmt, _dptr(w), n, k, _dptr(codes), _dptr(sup), _stream(stream)),
+           "ccq_encode_emb_device")
+    return codes, sup
 
 
 def ccq_quantize_w4_host(w: np.ndarray, threads: int = 0):

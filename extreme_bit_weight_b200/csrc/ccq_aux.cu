@@ -127,6 +127,39 @@ __global__ void dequant_std_kernel(const uint8_t *__restrict__ codes, const floa
     }
 }
 
+// Formats with the group scale in the redundant bits (CCQ §3.5 Algorithm 2; Table 1 rows (4,3,2) and
+// (3,3,2)(3,4,2)), one thread per (row, group).  kind 1: 22 one-byte codes per group, states at
+// shifts 4, 2, 0 (mask 0xF, zero-point 8), code 21 = weight 63's state (top nibble) and the 4-bit
+// scale (low nibble).  kind 2: ten little-endian 16-bit words, states at shifts 13, 11, 9, 6, 4, 2,
+// 0 (mask 0x7, zero-point 4), word 9 = weight 63's state (top 3 bits) and the 13-bit scale.
+// s = bf16(fl32(q * super[row])); w = bf16((u - zp) * s), an exact product rounded once.
+__global__ void dequant_emb_kernel(int kind, const uint8_t *__restrict__ codes, const float *__restrict__ super,
+                                   int rows, int K, uint16_t *__restrict__ out) {
+    const int ng = K / 64, gb = kind == 1 ? 22 : 20;
+    const int kShift[7] = {13, 11, 9, 6, 4, 2, 0};
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < (size_t)rows * ng;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int r = (int)(idx / ng), g = (int)(idx % ng);
+        const uint8_t *c = codes + idx * gb;
+        const uint32_t q = kind == 1 ? (c[21] & 0xFu) : (((uint32_t)c[18] | ((uint32_t)c[19] << 8)) & 0x1FFFu);
+        const float s = bf16_bits_to_float(float_to_bf16_bits(__fmul_rn((float)q, __ldg(super + r))));
+        uint16_t *o = out + (size_t)r * K + (size_t)g * 64;
+        for (int i = 0; i < 64; ++i) {
+            int u;
+            if (kind == 1) {
+                const int j = i < 63 ? i / 3 : 21, sh = i < 63 ? 4 - 2 * (i % 3) : 4;
+                u = (c[j] >> sh) & 0xF;
+                u -= 8;
+            } else {
+                const int j = i < 63 ? i / 7 : 9, sh = i < 63 ? kShift[i % 7] : 13;
+                const uint32_t word = (uint32_t)c[2 * j] | ((uint32_t)c[2 * j + 1] << 8);
+                u = (int)((word >> sh) & 0x7u) - 4;
+            }
+            o[i] = float_to_bf16_bits(__fmul_rn((float)u, s));
+        }
+    }
+}
+
 // WINT2-Standard round-to-nearest, one warp per (row, 64-column group); lane l holds columns 2l,
 // 2l+1.  s = bf16(max|w| / 2); the level round_half_even(w / s) clipped to [-2, 1] is decided by
 // comparing w with s/2 and 3s/2, which are exact in fp32 for a BF16 s, so the decision equals the
@@ -353,6 +386,9 @@ cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, c
             codes, q4 ? nullptr : scales, alpha, beta, rows, K, out, scale_q4, super);
     } else if (fmt == CCQ_FMT_W2_STD_G64) {
         dequant_std_kernel<<<grid_for((size_t)rows * K / 4, 256), 256, 0, s>>>(codes, scales, rows, K, out);
+    } else if (fmt == CCQ_FMT_W275_432 || fmt == CCQ_FMT_W25_HYBRID) {
+        dequant_emb_kernel<<<grid_for((size_t)rows * (K / 64), 128), 128, 0, s>>>(fmt == CCQ_FMT_W275_432 ? 1 : 2, codes,
+                                                                                   super, rows, K, out);
     } else {
         dequant_w4_kernel<<<grid_for((size_t)rows * K / 2, 256), 256, 0, s>>>(codes, scales, rows, K, out);
     }

@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/ccq.h"
 #include "ccq_device.cuh"
@@ -51,10 +52,18 @@ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 ccq_status check_weight(const ccq_weight *w, int experts) {
     if (!w || experts <= 0) return CCQ_ERR_INVALID_ARG;
     if (w->fmt != CCQ_FMT_W2_CCQ_G64 && w->fmt != CCQ_FMT_W4_PER_CHANNEL && w->fmt != CCQ_FMT_W2_CCQ_G64_Q4SCALE &&
-        w->fmt != CCQ_FMT_W2_STD_G64)
+        w->fmt != CCQ_FMT_W2_STD_G64 && w->fmt != CCQ_FMT_W275_432 && w->fmt != CCQ_FMT_W25_HYBRID)
         return CCQ_ERR_UNSUPPORTED;
     if (w->n <= 0 || w->k <= 0 || w->n % 16 || w->k % 64) return CCQ_ERR_INVALID_ARG;
     if (!w->codes || !aligned16(w->codes)) return CCQ_ERR_INVALID_ARG;
+    if (w->fmt == CCQ_FMT_W275_432 || w->fmt == CCQ_FMT_W25_HYBRID) {
+        if (w->group != 64) return CCQ_ERR_UNSUPPORTED;
+        // the code rows' pitch must be a multiple of 16 bytes (TMA)
+        if (w->k % (w->fmt == CCQ_FMT_W275_432 ? 512 : 256)) return CCQ_ERR_INVALID_ARG;
+        if (!w->super_scale || !aligned16(w->super_scale)) return CCQ_ERR_INVALID_ARG;
+        if ((size_t)experts * w->n > (size_t)INT32_MAX) return CCQ_ERR_INVALID_ARG;
+        return CCQ_OK;
+    }
     if (w->fmt == CCQ_FMT_W2_CCQ_G64_Q4SCALE) {
         if (w->group != 64) return CCQ_ERR_UNSUPPORTED;
         if (w->k % 128 || !w->scale_q4 || !w->super_scale || !w->alpha || !w->beta) return CCQ_ERR_INVALID_ARG;
@@ -72,9 +81,15 @@ ccq_status check_weight(const ccq_weight *w, int experts) {
     return CCQ_OK;
 }
 
+// Formats with the scale in the redundant bits: 1 = (4,3,2), 2 = hybrid, 0 otherwise.
+inline int emb_kind(const ccq_weight *w) {
+    return w->fmt == CCQ_FMT_W275_432 ? 1 : w->fmt == CCQ_FMT_W25_HYBRID ? 2 : 0;
+}
+
 // The weight-format fields of a kernel parameter block.
 template <class Params>
 void set_format(Params &p, const ccq_weight *w) {
+    if constexpr (std::is_same<Params, TcGemmParams>::value) p.emb = emb_kind(w);
     p.scales = w->scales;
     p.alpha = w->alpha;
     p.beta = w->beta;
@@ -173,7 +188,7 @@ int sm_count() {
 
 GemmWs gemm_layout(const ccq_weight *w, int m) {
     GemmWs L{};
-    if (m >= kTcMinM) {
+    if (m >= kTcMinM || emb_kind(w)) {  // (the embedded-scale formats run on the tcgen05 kernel only)
         L.tc = true;
         L.P = m;
         L.xt = 0;
@@ -229,6 +244,7 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     L.P = (pairs + 3) & ~3;
     L.tc = (double)pairs / E >= kTcMinRowsPerExpert;
     L.max_tiles = L.P / 128 + E + 1;  // enough for 128-token tiles
+    // (the tile list is always laid out: the embedded-scale formats take the tcgen05 path at any size)
     size_t off = 0;
     L.err = off; off = up256(off + 16);
     L.seg = off; off = up256(off + sizeof(int) * (size_t)(E + 1));
@@ -245,8 +261,8 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     L.gs_x = off; if (!L.tc) off = up256(off + (size_t)L.P * gsum_ld(H) * 16);
     L.xa_h = off; off = up256(off + (size_t)L.P * I * 2);
     L.gs_h = off; if (!L.tc) off = up256(off + (size_t)L.P * gsum_ld(I) * 16);
-    L.tiles = off; if (L.tc) off = up256(off + sizeof(int2) * (size_t)L.max_tiles);
-    L.tcount = off; if (L.tc) off = up256(off + 16);
+    L.tiles = off; off = up256(off + sizeof(int2) * (size_t)L.max_tiles);
+    L.tcount = off; off = up256(off + 16);
     L.slot = off; off = up256(off + (size_t)L.P * H * 4);
     L.total = off;
     return L;
@@ -261,7 +277,15 @@ bool tc_maps(CUtensorMap &ta, CUtensorMap &tcodes, const ccq_weight *w, int expe
         if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return false;
     }
-    {
+    if (const int emb = emb_kind(w)) {
+        // rows of K/64 groups of 22 or 20 bytes; a code stage (4 groups) is one 112- or 80-byte box
+        const cuuint64_t row_bytes = (cuuint64_t)(K / 64) * (emb == 1 ? 22 : 20);
+        cuuint64_t dims[2] = {row_bytes, (cuuint64_t)experts * w->n};
+        cuuint64_t str[1] = {row_bytes};
+        cuuint32_t box[2] = {emb == 1 ? 112u : 80u, 128};
+        if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w->codes, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return false;
+    } else {
         const cuuint64_t row_bytes = (cuuint64_t)(w->fmt == CCQ_FMT_W4_PER_CHANNEL ? K / 2 : K / 4);
         cuuint64_t dims[2] = {row_bytes, (cuuint64_t)experts * w->n};
         cuuint64_t str[1] = {row_bytes};
@@ -455,7 +479,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         e = launch_moe_route(expert_ids, routing_w, T, topk, num_experts, seg, cursor, tok, rwp, inv, dep, err, s);
     if (e == cudaSuccess) e = trace(events, 1, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
-    if (L.tc) {
+    if (L.tc || emb_kind(w13) || emb_kind(w2)) {
         // prefill-sized: tcgen05 grouped GEMMs over (expert, 256-token tile) entries
         int2 *tiles = reinterpret_cast<int2 *>(base + L.tiles);
         int *tcount = reinterpret_cast<int *>(base + L.tcount);
@@ -593,6 +617,16 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     if (e == cudaSuccess) e = launch_moe_combine(slot, inv, T, topk, H, static_cast<uint16_t *>(y_bf16), s);
     if (e == cudaSuccess) e = trace(events, 6, s);
     return cuda_status(e);
+}
+
+ccq_status ccq_encode_emb_device(int32_t fmt, const float *w, int32_t n, int32_t k, uint8_t *codes,
+                                 float *super_scale, ccq_stream_t stream) {
+    if (fmt != CCQ_FMT_W275_432 && fmt != CCQ_FMT_W25_HYBRID) return CCQ_ERR_UNSUPPORTED;
+    if (!w || !codes || !super_scale || n < 0 || k <= 0 || k % 64) return CCQ_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(codes) || !aligned16(super_scale)) return CCQ_ERR_INVALID_ARG;
+    if ((long long)n * (k / 64) > 0x3FFFFFFFll) return CCQ_ERR_INVALID_ARG;
+    return cuda_status(launch_encode_emb(fmt == CCQ_FMT_W275_432 ? 1 : 2, w, n, k, codes, super_scale,
+                                         (cudaStream_t)stream));
 }
 
 ccq_status ccq_quantize_std_device(const float *w, int32_t n, int32_t k, uint8_t *codes, float *scales,

@@ -17,6 +17,7 @@
 
 #include "../../include/ccq.h"
 #include "ccq_device.cuh"
+#include "ccq_kernels.cuh"
 
 namespace ccq {
 namespace {
@@ -246,7 +247,128 @@ __global__ void __launch_bounds__(256) enc_bytes_kernel(const float *__restrict_
     if (live) codes[(size_t)r * (k / 4) + j] = byte;
 }
 
+// ---- formats with the scale in the redundant bits (§3.2, §3.4, Algorithm 2) -----------------------
+// kind 1, (4,3,2): 22 one-byte codes per 64 weights, states at shifts 4, 2, 0 (mask 0xF), zero-point
+//   8, 4-bit scale in code 21's low nibble.
+// kind 2, hybrid (3,3,2)+(3,4,2): 10 little-endian 16-bit words per 64 weights; word j < 9 = a 7-bit
+//   (3,3,2) code (states at 4, 2, 0 of it) above a 9-bit (3,4,2) code (states at 6, 4, 2, 0), mask
+//   0x7, zero-point 4; 13-bit scale in word 9's low 13 bits.
+// Scale: raw r_g = max|w_g| / (7 or 3) (fp32), super = max_g r_g / (15 or 8191) (fp32), q_g =
+// clip(round-half-even(r_g / super), 0, 15 or 8191) (0 when super = 0), s = bf16(fl32(q_g * super)).
+// Each full code is the argmin of its decoded weights' squared error over every code of its width
+// (ties to the smallest); the last code's state is the nearest level for weight 63.
+
+__device__ __forceinline__ double emb_raw(const float *g, int kind) {
+    double amax = 0.0;
+    for (int i = 0; i < 64; ++i) amax = fmax(amax, fabs((double)g[i]));
+    return (double)__double2float_rn(__ddiv_rn(amax, kind == 1 ? 7.0 : 3.0));
+}
+
+// 1: one block per row: its super scale
+__global__ void __launch_bounds__(128) enc_emb_super_kernel(int kind, const float *__restrict__ w, int n, int k,
+                                                            float *__restrict__ super) {
+    __shared__ double red[128];
+    const int r = blockIdx.x, ng = k / 64;
+    double m = 0.0;
+    for (int g = threadIdx.x; g < ng; g += blockDim.x) m = fmax(m, emb_raw(w + (size_t)r * k + (size_t)g * 64, kind));
+    red[threadIdx.x] = m;
+    __syncthreads();
+    for (int h = 64; h > 0; h >>= 1) {
+        if (threadIdx.x < h) red[threadIdx.x] = fmax(red[threadIdx.x], red[threadIdx.x + h]);
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) super[r] = __double2float_rn(__ddiv_rn(red[0], kind == 1 ? 15.0 : 8191.0));
+}
+
+// squared error of n consecutive weights v[0..n) against states taken from code c at the given shifts
+template <int N>
+__device__ __forceinline__ double emb_err(const double *v, uint32_t c, const int (&sh)[N], uint32_t mask,
+                                          const double *lev) {
+    double e = 0.0;
+#pragma unroll
+    for (int t = 0; t < N; ++t) {
+        const double d = __dsub_rn(v[t], lev[(c >> sh[t]) & mask]);
+        e = __dadd_rn(e, __dmul_rn(d, d));
+    }
+    return e;
+}
+
+// 2: one warp per (row, group); lane j searches code j
+__global__ void __launch_bounds__(256) enc_emb_codes_kernel(int kind, const float *__restrict__ w, int n, int k,
+                                                            const float *__restrict__ super,
+                                                            uint8_t *__restrict__ codes) {
+    __shared__ double sv[8][64];
+    __shared__ double slev[8][16];
+    const int wv = threadIdx.x >> 5, lane = threadIdx.x & 31, ng = k / 64;
+    const long long unit = (long long)blockIdx.x * 8 + wv;
+    if (unit >= (long long)n * ng) return;  // whole warps only: no barrier below
+    const int r = (int)(unit / ng), g = (int)(unit % ng);
+    const float *gw = w + (size_t)r * k + (size_t)g * 64;
+    sv[wv][lane] = (double)gw[lane];
+    sv[wv][lane + 32] = (double)gw[lane + 32];
+    __syncwarp();
+    const float sup = super[r];
+    const double raw = emb_raw(gw, kind);
+    const double qmax = kind == 1 ? 15.0 : 8191.0;
+    double qq = sup > 0.0f ? rint(__ddiv_rn(raw, (double)sup)) : 0.0;
+    qq = fmin(fmax(qq, 0.0), qmax);
+    const uint32_t q = (uint32_t)qq;
+    const float sb = to_bf16(__fmul_rn((float)q, sup));
+    const int zp = kind == 1 ? 8 : 4, L = kind == 1 ? 4 : 3;
+    if (lane < (1 << L)) slev[wv][lane] = (double)to_bf16(__fmul_rn((float)(lane - zp), sb));
+    __syncwarp();
+    const double *v = sv[wv], *lev = slev[wv];
+    const int nw = kind == 1 ? 22 : 10;
+    uint8_t *dst = codes + ((size_t)r * ng + g) * (size_t)(kind == 1 ? 22 : 20);
+    if (lane < nw - 1) {
+        if (kind == 1) {
+            const int sh[3] = {4, 2, 0};
+            double best = INFINITY;
+            uint32_t bc = 0;
+            for (uint32_t c = 0; c < 256; ++c) {
+                const double e = emb_err<3>(v + 3 * lane, c, sh, 0xFu, lev);
+                if (e < best) { best = e; bc = c; }
+            }
+            dst[lane] = (uint8_t)bc;
+        } else {
+            const int sh7[3] = {4, 2, 0}, sh9[4] = {6, 4, 2, 0};
+            double best = INFINITY;
+            uint32_t b7 = 0, b9 = 0;
+            for (uint32_t c = 0; c < 128; ++c) {
+                const double e = emb_err<3>(v + 7 * lane, c, sh7, 0x7u, lev);
+                if (e < best) { best = e; b7 = c; }
+            }
+            best = INFINITY;
+            for (uint32_t c = 0; c < 512; ++c) {
+                const double e = emb_err<4>(v + 7 * lane + 3, c, sh9, 0x7u, lev);
+                if (e < best) { best = e; b9 = c; }
+            }
+            reinterpret_cast<uint16_t *>(dst)[lane] = (uint16_t)((b7 << 9) | b9);
+        }
+    } else if (lane == nw - 1) {
+        double best = INFINITY;
+        uint32_t bu = 0;
+        for (uint32_t u = 0; u < (1u << L); ++u) {
+            const double d = __dsub_rn(v[63], lev[u]);
+            const double e = __dmul_rn(d, d);
+            if (e < best) { best = e; bu = u; }
+        }
+        if (kind == 1) dst[21] = (uint8_t)((bu << 4) | q);
+        else reinterpret_cast<uint16_t *>(dst)[9] = (uint16_t)((bu << 13) | q);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_encode_emb(int kind, const float *w, int rows, int K, void *codes, float *super, cudaStream_t s) {
+    if (rows <= 0) return cudaSuccess;
+    enc_emb_super_kernel<<<rows, 128, 0, s>>>(kind, w, rows, K, super);
+    const long long units = (long long)rows * (K / 64);
+    enc_emb_codes_kernel<<<(unsigned)((units + 7) / 8), 256, 0, s>>>(kind, w, rows, K, super,
+                                                                     static_cast<uint8_t *>(codes));
+    return cudaGetLastError();
+}
+
 }  // namespace ccq
 
 using namespace ccq;

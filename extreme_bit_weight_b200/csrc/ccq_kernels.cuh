@@ -124,6 +124,9 @@ struct TcGemmParams {
     const uint8_t *scale_q4;
     const float *super_scale;
     int std2;              // 1: WINT2-Standard plain 2-bit fields (no alpha/beta)
+    // 1 / 2: the (4,3,2) / hybrid format with the group scale in the redundant bits (codes and
+    // super_scale only)
+    int emb;
     uint32_t *err;
     // split-K (dense matmul with few tiles): ksplit > 1 splits the 64-column groups into ranges of
     // kg groups (a multiple of 4); each range writes EPI_PARTIAL_F32 sums at out + ks*out_split_stride
@@ -140,6 +143,10 @@ cudaError_t launch_pack_xt(const uint16_t *x, const int *tok_of, int P_valid, in
 cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, const float *alpha,
                            const float *beta, int rows, int K, uint16_t *out, cudaStream_t s,
                            const uint8_t *scale_q4 = nullptr, const float *super = nullptr);
+
+// Encoder for the formats with the scale in the redundant bits (kind 1 / 2): w fp32 [rows][K] ->
+// codes [rows][K/64 * (22 or 20) bytes] and super [rows].
+cudaError_t launch_encode_emb(int kind, const float *w, int rows, int K, void *codes, float *super, cudaStream_t s);
 
 // WINT2-Standard round-to-nearest: w fp32 [rows][K] -> codes [rows][K/4], scales [rows][K/64]
 cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes, float *scales, cudaStream_t s);

@@ -42,13 +42,20 @@ constexpr int kSBof = MT == 1 ? 3 : 2;
 constexpr int kSC = 2;   // code stages (4 groups each)
 constexpr int kATile = 128 * 64 * 2;   // 16 KB per 128-token sub-tile
 constexpr int kBTile = 256 * 64 * 2;   // 32 KB
-constexpr int kCTile = 2 * 128 * 64;   // 16 KB: two 128-row halves x 64 code bytes
+// Code bytes per row in one code stage (4 groups; W4: 2): 64 for CCQ, W4 and STD.  The formats with
+// the scale in the redundant bits (EMB) have 22 (kind 1) or 20 (kind 2) bytes per group: a kind-1
+// stage's 88 bytes start at an 8-byte boundary every other stage, and TMA boxes start at 16-byte
+// boundaries, so its box is 112 bytes wide, starting at the 16-byte boundary at or below.
+template <int EMB>
+constexpr int kCRowOf = EMB == 1 ? 112 : EMB == 2 ? 80 : 64;
+template <int EMB>
+constexpr int kCTileOf = 2 * 128 * kCRowOf<EMB>;  // two 128-row halves
 
-template <int MT>
+template <int MT, int EMB = 0>
 struct TcSmem {
     static constexpr int kA = kSA * MT * kATile;
     static constexpr int kB = kSBof<MT> * kBTile;
-    static constexpr int kC = kSC * kCTile;
+    static constexpr int kC = kSC * kCTileOf<EMB>;
     static constexpr int kTotal = kA + kB + kC + 1024;
     static_assert(kTotal + 512 <= 227 * 1024, "shared memory per CTA");
 };
@@ -197,7 +204,50 @@ __device__ __forceinline__ void decode_word_std_bf16(uint32_t w, uint32_t s2, ui
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
 // position p of a 16-column block holds column 4*(p%4) + p/4 (and the map is its own inverse)
-__device__ __forceinline__ int perm16(int p) { return ((p & 3) << 2) | (p >> 2); }
+__host__ __device__ constexpr int perm16(int p) { return ((p & 3) << 2) | (p >> 2); }
+
+// Algorithm 2 formats: the 32 states u[0..31] of this thread's half of a group (natural column
+// order) -> the two 16-column blocks of BF16 (u - zp) * s in position order.  Each register pairs
+// two states as BF16 (128 + u), subtracts 128 + zp exactly and multiplies by s once.
+template <int ZP>
+__device__ __forceinline__ void emb_pack(const uint32_t (&u)[32], uint32_t s2, uint32_t (&o)[2][8]) {
+    constexpr uint32_t Z = (uint32_t)(0x4300 + ZP) * 0x10001u;  // bf16x2(128 + zp)
+#pragma unroll
+    for (int b = 0; b < 2; ++b)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const uint32_t v = u[16 * b + perm16(2 * q)] | (u[16 * b + perm16(2 * q + 1)] << 16) | 0x43004300u;
+            o[b][q] = bmul2(bsub2(v, Z), s2);
+        }
+}
+
+// kind 1, (4,3,2): code j < 21 holds weights 3j..3j+2 at shifts 4, 2, 0 (mask 0xF); code 21 holds
+// weight 63 in its top nibble.  c[] holds codes 10*PT .. 10*PT+11 of the group, one per entry.
+template <int PT>
+__device__ __forceinline__ void emb1_states(const uint32_t (&c)[12], uint32_t (&u)[32]) {
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+        const int wi = 32 * PT + m;
+        const int j = wi < 63 ? wi / 3 : 21;
+        const int sh = wi < 63 ? 4 - 2 * (wi % 3) : 4;
+        u[m] = (c[j - 10 * PT] >> sh) & 0xFu;
+    }
+}
+
+// kind 2, hybrid: word j < 9 holds weights 7j..7j+6 at shifts 13, 11, 9 (its (3,3,2) code) and 6,
+// 4, 2, 0 (its (3,4,2) code), mask 0x7; word 9 holds weight 63 in its top 3 bits.  w[] holds the
+// group's ten words two per entry in w[0..4] (word 2i in the low half of w[i]).
+template <int PT>
+__device__ __forceinline__ void emb2_states(const uint32_t (&w)[12], uint32_t (&u)[32]) {
+    constexpr int kShift[7] = {13, 11, 9, 6, 4, 2, 0};
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+        const int wi = 32 * PT + m;
+        const int j = wi < 63 ? wi / 7 : 9;
+        const int sh = wi < 63 ? kShift[wi % 7] : 13;
+        u[m] = (w[j >> 1] >> (16 * (j & 1) + sh)) & 0x7u;
+    }
+}
 
 // Position in a ring of N shared-memory stages: slot and the parity of the current round (no
 // division by N in the loops).
@@ -237,11 +287,14 @@ __device__ __forceinline__ bool tile_of(const TcGemmParams &p, int w, TileInfo &
 }
 
 // STD: WINT2-Standard plain 2-bit fields (no per-row constants)
-template <int MT, bool W4, bool Q4 = false, bool STD = false>
+// EMB: 1 = (4,3,2), 2 = hybrid (3,3,2)+(3,4,2), the formats with the scale in the redundant bits
+template <int MT, bool W4, bool Q4 = false, bool STD = false, int EMB = 0>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_codes,
                   const TcGemmParams p) {
-    using S = TcSmem<MT>;
+    using S = TcSmem<MT, EMB>;
+    constexpr int kCRow = kCRowOf<EMB>;
+    constexpr int kCTile = kCTileOf<EMB>;
     constexpr int kSB = kSBof<MT>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned start, kept as an offset from the shared array so that loads and stores
@@ -298,8 +351,11 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                         if (ci >= kSC) ok = mbar_wait(&c_empty[s], rc.phase ^ 1u, p.err);
                         if (!ok) break;
                         mbar_arrive_expect_tx(&c_full[s], kCTile);
-                        tma_load_2d(sC + s * kCTile, &tm_codes, &c_full[s], (ks / kKsPerCode) * 64, rowA);
-                        tma_load_2d(sC + s * kCTile + kCTile / 2, &tm_codes, &c_full[s], (ks / kKsPerCode) * 64, rowB);
+                        // the stage's first code byte, rounded down to a 16-byte boundary (EMB 1)
+                        const int cs_no = ks / kKsPerCode;
+                        const int x = EMB == 1 ? (88 * cs_no) & ~15 : EMB == 2 ? 80 * cs_no : 64 * cs_no;
+                        tma_load_2d(sC + s * kCTile, &tm_codes, &c_full[s], x, rowA);
+                        tma_load_2d(sC + s * kCTile + kCTile / 2, &tm_codes, &c_full[s], x, rowB);
                         ++ci;
                         rc.advance();
                     }
@@ -362,8 +418,10 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         // ------------------------------ decoders ------------------------------
         // two threads per weight row: thread part pt decodes words 2pt, 2pt+1 (W2: bytes 8pt..8pt+7 of
         // the row's 16 bytes of the group; W4: the second 16-byte chunk of the row's 32 bytes)
+        // (EMB: each warp decodes one half of 32 rows' groups, so its code path is warp-uniform)
         const int d = threadIdx.x - 64;
-        const int r = d >> 1, pt = d & 1;  // weight row within the tile, 0..255; part
+        const int r = EMB ? ((d >> 6) << 5) + (d & 31) : d >> 1;  // weight row within the tile, 0..255
+        const int pt = EMB ? (d >> 5) & 1 : d & 1;                 // part
         const int half = r >> 7, rr = r & 127;
         uint32_t bi = 0;
         Ring<kSB> rb;
@@ -378,17 +436,17 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             const int local = t.nt * p.row_block_stride + half * p.half_stride + rr;
             const bool valid = local < p.N;
             const size_t grow = (size_t)t.e * p.N + (valid ? local : 0);
-            const float alpha = (W4 || STD) ? 0.0f : __ldg(p.alpha + grow);
-            const float beta = (W4 || STD) ? 0.0f : __ldg(p.beta + grow);
+            const float alpha = (W4 || STD || EMB) ? 0.0f : __ldg(p.alpha + grow);
+            const float beta = (W4 || STD || EMB) ? 0.0f : __ldg(p.beta + grow);
             rp.ab = fpk2(alpha, alpha);
             rp.bb = fpk2(beta, beta);
-            const float *srow = p.scales + grow * (W4 ? 1 : nk);
+            const float *srow = EMB ? nullptr : p.scales + grow * (W4 ? 1 : nk);
             const float sc_row = W4 ? bf16_bits_to_float(float_to_bf16_bits(__ldg(srow))) : 0.0f;
             // W2 group scales, four groups (one code stage) at a time and one stage ahead, so the
             // global read is off the decode's critical path
-            const float sup_row = Q4 ? __ldg(p.super_scale + grow) : 0.0f;
+            const float sup_row = (Q4 || EMB) ? __ldg(p.super_scale + grow) : 0.0f;
             auto load_sc4 = [&](int g0) -> float4 {
-                if (W4 || g0 >= nk) return make_float4(0.f, 0.f, 0.f, 0.f);
+                if (W4 || EMB || g0 >= nk) return make_float4(0.f, 0.f, 0.f, 0.f);
                 if (Q4) {
                     // 4-bit group scales: groups g0..g0+3 in two bytes (even group in the low nibble)
                     const int qpr = p.K / 128;
@@ -404,7 +462,7 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             };
             float4 sc_cur = make_float4(0.f, 0.f, 0.f, 0.f), sc_next = load_sc4(t.g0);
             for (int ks = t.g0; ks < t.g1 && ok; ++ks) {
-                if (!W4 && (ks & 3) == 0) {
+                if (!W4 && !EMB && (ks & 3) == 0) {
                     sc_cur = sc_next;
                     sc_next = load_sc4(ks + 4);
                 }
@@ -413,12 +471,34 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                     ok = mbar_wait(&c_full[cs], rc.phase, p.err);
                     if (!ok) break;
                 }
-                // this thread's code bytes of group ks (64-byte rows, 64B swizzle)
-                const uint8_t *crow = sC + cs * kCTile + half * (kCTile / 2) + rr * 64;
+                // this thread's code bytes of group ks (64-byte rows, 64B swizzle; EMB: unswizzled
+                // rows of kCRow bytes)
+                const uint8_t *crow = sC + cs * kCTile + half * (kCTile / 2) + rr * kCRow;
                 const uint32_t swz = ((uint32_t)rr >> 1) & 3u;
                 uint2 q2w = make_uint2(0, 0);
                 uint4 q4w = make_uint4(0, 0, 0, 0);
-                if (!W4) {
+                uint32_t ec[12];  // EMB 1: codes 10pt .. 10pt+11 of the group, one per entry; EMB 2:
+                                  // the ten words, two per entry, in ec[0..4]
+                uint32_t eq = 0;  // EMB: the group's quantized scale
+                if constexpr (EMB == 1) {
+                    // the group's first code sits (88 * stage) mod 16 + 22 * (ks mod 4) bytes into the
+                    // row's line: an even offset, so 16-bit loads are aligned
+                    const uint8_t *gb = crow + ((88 * (ks >> 2)) & 15) + 22 * (ks & 3);
+                    const uint16_t *g16 = reinterpret_cast<const uint16_t *>(gb + 10 * pt);
+#pragma unroll
+                    for (int i = 0; i < 6; ++i) {
+                        const uint32_t h = g16[i];
+                        ec[2 * i] = h & 0xFFu;
+                        ec[2 * i + 1] = h >> 8;
+                    }
+                    // the scale: the low nibble of code 21 (the high byte of the 16-bit word at 20)
+                    eq = ((uint32_t)*reinterpret_cast<const uint16_t *>(gb + 20) >> 8) & 0xFu;
+                } else if constexpr (EMB == 2) {
+                    const uint32_t *g32 = reinterpret_cast<const uint32_t *>(crow + 20 * (ks & 3));
+#pragma unroll
+                    for (int i = 0; i < 5; ++i) ec[i] = g32[i];
+                    eq = (ec[4] >> 16) & 0x1FFFu;
+                } else if (!W4) {
                     q2w = *reinterpret_cast<const uint2 *>(crow + ((((uint32_t)(ks & 3)) ^ swz) << 4) + 8 * pt);
                 } else {
                     const uint32_t c0 = 2u * (uint32_t)(ks & 1) + (uint32_t)pt;
@@ -430,7 +510,20 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                     rc.advance();
                 }
                 uint32_t o[2][8];
-                if (!W4) {
+                if constexpr (EMB != 0) {
+                    const float sc = bf16_bits_to_float(float_to_bf16_bits(__fmul_rn((float)eq, sup_row)));
+                    const uint32_t s2 = pack_bf16x2(sc, sc);
+                    uint32_t u[32];
+                    if constexpr (EMB == 1) {
+                        if (pt == 0) emb1_states<0>(ec, u);
+                        else emb1_states<1>(ec, u);
+                        emb_pack<8>(u, s2, o);
+                    } else {
+                        if (pt == 0) emb2_states<0>(ec, u);
+                        else emb2_states<1>(ec, u);
+                        emb_pack<4>(u, s2, o);
+                    }
+                } else if (!W4) {
                     const int gi = ks & 3;
                     const float sraw = gi == 0 ? sc_cur.x : gi == 1 ? sc_cur.y : gi == 2 ? sc_cur.z : sc_cur.w;
                     const float sc = bf16_bits_to_float(float_to_bf16_bits(sraw));
@@ -612,11 +705,13 @@ __global__ void pack_xt_kernel(const uint16_t *__restrict__ x, const int *__rest
 
 template <int MT>
 cudaError_t launch_tc_mt(const TcGemmParams &p, const CUtensorMap &ta, const CUtensorMap &tc, int grid, cudaStream_t s) {
-    auto kern = p.w4     ? tc_gemm_w2_kernel<MT, true>
-                : p.q4   ? tc_gemm_w2_kernel<MT, false, true>
-                : p.std2 ? tc_gemm_w2_kernel<MT, false, false, true>
-                         : tc_gemm_w2_kernel<MT, false>;
-    const int smem = TcSmem<MT>::kTotal;
+    auto kern = p.emb == 1 ? tc_gemm_w2_kernel<MT, false, false, false, 1>
+                : p.emb == 2 ? tc_gemm_w2_kernel<MT, false, false, false, 2>
+                : p.w4       ? tc_gemm_w2_kernel<MT, true>
+                : p.q4       ? tc_gemm_w2_kernel<MT, false, true>
+                : p.std2     ? tc_gemm_w2_kernel<MT, false, false, true>
+                             : tc_gemm_w2_kernel<MT, false>;
+    const int smem = p.emb == 1 ? TcSmem<MT, 1>::kTotal : p.emb == 2 ? TcSmem<MT, 2>::kTotal : TcSmem<MT>::kTotal;
     cudaError_t err = kernel_setup(reinterpret_cast<const void *>(kern), smem, kTcThreads, 0, nullptr);
     if (err != cudaSuccess) return err;
     kern<<<grid, kTcThreads, smem, s>>>(ta, tc, p);

@@ -72,17 +72,34 @@ typedef enum {
  *     codes[n][k/4] uint8, bits 2i..2i+1 of byte j hold the level q of weight k = 4j + i;
  *     scales[n][k/64] fp32 group scales (used as bf16_rn(scale));
  *     w = bf16_rn((q - 2) * bf16_rn(scales[n][k/64]))          (levels -2, -1, 0, 1).
+ * CCQ_FMT_W275_432 and CCQ_FMT_W25_HYBRID: the CCQ formats without code cluster whose group scale
+ *   sits in the group's redundant bits (§3.2 "Hybrid Encoding", §3.4 "Scale Compression", §3.5
+ *   Algorithm 2, Table 1 rows (4,3,2) and (3,3,2)(3,4,2)).  Per row: `codes` is the row's groups of
+ *   64 weights back to back, and super_scale[n] is fp32; scales, alpha, beta, scale_q4 are unused.
+ *   CCQ_FMT_W275_432, (L,N,S) = (4,3,2), 2.75 bpw: a group is 22 one-byte codes; code j < 21
+ *     holds weights 3j..3j+2 as states (c >> 4) & 15, (c >> 2) & 15, c & 15; code 21 holds weight
+ *     63 in its top nibble and the group's 4-bit scale q in its low nibble.  Zero-point 8.
+ *     k must be a multiple of 512 (row pitch a multiple of 16 bytes).
+ *   CCQ_FMT_W25_HYBRID, (3,3,2)+(3,4,2), 2.5 bpw: a group is ten little-endian 16-bit words; word
+ *     j < 9 holds weights 7j..7j+6 as states (x >> 13, 11, 9, 6, 4, 2, 0) & 7; word 9 holds weight
+ *     63 in its top 3 bits and the 13-bit scale q in its low 13 bits.  Zero-point 4.  k must be a
+ *     multiple of 256.
+ *   Weight: w = bf16_rn((u - zp) * bf16_rn(fl32(q * super_scale[n]))).
+ *   Every matmul with these formats runs on the tcgen05 kernel (any m).
  */
 enum {
     CCQ_FMT_W2_CCQ_G64 = 1,
     CCQ_FMT_W4_PER_CHANNEL = 2,
     CCQ_FMT_W2_CCQ_G64_Q4SCALE = 3,
-    CCQ_FMT_W2_STD_G64 = 4
+    CCQ_FMT_W2_STD_G64 = 4,
+    CCQ_FMT_W275_432 = 5,
+    CCQ_FMT_W25_HYBRID = 6
 };
 
 /* One linear layer, or `num_experts` layers of the same shape stacked back to back: expert e's
  * arrays start at codes + e*n*(k/4) (W2) or e*n*(k/2) (W4), scales + e*n*(k/64) (W2) or e*n (W4),
- * alpha/beta/super_scale + e*n, scale_q4 + e*n*(k/128).  All device pointers, 16-byte aligned.
+ * alpha/beta/super_scale + e*n, scale_q4 + e*n*(k/128); for CCQ_FMT_W275_432 / CCQ_FMT_W25_HYBRID
+ * codes + e*n*(k/64)*22 / 20.  All device pointers, 16-byte aligned.
  * y = x W^T: W is [n][k]. */
 typedef struct {
     int32_t fmt;          /* CCQ_FMT_* */
@@ -158,6 +175,20 @@ ccq_status ccq_encode_host_q4(const float *w, int32_t n, int32_t k, int32_t grou
  *   bad shapes, misaligned pointers: all three 16-byte aligned) return before any launch. */
 ccq_status ccq_quantize_std_device(const float *w, int32_t n, int32_t k, uint8_t *codes, float *scales,
                                    ccq_stream_t stream);
+
+/* ccq_encode_emb_device - encoder for CCQ_FMT_W275_432 / CCQ_FMT_W25_HYBRID on the GPU (the pages
+ * print no encoder for these formats; plain reading of Algorithm 1 and §3.4):
+ *   raw group scale r_g = max|w_g| / (2^(L-1) - 1) (fp32; 7 or 3); super_scale[n] = max_g r_g /
+ *   (2^b - 1) (fp32; b = 4 or 13 scale bits); q_g = clip(round_half_even(r_g / super), 0, 2^b - 1)
+ *   in fp64 (0 when super is 0); group scale bf16(fl32(q_g * super)).  Every full code is the one,
+ *   over all codes of its width, whose decoded weights have the least squared error (fp64, ties to
+ *   the smallest code); the last code's state is the nearest level for weight 63.
+ *   fmt    CCQ_FMT_W275_432 or CCQ_FMT_W25_HYBRID (else CCQ_ERR_UNSUPPORTED)
+ *   w      (device) fp32 [n][k], k % 64 == 0;  codes (device) out [n][k/64 * (22 or 20) bytes];
+ *   super_scale (device) out fp32 [n].  Asynchronous on `stream`; argument errors (null or
+ *   misaligned pointers, bad shapes) return before any launch. */
+ccq_status ccq_encode_emb_device(int32_t fmt, const float *w, int32_t n, int32_t k, uint8_t *codes,
+                                 float *super_scale, ccq_stream_t stream);
 
 /* ccq_quantize_w4_host - W4 per-channel round-to-nearest ("GPTQ and AWQ" Part 2 rtn/pack_int4):
  * s = bf16(max|w_row|/7), q = clip(round_half_even(w/s), -8, 7) (w/s in fp64), two codes per byte,

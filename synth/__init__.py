@@ -123,3 +123,16 @@ def std_format_random(n: int, k: int, seed: int, group: int = 64, scale_std: flo
     codes = g.integers(0, 256, size=(n, k // 4), dtype=np.uint8)
     scales = (np.abs(g.normal(2.5, 0.4, size=(n, k // group))) * scale_std / 2.0).astype(np.float32)
     return codes, scales
+
+
+def emb_format_random(kind: int, n: int, k: int, seed: int, scale_std: float = 0.02):
+    """Random parameters of the formats with the scale in the redundant bits (kind 1: (4,3,2), 22
+    bytes per 64 weights; kind 2: hybrid, 20 bytes): uniform code bytes (every byte and 16-bit word
+    is a valid code; the scale bits are uniform too) and per-row super scales of the magnitude a
+    N(0, scale_std^2) row gives."""
+    g = rng(seed)
+    gb = 22 if kind == 1 else 20
+    codes = g.integers(0, 256, size=(n, k // 64 * gb), dtype=np.uint8)
+    levels, qmax = (7.0, 15.0) if kind == 1 else (3.0, 8191.0)
+    sup = (np.abs(g.normal(3.0, 0.3, size=n)) * scale_std / levels / qmax).astype(np.float32)
+    return codes, sup

@@ -84,6 +84,20 @@ def test_host_validation_returns_before_launch(ccq):
     assert q(fake, 4, 96, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG      # k % 64
     assert q(fake, -1, 64, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG
     assert q(fake + 8, 4, 64, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG  # misaligned w
+    # formats with the scale in the redundant bits: k pitch rules, super scale required, encoder args
+    for fmt, kbad in ((ccq.CCQ_FMT_W275_432, 768), (ccq.CCQ_FMT_W25_HYBRID, 320)):
+        w = ccq.ccq_weight(fmt, 256, kbad, 64, fake, None, None, None, None, fake)
+        assert lib.ccq_w2a16_gemm(ctypes.byref(w), fake, 4, fake, fake, 1 << 30, None) == ccq.CCQ_ERR_INVALID_ARG
+        w = ccq.ccq_weight(fmt, 256, 1024, 64, fake, None, None, None, None, None)
+        assert lib.ccq_w2a16_gemm(ctypes.byref(w), fake, 4, fake, fake, 1 << 30, None) == ccq.CCQ_ERR_INVALID_ARG
+        w = ccq.ccq_weight(fmt, 256, 1024, 64, fake, None, None, None, None, fake)
+        assert lib.ccq_w2a16_gemm(ctypes.byref(w), fake, 4, fake, fake, 0, None) == ccq.CCQ_ERR_INVALID_ARG
+        assert lib.ccq_gemm_workspace_size(ctypes.byref(w), 1) > 0
+        e = lib.ccq_encode_emb_device
+        assert e(fmt, None, 4, 64, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG
+        assert e(fmt, fake, 4, 96, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG
+        assert e(fmt, fake + 4, 4, 64, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG
+    assert lib.ccq_encode_emb_device(ccq.CCQ_FMT_W2_CCQ_G64, fake, 4, 64, fake, fake, None) == ccq.CCQ_ERR_UNSUPPORTED
 
 
 def test_encoder_matches_oracle(ccq):

@@ -329,7 +329,7 @@ def test_gemm_w4_shapes(ccq, m, n, k):
 
 # formats by name: "ccq" (W2 g64, fp32 scales), "q4" (W2 g64, 4-bit scales), "w4" (per channel),
 # "std" (WINT2-Standard); FMT_SEED gives each a number for the seeds
-FMT_SEED = {"ccq": 2, "q4": 3, "w4": 4, "std": 5}
+FMT_SEED = {"ccq": 2, "q4": 3, "w4": 4, "std": 5, "w275": 6, "w25": 7}
 
 
 def moe_weights_fmt(ccq, E, H, I, seed, fmt13, fmt2):
@@ -345,6 +345,10 @@ def moe_weights_fmt(ccq, E, H, I, seed, fmt13, fmt2):
             c, sc = synth.std_format_random(rows, k, s)
             return (ccq.CcqWeight(ccq.CCQ_FMT_W2_STD_G64, rows // E, k, c, sc, experts=E),
                     oracle.dequant_w2std(c, sc))
+        if fmt in ("w275", "w25"):
+            kind = 1 if fmt == "w275" else 2
+            c, sup = synth.emb_format_random(kind, rows, k, s)
+            return emb_weight(ccq, kind, c, sup, experts=E), emb_oracle(kind, c, sup)
         assert fmt == "ccq"
         c, sc, a, b = synth.w2_format_random(rows, k, s)
         return (ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, rows // E, k, c, sc, a, b, experts=E),
@@ -563,6 +567,107 @@ def test_moe_std_quantized_layer_matches_oracle(ccq):
     W2, d2 = q(E * H, I, 8501)
     x = synth.activations(T, H, 8502)
     ids, rw = synth.routing_uniform(T, E, topk, 8503)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    ref = oracle.moe_f64(synth.bf16_bits(x), d13.reshape(E, 2 * I, H), d2.reshape(E, H, I), ids, rw, round_h=True)
+    assert rel_err(y, ref) <= TOL
+
+
+# ----------------------------------------------------------------------------------------------
+# formats with the scale in the redundant bits (CCQ §3.5 Algorithm 2): (4,3,2) 2.75 bpw and
+# hybrid (3,3,2)+(3,4,2) 2.5 bpw; every matmul runs on the tcgen05 kernel
+# ----------------------------------------------------------------------------------------------
+def emb_weight(ccq, kind, codes, sup, experts=1):
+    fmt = ccq.CCQ_FMT_W275_432 if kind == 1 else ccq.CCQ_FMT_W25_HYBRID
+    n = codes.shape[0] // experts
+    k = codes.shape[1] // (22 if kind == 1 else 20) * 64
+    return ccq.CcqWeight(fmt, n, k, codes, None, experts=experts, super_scale=sup)
+
+
+def emb_oracle(kind, codes, sup):
+    codes = np.ascontiguousarray(codes)
+    return oracle.dequant_emb(kind, codes if kind == 1 else codes.view(np.uint16), sup)
+
+
+@pytest.mark.parametrize("kind", [1, 2])
+@pytest.mark.parametrize("n,k,E", [(16, 512, 1), (48, 1024, 3), (1024, 8192, 1)])
+def test_dequant_emb_bitexact(ccq, kind, n, k, E):
+    codes, sup = synth.emb_format_random(kind, n * E, k, 9000 + n + k + kind)
+    got = bits_of(ccq.ccq_dequant_bf16(emb_weight(ccq, kind, codes, sup, experts=E))).reshape(n * E, k)
+    assert np.array_equal(got, emb_oracle(kind, codes, sup))
+
+
+@pytest.mark.parametrize("kind", [1, 2])
+@pytest.mark.parametrize("n,k", [(6, 512), (33, 1024)])
+def test_encode_emb_device_matches_oracle(ccq, kind, n, k):
+    w = synth.weights_normal(n, k, 9100 + n + kind)
+    w[min(2, n - 1)] = 0.0                       # an all-zero row (super scale 0)
+    w[0, 64:128] = 0.0                           # an all-zero group
+    fmt = ccq.CCQ_FMT_W275_432 if kind == 1 else ccq.CCQ_FMT_W25_HYBRID
+    c, sup = (t.cpu().numpy() for t in ccq.ccq_encode_emb_device(fmt, torch.from_numpy(w).cuda()))
+    oc, osup = oracle.encode_emb(kind, w)
+    assert np.array_equal(sup, osup)
+    assert np.array_equal(c if kind == 1 else c.view(np.uint16), oc)
+
+
+@pytest.mark.parametrize("kind", [1, 2])
+def test_gemm_emb_one_hot_identity(ccq, kind):
+    n, k = 272, 1024
+    codes, sup = synth.emb_format_random(kind, n, k, 9200 + kind)
+    W = emb_weight(ccq, kind, codes, sup)
+    ref = oracle.bf16_to_f64(emb_oracle(kind, codes, sup)).T.astype(np.float32)
+    eye = synth.one_hot_rows(k).cuda()
+    for j in range(0, 64, 16):  # small m: still the tcgen05 kernel
+        y = ccq.ccq_w2a16_gemm(W, eye[j:j + 16].contiguous()).float().cpu().numpy()
+        assert np.array_equal(y, ref[j:j + 16]), j
+    y = ccq.ccq_w2a16_gemm(W, eye).float().cpu().numpy()
+    assert np.array_equal(y, ref)
+
+
+@pytest.mark.parametrize("kind", [1, 2])
+@pytest.mark.parametrize("m,n,k", [(1, 256, 512), (4, 1024, 4096), (33, 272, 1024), (128, 512, 1536),
+                                   (300, 272, 1024), (1, 8192, 8192)])
+def test_gemm_emb_shapes(ccq, kind, m, n, k):
+    if kind == 1 and k % 512:
+        k += 512 - k % 512
+    codes, sup = synth.emb_format_random(kind, n, k, 9300 + m + n + kind)
+    W = emb_weight(ccq, kind, codes, sup)
+    x = synth.activations(m, k, 9301 + m)
+    y = ccq.ccq_w2a16_gemm(W, x.cuda()).float().cpu().numpy()
+    ref = oracle.gemm_f64(synth.bf16_bits(x), emb_oracle(kind, codes, sup))
+    e = rel_err(y, ref)
+    assert e <= TOL
+    assert e <= 4e-3
+
+
+@pytest.mark.parametrize("fmts", [("w275", "w275"), ("w25", "w25"), ("ccq", "w275"), ("w25", "ccq")])
+@pytest.mark.parametrize("T", [6, 300])
+def test_moe_emb_formats(ccq, fmts, T):
+    E, H, I, topk = 8, 1024, 512, 2
+    W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 9400 + T + 10 * FMT_SEED[fmts[0]] + FMT_SEED[fmts[1]], *fmts)
+    x = synth.activations(T, H, 9401 + T)
+    ids, rw = synth.routing_uniform(T, E, topk, 9402 + T)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    ref = oracle.moe_f64(synth.bf16_bits(x), d13, d2, ids, rw, round_h=True)
+    assert rel_err(y, ref) <= TOL
+
+
+@pytest.mark.parametrize("kind", [1, 2])
+def test_moe_emb_encoded_layer_matches_oracle(ccq, kind):
+    # weights through the device encoder, decode-sized token count (still the tcgen05 kernel)
+    E, H, I, topk, T = 8, 1024, 512, 2, 16
+    fmt = ccq.CCQ_FMT_W275_432 if kind == 1 else ccq.CCQ_FMT_W25_HYBRID
+
+    def q(rows, k, seed):
+        w = synth.weights_normal(rows, k, seed)
+        c, sup = (t.cpu().numpy() for t in ccq.ccq_encode_emb_device(fmt, torch.from_numpy(w).cuda()))
+        return emb_weight(ccq, kind, c, sup, experts=E), emb_oracle(kind, c, sup)
+
+    W13, d13 = q(E * 2 * I, H, 9500 + kind)
+    W2, d2 = q(E * H, I, 9510 + kind)
+    x = synth.activations(T, H, 9502)
+    ids, rw = synth.routing_uniform(T, E, topk, 9503)
     y, st = run_moe(ccq, W13, W2, x, ids, rw)
     assert st == ccq.CCQ_OK
     ref = oracle.moe_f64(synth.bf16_bits(x), d13.reshape(E, 2 * I, H), d2.reshape(E, H, I), ids, rw, round_h=True)
