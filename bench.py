@@ -32,7 +32,9 @@ NOMINAL_HBM_GBS = 8000.0
 METRIC = "W2A16 MoE layer tokens/s; packed-weight HBM GB/s (% of 8 TB/s), 1 B200"
 WORKLOAD = "moe_ffn_decode_T32_H8192_I3584_E64_top8_ccq_w2_g64"
 SCALES = "fp32"       # group scale storage: fp32 (the benchmark format) or q4 (CCQ's 2.06-bpw form)
-CODES = "ccq"         # 2-bit codes: ccq (code cluster) or std (plain WINT2-Standard fields, CCQ Table 4)
+CODES = "ccq"         # codes: ccq (code cluster), std (plain WINT2-Standard fields, CCQ Table 4), or the
+                      # Algorithm 2 formats w275 ((4,3,2), 2.75 bpw) and w25 (hybrid, 2.5 bpw)
+EMB_CODES = {"w275": (5, 22), "w25": (6, 20)}  # format constant, code bytes per 64 weights
 
 
 def parse():
@@ -51,9 +53,11 @@ def parse():
     ap.add_argument("--m", type=int, default=0, help="tokens for --workload gemm (default 1) / stack (default 32)")
     ap.add_argument("--scales", default="fp32", choices=["fp32", "q4"],
                     help="W2 group scales: fp32 (default) or 4-bit x per-channel super scale (2.06 bpw)")
-    ap.add_argument("--codes", default="ccq", choices=["ccq", "std"],
-                    help="2-bit codes: ccq (code cluster, default) or std (plain 2-bit WINT2-Standard fields, "
-                         "the comparison format of CCQ Table 4; fp32 scales only)")
+    ap.add_argument("--codes", default="ccq", choices=["ccq", "std", "w275", "w25"],
+                    help="codes: ccq (code cluster, default), std (plain 2-bit WINT2-Standard fields, the "
+                         "comparison format of CCQ Table 4), w275 ((4,3,2), 2.75 bpw) or w25 (hybrid "
+                         "(3,3,2)+(3,4,2), 2.5 bpw), the last two with the scale in the codes (Algorithm 2); "
+                         "all but ccq take --scales fp32 only")
     ap.add_argument("--shape", default="8192x8192",
                     help="--workload gemm: input x output size KxN (CCQ Table 4: 4096x4096, 4096x1024, "
                          "8192x8192, 8192x1024)")
@@ -61,8 +65,8 @@ def parse():
     global T, E, WORKLOAD, SCALES, CODES
     SCALES = args.scales
     CODES = args.codes
-    if CODES == "std" and SCALES != "fp32":
-        ap.error("--codes std takes fp32 scales only")
+    if CODES != "ccq" and SCALES != "fp32":
+        ap.error("--scales q4 applies to --codes ccq only")
     if args.workload == "prefill":
         T = 4096
         WORKLOAD = "moe_ffn_prefill_T4096_zipf1.1_H8192_I3584_E64_top8_ccq_w2_g64"
@@ -72,6 +76,10 @@ def parse():
         WORKLOAD = WORKLOAD.replace("ccq_w2_g64", "ccq_w2_g64_q4scale")
     if CODES == "std":
         WORKLOAD = WORKLOAD.replace("ccq_w2_g64", "std_w2_g64")
+    if CODES == "w275":
+        WORKLOAD = WORKLOAD.replace("ccq_w2_g64", "ccq_w275_432_g64")
+    if CODES == "w25":
+        WORKLOAD = WORKLOAD.replace("ccq_w2_g64", "ccq_w25_hybrid_g64")
     return args
 
 
@@ -137,7 +145,12 @@ def config_dict():
         "workload": WORKLOAD,
         "tokens": T, "hidden": H, "intermediate": I, "experts": E, "topk": TOPK,
         "weight_format": ("WINT2-Standard plain 2-bit fields, 4 weights/byte, fp32 group-64 scales"
-                          if CODES == "std" else "CCQ (6,4,3) code cluster, 4 weights/byte, " + (
+                          if CODES == "std" else
+                          "CCQ (4,3,2), 22 one-byte codes per 64 weights, 4-bit scale in the last code x fp32 "
+                          "per-channel super scale (2.75 bpw)" if CODES == "w275" else
+                          "CCQ hybrid (3,3,2)+(3,4,2), ten 16-bit words per 64 weights, 13-bit scale in the last "
+                          "word x fp32 per-channel super scale (2.5 bpw)" if CODES == "w25" else
+                          "CCQ (6,4,3) code cluster, 4 weights/byte, " + (
                               "4-bit group-64 scales x fp32 per-channel super scale (2.06 bpw)" if SCALES == "q4"
                               else "fp32 group-64 scales")),
         "routing": ("Zipf(1.1) expert popularity, top-8 by Gumbel-max; " if prefill else "uniform distinct top-8, ")
@@ -147,6 +160,8 @@ def config_dict():
                     if SCALES == "q4" else
                     f"N(0,0.02) per expert (seeded device RNG), all {E} quantized by ccq_quantize_std_device"
                     if CODES == "std" else
+                    f"N(0,0.02) (seeded device RNG) encoded by ccq_encode_emb_device for {DISTINCT} experts, "
+                    f"copied to all {E}" if CODES in EMB_CODES else
                     f"N(0,0.02) per expert (seeded device RNG), all {E} encoded by ccq_encode_device"),
         "l2": "inputs larger than L2: ~1.74 GB of packed weights touched per step vs 126 MB L2",
         "parallelism": "replicas",
@@ -160,6 +175,28 @@ def make_layer_device(ccq, torch, device, seed_base: int = 3100):
     """Every expert its own N(0, 0.02) weights (seeded device RNG), encoded by ccq_encode_device
     (or, for the WINT2-Standard codes, quantized by ccq_quantize_std_device)."""
     std = CODES == "std"
+    if CODES in EMB_CODES:
+        fmt, gb = EMB_CODES[CODES]
+
+        def stack_emb(n, k, seed):
+            codes = torch.empty((E * n, k // 64 * gb), dtype=torch.uint8, device=device)
+            sup = torch.empty((E * n,), dtype=torch.float32, device=device)
+            g = torch.Generator(device=device)
+            # the exhaustive code search costs seconds per expert: DISTINCT experts are encoded and
+            # copied into every slot (each slot its own memory; decode cost does not depend on values)
+            for e in range(E):
+                if e < DISTINCT:
+                    g.manual_seed(seed + e)
+                    w = torch.randn((n, k), generator=g, device=device, dtype=torch.float32) * 0.02
+                    c, su = ccq.ccq_encode_emb_device(fmt, w)
+                else:
+                    d = e % DISTINCT
+                    c, su = codes[d * n:(d + 1) * n], sup[d * n:(d + 1) * n]
+                codes[e * n:(e + 1) * n].copy_(c)
+                sup[e * n:(e + 1) * n].copy_(su)
+            return ccq.CcqWeight(fmt, n, k, codes, None, experts=E, device=device, super_scale=sup)
+
+        return stack_emb(2 * I, H, seed_base), stack_emb(H, I, seed_base + 100)
 
     def stack(n, k, seed):
         codes = torch.empty((E * n, k // 4), dtype=torch.uint8, device=device)
@@ -235,6 +272,10 @@ def touched_bytes(ids):
     if CODES == "std":
         per13 = 2 * I * (H // 4) + 2 * I * (H // 64) * 4
         per2 = H * (I // 4) + H * (I // 64) * 4
+    elif CODES in EMB_CODES:
+        gb = EMB_CODES[CODES][1]
+        per13 = 2 * I * ((H // 64) * gb + 4)
+        per2 = H * ((I // 64) * gb + 4)
     elif SCALES == "q4":
         per13 = 2 * I * (H // 4) + 2 * I * (H // 128) + 2 * I * 12
         per2 = H * (I // 4) + H * (I // 128) + H * 12
@@ -526,7 +567,8 @@ def run_ours(args, rank, world, local):
              "traffic": FUSED_DECODE_DRAM_BYTES_PER_EXPERT * ne if (SCALES, CODES) == ("fp32", "ccq") else None,
              "traffic_source": "ncu dram__bytes_read+write of the 16-expert capture, scaled by touched experts",
              "launch_ms": gemm1_ms, "algorithmic_bytes_per_launch": b13 + b2} if fused else
-            {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (gate/up, SiLU epilogue)",
+            {"bound": "hbm", "kernel": ("tc_gemm_w2_kernel" if CODES in EMB_CODES else "decode_gemm_w2_kernel")
+                                       + " (gate/up, SiLU epilogue)",
              "achieved": ach13, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "unit": "GB/s",
              "frac": ach13 / hbm, "traffic": None, "launch_ms": gemm1_ms,
              "algorithmic_bytes_per_launch": b13,
@@ -582,6 +624,11 @@ def run_gemm(args, rank, world, local):
         c, sc = (t.cpu().numpy() for t in ccq.ccq_quantize_std_device(torch.from_numpy(w).to(device)))
         per_copy = c.nbytes + sc.nbytes
         mk = lambda: ccq.CcqWeight(ccq.CCQ_FMT_W2_STD_G64, ND, KD, c, sc, device=device)
+    elif CODES in EMB_CODES:
+        fmt = EMB_CODES[CODES][0]
+        c, su = (t.cpu().numpy() for t in ccq.ccq_encode_emb_device(fmt, torch.from_numpy(w).to(device)))
+        per_copy = c.nbytes + su.nbytes
+        mk = lambda: ccq.CcqWeight(fmt, ND, KD, c, None, device=device, super_scale=su)
     elif SCALES == "q4":
         c, sq, sup, al, be, _ = ccq.ccq_encode_host_q4(w, 64, 0, 0)
         per_copy = c.nbytes + sq.nbytes + sup.nbytes + al.nbytes + be.nbytes
@@ -632,10 +679,12 @@ def run_gemm(args, rank, world, local):
              "unit": "TFLOP/s", "frac": flops / (ms * 1e-3) / 1e12 / tf} if tensor else
             {"bound": "hbm", "achieved": gbs, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "unit": "GB/s",
              "frac": gbs / hbm})
-    roof.update({"kernel": "whole ccq_w2a16_gemm call (" + ("tcgen05 kernel" if tensor else
+    roof.update({"kernel": "whole ccq_w2a16_gemm call (" + ("activation packing, tcgen05 kernel, split-K reduce"
+                                                            if tensor or CODES in EMB_CODES else
                  "activation packing, decode kernel, split-K reduce") + ")", "traffic": None,
                  "algorithmic_bytes_per_call": per_copy, "algorithmic_flops_per_call": flops})
-    fmt_tag = "std_w2_g64" if CODES == "std" else "ccq_w2_g64" + ("_q4scale" if SCALES == "q4" else "")
+    fmt_tag = ("std_w2_g64" if CODES == "std" else "ccq_w275_432_g64" if CODES == "w275" else
+               "ccq_w25_hybrid_g64" if CODES == "w25" else "ccq_w2_g64" + ("_q4scale" if SCALES == "q4" else ""))
     line = {"metric": f"W2A16 dense linear tokens/s (K={KD}, N={ND})", "value": M / (ms * 1e-3), "unit": "tokens/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "us_per_call": 1000.0 * ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -643,6 +692,7 @@ def run_gemm(args, rank, world, local):
             "config": {"workload": f"dense_gemm_M{M}_K{KD}_N{ND}_{fmt_tag}",
                        "m": M, "k": KD, "n": ND,
                        "weights": "N(0,0.02) " + ("quantized by ccq_quantize_std_device" if CODES == "std" else
+                                                  "encoded by ccq_encode_emb_device" if CODES in EMB_CODES else
                                                   "encoded by ccq_encode_host" + ("_q4" if SCALES == "q4" else "")),
                        "l2": f"{R} rotating weight copies ({R * per_copy / 1e6:.0f} MB) vs {l2 / 1e6:.0f} MB L2"},
             "packed_weight_gbs": gbs, "roofline": roof,
