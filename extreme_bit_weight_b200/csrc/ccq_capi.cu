@@ -173,8 +173,16 @@ int tc_mt(double rows_per_expert) { return rows_per_expert > 96.0 ? 2 : 1; }
 struct GemmWs {
     size_t xa, gs, partial, xt, work, total;
     int P, ksplit, spp, row_blocks, nt;
+    int sn;  // tcgen05 path: small-token tile width (0: 128-token tiles)
     bool tc;
 };
+
+// Small-token tiles on the tcgen05 path (embedded-scale formats, at most 64 tokens per expert or
+// call): the tile width for a mean of `rows` tokens.
+inline int pick_sn(const ccq_weight *w, double rows) {
+    if (!emb_kind(w) || rows > 64.0) return 0;
+    return rows <= 16.0 ? 16 : rows <= 32.0 ? 32 : 64;
+}
 
 int sm_count() {
     static int n = 0;
@@ -192,11 +200,12 @@ GemmWs gemm_layout(const ccq_weight *w, int m) {
         L.tc = true;
         L.P = m;
         L.xt = 0;
+        L.sn = pick_sn(w, (double)m);
         size_t off = up256((size_t)m * w->k * 2);
         // split-K when the (token tile, row tile) items cannot fill the SMs: ranges of kg groups
         // (a multiple of 4, one code stage), as many ranges as keep every item on its own SM
         const int nk = w->k / 64;
-        const int items = ceil_div(m, 128 * tc_mt((double)m)) * ceil_div(w->n, 256);
+        const int items = ceil_div(m, L.sn ? L.sn : 128 * tc_mt((double)m)) * ceil_div(w->n, 256);
         const int sms = sm_count();
         L.ksplit = 1;
         L.spp = nk;
@@ -243,7 +252,7 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     const int pairs = T * topk;
     L.P = (pairs + 3) & ~3;
     L.tc = (double)pairs / E >= kTcMinRowsPerExpert;
-    L.max_tiles = L.P / 128 + E + 1;  // enough for 128-token tiles
+    L.max_tiles = L.P / 16 + E + 1;  // enough for the smallest (16-token) tiles
     // (the tile list is always laid out: the embedded-scale formats take the tcgen05 path at any size)
     size_t off = 0;
     L.err = off; off = up256(off + 16);
@@ -268,12 +277,14 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     return L;
 }
 
-bool tc_maps(CUtensorMap &ta, CUtensorMap &tcodes, const ccq_weight *w, int experts, const uint16_t *a, int P) {
+// box_rows: token rows per activation load (128, or the small-token tile width)
+bool tc_maps(CUtensorMap &ta, CUtensorMap &tcodes, const ccq_weight *w, int experts, const uint16_t *a, int P,
+             int box_rows = 128) {
     const int K = w->k;
     {
         cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)P};
         cuuint64_t str[1] = {(cuuint64_t)K * 2};
-        cuuint32_t box[2] = {64, 128};
+        cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
         if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return false;
     }
@@ -354,15 +365,16 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
         cudaError_t e = launch_pack_xt(static_cast<const uint16_t *>(x_bf16), nullptr, m, w->k, xt, s);
         if (e != cudaSuccess) return CCQ_ERR_CUDA;
         CUtensorMap ta, tcodes;
-        if (!tc_maps(ta, tcodes, w, 1, xt, m)) return CCQ_ERR_CUDA;
+        if (!tc_maps(ta, tcodes, w, 1, xt, m, L.sn ? L.sn : 128)) return CCQ_ERR_CUDA;
         TcGemmParams p{};
         p.N = w->n;
         p.K = w->k;
         p.row_block_stride = 256;
         p.half_stride = 128;
         p.n_tiles = ceil_div(w->n, 256);
-        const int mt = tc_mt((double)m);
-        p.m_tile = 128 * mt;
+        const int mt = L.sn ? 1 : tc_mt((double)m);
+        p.sn = L.sn;
+        p.m_tile = L.sn ? L.sn : 128 * mt;
         p.static_tiles = ceil_div(m, p.m_tile);
         p.M = m;
         p.out_ld = w->n;
@@ -483,13 +495,18 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         // prefill-sized: tcgen05 grouped GEMMs over (expert, 256-token tile) entries
         int2 *tiles = reinterpret_cast<int2 *>(base + L.tiles);
         int *tcount = reinterpret_cast<int *>(base + L.tcount);
-        const int mt = tc_mt((double)pairs / num_experts);
+        // small-token tiles when both weights take them (one tile list serves both projections)
+        const double rows = (double)pairs / num_experts;
+        const int sn = (pick_sn(w13, rows) && pick_sn(w2, rows)) ? pick_sn(w13, rows) : 0;
+        const int mt = sn ? 1 : tc_mt(rows);
+        const int m_tile = sn ? sn : 128 * mt;
         e = launch_pack_xt(static_cast<const uint16_t *>(x_bf16), tok, pairs, H, xa_x, s);
-        if (e == cudaSuccess) e = launch_build_tiles(seg, num_experts, 128 * mt, tiles, tcount, s);
+        if (e == cudaSuccess) e = launch_build_tiles(seg, num_experts, m_tile, tiles, tcount, s);
         if (e == cudaSuccess) e = trace(events, 2, s);
         if (e != cudaSuccess) return CCQ_ERR_CUDA;
         CUtensorMap ta1, tc1, ta2, tc2;
-        if (!tc_maps(ta1, tc1, w13, num_experts, xa_x, L.P) || !tc_maps(ta2, tc2, w2, num_experts, xa_h, L.P))
+        if (!tc_maps(ta1, tc1, w13, num_experts, xa_x, L.P, sn ? sn : 128) ||
+            !tc_maps(ta2, tc2, w2, num_experts, xa_h, L.P, sn ? sn : 128))
             return CCQ_ERR_CUDA;
         TcGemmParams q1{};
         q1.N = w13->n;
@@ -499,7 +516,8 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q1.n_tiles = ceil_div(I, 128);
         q1.tile_list = tiles;
         q1.tile_count = tcount;
-        q1.m_tile = 128 * mt;
+        q1.m_tile = m_tile;
+        q1.sn = sn;
         q1.seg_off = seg;
         q1.mode = EPI_GATEUP;
         q1.out = xa_h;

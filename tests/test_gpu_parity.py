@@ -672,3 +672,34 @@ def test_moe_emb_encoded_layer_matches_oracle(ccq, kind):
     assert st == ccq.CCQ_OK
     ref = oracle.moe_f64(synth.bf16_bits(x), d13.reshape(E, 2 * I, H), d2.reshape(E, H, I), ids, rw, round_h=True)
     assert rel_err(y, ref) <= TOL
+
+
+@pytest.mark.parametrize("kind", [1, 2])
+@pytest.mark.parametrize("m", [17, 40, 64])
+def test_gemm_emb_small_token_tiles(ccq, kind, m):
+    # token tiles of 32 / 64 tokens on the MMA's N side, several tiles per call
+    n, k = 512, 1024
+    codes, sup = synth.emb_format_random(kind, n, k, 9600 + m + kind)
+    W = emb_weight(ccq, kind, codes, sup)
+    x = synth.activations(m, k, 9601 + m)
+    y = ccq.ccq_w2a16_gemm(W, x.cuda()).float().cpu().numpy()
+    ref = oracle.gemm_f64(synth.bf16_bits(x), emb_oracle(kind, codes, sup))
+    assert rel_err(y, ref) <= 4e-3
+
+
+@pytest.mark.parametrize("fmts", [("w275", "w275"), ("w25", "w25")])
+@pytest.mark.parametrize("T,zipf", [(48, False), (200, False), (120, True)])
+def test_moe_emb_small_token_tiles(ccq, fmts, T, zipf):
+    # 12 / 50 / 30 rows per expert on average: 16-, 64- and 32-token tiles, with experts that span
+    # several tiles (and, under Zipf routing, experts with none)
+    E, H, I, topk = 8, 1024, 512, 2
+    W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 9700 + T + FMT_SEED[fmts[0]], *fmts)
+    x = synth.activations(T, H, 9701 + T)
+    if zipf:
+        ids, rw = synth.routing_zipf(T, E, topk, 9702 + T, s=1.1)
+    else:
+        ids, rw = synth.routing_uniform(T, E, topk, 9702 + T)
+    y, st = run_moe(ccq, W13, W2, x, ids, rw)
+    assert st == ccq.CCQ_OK
+    ref = oracle.moe_f64(synth.bf16_bits(x), d13, d2, ids, rw, round_h=True)
+    assert rel_err(y, ref) <= TOL
