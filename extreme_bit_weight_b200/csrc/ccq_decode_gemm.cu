@@ -43,17 +43,26 @@ namespace ccq {
 namespace {
 
 constexpr int kRowWarps = 8;                       // warps per 16-row slot set (256 rows per CTA)
-constexpr int kConsumerWarps = 2 * kRowWarps;       // two warps per row slot: groups 0-3 / 4-7 of a stage
 constexpr int kProducerWarps = 4;                   // one warpgroup; lane 0 of its first warp issues the loads
-constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
-// Register split: the CTA launches with kLaunchRegs per thread (the most 640 threads can have), the
+constexpr int kProducerRegs = 24;
+// Consumer layout.  KH = 2: two warps per row slot, groups 0-3 / 4-7 of a stage, whose sums meet at
+// the end of a chunk (640 threads).  KH = 1: one warp per row slot takes all 8 groups (384 threads,
+// each consumer with twice the registers).
+// Register split: the CTA launches with kLaunchRegs per thread (the most its threads can have), the
 // producer warpgroup hands registers back and the consumer warpgroups take them.  The split must
 // fit in the launch allocation, or the consumers' increase would wait for registers forever; the
 // launcher also checks that the compiled kernel really launches with kLaunchRegs.
-constexpr int kLaunchRegs = 96, kProducerRegs = 24, kConsumerRegs = 112;
-static_assert(kProducerWarps * 32 * kProducerRegs + kConsumerWarps * 32 * kConsumerRegs <= kThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
-static_assert(65536 / kThreads >= kLaunchRegs, "launch registers");
+template <int KH>
+struct Cfg {
+    static constexpr int kConsumerWarps = kRowWarps * KH;
+    static constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
+    static constexpr int kLaunchRegs = KH == 2 ? 96 : 168;
+    static constexpr int kConsumerRegs = KH == 2 ? 112 : 240;
+    static constexpr int kGroups = 8 / KH;  // groups of a stage per consumer warp
+    static_assert(kProducerWarps * 32 * kProducerRegs + kConsumerWarps * 32 * kConsumerRegs <= kThreads * kLaunchRegs,
+                  "register split exceeds the launch allocation");
+    static_assert(65536 / kThreads >= kLaunchRegs, "launch registers");
+};
 constexpr int kCodeTileBytes = 128 * 128;  // [128 rows][128 B] = 8 groups of 16 bytes
 
 template <int NT, bool W4 = false, bool Q4 = false>
@@ -397,12 +406,15 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
 // Persistent: CTA b walks units b, b + gridDim.x, ...; its producer streams every stage of every
 // unit through one ring, so the next unit's first stages load while this unit finishes.
 // FUSED: the launch holds the MoE gate/up units (p, m1) followed by the down units (p2, m2).
-// STD: WINT2-Standard plain 2-bit fields (no per-row constants).
-template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false, bool STD = false>
-__global__ void __launch_bounds__(kThreads, 1)
+// STD: WINT2-Standard plain 2-bit fields (no per-row constants).  KH: consumer layout (Cfg; KH = 1
+// only with TMA-staged fp32 scales).
+template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false, bool STD = false, int KH = 2>
+__global__ void __launch_bounds__(Cfg<KH>::kThreads, 1)
 decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__ MapSet m2,
                       const __grid_constant__ DecodeGemmParams p, const __grid_constant__ DecodeGemmParams p2) {
+    static_assert(KH == 2 || (TMA_SC && !W4 && !Q4), "one warp per row slot needs TMA-staged fp32 scales");
     using S = Smem<NT, W4, Q4>;
+    using C = Cfg<KH>;
     constexpr int MP = S::MP;
     constexpr int kStages = S::kStages;
     constexpr int kCodeOff = 0;                       // code tiles of the stage
@@ -422,7 +434,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full_bar[i], 1);
-            mbar_init(&empty_bar[i], kConsumerWarps);
+            mbar_init(&empty_bar[i], C::kConsumerWarps);
         }
         mbar_init(&red_full, kRowWarps);
         mbar_init(&red_empty, kRowWarps);
@@ -552,9 +564,9 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             P.st = st + 1 == U.s_end ? U.s_begin : st + 1;
         }
     };
-    if (warp >= kConsumerWarps) {
+    if (warp >= C::kConsumerWarps) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
-        if (warp == kConsumerWarps && lane == 0) {
+        if (warp == C::kConsumerWarps && lane == 0) {
             P.u = blockIdx.x;
             P.pi = P.slot = P.round = 0;
             p_ord = 0;
@@ -585,12 +597,12 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
         }
         return;
     }
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kConsumerRegs));
 
     // ---------------- consumers ----------------
     const int g = lane >> 2, tig = lane & 3;
     const int wslot = warp & (kRowWarps - 1);  // row slot: 16 rows inside each 128-row half
-    const int khalf = warp / kRowWarps;        // 0: groups 0-3 of every stage, 1: groups 4-7
+    const int khalf = KH == 2 ? warp / kRowWarps : 0;  // KH 2: 0 = groups 0-3 of every stage, 1 = 4-7
     const int Gh = 4 * khalf;
     const int wrow = wslot * 16;
 
@@ -603,10 +615,11 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     kc.wmask = (W4 ? 0x000F000Fu : STD ? 0x00030003u : 0x003F003Fu) ^ opaque;
     kc.wexp = (W4 ? 0x43084308u : 0x43004300u) ^ opaque;   // BF16 128 (W4: and the nibble sign flip)
 
-    // per-thread shared-memory offsets inside a stage, for this warp's four groups Gh..Gh+3
-    uint32_t coff[4];
+    // per-thread shared-memory offsets inside a stage, for this warp's groups Gh..Gh+kGroups-1
+    constexpr int kG = C::kGroups;
+    uint32_t coff[kG];
 #pragma unroll
-    for (int G = 0; G < 4; ++G) {
+    for (int G = 0; G < kG; ++G) {
         if constexpr (!W4) {
             // word tig of row wrow+g in 16-byte chunk (Gh+G) ^ g (128-byte swizzle)
             coff[G] = kCodeOff + (uint32_t)(wrow + g) * 128u + 4u * (uint32_t)tig + ((uint32_t)((Gh + G) ^ g) << 4);
@@ -716,22 +729,35 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             });
         } else if (TMA_SC) {
             // full stage: groups beyond K read TMA zero fill (scale 0, activations 0) and add nothing
-            const uint32_t sa = sb + sc_thr;
-            const float4 s0 = lds128f_at<0>(sa);
-            const float4 s1 = lds128f_at<256>(sa);
-            const float4 s2 = lds128f_at<4096>(sa);
-            const float4 s3 = lds128f_at<4096 + 256>(sa);
-            const float v0[4] = {s0.x, s0.y, s0.z, s0.w}, v1[4] = {s1.x, s1.y, s1.z, s1.w};
-            const float v2[4] = {s2.x, s2.y, s2.z, s2.w}, v3[4] = {s3.x, s3.y, s3.z, s3.w};
-            const uint32_t xs = sb + xa_thr, gs = sb + gs_thr;
-            static_for<4>([&](auto Gc) {
-                constexpr int G = decltype(Gc)::value;
-                const float sc[4] = {round_bf16(v0[G]), round_bf16(v1[G]), round_bf16(v2[G]), round_bf16(v3[G])};
-                group_w2<NT, G, STD>(sb + coff[G], xs, gs, sc, rd, kc, acc);
-            });
+            // this warp's groups, four at a time: groups 4Q..4Q+3 sit 16Q bytes further in the scale
+            // rows, 16 MP 32 Q bytes further in the XA slice, 64Q in the gsq entries, and in the
+            // 128-byte-swizzled chunk (G ^ g) ^ 4Q, i.e. with code address bit 6 flipped
+            auto quad = [&](int Q) {
+                const uint32_t sa = sb + sc_thr + 16u * (uint32_t)Q;
+                const uint32_t xs = sb + xa_thr + (uint32_t)(Q * 16 * MP * 32), gs = sb + gs_thr + 64u * (uint32_t)Q;
+                const uint32_t cflip = (uint32_t)Q << 6;
+                const float4 s0 = lds128f_at<0>(sa);
+                const float4 s1 = lds128f_at<256>(sa);
+                const float4 s2 = lds128f_at<4096>(sa);
+                const float4 s3 = lds128f_at<4096 + 256>(sa);
+                const float v0[4] = {s0.x, s0.y, s0.z, s0.w}, v1[4] = {s1.x, s1.y, s1.z, s1.w};
+                const float v2[4] = {s2.x, s2.y, s2.z, s2.w}, v3[4] = {s3.x, s3.y, s3.z, s3.w};
+                static_for<4>([&](auto Gc) {
+                    constexpr int G = decltype(Gc)::value;
+                    const float sc[4] = {round_bf16(v0[G]), round_bf16(v1[G]), round_bf16(v2[G]), round_bf16(v3[G])};
+                    group_w2<NT, G, STD>(sb + (coff[G] ^ cflip), xs, gs, sc, rd, kc, acc);
+                });
+            };
+            if constexpr (NT >= 4) {
+                // (4 token tiles: one quad's code at a time keeps the accumulators in registers)
+#pragma unroll 1
+                for (int Q = 0; Q < kG / 4; ++Q) quad(Q);
+            } else {
+                static_for<kG / 4>([&](auto Qc) { quad(decltype(Qc)::value); });
+            }
         } else {
             const int ngroups = pq.K / 64;
-            const int g_lim = min(4, ngroups - st * 8 - Gh);
+            const int g_lim = min(kG, ngroups - st * 8 - Gh);
 #pragma unroll 1
             for (int G = 0; G < g_lim; ++G) {
                 const int gg = st * 8 + Gh + G;
@@ -758,9 +784,11 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
         i = 0;
 
         // ---------------- epilogue for token chunk c ----------------
-        // the second warp of each row slot hands its partial sums to the first (bounded waits)
+        // KH 2: the second warp of each row slot hands its partial sums to the first (bounded waits)
         float *red = reinterpret_cast<float *>(smem + kStages * S::kStageBytes) + (wslot * 32 + lane) * (2 * NT * 4);
-        if (khalf == 1) {
+        if (KH == 1) {
+            // one warp per row slot: its sums are complete
+        } else if (khalf == 1) {
             if (cc > 0 && !mbar_wait(&red_empty, (cc - 1) & 1, p.err)) {
                 ok = false;
                 break;
@@ -900,9 +928,13 @@ using DecodeKernel = void (*)(MapSet, MapSet, DecodeGemmParams, DecodeGemmParams
 
 // Checks the kernel's launch register count (the register split assumes kLaunchRegs), sets its
 // dynamic shared memory and returns the CTAs that fit per SM (once per kernel and device).
+template <int KH>
 cudaError_t prepare_kernel(DecodeKernel kern, int smem, int *per_sm = nullptr) {
-    return kernel_setup(reinterpret_cast<const void *>(kern), smem, kThreads, kLaunchRegs, per_sm);
+    return kernel_setup(reinterpret_cast<const void *>(kern), smem, Cfg<KH>::kThreads, Cfg<KH>::kLaunchRegs, per_sm);
 }
+
+// Consumer layout for the fp32-scale 2-bit kernels (CCQ and STD); the others use KH = 2.
+constexpr int kFastKH = 1;
 
 int device_sms(cudaError_t &err) {
     int dev = 0, sms = 0;
@@ -916,7 +948,7 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
                       const CUtensorMap &c, const CUtensorMap &d, int row_blocks, int ksplit, int experts,
                       cudaStream_t s) {
     DecodeKernel kern = nullptr;
-    int smem = 0;
+    int smem = 0, kh = 2;
     if constexpr (NT <= 2) {  // W4 keeps at most 16 tokens per chunk (its code tiles are twice as wide)
         if (p.w4) {
             kern = decode_gemm_w2_kernel<NT, false, true, false>;
@@ -924,20 +956,23 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
         }
     }
     if (!p.w4 && p.std2) {
-        kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false, false, false, true>
+        kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false, false, false, true, kFastKH>
                             : decode_gemm_w2_kernel<NT, false, false, false, false, true>;
+        kh = p.tma_scales ? kFastKH : 2;
         smem = Smem<NT, false>::kTotal;
     } else if (!p.w4 && p.q4) {
         kern = decode_gemm_w2_kernel<NT, false, false, false, true>;
         smem = Smem<NT, false, true>::kTotal;
     } else if (!p.w4) {
-        kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false, false>
+        kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false, false, false, false, kFastKH>
                             : decode_gemm_w2_kernel<NT, false, false, false>;
+        kh = p.tma_scales ? kFastKH : 2;
         smem = Smem<NT, false>::kTotal;
     }
     if (!kern) return cudaErrorInvalidValue;
-    cudaError_t err = prepare_kernel(kern, smem);
+    cudaError_t err = kh == 1 ? prepare_kernel<1>(kern, smem) : prepare_kernel<2>(kern, smem);
     if (err != cudaSuccess) return err;
+    const int threads = kh == 1 ? Cfg<1>::kThreads : Cfg<2>::kThreads;
     DecodeGemmParams q = p;
     q.row_blocks = row_blocks;
     q.ksplit = ksplit;
@@ -946,7 +981,7 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
     const int sms = device_sms(err);
     if (err != cudaSuccess) return err;
     MapSet m{a, b, c, d};
-    kern<<<std::min(q.units, sms), kThreads, smem, s>>>(m, m, q, q);
+    kern<<<std::min(q.units, sms), threads, smem, s>>>(m, m, q, q);
     return cudaGetLastError();
 }
 
@@ -955,12 +990,14 @@ cudaError_t launch_fused_nt(const DecodeGemmParams &p1, const MapSet &m1, int ro
                             const MapSet &m2, int row_blocks2, int experts, cudaStream_t s) {
     // fp32 group scales staged by TMA, or 4-bit scales read by the consumers (both projections alike)
     DecodeKernel kern = p1.q4     ? decode_gemm_w2_kernel<NT, false, false, true, true>
-                        : p1.std2 ? decode_gemm_w2_kernel<NT, true, false, true, false, true>
-                                  : decode_gemm_w2_kernel<NT, true, false, true>;
+                        : p1.std2 ? decode_gemm_w2_kernel<NT, true, false, true, false, true, kFastKH>
+                                  : decode_gemm_w2_kernel<NT, true, false, true, false, false, kFastKH>;
+    const int kh = p1.q4 ? 2 : kFastKH;
     const int smem = p1.q4 ? Smem<NT, false, true>::kTotal : Smem<NT, false>::kTotal;
     int per_sm = 0;
-    cudaError_t err = prepare_kernel(kern, smem, &per_sm);
+    cudaError_t err = kh == 1 ? prepare_kernel<1>(kern, smem, &per_sm) : prepare_kernel<2>(kern, smem, &per_sm);
     if (err != cudaSuccess) return err;
+    const int threads = kh == 1 ? Cfg<1>::kThreads : Cfg<2>::kThreads;
     DecodeGemmParams q1 = p1, q2 = p2;
     q1.row_blocks = row_blocks1;
     q1.ksplit = 1;
@@ -978,7 +1015,7 @@ cudaError_t launch_fused_nt(const DecodeGemmParams &p1, const MapSet &m1, int ro
     const int grid = std::min(q1.units + q2.units, sms * per_sm);
     MapSet a = m1, b = m2;
     void *args[] = {&a, &b, &q1, &q2};
-    err = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), dim3(grid), dim3(kThreads), args, smem, s);
+    err = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), dim3(grid), dim3(threads), args, smem, s);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
