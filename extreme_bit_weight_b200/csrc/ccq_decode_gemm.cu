@@ -44,7 +44,6 @@ namespace {
 
 constexpr int kRowWarps = 8;                       // warps per 16-row slot set (256 rows per CTA)
 constexpr int kProducerWarps = 4;                   // one warpgroup; lane 0 of its first warp issues the loads
-constexpr int kProducerRegs = 24;
 // Consumer layout.  KH = 2: two warps per row slot, groups 0-3 / 4-7 of a stage, whose sums meet at
 // the end of a chunk (640 threads).  KH = 1: one warp per row slot takes all 8 groups (384 threads,
 // each consumer with twice the registers).
@@ -57,10 +56,14 @@ struct Cfg {
     static constexpr int kConsumerWarps = kRowWarps * KH;
     static constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
     static constexpr int kLaunchRegs = KH == 2 ? 96 : 168;
-    static constexpr int kConsumerRegs = KH == 2 ? 112 : 240;
+    // the producer warpgroup keeps what the consumers leave: its issue loop (and, KH 1, the scale
+    // expanders holding three rows' loads in flight) then runs without spills
+    static constexpr int kProducerRegs = KH == 2 ? 32 : 40;
+    static constexpr int kConsumerRegs = KH == 2 ? 112 : 232;
     static constexpr int kGroups = 8 / KH;  // groups of a stage per consumer warp
     static_assert(kProducerWarps * 32 * kProducerRegs + kConsumerWarps * 32 * kConsumerRegs <= kThreads * kLaunchRegs,
                   "register split exceeds the launch allocation");
+    static_assert(kProducerRegs % 8 == 0 && kConsumerRegs % 8 == 0 && kConsumerRegs <= 256, "setmaxnreg counts");
     static_assert(65536 / kThreads >= kLaunchRegs, "launch registers");
 };
 constexpr int kCodeTileBytes = 128 * 128;  // [128 rows][128 B] = 8 groups of 16 bytes
@@ -71,10 +74,11 @@ struct Smem {
     static constexpr int kCodeBytes = (W4 ? 2 : 1) * 2 * kCodeTileBytes;  // both halves, one stage
     static constexpr int kXaBytes = 32 * MP * 16 * 2;  // [G*4+i = 32][MP][16] bf16
     static constexpr int kGsBytes = MP * 8 * 16;       // [MP][8] gsq float4 entries
-    // [2 halves][128 rows][8 groups] fp32 scales (none for W4; 4-bit scales are read from global)
-    static constexpr int kScBytes = (W4 || Q4) ? 0 : 2 * 128 * 8 * 4;
-    // [4][128] fp32: alpha A, alpha B, beta A, beta B (W4: scales A, B); Q4: then super A, super B
-    static constexpr int kRowsBytes = Q4 ? 3072 : 2048;
+    // [2 halves][128 rows][8 groups] fp32 scales (none for W4; 4-bit scales are expanded into it by
+    // the producer warpgroup)
+    static constexpr int kScBytes = W4 ? 0 : 2 * 128 * 8 * 4;
+    // [4][128] fp32: alpha A, alpha B, beta A, beta B (W4: scales A, B)
+    static constexpr int kRowsBytes = 2048;
     static constexpr int kStageBytes = ((kCodeBytes + kXaBytes + kGsBytes + kScBytes + kRowsBytes) + 1023) & ~1023;
     static constexpr int kRedBytes = kRowWarps * 32 * 2 * NT * 4 * 4;  // partial sums of the second warp half
     static constexpr int kStages = ((227 * 1024 - 2048 - kRedBytes) / kStageBytes) < 4
@@ -412,7 +416,8 @@ template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false, bool STD = 
 __global__ void __launch_bounds__(Cfg<KH>::kThreads, 1)
 decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__ MapSet m2,
                       const __grid_constant__ DecodeGemmParams p, const __grid_constant__ DecodeGemmParams p2) {
-    static_assert(KH == 2 || (TMA_SC && !W4 && !Q4), "one warp per row slot needs TMA-staged fp32 scales");
+    static_assert(KH == 2 || (!W4 && (TMA_SC || Q4)), "one warp per row slot needs staged fp32 scales");
+    static_assert(!Q4 || (KH == 1 && !TMA_SC), "4-bit scales: expanded by the producer warpgroup");
     using S = Smem<NT, W4, Q4>;
     using C = Cfg<KH>;
     constexpr int MP = S::MP;
@@ -428,12 +433,22 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     __shared__ uint64_t full_bar[kStages], empty_bar[kStages], red_full, red_empty;
     __shared__ float epi_gs[FUSED ? kRowWarps : 1][FUSED ? MP : 1];  // fused gate/up epilogue sums
     __shared__ uint64_t epi_bar[2];  // fused gate/up epilogue: the 8 first-half warps meet twice per chunk
+    // Q4: the stage each ring slot holds, published by the producer for the scale expanders (warps
+    // 1-3 of the producer warpgroup), which complete the slot's full barrier once they have written
+    // its fp32 scales
+    struct StageDesc {
+        int rowA, rowB, nA, nB, st, phase;  // phase < 0: the end marker
+    };
+    __shared__ StageDesc sdesc[Q4 ? kStages : 1];
+    __shared__ uint64_t desc_bar[Q4 ? kStages : 1];
+    constexpr int kExpanderWarps = 3;
 
     const int units = p.units + (FUSED ? p2.units : 0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&full_bar[i], 1);
+            mbar_init(&full_bar[i], Q4 ? 1 + kExpanderWarps : 1);
+            if (Q4) mbar_init(&desc_bar[i], 1);
             mbar_init(&empty_bar[i], C::kConsumerWarps);
         }
         mbar_init(&red_full, kRowWarps);
@@ -513,8 +528,13 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             }
             fence_proxy_async_global();  // the generic-proxy writes of h are visible to TMA from here
         }
-        const uint32_t row_bytes =
-            (first && !STD) ? (uint32_t)(U.nA + U.nB) * 4u * (W4 ? 1u : Q4 ? 3u : 2u) : 0u;
+        if constexpr (Q4) {
+            // the stage this slot will hold, for the scale expanders (the slot is free: the empty
+            // barrier was passed before this call)
+            sdesc[slot] = StageDesc{rowA, rowB, U.nA, U.nB, st, U.phase};
+            mbar_arrive(&desc_bar[slot]);
+        }
+        const uint32_t row_bytes = (first && !STD) ? (uint32_t)(U.nA + U.nB) * 4u * (W4 ? 1u : 2u) : 0u;
         mbar_arrive_expect_tx(bar, S::kTxBytes + ((TMA_SC && !W4) ? S::kScBytes : 0) + row_bytes);
         if (first && !STD) {
             // the unit's per-row constants: alpha, beta (W2) or the channel scales (W4) of both halves
@@ -524,10 +544,6 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             if (!W4) {
                 if (U.nA) bulk_g2s(base + kRowsOff + 1024, q.beta + rowA, U.nA * 4u, bar);
                 if (U.nB) bulk_g2s(base + kRowsOff + 1536, q.beta + rowB, U.nB * 4u, bar);
-            }
-            if (Q4) {
-                if (U.nA) bulk_g2s(base + kRowsOff + 2048, q.super_scale + rowA, U.nA * 4u, bar);
-                if (U.nB) bulk_g2s(base + kRowsOff + 2560, q.super_scale + rowB, U.nB * 4u, bar);
             }
         }
         if (TMA_SC && !W4) {
@@ -565,7 +581,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
         }
     };
     if (warp >= C::kConsumerWarps) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kProducerRegs));
         if (warp == C::kConsumerWarps && lane == 0) {
             P.u = blockIdx.x;
             P.pi = P.slot = P.round = 0;
@@ -581,10 +597,15 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                 issue_next();
             }
             if (pok && !(P.pi >= kStages && !mbar_wait(&empty_bar[P.slot], (P.round & 1) ^ 1, p.err))) {
-                // end marker: a ring slot without loads whose descriptor stops the consumers
+                // end marker: a ring slot without loads whose descriptor stops the consumers (and
+                // the scale expanders, which then complete the slot's barrier too)
                 Unit end{};
                 end.e = -1;
                 udesc[p_ord++ % kUnitRing] = end;
+                if constexpr (Q4) {
+                    sdesc[P.slot] = StageDesc{0, 0, 0, 0, 0, -1};
+                    mbar_arrive(&desc_bar[P.slot]);
+                }
                 mbar_arrive(&full_bar[P.slot]);
             } else {
                 pok = false;
@@ -593,6 +614,55 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                 // consumers stopped releasing: let the copies in flight land before exiting (bounded)
                 for (int j = max(0, P.pi - kStages); j < P.pi; ++j)
                     if (!mbar_wait(&full_bar[j % kStages], (j / kStages) & 1, p.err)) break;
+            }
+        } else if (Q4 && warp > C::kConsumerWarps) {
+            // scale expanders: for each slot in ring order, the 4-bit scales of the stage's rows ->
+            // fp32 s = fl32(q4 * super[row]) in the [half][row][8 groups] layout the consumers read
+            const int et = (warp - C::kConsumerWarps - 1) * 32 + lane;  // 0..95
+            for (int j = 0;; ++j) {
+                const int slot = j % kStages;
+                if (!mbar_wait(&desc_bar[slot], (j / kStages) & 1, p.err)) break;
+                const StageDesc d = sdesc[slot];
+                if (d.phase >= 0) {
+                    const DecodeGemmParams &q = (FUSED && d.phase) ? p2 : p;
+                    const int qpr = q.K / 128;  // scale bytes per row
+                    float *sc = reinterpret_cast<float *>(smem + slot * S::kStageBytes + kScOff);
+                    // rows et, et + 96, et + 192 (< 256): every load issued before any is used
+                    constexpr int kR = (256 + 32 * kExpanderWarps - 1) / (32 * kExpanderWarps);
+                    float sup[kR];
+                    uint32_t bytes[kR][4];
+#pragma unroll
+                    for (int k = 0; k < kR; ++k) {
+                        const int idx = et + 32 * kExpanderWarps * k;
+                        const int half = idx >> 7, r = idx & 127;
+                        const bool live = idx < 256 && r < (half ? d.nB : d.nA);
+                        const int row = (half ? d.rowB : d.rowA) + r;
+                        sup[k] = live ? __ldg(q.super_scale + row) : 0.0f;
+                        const uint8_t *src = q.scale_q4 + (size_t)(live ? row : 0) * qpr;
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            const int at = 4 * d.st + b;  // groups 8 st + 2b, 8 st + 2b + 1
+                            bytes[k][b] = (live && at < qpr) ? (uint32_t)__ldg(src + at) : 0u;
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < kR; ++k) {
+                        const int idx = et + 32 * kExpanderWarps * k;
+                        if (idx >= 256) break;
+                        float v[8];
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            v[2 * b] = __fmul_rn((float)(bytes[k][b] & 0xFu), sup[k]);
+                            v[2 * b + 1] = __fmul_rn((float)(bytes[k][b] >> 4), sup[k]);
+                        }
+                        float4 *dst = reinterpret_cast<float4 *>(sc + idx * 8);  // [half][row][8]
+                        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+                        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_bar[slot]);
+                if (d.phase < 0) break;
             }
         }
         return;
@@ -640,8 +710,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     int it = 0, slot = 0, round = 0, cc = 0;  // iteration (over all units), ring slot and round, chunk count
     int ec = 0;                               // fused gate/up chunks done (epilogue meeting parity)
     RowDecode rd[4];
-    float sc_row[4];  // W4: per-channel scales, bf16-rounded; Q4: the rows' super scales
-    uint32_t q4cur[4] = {0, 0, 0, 0}, q4nxt[4] = {0, 0, 0, 0};  // Q4: this / the next stage's scale nibbles
+    float sc_row[4];  // W4: per-channel scales, bf16-rounded
     float acc[2][NT][4];
 #pragma unroll
     for (int t = 0; t < 2; ++t)
@@ -673,10 +742,6 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                 rd[1].ab = f2_pack(r1, r1); rd[1].bb = f2_pack(b1, b1);
                 rd[2].ab = f2_pack(r2, r2); rd[2].bb = f2_pack(b2, b2);
                 rd[3].ab = f2_pack(r3, r3); rd[3].bb = f2_pack(b3, b3);
-                if constexpr (Q4) {
-                    sc_row[0] = lds_f32(ra + 2048); sc_row[1] = lds_f32(ra + 2080);
-                    sc_row[2] = lds_f32(ra + 2560); sc_row[3] = lds_f32(ra + 2592);
-                }
             } else {
                 sc_row[0] = round_bf16(r0); sc_row[1] = round_bf16(r1);
                 sc_row[2] = round_bf16(r2); sc_row[3] = round_bf16(r3);
@@ -689,46 +754,9 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                 constexpr int G = decltype(Gc)::value;
                 group_w4<NT, G>(sb + coff[G], xs, gs, sc_row, kc, acc);
             });
-        } else if (Q4) {
-            // 4-bit group scales: this thread's 4 nibbles (groups Gh..Gh+3) of each of its rows, read
-            // from global memory one stage ahead; s = bf16(fl32(q4 * super)).  Groups beyond K
-            // read activations 0 (TMA zero fill) and add nothing.
-            const int nst = U.s_end - U.s_begin;
-            auto q4_load = [&](int stg, uint32_t (&dst)[4]) {
-                const int qpr = pq.K / 128;  // scale bytes per row
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int lr = (r < 2 ? U.localA : U.localB) + wrow + g + 8 * (r & 1);
-                    const int grow = U.e * pq.N + (lr < pq.N ? lr : 0);
-                    // two single bytes: a row's scale bytes need not be 2-byte aligned, and the
-                    // last stage may end inside the row
-                    const int byte = stg * 4 + khalf * 2;
-                    const uint8_t *src = pq.scale_q4 + (size_t)grow * qpr + byte;
-                    const uint32_t lo = byte < qpr ? (uint32_t)__ldg(src) : 0u;
-                    const uint32_t hi = byte + 1 < qpr ? (uint32_t)__ldg(src + 1) : 0u;
-                    dst[r] = lo | (hi << 8);
-                }
-            };
-            if (first) q4_load(st, q4cur);
-            else {
-#pragma unroll
-                for (int r = 0; r < 4; ++r) q4cur[r] = q4nxt[r];
-            }
-            if (i + 1 < nst) q4_load(st + 1 == U.s_end ? U.s_begin : st + 1, q4nxt);
-            const uint32_t xs = sb + xa_thr, gs = sb + gs_thr;
-            static_for<4>([&](auto Gc) {
-                constexpr int G = decltype(Gc)::value;
-                float sc[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    // the nibble as a float: its bits under the exponent of 2^23, minus 2^23
-                    const float qf = __uint_as_float(0x4B000000u | ((q4cur[r] >> (4 * G)) & 0xFu)) - 8388608.0f;
-                    sc[r] = round_bf16(__fmul_rn(qf, sc_row[r]));
-                }
-                group_w2<NT, G, STD>(sb + coff[G], xs, gs, sc, rd, kc, acc);
-            });
-        } else if (TMA_SC) {
-            // full stage: groups beyond K read TMA zero fill (scale 0, activations 0) and add nothing
+        } else if (TMA_SC || Q4) {
+            // full stage (scales staged by TMA, or expanded from 4 bits by the producer warpgroup):
+            // groups beyond K read zero scales and activations and add nothing
             // this warp's groups, four at a time: groups 4Q..4Q+3 sit 16Q bytes further in the scale
             // rows, 16 MP 32 Q bytes further in the XA slice, 64Q in the gsq entries, and in the
             // 128-byte-swizzled chunk (G ^ g) ^ 4Q, i.e. with code address bit 6 flipped
@@ -933,7 +961,8 @@ cudaError_t prepare_kernel(DecodeKernel kern, int smem, int *per_sm = nullptr) {
     return kernel_setup(reinterpret_cast<const void *>(kern), smem, Cfg<KH>::kThreads, Cfg<KH>::kLaunchRegs, per_sm);
 }
 
-// Consumer layout for the fp32-scale 2-bit kernels (CCQ and STD); the others use KH = 2.
+// Consumer layout for the fp32-scale 2-bit kernels (CCQ and STD); 4-bit scales always take KH = 1 (their
+// expansion runs in the producer warpgroup), W4 and unstaged scales KH = 2.
 constexpr int kFastKH = 1;
 
 int device_sms(cudaError_t &err) {
@@ -961,7 +990,8 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
         kh = p.tma_scales ? kFastKH : 2;
         smem = Smem<NT, false>::kTotal;
     } else if (!p.w4 && p.q4) {
-        kern = decode_gemm_w2_kernel<NT, false, false, false, true>;
+        kern = decode_gemm_w2_kernel<NT, false, false, false, true, false, 1>;
+        kh = 1;
         smem = Smem<NT, false, true>::kTotal;
     } else if (!p.w4) {
         kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false, false, false, false, kFastKH>
@@ -989,10 +1019,10 @@ template <int NT>
 cudaError_t launch_fused_nt(const DecodeGemmParams &p1, const MapSet &m1, int row_blocks1, const DecodeGemmParams &p2,
                             const MapSet &m2, int row_blocks2, int experts, cudaStream_t s) {
     // fp32 group scales staged by TMA, or 4-bit scales read by the consumers (both projections alike)
-    DecodeKernel kern = p1.q4     ? decode_gemm_w2_kernel<NT, false, false, true, true>
+    DecodeKernel kern = p1.q4     ? decode_gemm_w2_kernel<NT, false, false, true, true, false, 1>
                         : p1.std2 ? decode_gemm_w2_kernel<NT, true, false, true, false, true, kFastKH>
                                   : decode_gemm_w2_kernel<NT, true, false, true, false, false, kFastKH>;
-    const int kh = p1.q4 ? 2 : kFastKH;
+    const int kh = p1.q4 ? 1 : kFastKH;
     const int smem = p1.q4 ? Smem<NT, false, true>::kTotal : Smem<NT, false>::kTotal;
     int per_sm = 0;
     cudaError_t err = kh == 1 ? prepare_kernel<1>(kern, smem, &per_sm) : prepare_kernel<2>(kern, smem, &per_sm);
