@@ -220,6 +220,8 @@ __device__ __forceinline__ void store_gsq(float *gsq, int pr, int G, int ld, int
 __global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__restrict__ tok_of, int P_valid,
                                int P, int K, float level, uint16_t *__restrict__ xa, float *__restrict__ gsq,
                                int *zero_ctr) {
+    pdl_wait();     // x, tok_of: written by earlier work
+    pdl_trigger();  // the matmul may load its prologue meanwhile; it waits for this grid's results
     if (zero_ctr && blockIdx.x == 0 && threadIdx.x == 0) *zero_ctr = 0;
     const int ng = K / 64, ld = gsum_ld(K);
     const size_t total = (size_t)P_valid * ng * 4;  // a multiple of 4: the lanes of one group stay together
@@ -275,6 +277,8 @@ __global__ void gsum_from_xa_kernel(const uint16_t *__restrict__ xa, int P_valid
 
 __global__ void splitk_reduce_kernel(const float *__restrict__ partial, int ksplit, size_t split_stride, int M,
                                      int N, uint16_t *__restrict__ y) {
+    pdl_wait();  // the partial sums of the matmul before
+    pdl_trigger();
     const size_t total = (size_t)M * N;
     for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
          idx += (size_t)gridDim.x * blockDim.x) {
@@ -404,9 +408,8 @@ cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes,
 cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,
                            uint16_t *xa, float *gsq, cudaStream_t s, int *zero_ctr) {
     if (P_valid <= 0) return cudaSuccess;
-    pack_xa_kernel<<<grid_for((size_t)P_valid * (K / 64) * 4, 128), 128, 0, s>>>(x, tok_of, P_valid, P, K, level, xa,
-                                                                                 gsq, zero_ctr);
-    return cudaGetLastError();
+    return launch_pdl(pack_xa_kernel, dim3(grid_for((size_t)P_valid * (K / 64) * 4, 128)), dim3(128), 0, s, x, tok_of,
+                      P_valid, P, K, level, xa, gsq, zero_ctr);
 }
 
 cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float level, float *gsq,
@@ -419,8 +422,8 @@ cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, f
 cudaError_t launch_splitk_reduce(const float *partial, int ksplit, size_t split_stride, int M, int N,
                                  uint16_t *y, cudaStream_t s) {
     if ((size_t)M * N == 0) return cudaSuccess;
-    splitk_reduce_kernel<<<grid_for((size_t)M * N, 256), 256, 0, s>>>(partial, ksplit, split_stride, M, N, y);
-    return cudaGetLastError();
+    return launch_pdl(splitk_reduce_kernel, dim3(grid_for((size_t)M * N, 256)), dim3(256), 0, s, partial, ksplit,
+                      split_stride, M, N, y);
 }
 
 cudaError_t launch_moe_route(const int *ids, const float *rw, int T, int topk, int E, int *seg_off, int *cursor,

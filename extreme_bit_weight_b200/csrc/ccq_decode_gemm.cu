@@ -445,6 +445,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
 
     const int units = p.units + (FUSED ? p2.units : 0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_trigger();  // a dependent grid cannot fit beside this one; it is scheduled as CTAs retire
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full_bar[i], Q4 ? 1 + kExpanderWarps : 1);
@@ -583,6 +584,10 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     if (warp >= C::kConsumerWarps) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kProducerRegs));
         if (warp == C::kConsumerWarps && lane == 0) {
+            // the work counter, the activation operand and its gsq table come from the kernel before
+            // (with programmatic launch this grid may start while it still runs); everything the
+            // consumers and expanders do follows this thread's loads
+            pdl_wait();
             P.u = blockIdx.x;
             P.pi = P.slot = P.round = 0;
             p_ord = 0;
@@ -1011,8 +1016,7 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
     const int sms = device_sms(err);
     if (err != cudaSuccess) return err;
     MapSet m{a, b, c, d};
-    kern<<<std::min(q.units, sms), threads, smem, s>>>(m, m, q, q);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(std::min(q.units, sms)), dim3(threads), (size_t)smem, s, m, m, q, q);
 }
 
 template <int NT>

@@ -35,6 +35,13 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
+// Programmatic dependent launch.  pdl_wait: block until the grids this one depends on have
+// completed and their memory is visible (a no-op when the launch carries no such dependency).
+// pdl_trigger: let the next grid in the stream, if launched with programmatic serialization, be
+// scheduled now (it still waits in its own pdl_wait before touching this grid's results).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

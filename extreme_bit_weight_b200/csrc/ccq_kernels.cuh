@@ -12,6 +12,24 @@ namespace ccq {
 // runtime, so a small call's host cost is its launches.  per_sm may be NULL.
 cudaError_t kernel_setup(const void *kern, int smem, int threads, int want_regs, int *per_sm);
 
+// Launch `kern` with programmatic stream serialization: the grid may be scheduled while the previous
+// kernel in the stream finishes; the kernel itself waits (pdl_wait) before touching that kernel's
+// results.  Used for the dense matmul's chain (packing, decode kernel, split-K reduce).
+template <class... Params, class... Args>
+cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // Epilogue modes of the decode-sized grouped kernel.
 enum EpiMode : int {
     EPI_PARTIAL_F32 = 0,  // out_f32[ks][m][n] = partial sum over this CTA's k range
