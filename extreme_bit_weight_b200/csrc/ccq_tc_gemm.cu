@@ -34,11 +34,13 @@ namespace {
 constexpr int kDecWarps = 16;  // two threads per weight row of the 256-row tile
 constexpr int kEpiWarps = 4;
 constexpr int kTcThreads = (2 + kDecWarps + kEpiWarps) * 32;  // 704
-constexpr int kSA = 3;   // activation stages
-// decoded-weight stages: 3 with 128-token tiles (the MMA of a stage is short, so the decoders need
-// more room ahead), 2 with 256-token tiles (shared memory)
+// Ring depths.  Activation stages: 3 with 128-token tiles, 2 with 256-token tiles.  Decoded-weight
+// stages: as many as shared memory leaves (4 / 3; 3 with 128-token tiles of the embedded-scale
+// formats, whose code ring is wider), so that the decoders can run ahead of the MMA.
 template <int MT>
-constexpr int kSBof = MT == 1 ? 3 : 2;
+constexpr int kSAof = MT == 1 ? 3 : 2;
+template <int MT, int EMB>
+constexpr int kSBof = MT == 1 ? (EMB ? 3 : 4) : 3;
 constexpr int kSC = 2;   // code stages (4 groups each)
 constexpr int kATile = 128 * 64 * 2;   // 16 KB per 128-token sub-tile
 constexpr int kBTile = 256 * 64 * 2;   // 32 KB
@@ -53,8 +55,8 @@ constexpr int kCTileOf = 2 * 128 * kCRowOf<EMB>;  // two 128-row halves
 
 template <int MT, int EMB = 0>
 struct TcSmem {
-    static constexpr int kA = kSA * MT * kATile;
-    static constexpr int kB = kSBof<MT> * kBTile;
+    static constexpr int kA = kSAof<MT> * MT * kATile;
+    static constexpr int kB = kSBof<MT, EMB> * kBTile;
     static constexpr int kC = kSC * kCTileOf<EMB>;
     static constexpr int kTotal = kA + kB + kC + 1024;
     static_assert(kTotal + 512 <= 227 * 1024, "shared memory per CTA");
@@ -303,7 +305,8 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     using S = TcSmem<MT, EMB>;
     constexpr int kCRow = kCRowOf<EMB>;
     constexpr int kCTile = kCTileOf<EMB>;
-    constexpr int kSB = kSBof<MT>;
+    constexpr int kSA = kSAof<MT>;
+    constexpr int kSB = kSBof<MT, EMB>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned start, kept as an offset from the shared array so that loads and stores
     // through it stay shared-memory instructions
