@@ -86,6 +86,7 @@ _lib.ccq_moe_w2a16_forward.argtypes = [ctypes.POINTER(ccq_weight), ctypes.POINTE
 _lib.ccq_moe_w2a16_forward_traced.argtypes = [ctypes.POINTER(ccq_weight), ctypes.POINTER(ccq_weight), _I, _P, _I,
                                               _P, _P, _I, _P, _P, ctypes.c_size_t, _P, _P]
 _lib.ccq_check_device_error.argtypes = [_P, _P]
+_lib.ccq_selftest_bounded_wait.argtypes = [_P, _I, _I, _P]
 _lib.ccq_w2a16_gemm_noalloc.argtypes = [ctypes.POINTER(ccq_weight), _P, _I, _P, _P]
 _lib.ccq_w2a16_gemm_noalloc_max_scratch.restype = ctypes.c_size_t
 CCQ_MOE_TRACE_POINTS = 7
@@ -345,3 +346,10 @@ def exported_symbols():
     with open(hdr) as f:
         txt = f.read()
     return sorted(set(re.findall(r"\b(ccq_[a-z0-9_]+)\s*\(", txt)))
+
+
+def ccq_selftest_bounded_wait(ws: torch.Tensor, kind: int, limit_us: int = 20000, stream=None) -> None:
+    """Failure-detection self-test: a kernel whose bounded wait cannot be satisfied (kind 0: an
+    mbarrier phase, 1: a global counter) gives up after limit_us and records a timeout in ws's error
+    word; read it with ccq_check_device_error."""
+    _check(_lib.ccq_selftest_bounded_wait(_dptr(ws), kind, limit_us, _stream(stream)), "ccq_selftest_bounded_wait")

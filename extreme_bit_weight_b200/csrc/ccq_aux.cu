@@ -160,6 +160,24 @@ __global__ void dequant_emb_kernel(int kind, const uint8_t *__restrict__ codes, 
     }
 }
 
+// Failure-detection self-test: one CTA whose bounded waits can never be satisfied -- kind 0 an
+// mbarrier phase that nothing completes, kind 1 a global counter that nothing increments (it is
+// zeroed first).  Each wait gives up after limit_ns and records DEV_ERR_TIMEOUT in the error word,
+// as the matmul kernels' waits do; the kernel then returns normally.
+__global__ void bounded_wait_probe_kernel(uint32_t *err, int *never, int kind, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    if (kind == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        (void)mbar_wait(&bar, 0, err, limit_ns);  // nobody arrives
+    } else {
+        *never = 0;
+        __threadfence();
+        (void)wait_counter(never, 1, err, limit_ns);  // nobody adds
+    }
+}
+
 // WINT2-Standard round-to-nearest, one warp per (row, 64-column group); lane l holds columns 2l,
 // 2l+1.  s = bf16(max|w| / 2); the level round_half_even(w / s) clipped to [-2, 1] is decided by
 // comparing w with s/2 and 3s/2, which are exact in fp32 for a BF16 s, so the decision equals the
@@ -396,6 +414,11 @@ cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, c
     } else {
         dequant_w4_kernel<<<grid_for((size_t)rows * K / 2, 256), 256, 0, s>>>(codes, scales, rows, K, out);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bounded_wait_probe(uint32_t *err, int *never, int kind, uint64_t limit_ns, cudaStream_t s) {
+    bounded_wait_probe_kernel<<<1, 32, 0, s>>>(err, never, kind, limit_ns);
     return cudaGetLastError();
 }
 

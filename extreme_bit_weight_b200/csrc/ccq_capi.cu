@@ -655,6 +655,14 @@ ccq_status ccq_quantize_std_device(const float *w, int32_t n, int32_t k, uint8_t
     return cuda_status(launch_quantize_std(w, n, k, codes, scales, (cudaStream_t)stream));
 }
 
+ccq_status ccq_selftest_bounded_wait(void *ws, int32_t kind, int32_t limit_us, ccq_stream_t stream) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15u) || (kind != 0 && kind != 1)) return CCQ_ERR_INVALID_ARG;
+    if (limit_us < 1 || limit_us > 2000000) return CCQ_ERR_INVALID_ARG;
+    uint32_t *err = static_cast<uint32_t *>(ws);
+    int *never = reinterpret_cast<int *>(static_cast<uint8_t *>(ws) + 8);
+    return cuda_status(launch_bounded_wait_probe(err, never, kind, (uint64_t)limit_us * 1000u, (cudaStream_t)stream));
+}
+
 ccq_status ccq_check_device_error(void *ws, ccq_stream_t stream) {
     if (!ws) return CCQ_ERR_INVALID_ARG;
     uint32_t h[2] = {0, 0};

@@ -368,29 +368,11 @@ __device__ __forceinline__ bool load_unit_any(const DecodeGemmParams &p, const D
     return ok;
 }
 
-__device__ __forceinline__ int ld_acquire_gpu(const int *ptr) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-    return v;
-}
 __device__ __forceinline__ void red_release_gpu_add(int *ptr, int v) {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Bounded wait until *ctr >= need (another CTA's release); false after kWaitLimitNs.
-__device__ __forceinline__ bool wait_counter(const int *ctr, int need, uint32_t *err) {
-    if (ld_acquire_gpu(ctr) >= need) return true;
-    const uint64_t t0 = global_ns();
-    for (;;) {
-        __nanosleep(200);
-        if (ld_acquire_gpu(ctr) >= need) return true;
-        if (global_ns() - t0 > kWaitLimitNs) break;
-    }
-    record_error(err, DEV_ERR_TIMEOUT, 0xFFFFFFFEu);
-    return false;
 }
 
 // 1D bulk copy global -> shared completing on an mbarrier (16-byte aligned, size a multiple of 16)

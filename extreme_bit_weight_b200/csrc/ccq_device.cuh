@@ -101,16 +101,38 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t pa
 }
 
 // Bounded wait on phase `parity`; returns false (and records a timeout) if it does not complete
-// within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err) {
+// within limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (;;) {
         for (int i = 0; i < 8; ++i)
             if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
-        if (global_ns() - t0 > kWaitLimitNs) break;
+        if (global_ns() - t0 > limit_ns) break;
     }
     record_error(err, DEV_ERR_TIMEOUT, 0xFFFFFFFFu);
+    return false;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *ptr) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+// Bounded wait until *ctr >= need (another CTA's release); false (and a recorded timeout) after
+// limit_ns.
+__device__ __forceinline__ bool wait_counter(const int *ctr, int need, uint32_t *err,
+                                             uint64_t limit_ns = kWaitLimitNs) {
+    if (ld_acquire_gpu(ctr) >= need) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        __nanosleep(200);
+        if (ld_acquire_gpu(ctr) >= need) return true;
+        if (global_ns() - t0 > limit_ns) break;
+    }
+    record_error(err, DEV_ERR_TIMEOUT, 0xFFFFFFFEu);
     return false;
 }
 

@@ -169,6 +169,9 @@ cudaError_t launch_dequant(int fmt, const uint8_t *codes, const float *scales, c
 // codes [rows][K/64 * (22 or 20) bytes] and super [rows].
 cudaError_t launch_encode_emb(int kind, const float *w, int rows, int K, void *codes, float *super, cudaStream_t s);
 
+// Failure-detection self-test (see ccq_selftest_bounded_wait in ccq.h).
+cudaError_t launch_bounded_wait_probe(uint32_t *err, int *never, int kind, uint64_t limit_ns, cudaStream_t s);
+
 // WINT2-Standard round-to-nearest: w fp32 [rows][K] -> codes [rows][K/4], scales [rows][K/64]
 cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes, float *scales, cudaStream_t s);
 

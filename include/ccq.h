@@ -277,6 +277,15 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
  * workspace used by ccq_moe_w2a16_forward.  CCQ_OK, or CCQ_ERR_DEVICE_CHECK / CCQ_ERR_TIMEOUT. */
 ccq_status ccq_check_device_error(void *ws, ccq_stream_t stream);
 
+/* ccq_selftest_bounded_wait - failure-detection self-test (no paper counterpart).  Launches one
+ * CTA whose bounded wait can never be satisfied, with the same wait primitive the matmul kernels
+ * use: kind 0 waits on an mbarrier phase that nothing completes, kind 1 on a global counter that
+ * nothing increments.  The wait gives up after limit_us microseconds (1 .. 2 000 000), records
+ * CCQ_ERR_TIMEOUT in the error word at the start of `ws`, and the kernel returns; the context stays
+ * usable.  ws (device): at least 16 bytes, 16-byte aligned (a MoE workspace will do; bytes 8..11
+ * are overwritten).  Read the result with ccq_check_device_error. */
+ccq_status ccq_selftest_bounded_wait(void *ws, int32_t kind, int32_t limit_us, ccq_stream_t stream);
+
 /* ccq_status_string - static description of a status code. */
 const char *ccq_status_string(ccq_status s);
 

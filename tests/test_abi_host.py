@@ -98,6 +98,13 @@ def test_host_validation_returns_before_launch(ccq):
         assert e(fmt, fake, 4, 96, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG
         assert e(fmt, fake + 4, 4, 64, fake, fake, None) == ccq.CCQ_ERR_INVALID_ARG
     assert lib.ccq_encode_emb_device(ccq.CCQ_FMT_W2_CCQ_G64, fake, 4, 64, fake, fake, None) == ccq.CCQ_ERR_UNSUPPORTED
+    # failure-detection self-test: argument checks before any launch
+    t = lib.ccq_selftest_bounded_wait
+    assert t(None, 0, 1000, None) == ccq.CCQ_ERR_INVALID_ARG
+    assert t(fake + 4, 0, 1000, None) == ccq.CCQ_ERR_INVALID_ARG
+    assert t(fake, 2, 1000, None) == ccq.CCQ_ERR_INVALID_ARG
+    assert t(fake, 0, 0, None) == ccq.CCQ_ERR_INVALID_ARG
+    assert t(fake, 1, 3000000, None) == ccq.CCQ_ERR_INVALID_ARG
 
 
 def test_encoder_matches_oracle(ccq):

@@ -703,3 +703,22 @@ def test_moe_emb_small_token_tiles(ccq, fmts, T, zipf):
     assert st == ccq.CCQ_OK
     ref = oracle.moe_f64(synth.bf16_bits(x), d13, d2, ids, rw, round_h=True)
     assert rel_err(y, ref) <= TOL
+
+
+# ----------------------------------------------------------------------------------------------
+# failure detection: bounded waits give up, report, and leave the context usable
+# ----------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("kind", [0, 1])
+def test_bounded_wait_reports_timeout_and_context_survives(ccq, kind):
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ccq.ccq_selftest_bounded_wait(ws, kind, limit_us=20000)
+    assert ccq.ccq_check_device_error(ws) == ccq.CCQ_ERR_TIMEOUT
+    assert ccq.ccq_check_device_error(ws) == ccq.CCQ_OK  # the check clears the word
+    # the same context still computes exactly
+    n, k = 256, 512
+    codes, scales, a, b = synth.w2_format_random(n, k, 9900 + kind)
+    W = w2_weight(ccq, codes, scales, a, b)
+    eye = synth.one_hot_rows(k)[:16].contiguous().cuda()
+    y = ccq.ccq_w2a16_gemm(W, eye).float().cpu().numpy()
+    ref = oracle.bf16_to_f64(oracle.dequant_w2(codes, scales, a, b)).T.astype(np.float32)[:16]
+    assert np.array_equal(y, ref)
