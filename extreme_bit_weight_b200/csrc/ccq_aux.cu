@@ -279,6 +279,55 @@ __global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__rest
     }
 }
 
+// The (4,3,2) operand order (w275_pos): one thread per (operand row, group) gathers the group's 64
+// values, writes each to its position and sums L(k) x_k in column order (every product is exact:
+// an 8-bit level times a BF16 value).
+__global__ void pack_xa_w275_kernel(const uint16_t *__restrict__ x, const int *__restrict__ tok_of, int P_valid,
+                                    int P, int K, uint16_t *__restrict__ xa, float *__restrict__ gsq, int *zero_ctr) {
+    pdl_wait();
+    pdl_trigger();
+    if (zero_ctr && blockIdx.x == 0 && threadIdx.x == 0) *zero_ctr = 0;
+    const int ng = K / 64, ld = gsum_ld(K);
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < (size_t)P_valid * ng;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int pr = (int)(idx / ng), G = (int)(idx % ng);
+        const int src = tok_of ? __ldg(tok_of + pr) : pr;
+        const uint4 *blk = reinterpret_cast<const uint4 *>(x + (size_t)src * K + (size_t)G * 64);
+        float sum = 0.0f;
+        for (int q = 0; q < 8; ++q) {
+            const uint4 w4 = __ldg(blk + q);
+            const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+                const int k = 8 * q + h;
+                const uint16_t v = (uint16_t)(ws[h >> 1] >> (16 * (h & 1)));
+                int i, tig, b;
+                w275_pos(k, i, tig, b);
+                sum += w275_level(i, b) * bf16_bits_to_float(v);
+                xa[xa_index_perm((size_t)pr, (size_t)G * 64 + k, (size_t)P, 1)] = v;
+            }
+        }
+        store_gsq(gsq, pr, G, ld, P_valid, sum);
+    }
+}
+
+__global__ void gsum_from_xa_w275_kernel(const uint16_t *__restrict__ xa, int P_valid, int P, int K,
+                                         float *__restrict__ gsq) {
+    const int ng = K / 64, ld = gsum_ld(K);
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < (size_t)P_valid * ng;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int pr = (int)(idx / ng), G = (int)(idx % ng);
+        float sum = 0.0f;
+        for (int k = 0; k < 64; ++k) {
+            int i, tig, b;
+            w275_pos(k, i, tig, b);
+            sum += w275_level(i, b) *
+                   bf16_bits_to_float(xa[xa_index_perm((size_t)pr, (size_t)G * 64 + k, (size_t)P, 1)]);
+        }
+        store_gsq(gsq, pr, G, ld, P_valid, sum);
+    }
+}
+
 __global__ void gsum_from_xa_kernel(const uint16_t *__restrict__ xa, int P_valid, int P, int K, float level,
                                     float *__restrict__ gsq) {
     const int ng = K / 64, ld = gsum_ld(K);
@@ -429,15 +478,22 @@ cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes,
 }
 
 cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,
-                           uint16_t *xa, float *gsq, cudaStream_t s, int *zero_ctr) {
+                           uint16_t *xa, float *gsq, cudaStream_t s, int *zero_ctr, int perm) {
     if (P_valid <= 0) return cudaSuccess;
+    if (perm == 1)
+        return launch_pdl(pack_xa_w275_kernel, dim3(grid_for((size_t)P_valid * (K / 64), 128)), dim3(128), 0, s, x,
+                          tok_of, P_valid, P, K, xa, gsq, zero_ctr);
     return launch_pdl(pack_xa_kernel, dim3(grid_for((size_t)P_valid * (K / 64) * 4, 128)), dim3(128), 0, s, x, tok_of,
                       P_valid, P, K, level, xa, gsq, zero_ctr);
 }
 
 cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float level, float *gsq,
-                                cudaStream_t s) {
+                                cudaStream_t s, int perm) {
     if (P_valid <= 0) return cudaSuccess;
+    if (perm == 1) {
+        gsum_from_xa_w275_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(xa, P_valid, P, K, gsq);
+        return cudaGetLastError();
+    }
     gsum_from_xa_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(xa, P_valid, P, K, level, gsq);
     return cudaGetLastError();
 }

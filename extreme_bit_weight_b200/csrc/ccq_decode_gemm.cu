@@ -68,15 +68,19 @@ struct Cfg {
 };
 constexpr int kCodeTileBytes = 128 * 128;  // [128 rows][128 B] = 8 groups of 16 bytes
 
-template <int NT, bool W4 = false, bool Q4 = false>
+// The (4,3,2) format's code rows: 8 groups x 22 bytes per stage and row (unswizzled TMA boxes)
+constexpr int kW275Row = 176;
+constexpr int kW275Half = 128 * kW275Row;
+
+template <int NT, bool W4 = false, bool Q4 = false, bool W275 = false>
 struct Smem {
     static constexpr int MP = 8 * NT;
-    static constexpr int kCodeBytes = (W4 ? 2 : 1) * 2 * kCodeTileBytes;  // both halves, one stage
+    static constexpr int kCodeBytes = W275 ? 2 * kW275Half : (W4 ? 2 : 1) * 2 * kCodeTileBytes;  // both halves
     static constexpr int kXaBytes = 32 * MP * 16 * 2;  // [G*4+i = 32][MP][16] bf16
     static constexpr int kGsBytes = MP * 8 * 16;       // [MP][8] gsq float4 entries
     // [2 halves][128 rows][8 groups] fp32 scales (none for W4; 4-bit scales are expanded into it by
     // the producer warpgroup)
-    static constexpr int kScBytes = W4 ? 0 : 2 * 128 * 8 * 4;
+    static constexpr int kScBytes = (W4 || W275) ? 0 : 2 * 128 * 8 * 4;
     // [4][128] fp32: alpha A, alpha B, beta A, beta B (W4: scales A, B)
     static constexpr int kRowsBytes = 2048;
     static constexpr int kStageBytes = ((kCodeBytes + kXaBytes + kGsBytes + kScBytes + kRowsBytes) + 1023) & ~1023;
@@ -324,6 +328,49 @@ __device__ __forceinline__ void group_w4(uint32_t ca, uint32_t xs, uint32_t gs, 
     group_mma<NT, G>(R[0], R[1], R[2], R[3], xs, gs, sc, acc);
 }
 
+template <int OFF>
+__device__ __forceinline__ uint32_t lds16_at(uint32_t a) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1+%2];" : "=h"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ uint32_t lds8_at(uint32_t a) {
+    uint16_t v;
+    asm volatile("ld.shared.u8 %0, [%1+%2];" : "=h"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+
+// (4,3,2) format: one row's part of group G for this thread (operand order w275_pos): the word of
+// codes 4tig..4tig+3, code 16+tig and the extra code's byte, decoded into the eight A-fragment
+// registers as BF16 2^(7-T) + u (T = 0, 2, 3: shift-0 states as they are, shift-2 states two bits
+// up, shift-4 states moved down by one), and the group's scale bf16(fl32(q * super)), q the low
+// nibble of code 21.  rb: the row's code line; o_w = 4 tig, o_b = 16 + tig, o_e = 20 + (tig == 3),
+// sh_e: the extra state's shift (4 - 2 tig, or 4 for tig 3).
+template <int G>
+__device__ __forceinline__ void decode_w275_row(uint32_t rb, uint32_t o_w, uint32_t o_b, uint32_t o_e, uint32_t sh_e,
+                                                float sup, uint32_t (&R)[8], float &s) {
+    uint32_t W;
+    if constexpr ((G & 1) == 0) {
+        W = lds32_at<22 * G>(rb + o_w);  // group start 22 G: 4-byte aligned for even G
+    } else {
+        W = lds16_at<22 * G>(rb + o_w) | (lds16_at<22 * G + 2>(rb + o_w) << 16);
+    }
+    const uint32_t b16 = lds8_at<22 * G>(rb + o_b);
+    const uint32_t ex = lds8_at<22 * G>(rb + o_e);
+    const uint32_t q = lds8_at<22 * G + 21>(rb) & 0xFu;
+    const uint32_t W8 = W >> 8, W1 = W >> 1, W9 = W >> 9;
+    R[0] = and_or(W, 0x000F000Fu, 0x43004300u);   // shift-0 states of bytes 0, 2: 128 + u
+    R[1] = and_or(W8, 0x000F000Fu, 0x43004300u);  // bytes 1, 3
+    R[2] = and_or(W, 0x003C003Cu, 0x42004200u);   // shift-2 states: 32 + u
+    R[3] = and_or(W8, 0x003C003Cu, 0x42004200u);
+    R[4] = and_or(W1, 0x00780078u, 0x41804180u);  // shift-4 states, one bit down: 16 + u
+    R[5] = and_or(W9, 0x00780078u, 0x41804180u);
+    R[6] = and_or(b16 * 0x10001u, 0x003C000Fu, 0x42004300u);  // code 16+tig: shift 0 | shift 2
+    R[7] = and_or(((ex >> sh_e) << 16) + (b16 >> 1), 0x000F0078u, 0x43004180u);  // its shift 4 | the extra
+    s = round_bf16(__fmul_rn(__uint_as_float(0x4B000000u | q) - 8388608.0f, sup));
+}
+
 // One work unit of the persistent kernel: expert e, 256-row block rb (two 128-row halves), k split ks.
 // A unit walks its stages starting at s_begin + rot (wrapping): units that run at the same time
 // then read different 128-byte column slabs of their rows, which spreads the loads over the DRAM
@@ -394,13 +441,16 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
 // FUSED: the launch holds the MoE gate/up units (p, m1) followed by the down units (p2, m2).
 // STD: WINT2-Standard plain 2-bit fields (no per-row constants).  KH: consumer layout (Cfg; KH = 1
 // only with TMA-staged fp32 scales).
-template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false, bool STD = false, int KH = 2>
+template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false, bool STD = false, int KH = 2,
+          bool W275 = false>
 __global__ void __launch_bounds__(Cfg<KH>::kThreads, 1)
 decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__ MapSet m2,
                       const __grid_constant__ DecodeGemmParams p, const __grid_constant__ DecodeGemmParams p2) {
-    static_assert(KH == 2 || (!W4 && (TMA_SC || Q4)), "one warp per row slot needs staged fp32 scales");
+    static_assert(KH == 2 || (!W4 && (TMA_SC || Q4 || W275)), "one warp per row slot needs staged scales");
     static_assert(!Q4 || (KH == 1 && !TMA_SC), "4-bit scales: expanded by the producer warpgroup");
-    using S = Smem<NT, W4, Q4>;
+    static_assert(!W275 || (KH == 1 && !TMA_SC && !W4 && !Q4 && !STD), "(4,3,2): scales come with the codes");
+    using S = Smem<NT, W4, Q4, W275>;
+    constexpr int kCodeHalf = W275 ? kW275Half : kCodeTileBytes;  // second half's code tile
     using C = Cfg<KH>;
     constexpr int MP = S::MP;
     constexpr int kStages = S::kStages;
@@ -517,14 +567,15 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             sdesc[slot] = StageDesc{rowA, rowB, U.nA, U.nB, st, U.phase};
             mbar_arrive(&desc_bar[slot]);
         }
-        const uint32_t row_bytes = (first && !STD) ? (uint32_t)(U.nA + U.nB) * 4u * (W4 ? 1u : 2u) : 0u;
+        const uint32_t row_bytes = (first && !STD) ? (uint32_t)(U.nA + U.nB) * 4u * ((W4 || W275) ? 1u : 2u) : 0u;
         mbar_arrive_expect_tx(bar, S::kTxBytes + ((TMA_SC && !W4) ? S::kScBytes : 0) + row_bytes);
         if (first && !STD) {
-            // the unit's per-row constants: alpha, beta (W2) or the channel scales (W4) of both halves
-            const float *ra = W4 ? q.scales : q.alpha;
+            // the unit's per-row constants: alpha, beta (W2), the channel scales (W4) or the super
+            // scales ((4,3,2)) of both halves
+            const float *ra = W4 ? q.scales : W275 ? q.super_scale : q.alpha;
             if (U.nA) bulk_g2s(base + kRowsOff, ra + rowA, U.nA * 4u, bar);
             if (U.nB) bulk_g2s(base + kRowsOff + 512, ra + rowB, U.nB * 4u, bar);
-            if (!W4) {
+            if (!W4 && !W275) {
                 if (U.nA) bulk_g2s(base + kRowsOff + 1024, q.beta + rowA, U.nA * 4u, bar);
                 if (U.nB) bulk_g2s(base + kRowsOff + 1536, q.beta + rowB, U.nB * 4u, bar);
             }
@@ -534,12 +585,12 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             tma_load_2d(sc, &m.sc, bar, st * 8, rowA);
             tma_load_2d(sc + S::kScBytes / 2, &m.sc, bar, st * 8, rowB);
         }
-        // W2: 128 code bytes per row per stage; W4: 256, as two 128-byte boxes
+        // W2: 128 code bytes per row per stage; W4: 256, as two 128-byte boxes; (4,3,2): one 176-byte box
 #pragma unroll
         for (int bx = 0; bx < (W4 ? 2 : 1); ++bx) {
-            const int x = st * (W4 ? 256 : 128) + bx * 128;
+            const int x = W275 ? st * kW275Row : st * (W4 ? 256 : 128) + bx * 128;
             tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes, &m.codes, bar, x, rowA);
-            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes + kCodeTileBytes, &m.codes, bar, x, rowB);
+            tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes + kCodeHalf, &m.codes, bar, x, rowB);
         }
         tma_load_3d(base + kXaOff, &m.xa, bar, 0, U.seg0 + c * MP, st * 32);
         tma_load_2d(base + kGsOff, &m.gs, bar, st * 32, U.seg0 + c * MP);
@@ -692,6 +743,13 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     const uint32_t sc_thr = kScOff + (uint32_t)(wrow + g) * 32u + (uint32_t)Gh * 4u;   // row wrow+g, groups Gh..
     const uint32_t rows_thr = kRowsOff + (uint32_t)(wrow + g) * 4u;                     // row wrow+g of half A
     const uint32_t sbase = smem_u32(smem);
+    // (4,3,2): this thread's four code lines (rows g, g+8 of both halves) and byte offsets
+    uint32_t w_row[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+        w_row[r] = kCodeOff + (uint32_t)(r >> 1) * (uint32_t)kW275Half + (uint32_t)(wrow + g + 8 * (r & 1)) * kW275Row;
+    const uint32_t w_ow = 4u * (uint32_t)tig, w_ob = 16u + (uint32_t)tig, w_oe = 20u + (tig == 3 ? 1u : 0u);
+    const uint32_t w_she = tig < 3 ? 4u - 2u * (uint32_t)tig : 4u;
 
     bool ok = true;
     int it = 0, slot = 0, round = 0, cc = 0;  // iteration (over all units), ring slot and round, chunk count
@@ -722,7 +780,9 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             // this unit's per-row constants arrived with its first stage
             const uint32_t ra = sb + rows_thr;
             const float r0 = lds_f32(ra), r1 = lds_f32(ra + 32), r2 = lds_f32(ra + 512), r3 = lds_f32(ra + 544);
-            if constexpr (!W4) {
+            if constexpr (W275) {
+                sc_row[0] = r0; sc_row[1] = r1; sc_row[2] = r2; sc_row[3] = r3;  // super scales
+            } else if constexpr (!W4) {
                 const float b0 = lds_f32(ra + 1024), b1 = lds_f32(ra + 1056), b2 = lds_f32(ra + 1536),
                             b3 = lds_f32(ra + 1568);
                 rd[0].ab = f2_pack(r0, r0); rd[0].bb = f2_pack(b0, b0);
@@ -740,6 +800,20 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             static_for<4>([&](auto Gc) {
                 constexpr int G = decltype(Gc)::value;
                 group_w4<NT, G>(sb + coff[G], xs, gs, sc_row, kc, acc);
+            });
+        } else if (W275) {
+            // (4,3,2): all 8 groups of the stage; each group's scale comes with its codes.  Groups
+            // beyond K read zero codes (scale 0) and zero activations and add nothing.
+            const uint32_t xs = sb + xa_thr, gs = sb + gs_thr;
+            static_for<8>([&](auto Gc) {
+                constexpr int G = decltype(Gc)::value;
+                uint32_t RA0[8], RA1[8], RB0[8], RB1[8];
+                float sc[4];
+                decode_w275_row<G>(sb + w_row[0], w_ow, w_ob, w_oe, w_she, sc_row[0], RA0, sc[0]);
+                decode_w275_row<G>(sb + w_row[1], w_ow, w_ob, w_oe, w_she, sc_row[1], RA1, sc[1]);
+                decode_w275_row<G>(sb + w_row[2], w_ow, w_ob, w_oe, w_she, sc_row[2], RB0, sc[2]);
+                decode_w275_row<G>(sb + w_row[3], w_ow, w_ob, w_oe, w_she, sc_row[3], RB1, sc[3]);
+                group_mma<NT, G>(RA0, RA1, RB0, RB1, xs, gs, sc, acc);
             });
         } else if (TMA_SC || Q4) {
             // full stage (scales staged by TMA, or expanded from 4 bits by the producer warpgroup):
@@ -851,8 +925,17 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                     const float h = silu(acc[0][n][q]) * acc[1][n][q];
                     const size_t pr = (size_t)(U.seg0 + tok);
                     const uint16_t hb = float_to_bf16_bits(h);
-                    reinterpret_cast<uint16_t *>(pq.out)[xa_index(pr, (size_t)r, (size_t)pq.h_P)] = hb;
-                    if constexpr (FUSED) hsum[n][q & 1] += bf16_bits_to_float(hb);
+                    reinterpret_cast<uint16_t *>(pq.out)[xa_index_perm(pr, (size_t)r, (size_t)pq.h_P, pq.h_perm)] = hb;
+                    if constexpr (FUSED) {
+                        // (4,3,2) down weight: each column carries its own level offset
+                        float lw = 1.0f;
+                        if (pq.h_perm) {
+                            int li, lt, lb;
+                            w275_pos(r & 63, li, lt, lb);
+                            lw = w275_level(li, lb);
+                        }
+                        hsum[n][q & 1] += lw * bf16_bits_to_float(hb);
+                    }
                     continue;
                 }
 #pragma unroll
@@ -905,7 +988,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                         }
                         if (t0 + 1 >= U.Me) s1 = 0.0f;
                         const int G = U.localA / 64 + (wslot >> 2);
-                        const float L = pq.fuse_level;
+                        const float L = pq.h_perm ? 1.0f : pq.fuse_level;  // (perm 1: levels applied per column)
                         reinterpret_cast<float4 *>(pq.fuse_gsq)[(size_t)(U.seg0 + t0) * pq.fuse_gsq_ld + G] =
                             make_float4(L * s0, L * s1, L * s0, L * s1);
                     }
@@ -971,7 +1054,11 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
             smem = Smem<NT, true>::kTotal;
         }
     }
-    if (!p.w4 && p.std2) {
+    if (p.emb == 1) {
+        kern = decode_gemm_w2_kernel<NT, false, false, false, false, false, 1, true>;
+        kh = 1;
+        smem = Smem<NT, false, false, true>::kTotal;
+    } else if (!p.w4 && p.std2) {
         kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false, false, false, true, kFastKH>
                             : decode_gemm_w2_kernel<NT, false, false, false, false, true>;
         kh = p.tma_scales ? kFastKH : 2;
@@ -1005,11 +1092,14 @@ template <int NT>
 cudaError_t launch_fused_nt(const DecodeGemmParams &p1, const MapSet &m1, int row_blocks1, const DecodeGemmParams &p2,
                             const MapSet &m2, int row_blocks2, int experts, cudaStream_t s) {
     // fp32 group scales staged by TMA, or 4-bit scales read by the consumers (both projections alike)
-    DecodeKernel kern = p1.q4     ? decode_gemm_w2_kernel<NT, false, false, true, true, false, 1>
-                        : p1.std2 ? decode_gemm_w2_kernel<NT, true, false, true, false, true, kFastKH>
-                                  : decode_gemm_w2_kernel<NT, true, false, true, false, false, kFastKH>;
-    const int kh = p1.q4 ? 1 : kFastKH;
-    const int smem = p1.q4 ? Smem<NT, false, true>::kTotal : Smem<NT, false>::kTotal;
+    DecodeKernel kern = p1.emb == 1 ? decode_gemm_w2_kernel<NT, false, false, true, false, false, 1, true>
+                        : p1.q4     ? decode_gemm_w2_kernel<NT, false, false, true, true, false, 1>
+                        : p1.std2   ? decode_gemm_w2_kernel<NT, true, false, true, false, true, kFastKH>
+                                    : decode_gemm_w2_kernel<NT, true, false, true, false, false, kFastKH>;
+    const int kh = (p1.q4 || p1.emb == 1) ? 1 : kFastKH;
+    const int smem = p1.emb == 1 ? Smem<NT, false, false, true>::kTotal
+                     : p1.q4     ? Smem<NT, false, true>::kTotal
+                                 : Smem<NT, false>::kTotal;
     int per_sm = 0;
     cudaError_t err = kh == 1 ? prepare_kernel<1>(kern, smem, &per_sm) : prepare_kernel<2>(kern, smem, &per_sm);
     if (err != cudaSuccess) return err;
@@ -1056,7 +1146,9 @@ cudaError_t launch_decode_moe_fused(const DecodeGemmParams &p1, const CUtensorMa
                                     const CUtensorMap &c2, const CUtensorMap &d2, int row_blocks2, int experts,
                                     int nt, cudaStream_t s) {
     const bool fp32_sc = !p1.q4 && !p2.q4 && p1.tma_scales && p2.tma_scales, q4_sc = p1.q4 && p2.q4;
-    if (p1.w4 || p2.w4 || !(fp32_sc || q4_sc) || p1.std2 != p2.std2 || (q4_sc && p1.std2) || p1.mode != EPI_GATEUP || p2.mode != EPI_DOWN ||
+    const bool emb_both = p1.emb == 1 && p2.emb == 1;
+    if (p1.w4 || p2.w4 || !(fp32_sc || q4_sc || emb_both) || p1.std2 != p2.std2 || p1.emb != p2.emb ||
+        (q4_sc && p1.std2) || p1.mode != EPI_GATEUP || p2.mode != EPI_DOWN ||
         !p1.dep || !p2.dep || !p1.fuse_gsq)
         return cudaErrorInvalidValue;
     const MapSet m1{a1, b1, c1, d1}, m2{a2, b2, c2, d2};

@@ -51,6 +51,50 @@ __host__ __device__ inline size_t xa_index(size_t p, size_t k, size_t P) {
     return ((((G * 4 + i) * P + p) * 4 + tig) * 4 + j);
 }
 __host__ __device__ inline int gsum_ld(int K) { return ((K / 64) + 3) & ~3; }
+
+// Operand order of the (4,3,2) format (CCQ_FMT_W275_432) in the decode-sized kernel.  Thread tig
+// of a fragment quad decodes, per row and 64-column group, the states of codes 4tig..4tig+3 (one
+// 32-bit word), of code 16+tig, and one more state (code 20's state tig, or code 21's first state for
+// tig 3); a code j < 21 holds weights 3j (its first state, shift 4), 3j+1 (shift 2), 3j+2 (shift 0).
+// Its registers, as (slice i, element b) of the mma A fragment:
+//   i = 0: the shift-0 states of codes 4tig, 4tig+2, 4tig+1, 4tig+3 (b = 0..3);
+//   i = 1: the same codes' shift-2 states;  i = 2: their shift-4 states;
+//   i = 3: code 16+tig's shift-0, shift-2 and shift-4 states, then the extra state.
+// Each state reaches the tensor core as the BF16 value 2^(7-T) + u with T its bit position in the
+// register half (0, 2 or 3), so the group's accumulator starts at sum_k L(k) x_k with
+// L = -(2^(7-T) + 8) per position (-136, -40, -24).  w275_pos maps a group column w (0..63) to
+// (i, tig, b); w275_level gives L for (i, b).
+__host__ __device__ inline void w275_pos(int w, int &i, int &tig, int &b) {
+    if (w >= 60) {  // the extra states: weights 60..62 (code 20) and 63 (code 21)
+        i = 3;
+        tig = w - 60;
+        b = 3;
+        return;
+    }
+    const int c = w / 3, x = w % 3;  // code, state index (0: shift 4, 1: shift 2, 2: shift 0)
+    if (c >= 16) {
+        i = 3;
+        tig = c - 16;
+        b = 2 - x;  // shift 0, 2, 4 -> b 0, 1, 2
+        return;
+    }
+    tig = c >> 2;
+    i = 2 - x;                        // shift 0 -> slice 0, shift 2 -> 1, shift 4 -> 2
+    const int cb = c & 3;             // byte of the thread's word
+    b = (cb & 1) ? 2 + (cb >> 1) : cb >> 1;  // bytes 0, 2 -> b 0, 1; bytes 1, 3 -> b 2, 3
+}
+__host__ __device__ inline float w275_level(int i, int b) {
+    const int slot = i < 3 ? i : (b < 3 ? b : 0);  // 0: T = 0, 1: T = 2, 2: T = 3
+    return slot == 0 ? -136.0f : slot == 1 ? -40.0f : -24.0f;
+}
+// The decode-sized operand position of element (p, k): perm 0 = the CCQ / STD / W4 order (xa_index),
+// perm 1 = the (4,3,2) order above.
+__host__ __device__ inline size_t xa_index_perm(size_t p, size_t k, size_t P, int perm) {
+    if (perm == 0) return xa_index(p, k, P);
+    int i, tig, b;
+    w275_pos((int)(k & 63), i, tig, b);
+    return (((((k >> 6) * 4 + (size_t)i) * P + p) * 4 + (size_t)tig) * 4 + (size_t)b);
+}
 // The decoders hand the tensor core BF16 (128 + u) for CCQ state u (weight level u - 32),
 // (128 + q + 8) for W4 nibble q and (128 + q) for a STD 2-bit field q (level q - 2): the per-group
 // accumulator starts at L * S with L = -160 / -136 / -130.
@@ -87,6 +131,8 @@ struct DecodeGemmParams {
     const uint8_t *scale_q4;   // [rows_total][K/128]
     const float *super_scale;  // [rows_total]
     int std2;                  // 1: WINT2-Standard plain 2-bit fields (no alpha/beta)
+    int emb;                   // 1: the (4,3,2) format (codes with the scale inside; super_scale per row)
+    int h_perm;                // EPI_GATEUP: operand order of h for the down projection (xa_index_perm)
     uint32_t *err;
     // work units (set by the launcher): unit u = (expert, k split, row block), row block fastest
     int row_blocks, ksplit, units;
@@ -177,11 +223,12 @@ cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes,
 
 // x (BF16 [rows][K], row r taken from x[tok_of ? tok_of[p] : p]) -> XA operand + group sums.
 // zero_ctr (may be NULL): an int the kernel sets to 0 (the following matmul's work counter).
+// perm: operand order (xa_index_perm); perm 1 sums L(k) x_k per group and ignores `level`.
 cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,
-                           uint16_t *xa, float *gsq, cudaStream_t s, int *zero_ctr = nullptr);
+                           uint16_t *xa, float *gsq, cudaStream_t s, int *zero_ctr = nullptr, int perm = 0);
 // group-sum table of an operand already in XA layout (rows [0, P_valid))
 cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float level, float *gsq,
-                                cudaStream_t s);
+                                cudaStream_t s, int perm = 0);
 
 cudaError_t launch_splitk_reduce(const float *partial, int ksplit, size_t split_stride, int M, int N,
                                  uint16_t *y, cudaStream_t s);
