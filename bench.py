@@ -567,8 +567,7 @@ def run_ours(args, rank, world, local):
              "traffic": FUSED_DECODE_DRAM_BYTES_PER_EXPERT * ne if (SCALES, CODES) == ("fp32", "ccq") else None,
              "traffic_source": "ncu dram__bytes_read+write of the 16-expert capture, scaled by touched experts",
              "launch_ms": gemm1_ms, "algorithmic_bytes_per_launch": b13 + b2} if fused else
-            {"bound": "hbm", "kernel": ("tc_gemm_w2_kernel" if CODES == "w25" else "decode_gemm_w2_kernel")
-                                       + " (gate/up, SiLU epilogue)",
+            {"bound": "hbm", "kernel": "decode_gemm_w2_kernel (gate/up, SiLU epilogue)",
              "achieved": ach13, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "unit": "GB/s",
              "frac": ach13 / hbm, "traffic": None, "launch_ms": gemm1_ms,
              "algorithmic_bytes_per_launch": b13,
@@ -680,7 +679,7 @@ def run_gemm(args, rank, world, local):
             {"bound": "hbm", "achieved": gbs, "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "unit": "GB/s",
              "frac": gbs / hbm})
     roof.update({"kernel": "whole ccq_w2a16_gemm call (" + ("activation packing, tcgen05 kernel, split-K reduce"
-                                                            if tensor or CODES == "w25" else
+                                                            if tensor else
                  "activation packing, decode kernel, split-K reduce") + ")", "traffic": None,
                  "algorithmic_bytes_per_call": per_copy, "algorithmic_flops_per_call": flops})
     fmt_tag = ("std_w2_g64" if CODES == "std" else "ccq_w275_432_g64" if CODES == "w275" else

@@ -279,51 +279,43 @@ __global__ void pack_xa_kernel(const uint16_t *__restrict__ x, const int *__rest
     }
 }
 
-// The (4,3,2) operand order (w275_pos): one thread per (operand row, group) gathers the group's 64
-// values, writes each to its position and sums L(k) x_k in column order (every product is exact:
-// an 8-bit level times a BF16 value).
-__global__ void pack_xa_w275_kernel(const uint16_t *__restrict__ x, const int *__restrict__ tok_of, int P_valid,
-                                    int P, int K, uint16_t *__restrict__ xa, float *__restrict__ gsq, int *zero_ctr) {
+// The (4,3,2) and hybrid operand orders (perm 1, 2; xa_index_perm): one warp per (operand row, group);
+// lane l takes columns 2l, 2l+1, writes them to their positions and the warp sums L(k) x_k (every
+// product is exact: an 8-bit level times a BF16 value) in a fixed shuffle order.
+__global__ void pack_xa_perm_kernel(const uint16_t *__restrict__ x, const int *__restrict__ tok_of, int P_valid,
+                                    int P, int K, uint16_t *__restrict__ xa, float *__restrict__ gsq, int *zero_ctr,
+                                    int perm) {
     pdl_wait();
     pdl_trigger();
     if (zero_ctr && blockIdx.x == 0 && threadIdx.x == 0) *zero_ctr = 0;
-    const int ng = K / 64, ld = gsum_ld(K);
-    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < (size_t)P_valid * ng;
-         idx += (size_t)gridDim.x * blockDim.x) {
-        const int pr = (int)(idx / ng), G = (int)(idx % ng);
+    const int ng = K / 64, ld = gsum_ld(K), lane = threadIdx.x & 31;
+    const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
+    for (size_t u = blockIdx.x * (size_t)(blockDim.x >> 5) + (threadIdx.x >> 5); u < (size_t)P_valid * ng;
+         u += warps) {
+        const int pr = (int)(u / ng), G = (int)(u % ng);
         const int src = tok_of ? __ldg(tok_of + pr) : pr;
-        const uint4 *blk = reinterpret_cast<const uint4 *>(x + (size_t)src * K + (size_t)G * 64);
-        float sum = 0.0f;
-        for (int q = 0; q < 8; ++q) {
-            const uint4 w4 = __ldg(blk + q);
-            const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+        const uint32_t w2 = __ldg(reinterpret_cast<const uint32_t *>(x + (size_t)src * K + (size_t)G * 64) + lane);
+        const uint16_t v0 = (uint16_t)(w2 & 0xFFFFu), v1 = (uint16_t)(w2 >> 16);
+        const int k0 = 2 * lane;
+        float sum = perm_level(perm, k0) * bf16_bits_to_float(v0) + perm_level(perm, k0 + 1) * bf16_bits_to_float(v1);
 #pragma unroll
-            for (int h = 0; h < 8; ++h) {
-                const int k = 8 * q + h;
-                const uint16_t v = (uint16_t)(ws[h >> 1] >> (16 * (h & 1)));
-                int i, tig, b;
-                w275_pos(k, i, tig, b);
-                sum += w275_level(i, b) * bf16_bits_to_float(v);
-                xa[xa_index_perm((size_t)pr, (size_t)G * 64 + k, (size_t)P, 1)] = v;
-            }
-        }
-        store_gsq(gsq, pr, G, ld, P_valid, sum);
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        xa[xa_index_perm((size_t)pr, (size_t)G * 64 + k0, (size_t)P, perm)] = v0;
+        xa[xa_index_perm((size_t)pr, (size_t)G * 64 + k0 + 1, (size_t)P, perm)] = v1;
+        if (lane == 0) store_gsq(gsq, pr, G, ld, P_valid, sum);
     }
 }
 
-__global__ void gsum_from_xa_w275_kernel(const uint16_t *__restrict__ xa, int P_valid, int P, int K,
-                                         float *__restrict__ gsq) {
+__global__ void gsum_from_xa_perm_kernel(const uint16_t *__restrict__ xa, int P_valid, int P, int K,
+                                         float *__restrict__ gsq, int perm) {
     const int ng = K / 64, ld = gsum_ld(K);
     for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < (size_t)P_valid * ng;
          idx += (size_t)gridDim.x * blockDim.x) {
         const int pr = (int)(idx / ng), G = (int)(idx % ng);
         float sum = 0.0f;
-        for (int k = 0; k < 64; ++k) {
-            int i, tig, b;
-            w275_pos(k, i, tig, b);
-            sum += w275_level(i, b) *
-                   bf16_bits_to_float(xa[xa_index_perm((size_t)pr, (size_t)G * 64 + k, (size_t)P, 1)]);
-        }
+        for (int k = 0; k < 64; ++k)
+            sum += perm_level(perm, k) *
+                   bf16_bits_to_float(xa[xa_index_perm((size_t)pr, (size_t)G * 64 + k, (size_t)P, perm)]);
         store_gsq(gsq, pr, G, ld, P_valid, sum);
     }
 }
@@ -480,9 +472,9 @@ cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes,
 cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,
                            uint16_t *xa, float *gsq, cudaStream_t s, int *zero_ctr, int perm) {
     if (P_valid <= 0) return cudaSuccess;
-    if (perm == 1)
-        return launch_pdl(pack_xa_w275_kernel, dim3(grid_for((size_t)P_valid * (K / 64), 128)), dim3(128), 0, s, x,
-                          tok_of, P_valid, P, K, xa, gsq, zero_ctr);
+    if (perm != 0)
+        return launch_pdl(pack_xa_perm_kernel, dim3(grid_for((size_t)P_valid * (K / 64) * 32, 256)), dim3(256), 0, s,
+                          x, tok_of, P_valid, P, K, xa, gsq, zero_ctr, perm);
     return launch_pdl(pack_xa_kernel, dim3(grid_for((size_t)P_valid * (K / 64) * 4, 128)), dim3(128), 0, s, x, tok_of,
                       P_valid, P, K, level, xa, gsq, zero_ctr);
 }
@@ -490,8 +482,9 @@ cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, in
 cudaError_t launch_gsum_from_xa(const uint16_t *xa, int P_valid, int P, int K, float level, float *gsq,
                                 cudaStream_t s, int perm) {
     if (P_valid <= 0) return cudaSuccess;
-    if (perm == 1) {
-        gsum_from_xa_w275_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(xa, P_valid, P, K, gsq);
+    if (perm != 0) {
+        gsum_from_xa_perm_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(xa, P_valid, P, K, gsq,
+                                                                                           perm);
         return cudaGetLastError();
     }
     gsum_from_xa_kernel<<<grid_for((size_t)P_valid * (K / 64), 128), 128, 0, s>>>(xa, P_valid, P, K, level, gsq);

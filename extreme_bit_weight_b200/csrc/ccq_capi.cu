@@ -108,8 +108,10 @@ float level_of(const ccq_weight *w) {
 // --- decode-sized path ----------------------------------------------------------------------
 int pick_nt(double rows_per_expert, int fmt = CCQ_FMT_W2_CCQ_G64) {
     if (rows_per_expert <= 8.0) return 1;
-    // W4 code tiles are twice as wide; the (4,3,2) decode holds more registers per group
-    if (rows_per_expert <= 16.0 || fmt == CCQ_FMT_W4_PER_CHANNEL || fmt == CCQ_FMT_W275_432) return 2;
+    // W4 code tiles are twice as wide; the embedded-scale decodes hold more registers per group
+    if (rows_per_expert <= 16.0 || fmt == CCQ_FMT_W4_PER_CHANNEL || fmt == CCQ_FMT_W275_432 ||
+        fmt == CCQ_FMT_W25_HYBRID)
+        return 2;
     return 4;
 }
 
@@ -122,16 +124,17 @@ bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t
                  int nt) {
     const int K = w->k;
     const bool w4 = w->fmt == CCQ_FMT_W4_PER_CHANNEL;
-    const bool w275 = w->fmt == CCQ_FMT_W275_432;
+    const int emb = emb_kind(w);
     const cuuint64_t rows = (cuuint64_t)experts * w->n;
-    const cuuint64_t row_bytes = (cuuint64_t)(w4 ? K / 2 : w275 ? K / 64 * 22 : K / 4);
+    const cuuint32_t emb_row = emb == 1 ? 176u : 160u;  // 8 groups of 22 / 20 bytes
+    const cuuint64_t row_bytes = (cuuint64_t)(w4 ? K / 2 : emb ? K / 64 * (emb == 1 ? 22 : 20) : K / 4);
     {
-        // (4,3,2): one 176-byte box per stage (8 groups of 22 bytes), unswizzled
+        // embedded-scale formats: one unswizzled box of a stage's 8 groups per row
         cuuint64_t dims[2] = {row_bytes, rows};
         cuuint64_t str[1] = {row_bytes};
-        cuuint32_t box[2] = {w275 ? 176u : 128u, 128};
+        cuuint32_t box[2] = {emb ? emb_row : 128u, 128};
         if (!make_map(&m.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w->codes, dims, str, box,
-                      w275 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B))
+                      emb ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B))
             return false;
     }
     {
@@ -152,7 +155,7 @@ bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t
             return false;
     }
     // group scales [rows][K/64] fp32: staged by TMA when the row pitch is a multiple of 16 bytes
-    m.tma_scales = !w4 && !w275 && w->fmt != CCQ_FMT_W2_CCQ_G64_Q4SCALE && (K / 64) % 4 == 0;
+    m.tma_scales = !w4 && !emb && w->fmt != CCQ_FMT_W2_CCQ_G64_Q4SCALE && (K / 64) % 4 == 0;
     if (m.tma_scales) {
         cuuint64_t dims[2] = {(cuuint64_t)(K / 64), rows};
         cuuint64_t str[1] = {(cuuint64_t)(K / 64) * 4};
@@ -199,7 +202,7 @@ int sm_count() {
 
 GemmWs gemm_layout(const ccq_weight *w, int m) {
     GemmWs L{};
-    if (m >= kTcMinM || emb_kind(w) == 2) {  // (the hybrid format runs on the tcgen05 kernel only)
+    if (m >= kTcMinM) {
         L.tc = true;
         L.P = m;
         L.xt = 0;
@@ -403,7 +406,7 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
     float *gs = reinterpret_cast<float *>(base + L.gs);
     int *work = reinterpret_cast<int *>(base + L.work);
     cudaError_t e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), nullptr, m, L.P, w->k,
-                                   level_of(w), xa, gs, s, work, emb_kind(w) == 1 ? 1 : 0);
+                                   level_of(w), xa, gs, s, work, emb_kind(w));
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     DecodeMaps maps;
     if (!decode_maps(maps, w, 1, xa, gs, L.P, L.nt)) return CCQ_ERR_CUDA;
@@ -494,7 +497,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         e = launch_moe_route(expert_ids, routing_w, T, topk, num_experts, seg, cursor, tok, rwp, inv, dep, err, s);
     if (e == cudaSuccess) e = trace(events, 1, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
-    if (L.tc || emb_kind(w13) == 2 || emb_kind(w2) == 2) {
+    if (L.tc) {
         // prefill-sized: tcgen05 grouped GEMMs over (expert, 256-token tile) entries
         int2 *tiles = reinterpret_cast<int2 *>(base + L.tiles);
         int *tcount = reinterpret_cast<int *>(base + L.tcount);
@@ -550,7 +553,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         return cuda_status(e);
     }
     e = launch_pack_xa(static_cast<const uint16_t *>(x_bf16), tok, pairs, L.P, H, level_of(w13), xa_x, gs_x, s,
-                       nullptr, emb_kind(w13) == 1 ? 1 : 0);
+                       nullptr, emb_kind(w13));
     if (e == cudaSuccess) e = trace(events, 2, s);
     if (e != cudaSuccess) return CCQ_ERR_CUDA;
     const int nt1 = pick_nt((double)pairs / num_experts, w13->fmt);
@@ -601,9 +604,9 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
     // epilogue also writes h's group-sum table and each down unit starts once its expert's
     // gate/up units are done.  Otherwise (or if the device refuses the cooperative launch) two
     // launches with the group sums computed in between.
-    p1.h_perm = emb_kind(w2) == 1 ? 1 : 0;  // h in the down projection's operand order
+    p1.h_perm = emb_kind(w2);  // h in the down projection's operand order
     bool fused = !p1.w4 && !p2.w4 && nt1 == nt2 && p1.std2 == p2.std2 && p1.emb == p2.emb &&
-                 ((p1.tma_scales && p2.tma_scales && !p1.q4 && !p2.q4) || (p1.q4 && p2.q4) || p1.emb == 1);
+                 ((p1.tma_scales && p2.tma_scales && !p1.q4 && !p2.q4) || (p1.q4 && p2.q4) || p1.emb != 0);
     if (fused) {
         p1.dep = dep;
         p1.fuse_gsq = gs_h;
@@ -630,7 +633,7 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         e = launch_decode_gemm_w2(p1, m1.codes, m1.xa, m1.gs, m1.sc, ceil_div(I, 128), 1, num_experts, nt1, s);
         if (e == cudaSuccess) e = trace(events, 3, s);
         if (e == cudaSuccess)
-            e = launch_gsum_from_xa(xa_h, pairs, L.P, I, level_of(w2), gs_h, s, emb_kind(w2) == 1 ? 1 : 0);
+            e = launch_gsum_from_xa(xa_h, pairs, L.P, I, level_of(w2), gs_h, s, emb_kind(w2));
         if (e == cudaSuccess) e = trace(events, 4, s);
         if (e == cudaSuccess)
             e = launch_decode_gemm_w2(p2, m2.codes, m2.xa, m2.gs, m2.sc, ceil_div(H, 256), 1, num_experts, nt2, s);

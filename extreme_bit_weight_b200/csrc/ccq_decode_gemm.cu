@@ -68,19 +68,20 @@ struct Cfg {
 };
 constexpr int kCodeTileBytes = 128 * 128;  // [128 rows][128 B] = 8 groups of 16 bytes
 
-// The (4,3,2) format's code rows: 8 groups x 22 bytes per stage and row (unswizzled TMA boxes)
-constexpr int kW275Row = 176;
-constexpr int kW275Half = 128 * kW275Row;
+// The code rows of the formats with the scale in the codes (EMBK 1: (4,3,2), 8 groups x 22 bytes per
+// stage and row; 2: hybrid, 8 x 20), as unswizzled TMA boxes
+template <int EMBK>
+constexpr int kEmbRow = EMBK == 1 ? 176 : 160;
 
-template <int NT, bool W4 = false, bool Q4 = false, bool W275 = false>
+template <int NT, bool W4 = false, bool Q4 = false, int EMBK = 0>
 struct Smem {
     static constexpr int MP = 8 * NT;
-    static constexpr int kCodeBytes = W275 ? 2 * kW275Half : (W4 ? 2 : 1) * 2 * kCodeTileBytes;  // both halves
+    static constexpr int kCodeBytes = EMBK ? 2 * 128 * kEmbRow<EMBK> : (W4 ? 2 : 1) * 2 * kCodeTileBytes;  // both halves
     static constexpr int kXaBytes = 32 * MP * 16 * 2;  // [G*4+i = 32][MP][16] bf16
     static constexpr int kGsBytes = MP * 8 * 16;       // [MP][8] gsq float4 entries
     // [2 halves][128 rows][8 groups] fp32 scales (none for W4; 4-bit scales are expanded into it by
     // the producer warpgroup)
-    static constexpr int kScBytes = (W4 || W275) ? 0 : 2 * 128 * 8 * 4;
+    static constexpr int kScBytes = (W4 || EMBK) ? 0 : 2 * 128 * 8 * 4;
     // [4][128] fp32: alpha A, alpha B, beta A, beta B (W4: scales A, B)
     static constexpr int kRowsBytes = 2048;
     static constexpr int kStageBytes = ((kCodeBytes + kXaBytes + kGsBytes + kScBytes + kRowsBytes) + 1023) & ~1023;
@@ -371,6 +372,28 @@ __device__ __forceinline__ void decode_w275_row(uint32_t rb, uint32_t o_w, uint3
     s = round_bf16(__fmul_rn(__uint_as_float(0x4B000000u | q) - 8388608.0f, sup));
 }
 
+// Hybrid format: one row's part of group G for this thread (operand order hyb_pos): words 2tig and
+// 2tig+1 (one 32-bit load), each state pair of the two words in one register as BF16 2^(7-T) + u (T 4
+// for states 0-4 moved down to bit 4, 2 for state 5, 0 for state 6), the extra pair (word 8's states
+// at shifts sha and shb, or word 8's state 6 and word 9's first state) at T = 0, and the group's scale
+// bf16(fl32(q * super)), q the low 13 bits of word 9.  rb: the row's code line; o_w = 4 tig.
+template <int G>
+__device__ __forceinline__ void decode_hyb_row(uint32_t rb, uint32_t o_w, uint32_t sha, uint32_t shb, float sup,
+                                               uint32_t (&R)[8], float &s) {
+    const uint32_t W = lds32_at<20 * G>(rb + o_w);  // group start 20 G: 4-byte aligned
+    const uint32_t W89 = lds32_at<20 * G + 16>(rb);  // words 8, 9
+    const uint32_t q = (W89 >> 16) & 0x1FFFu;
+    R[0] = and_or(W >> 9, 0x00700070u, 0x41004100u);  // state 0 (shift 13): 8 + u
+    R[1] = and_or(W >> 7, 0x00700070u, 0x41004100u);  // state 1 (shift 11)
+    R[2] = and_or(W >> 5, 0x00700070u, 0x41004100u);  // state 2 (shift 9)
+    R[3] = and_or(W >> 2, 0x00700070u, 0x41004100u);  // state 3 (shift 6)
+    R[4] = and_or(W, 0x00700070u, 0x41004100u);       // state 4 (shift 4)
+    R[5] = and_or(W, 0x001C001Cu, 0x42004200u);       // state 5 (shift 2): 32 + u
+    R[6] = and_or(W, 0x00070007u, 0x43004300u);       // state 6 (shift 0): 128 + u
+    R[7] = and_or(((W89 >> shb) << 16) | ((W89 >> sha) & 0x7u), 0x00070007u, 0x43004300u);
+    s = round_bf16(__fmul_rn(__uint_as_float(0x4B000000u | q) - 8388608.0f, sup));
+}
+
 // One work unit of the persistent kernel: expert e, 256-row block rb (two 128-row halves), k split ks.
 // A unit walks its stages starting at s_begin + rot (wrapping): units that run at the same time
 // then read different 128-byte column slabs of their rows, which spreads the loads over the DRAM
@@ -442,15 +465,17 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
 // STD: WINT2-Standard plain 2-bit fields (no per-row constants).  KH: consumer layout (Cfg; KH = 1
 // only with TMA-staged fp32 scales).
 template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false, bool STD = false, int KH = 2,
-          bool W275 = false>
+          int EMBK = 0>
 __global__ void __launch_bounds__(Cfg<KH>::kThreads, 1)
 decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__ MapSet m2,
                       const __grid_constant__ DecodeGemmParams p, const __grid_constant__ DecodeGemmParams p2) {
-    static_assert(KH == 2 || (!W4 && (TMA_SC || Q4 || W275)), "one warp per row slot needs staged scales");
+    static_assert(KH == 2 || (!W4 && (TMA_SC || Q4 || EMBK)), "one warp per row slot needs staged scales");
     static_assert(!Q4 || (KH == 1 && !TMA_SC), "4-bit scales: expanded by the producer warpgroup");
-    static_assert(!W275 || (KH == 1 && !TMA_SC && !W4 && !Q4 && !STD), "(4,3,2): scales come with the codes");
-    using S = Smem<NT, W4, Q4, W275>;
-    constexpr int kCodeHalf = W275 ? kW275Half : kCodeTileBytes;  // second half's code tile
+    static_assert(!EMBK || (KH == 1 && !TMA_SC && !W4 && !Q4 && !STD), "embedded scales come with the codes");
+    using S = Smem<NT, W4, Q4, EMBK>;
+    constexpr bool W275 = EMBK != 0;  // (formats with the scale in the codes: super scale per row, no scale region)
+    constexpr int kERow = EMBK ? kEmbRow<EMBK> : 0;
+    constexpr int kCodeHalf = EMBK ? 128 * kERow : kCodeTileBytes;  // second half's code tile
     using C = Cfg<KH>;
     constexpr int MP = S::MP;
     constexpr int kStages = S::kStages;
@@ -588,7 +613,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
         // W2: 128 code bytes per row per stage; W4: 256, as two 128-byte boxes; (4,3,2): one 176-byte box
 #pragma unroll
         for (int bx = 0; bx < (W4 ? 2 : 1); ++bx) {
-            const int x = W275 ? st * kW275Row : st * (W4 ? 256 : 128) + bx * 128;
+            const int x = W275 ? st * kERow : st * (W4 ? 256 : 128) + bx * 128;
             tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes, &m.codes, bar, x, rowA);
             tma_load_2d(base + kCodeOff + bx * 2 * kCodeTileBytes + kCodeHalf, &m.codes, bar, x, rowB);
         }
@@ -747,9 +772,13 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     uint32_t w_row[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int r = 0; r < 4; ++r)
-        w_row[r] = kCodeOff + (uint32_t)(r >> 1) * (uint32_t)kW275Half + (uint32_t)(wrow + g + 8 * (r & 1)) * kW275Row;
+        w_row[r] = kCodeOff + (uint32_t)(r >> 1) * (uint32_t)kCodeHalf + (uint32_t)(wrow + g + 8 * (r & 1)) * kERow;
     const uint32_t w_ow = 4u * (uint32_t)tig, w_ob = 16u + (uint32_t)tig, w_oe = 20u + (tig == 3 ? 1u : 0u);
     const uint32_t w_she = tig < 3 ? 4u - 2u * (uint32_t)tig : 4u;
+    // hybrid: the extra pair's shifts in words 8-9 (word 8's states 2tig, 2tig+1; tig 3: its state 6 and
+    // word 9's state 0, at bit 16 + 13)
+    const uint32_t h_sha = tig == 0 ? 13u : tig == 1 ? 9u : tig == 2 ? 4u : 0u;
+    const uint32_t h_shb = tig == 0 ? 11u : tig == 1 ? 6u : tig == 2 ? 2u : 29u;
 
     bool ok = true;
     int it = 0, slot = 0, round = 0, cc = 0;  // iteration (over all units), ring slot and round, chunk count
@@ -802,17 +831,24 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                 group_w4<NT, G>(sb + coff[G], xs, gs, sc_row, kc, acc);
             });
         } else if (W275) {
-            // (4,3,2): all 8 groups of the stage; each group's scale comes with its codes.  Groups
+            // (4,3,2) / hybrid: all 8 groups of the stage; each group's scale comes with its codes.  Groups
             // beyond K read zero codes (scale 0) and zero activations and add nothing.
             const uint32_t xs = sb + xa_thr, gs = sb + gs_thr;
             static_for<8>([&](auto Gc) {
                 constexpr int G = decltype(Gc)::value;
                 uint32_t RA0[8], RA1[8], RB0[8], RB1[8];
                 float sc[4];
-                decode_w275_row<G>(sb + w_row[0], w_ow, w_ob, w_oe, w_she, sc_row[0], RA0, sc[0]);
-                decode_w275_row<G>(sb + w_row[1], w_ow, w_ob, w_oe, w_she, sc_row[1], RA1, sc[1]);
-                decode_w275_row<G>(sb + w_row[2], w_ow, w_ob, w_oe, w_she, sc_row[2], RB0, sc[2]);
-                decode_w275_row<G>(sb + w_row[3], w_ow, w_ob, w_oe, w_she, sc_row[3], RB1, sc[3]);
+                if constexpr (EMBK == 1) {
+                    decode_w275_row<G>(sb + w_row[0], w_ow, w_ob, w_oe, w_she, sc_row[0], RA0, sc[0]);
+                    decode_w275_row<G>(sb + w_row[1], w_ow, w_ob, w_oe, w_she, sc_row[1], RA1, sc[1]);
+                    decode_w275_row<G>(sb + w_row[2], w_ow, w_ob, w_oe, w_she, sc_row[2], RB0, sc[2]);
+                    decode_w275_row<G>(sb + w_row[3], w_ow, w_ob, w_oe, w_she, sc_row[3], RB1, sc[3]);
+                } else {
+                    decode_hyb_row<G>(sb + w_row[0], w_ow, h_sha, h_shb, sc_row[0], RA0, sc[0]);
+                    decode_hyb_row<G>(sb + w_row[1], w_ow, h_sha, h_shb, sc_row[1], RA1, sc[1]);
+                    decode_hyb_row<G>(sb + w_row[2], w_ow, h_sha, h_shb, sc_row[2], RB0, sc[2]);
+                    decode_hyb_row<G>(sb + w_row[3], w_ow, h_sha, h_shb, sc_row[3], RB1, sc[3]);
+                }
                 group_mma<NT, G>(RA0, RA1, RB0, RB1, xs, gs, sc, acc);
             });
         } else if (TMA_SC || Q4) {
@@ -927,13 +963,8 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                     const uint16_t hb = float_to_bf16_bits(h);
                     reinterpret_cast<uint16_t *>(pq.out)[xa_index_perm(pr, (size_t)r, (size_t)pq.h_P, pq.h_perm)] = hb;
                     if constexpr (FUSED) {
-                        // (4,3,2) down weight: each column carries its own level offset
-                        float lw = 1.0f;
-                        if (pq.h_perm) {
-                            int li, lt, lb;
-                            w275_pos(r & 63, li, lt, lb);
-                            lw = w275_level(li, lb);
-                        }
+                        // (4,3,2) or hybrid down weight: each column carries its own level offset
+                        const float lw = pq.h_perm ? perm_level(pq.h_perm, r & 63) : 1.0f;
                         hsum[n][q & 1] += lw * bf16_bits_to_float(hb);
                     }
                     continue;
@@ -1054,10 +1085,11 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
             smem = Smem<NT, true>::kTotal;
         }
     }
-    if (p.emb == 1) {
-        kern = decode_gemm_w2_kernel<NT, false, false, false, false, false, 1, true>;
+    if (p.emb == 1 || p.emb == 2) {
+        kern = p.emb == 1 ? decode_gemm_w2_kernel<NT, false, false, false, false, false, 1, 1>
+                          : decode_gemm_w2_kernel<NT, false, false, false, false, false, 1, 2>;
         kh = 1;
-        smem = Smem<NT, false, false, true>::kTotal;
+        smem = p.emb == 1 ? Smem<NT, false, false, 1>::kTotal : Smem<NT, false, false, 2>::kTotal;
     } else if (!p.w4 && p.std2) {
         kern = p.tma_scales ? decode_gemm_w2_kernel<NT, true, false, false, false, true, kFastKH>
                             : decode_gemm_w2_kernel<NT, false, false, false, false, true>;
@@ -1092,12 +1124,14 @@ template <int NT>
 cudaError_t launch_fused_nt(const DecodeGemmParams &p1, const MapSet &m1, int row_blocks1, const DecodeGemmParams &p2,
                             const MapSet &m2, int row_blocks2, int experts, cudaStream_t s) {
     // fp32 group scales staged by TMA, or 4-bit scales read by the consumers (both projections alike)
-    DecodeKernel kern = p1.emb == 1 ? decode_gemm_w2_kernel<NT, false, false, true, false, false, 1, true>
+    DecodeKernel kern = p1.emb == 1 ? decode_gemm_w2_kernel<NT, false, false, true, false, false, 1, 1>
+                        : p1.emb == 2 ? decode_gemm_w2_kernel<NT, false, false, true, false, false, 1, 2>
                         : p1.q4     ? decode_gemm_w2_kernel<NT, false, false, true, true, false, 1>
                         : p1.std2   ? decode_gemm_w2_kernel<NT, true, false, true, false, true, kFastKH>
                                     : decode_gemm_w2_kernel<NT, true, false, true, false, false, kFastKH>;
-    const int kh = (p1.q4 || p1.emb == 1) ? 1 : kFastKH;
-    const int smem = p1.emb == 1 ? Smem<NT, false, false, true>::kTotal
+    const int kh = (p1.q4 || p1.emb) ? 1 : kFastKH;
+    const int smem = p1.emb == 1 ? Smem<NT, false, false, 1>::kTotal
+                     : p1.emb == 2 ? Smem<NT, false, false, 2>::kTotal
                      : p1.q4     ? Smem<NT, false, true>::kTotal
                                  : Smem<NT, false>::kTotal;
     int per_sm = 0;
@@ -1146,7 +1180,7 @@ cudaError_t launch_decode_moe_fused(const DecodeGemmParams &p1, const CUtensorMa
                                     const CUtensorMap &c2, const CUtensorMap &d2, int row_blocks2, int experts,
                                     int nt, cudaStream_t s) {
     const bool fp32_sc = !p1.q4 && !p2.q4 && p1.tma_scales && p2.tma_scales, q4_sc = p1.q4 && p2.q4;
-    const bool emb_both = p1.emb == 1 && p2.emb == 1;
+    const bool emb_both = p1.emb != 0 && p1.emb == p2.emb;
     if (p1.w4 || p2.w4 || !(fp32_sc || q4_sc || emb_both) || p1.std2 != p2.std2 || p1.emb != p2.emb ||
         (q4_sc && p1.std2) || p1.mode != EPI_GATEUP || p2.mode != EPI_DOWN ||
         !p1.dep || !p2.dep || !p1.fuse_gsq)

@@ -87,12 +87,46 @@ __host__ __device__ inline float w275_level(int i, int b) {
     const int slot = i < 3 ? i : (b < 3 ? b : 0);  // 0: T = 0, 1: T = 2, 2: T = 3
     return slot == 0 ? -136.0f : slot == 1 ? -40.0f : -24.0f;
 }
+// Operand order of the hybrid (3,3,2)+(3,4,2) format (CCQ_FMT_W25_HYBRID).  A group is ten 16-bit
+// words; word j < 9 holds weights 7j + s for its states s = 0..6 (shifts 13, 11, 9, 6, 4, 2, 0).
+// Thread tig decodes words 2tig (low half of one 32-bit load) and 2tig+1 (high half): register
+// k = 0..6 pairs the two words' state k, as (slice k/2, elements 2 (k mod 2), +1); register 7 holds
+// two more states: word 8's states 2tig, 2tig+1 (tig < 3), or word 8's state 6 and word 9's (weight
+// 63) for tig 3.  States reach the tensor core as 2^(7-T) + u (T = 4 for states 0-4, 2 for state 5,
+// 0 for state 6 and the extra pair), so L = -(2^(7-T) + 4) = -12, -36, -132.
+__host__ __device__ inline void hyb_pos(int w, int &i, int &tig, int &b) {
+    if (w >= 56) {
+        i = 3;
+        tig = (w - 56) >> 1;
+        b = 2 + (w & 1);
+        return;
+    }
+    const int j = w / 7, st = w % 7;
+    tig = j >> 1;
+    i = st >> 1;
+    b = (st & 1) * 2 + (j & 1);
+}
+__host__ __device__ inline float hyb_level(int i, int b) {
+    const int k = 2 * i + (b >> 1);  // register index
+    return k <= 4 ? -12.0f : k == 5 ? -36.0f : -132.0f;
+}
+// Position (slice, thread, element) and level offset of group column w under operand order perm
+// (1: (4,3,2), 2: hybrid).
+__host__ __device__ inline void perm_pos(int perm, int w, int &i, int &tig, int &b) {
+    if (perm == 1) w275_pos(w, i, tig, b);
+    else hyb_pos(w, i, tig, b);
+}
+__host__ __device__ inline float perm_level(int perm, int w) {
+    int i, tig, b;
+    perm_pos(perm, w, i, tig, b);
+    return perm == 1 ? w275_level(i, b) : hyb_level(i, b);
+}
 // The decode-sized operand position of element (p, k): perm 0 = the CCQ / STD / W4 order (xa_index),
-// perm 1 = the (4,3,2) order above.
+// 1 = the (4,3,2) order, 2 = the hybrid order.
 __host__ __device__ inline size_t xa_index_perm(size_t p, size_t k, size_t P, int perm) {
     if (perm == 0) return xa_index(p, k, P);
     int i, tig, b;
-    w275_pos((int)(k & 63), i, tig, b);
+    perm_pos(perm, (int)(k & 63), i, tig, b);
     return (((((k >> 6) * 4 + (size_t)i) * P + p) * 4 + (size_t)tig) * 4 + (size_t)b);
 }
 // The decoders hand the tensor core BF16 (128 + u) for CCQ state u (weight level u - 32),
@@ -131,7 +165,7 @@ struct DecodeGemmParams {
     const uint8_t *scale_q4;   // [rows_total][K/128]
     const float *super_scale;  // [rows_total]
     int std2;                  // 1: WINT2-Standard plain 2-bit fields (no alpha/beta)
-    int emb;                   // 1: the (4,3,2) format (codes with the scale inside; super_scale per row)
+    int emb;                   // 1 / 2: the (4,3,2) / hybrid format (codes with the scale inside; super_scale per row)
     int h_perm;                // EPI_GATEUP: operand order of h for the down projection (xa_index_perm)
     uint32_t *err;
     // work units (set by the launcher): unit u = (expert, k split, row block), row block fastest
@@ -223,7 +257,7 @@ cudaError_t launch_quantize_std(const float *w, int rows, int K, uint8_t *codes,
 
 // x (BF16 [rows][K], row r taken from x[tok_of ? tok_of[p] : p]) -> XA operand + group sums.
 // zero_ctr (may be NULL): an int the kernel sets to 0 (the following matmul's work counter).
-// perm: operand order (xa_index_perm); perm 1 sums L(k) x_k per group and ignores `level`.
+// perm: operand order (xa_index_perm); perms 1 and 2 sum L(k) x_k per group and ignore `level`.
 cudaError_t launch_pack_xa(const uint16_t *x, const int *tok_of, int P_valid, int P, int K, float level,
                            uint16_t *xa, float *gsq, cudaStream_t s, int *zero_ctr = nullptr, int perm = 0);
 // group-sum table of an operand already in XA layout (rows [0, P_valid))
