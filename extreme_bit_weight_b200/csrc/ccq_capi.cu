@@ -184,11 +184,8 @@ struct GemmWs {
 };
 
 // Small-token tiles on the tcgen05 path (embedded-scale formats, at most 64 tokens per expert or
-// call): the tile width for a mean of `rows` tokens.
-inline int pick_sn(const ccq_weight *w, double rows) {
-    if (!emb_kind(w) || rows > 64.0) return 0;
-    return rows <= 16.0 ? 16 : rows <= 32.0 ? 32 : 64;
-}
+// call; fewer than 48 take the decode-sized kernel): 64 tokens on the MMA's N side.
+inline int pick_sn(const ccq_weight *w, double rows) { return (emb_kind(w) && rows <= 64.0) ? 64 : 0; }
 
 int sm_count() {
     static int n = 0;

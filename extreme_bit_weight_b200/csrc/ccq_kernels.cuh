@@ -225,7 +225,7 @@ struct TcGemmParams {
     // 1 / 2: the (4,3,2) / hybrid format with the group scale in the redundant bits (codes and
     // super_scale only)
     int emb;
-    // 0: token tiles of 128*mt tokens on the MMA's M side; 16, 32, 64: tiles of sn tokens on the N side
+    // 0: token tiles of 128*mt tokens on the MMA's M side; 64: tiles of 64 tokens on the N side
     // (m_tile == sn, mt == 1; the embedded-scale formats only); the activation map's box has sn rows
     int sn;
     uint32_t *err;

@@ -787,12 +787,8 @@ cudaError_t launch_tc_sn(const TcGemmParams &p, const CUtensorMap &ta, const CUt
 template <int EMB>
 cudaError_t launch_tc_sn_any(const TcGemmParams &p, const CUtensorMap &ta, const CUtensorMap &tc, int grid,
                              cudaStream_t s) {
-    switch (p.sn) {
-        case 16: return launch_tc_sn<EMB, 16>(p, ta, tc, grid, s);
-        case 32: return launch_tc_sn<EMB, 32>(p, ta, tc, grid, s);
-        case 64: return launch_tc_sn<EMB, 64>(p, ta, tc, grid, s);
-        default: return cudaErrorInvalidValue;
-    }
+    if (p.sn != 64) return cudaErrorInvalidValue;  // (the only width the dispatch uses)
+    return launch_tc_sn<EMB, 64>(p, ta, tc, grid, s);
 }
 
 template <int MT>

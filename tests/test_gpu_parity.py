@@ -675,9 +675,9 @@ def test_moe_emb_encoded_layer_matches_oracle(ccq, kind):
 
 
 @pytest.mark.parametrize("kind", [1, 2])
-@pytest.mark.parametrize("m", [17, 40, 64])
+@pytest.mark.parametrize("m", [17, 40, 48, 57, 64])
 def test_gemm_emb_small_token_tiles(ccq, kind, m):
-    # token tiles of 32 / 64 tokens on the MMA's N side, several tiles per call
+    # below 48 tokens the decode-sized kernel; 48-64: one 64-token tile on the tcgen05 kernel's N side
     n, k = 512, 1024
     codes, sup = synth.emb_format_random(kind, n, k, 9600 + m + kind)
     W = emb_weight(ccq, kind, codes, sup)
@@ -688,10 +688,10 @@ def test_gemm_emb_small_token_tiles(ccq, kind, m):
 
 
 @pytest.mark.parametrize("fmts", [("w275", "w275"), ("w25", "w25")])
-@pytest.mark.parametrize("T,zipf", [(48, False), (200, False), (120, True)])
+@pytest.mark.parametrize("T,zipf", [(48, False), (200, False), (240, True)])
 def test_moe_emb_small_token_tiles(ccq, fmts, T, zipf):
-    # 12 / 50 / 30 rows per expert on average: 16-, 64- and 32-token tiles, with experts that span
-    # several tiles (and, under Zipf routing, experts with none)
+    # 12 rows per expert on average (decode-sized kernel), 50 and 60 (64-token tiles on the tcgen05
+    # kernel's N side), with experts that span several tiles (and, under Zipf routing, experts with none)
     E, H, I, topk = 8, 1024, 512, 2
     W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 9700 + T + FMT_SEED[fmts[0]], *fmts)
     x = synth.activations(T, H, 9701 + T)
