@@ -469,7 +469,7 @@ template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false, bool STD = 
 __global__ void __launch_bounds__(Cfg<KH>::kThreads, 1)
 decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__ MapSet m2,
                       const __grid_constant__ DecodeGemmParams p, const __grid_constant__ DecodeGemmParams p2) {
-    static_assert(KH == 2 || (!W4 && (TMA_SC || Q4 || EMBK)), "one warp per row slot needs staged scales");
+    static_assert(KH == 2 || W4 || TMA_SC || Q4 || EMBK, "one warp per row slot needs staged scales");
     static_assert(!Q4 || (KH == 1 && !TMA_SC), "4-bit scales: expanded by the producer warpgroup");
     static_assert(!EMBK || (KH == 1 && !TMA_SC && !W4 && !Q4 && !STD), "embedded scales come with the codes");
     using S = Smem<NT, W4, Q4, EMBK>;
@@ -757,10 +757,11 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             // word tig of row wrow+g in 16-byte chunk (Gh+G) ^ g (128-byte swizzle)
             coff[G] = kCodeOff + (uint32_t)(wrow + g) * 128u + 4u * (uint32_t)tig + ((uint32_t)((Gh + G) ^ g) << 4);
         } else {
-            // 32 bytes per row and group: this thread's 8 bytes sit in chunk (2G + tig/2) ^ g of the
-            // 128-byte line of box khalf
-            coff[G] = kCodeOff + (uint32_t)khalf * (2u * kCodeTileBytes) + (uint32_t)(wrow + g) * 128u +
-                      8u * ((uint32_t)tig & 1u) + ((uint32_t)((2 * G + (tig >> 1)) ^ g) << 4);
+            // 32 bytes per row and group: this thread's 8 bytes sit in chunk (2G' + tig/2) ^ g of the
+            // 128-byte line of box khalf (KH 2; G' = G) or of box G/4 (KH 1; G' = G mod 4)
+            const int box = KH == 2 ? khalf : G >> 2, Gb = G & 3;
+            coff[G] = kCodeOff + (uint32_t)box * (2u * kCodeTileBytes) + (uint32_t)(wrow + g) * 128u +
+                      8u * ((uint32_t)tig & 1u) + ((uint32_t)((2 * Gb + (tig >> 1)) ^ g) << 4);
         }
     }
     const uint32_t xa_thr = kXaOff + (uint32_t)(Gh * 4 * MP * 32) + (uint32_t)g * 32u + (uint32_t)tig * 8u;
@@ -826,7 +827,7 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
         if (W4) {
             // per-channel scales; groups beyond K read TMA zero fill (activations 0) and add nothing
             const uint32_t xs = sb + xa_thr, gs = sb + gs_thr;
-            static_for<4>([&](auto Gc) {
+            static_for<kG>([&](auto Gc) {
                 constexpr int G = decltype(Gc)::value;
                 group_w4<NT, G>(sb + coff[G], xs, gs, sc_row, kc, acc);
             });
@@ -1062,8 +1063,9 @@ cudaError_t prepare_kernel(DecodeKernel kern, int smem, int *per_sm = nullptr) {
     return kernel_setup(reinterpret_cast<const void *>(kern), smem, Cfg<KH>::kThreads, Cfg<KH>::kLaunchRegs, per_sm);
 }
 
-// Consumer layout for the fp32-scale 2-bit kernels (CCQ and STD); 4-bit scales always take KH = 1 (their
-// expansion runs in the producer warpgroup), W4 and unstaged scales KH = 2.
+// Consumer layout for the fp32-scale 2-bit kernels (CCQ and STD); 4-bit scales, the embedded-scale
+// formats and W4 always take KH = 1; unstaged fp32 scales (rows whose scale pitch is not a multiple of
+// 16 bytes) KH = 2.
 constexpr int kFastKH = 1;
 
 int device_sms(cudaError_t &err) {
@@ -1081,7 +1083,8 @@ cudaError_t launch_nt(const DecodeGemmParams &p, const CUtensorMap &a, const CUt
     int smem = 0, kh = 2;
     if constexpr (NT <= 2) {  // W4 keeps at most 16 tokens per chunk (its code tiles are twice as wide)
         if (p.w4) {
-            kern = decode_gemm_w2_kernel<NT, false, true, false>;
+            kern = decode_gemm_w2_kernel<NT, false, true, false, false, false, 1>;
+            kh = 1;
             smem = Smem<NT, true>::kTotal;
         }
     }
