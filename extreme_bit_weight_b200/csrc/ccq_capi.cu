@@ -168,9 +168,14 @@ bool decode_maps(DecodeMaps &m, const ccq_weight *w, int experts, const uint16_t
     return true;
 }
 
-// Token counts above these run on the tcgen05 kernel (dense GEMM: m; MoE: mean rows per expert).
-constexpr int kTcMinM = 48;
-constexpr double kTcMinRowsPerExpert = 48.0;
+// Token counts from which the tcgen05 kernel runs (dense GEMM: m; MoE: mean rows per expert).  The
+// decode-sized kernel takes at most 32 tokens of an expert per pass over its weight, and it is
+// bound by the decode, so a second 32-token chunk costs a second full decode: a dense call of 33
+// to 47 tokens took 60 us against 39 us on the tcgen05 kernel (8192 x 8192), and a MoE layer with
+// 32 / 40 tokens per expert 2.27 / 2.83 ms against 1.84 / 1.86 ms.  With 24 tokens per expert
+// (few experts over 32) the decode-sized kernel still wins, 1.64 against about 1.83 ms.
+constexpr int kTcMinM = 33;
+constexpr double kTcMinRowsPerExpert = 28.0;
 // 128-token sub-tiles per tcgen05 tile: 1 while experts average at most 96 rows (a half-empty
 // 256-token tile would double the MMA time, which bounds the kernel there, and few experts spill
 // into a second 128-token tile), else 2 (a second tile would decode the weights again)
@@ -179,13 +184,8 @@ int tc_mt(double rows_per_expert) { return rows_per_expert > 96.0 ? 2 : 1; }
 struct GemmWs {
     size_t xa, gs, partial, xt, work, total;
     int P, ksplit, spp, row_blocks, nt;
-    int sn;  // tcgen05 path: small-token tile width (0: 128-token tiles)
     bool tc;
 };
-
-// Small-token tiles on the tcgen05 path (embedded-scale formats, at most 64 tokens per expert or
-// call; fewer than 48 take the decode-sized kernel): 64 tokens on the MMA's N side.
-inline int pick_sn(const ccq_weight *w, double rows) { return (emb_kind(w) && rows <= 64.0) ? 64 : 0; }
 
 int sm_count() {
     static int n = 0;
@@ -203,12 +203,11 @@ GemmWs gemm_layout(const ccq_weight *w, int m) {
         L.tc = true;
         L.P = m;
         L.xt = 0;
-        L.sn = pick_sn(w, (double)m);
         size_t off = up256((size_t)m * w->k * 2);
         // split-K when the (token tile, row tile) items cannot fill the SMs: ranges of kg groups
         // (a multiple of 4, one code stage), as many ranges as keep every item on its own SM
         const int nk = w->k / 64;
-        const int items = ceil_div(m, L.sn ? L.sn : 128 * tc_mt((double)m)) * ceil_div(w->n, 256);
+        const int items = ceil_div(m, 128 * tc_mt((double)m)) * ceil_div(w->n, 256);
         const int sms = sm_count();
         L.ksplit = 1;
         L.spp = nk;
@@ -255,8 +254,7 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     const int pairs = T * topk;
     L.P = (pairs + 3) & ~3;
     L.tc = (double)pairs / E >= kTcMinRowsPerExpert;
-    L.max_tiles = L.P / 16 + E + 1;  // enough for the smallest (16-token) tiles
-    // (the tile list is always laid out: the embedded-scale formats take the tcgen05 path at any size)
+    L.max_tiles = L.P / 128 + E + 1;  // (expert, 128-token tile) entries: at most one partial tile per expert
     size_t off = 0;
     L.err = off; off = up256(off + 16);
     L.seg = off; off = up256(off + sizeof(int) * (size_t)(E + 1));
@@ -280,14 +278,12 @@ MoeWs moe_layout(int T, int topk, int H, int I, int E) {
     return L;
 }
 
-// box_rows: token rows per activation load (128, or the small-token tile width)
-bool tc_maps(CUtensorMap &ta, CUtensorMap &tcodes, const ccq_weight *w, int experts, const uint16_t *a, int P,
-             int box_rows = 128) {
+bool tc_maps(CUtensorMap &ta, CUtensorMap &tcodes, const ccq_weight *w, int experts, const uint16_t *a, int P) {
     const int K = w->k;
     {
         cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)P};
         cuuint64_t str[1] = {(cuuint64_t)K * 2};
-        cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+        cuuint32_t box[2] = {64, 128};
         if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return false;
     }
@@ -368,16 +364,15 @@ ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, vo
         cudaError_t e = launch_pack_xt(static_cast<const uint16_t *>(x_bf16), nullptr, m, w->k, xt, s);
         if (e != cudaSuccess) return CCQ_ERR_CUDA;
         CUtensorMap ta, tcodes;
-        if (!tc_maps(ta, tcodes, w, 1, xt, m, L.sn ? L.sn : 128)) return CCQ_ERR_CUDA;
+        if (!tc_maps(ta, tcodes, w, 1, xt, m)) return CCQ_ERR_CUDA;
         TcGemmParams p{};
         p.N = w->n;
         p.K = w->k;
         p.row_block_stride = 256;
         p.half_stride = 128;
         p.n_tiles = ceil_div(w->n, 256);
-        const int mt = L.sn ? 1 : tc_mt((double)m);
-        p.sn = L.sn;
-        p.m_tile = L.sn ? L.sn : 128 * mt;
+        const int mt = tc_mt((double)m);
+        p.m_tile = 128 * mt;
         p.static_tiles = ceil_div(m, p.m_tile);
         p.M = m;
         p.out_ld = w->n;
@@ -498,18 +493,14 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         // prefill-sized: tcgen05 grouped GEMMs over (expert, 256-token tile) entries
         int2 *tiles = reinterpret_cast<int2 *>(base + L.tiles);
         int *tcount = reinterpret_cast<int *>(base + L.tcount);
-        // small-token tiles when both weights take them (one tile list serves both projections)
-        const double rows = (double)pairs / num_experts;
-        const int sn = (pick_sn(w13, rows) && pick_sn(w2, rows)) ? pick_sn(w13, rows) : 0;
-        const int mt = sn ? 1 : tc_mt(rows);
-        const int m_tile = sn ? sn : 128 * mt;
+        const int mt = tc_mt((double)pairs / num_experts);
+        const int m_tile = 128 * mt;
         e = launch_pack_xt(static_cast<const uint16_t *>(x_bf16), tok, pairs, H, xa_x, s);
         if (e == cudaSuccess) e = launch_build_tiles(seg, num_experts, m_tile, tiles, tcount, s);
         if (e == cudaSuccess) e = trace(events, 2, s);
         if (e != cudaSuccess) return CCQ_ERR_CUDA;
         CUtensorMap ta1, tc1, ta2, tc2;
-        if (!tc_maps(ta1, tc1, w13, num_experts, xa_x, L.P, sn ? sn : 128) ||
-            !tc_maps(ta2, tc2, w2, num_experts, xa_h, L.P, sn ? sn : 128))
+        if (!tc_maps(ta1, tc1, w13, num_experts, xa_x, L.P) || !tc_maps(ta2, tc2, w2, num_experts, xa_h, L.P))
             return CCQ_ERR_CUDA;
         TcGemmParams q1{};
         q1.N = w13->n;
@@ -520,7 +511,6 @@ ccq_status ccq_moe_w2a16_forward_traced(const ccq_weight *w13, const ccq_weight 
         q1.tile_list = tiles;
         q1.tile_count = tcount;
         q1.m_tile = m_tile;
-        q1.sn = sn;
         q1.seg_off = seg;
         q1.mode = EPI_GATEUP;
         q1.out = xa_h;

@@ -225,9 +225,6 @@ struct TcGemmParams {
     // 1 / 2: the (4,3,2) / hybrid format with the group scale in the redundant bits (codes and
     // super_scale only)
     int emb;
-    // 0: token tiles of 128*mt tokens on the MMA's M side; 64: tiles of 64 tokens on the N side
-    // (m_tile == sn, mt == 1; the embedded-scale formats only); the activation map's box has sn rows
-    int sn;
     uint32_t *err;
     // split-K (dense matmul with few tiles): ksplit > 1 splits the 64-column groups into ranges of
     // kg groups (a multiple of 4); each range writes EPI_PARTIAL_F32 sums at out + ks*out_split_stride

@@ -74,17 +74,12 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 // kind::f16 instruction descriptor: fp32 accumulate, BF16 A and B, both K-major, M=128, N=256.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
 
-// Small-token tiles ("SN" tokens on the N side): M=128 weight rows, N = SN tokens.
-template <int SN>
-constexpr uint32_t kIdescSN = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(SN >> 3) << 17) | ((128u >> 4) << 24);
-
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate,
-                                            uint32_t idesc = kIdesc) {
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+        "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -295,10 +290,7 @@ __device__ __forceinline__ bool tile_of(const TcGemmParams &p, int w, TileInfo &
 
 // STD: WINT2-Standard plain 2-bit fields (no per-row constants)
 // EMB: 1 = (4,3,2), 2 = hybrid (3,3,2)+(3,4,2), the formats with the scale in the redundant bits.
-// SN: 0 = token tiles of 128*MT tokens on the MMA's M side (weights on N, 256 wide); 16, 32 or 64 =
-// token tiles of SN tokens on the N side and the weight tile's two 128-row halves as two M=128
-// MMAs (MT = 1): at a few tokens per expert the tensor work then scales with the real tokens.
-template <int MT, bool W4, bool Q4 = false, bool STD = false, int EMB = 0, int SN = 0>
+template <int MT, bool W4, bool Q4 = false, bool STD = false, int EMB = 0>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_codes,
                   const TcGemmParams p) {
@@ -373,15 +365,10 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                     const int s = ra.slot;
                     if (ai >= kSA) ok = mbar_wait(&a_empty[s], ra.phase ^ 1u, p.err);
                     if (!ok) break;
-                    if constexpr (SN != 0) {
-                        mbar_arrive_expect_tx(&a_full[s], SN * 128);  // SN rows of 64 BF16
-                        tma_load_2d(sA + s * MT * kATile, &tm_a, &a_full[s], ks * 64, t.seg0 + t.m0);
-                    } else {
-                        mbar_arrive_expect_tx(&a_full[s], MT * kATile);
+                    mbar_arrive_expect_tx(&a_full[s], MT * kATile);
 #pragma unroll
-                        for (int j = 0; j < MT; ++j)
-                            tma_load_2d(sA + (s * MT + j) * kATile, &tm_a, &a_full[s], ks * 64, t.seg0 + t.m0 + j * 128);
-                    }
+                    for (int j = 0; j < MT; ++j)
+                        tma_load_2d(sA + (s * MT + j) * kATile, &tm_a, &a_full[s], ks * 64, t.seg0 + t.m0 + j * 128);
                     ++ai;
                     ra.advance();
                 }
@@ -410,29 +397,14 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                     ok = mbar_wait(&a_full[sa], ra.phase, p.err) && mbar_wait(&b_full[sb], rb.phase, p.err);
                     if (!ok) break;
                     tc_fence_after();
-                    if constexpr (SN != 0) {
-                        // weights (two 128-row halves) as A, the SN tokens as B: D columns [0, SN) hold
-                        // the first half's rows, [SN, 2 SN) the second's
-                        const uint32_t abase = smem_u32(sA + sa * MT * kATile);
+#pragma unroll
+                    for (int j = 0; j < MT; ++j) {
+                        const uint32_t abase = smem_u32(sA + (sa * MT + j) * kATile);
                         const uint32_t bbase = smem_u32(sB + sb * kBTile);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t acc = (ks > t.g0 || kk > 0) ? 1u : 0u;
-                            mma_bf16_ss(tmem, smem_desc_sw128(bbase + kk * 32), smem_desc_sw128(abase + kk * 32), acc,
-                                        kIdescSN<SN>);
-                            mma_bf16_ss(tmem + SN, smem_desc_sw128(bbase + 128 * 128 + kk * 32),
-                                        smem_desc_sw128(abase + kk * 32), acc, kIdescSN<SN>);
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < MT; ++j) {
-                            const uint32_t abase = smem_u32(sA + (sa * MT + j) * kATile);
-                            const uint32_t bbase = smem_u32(sB + sb * kBTile);
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_bf16_ss(tmem + j * 256, smem_desc_sw128(abase + kk * 32),
-                                            smem_desc_sw128(bbase + kk * 32), (ks > t.g0 || kk > 0) ? 1u : 0u);
-                        }
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16_ss(tmem + j * 256, smem_desc_sw128(abase + kk * 32),
+                                        smem_desc_sw128(bbase + kk * 32), (ks > t.g0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(&a_empty[sa]);
                     mma_commit(&b_empty[sb]);
@@ -612,48 +584,8 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             if (!ok) break;
             tc_fence_after();
             const int localA = t.nt * p.row_block_stride;
-            if constexpr (SN != 0) {
-                // TMEM lane = weight row rr of each 128-row half; column = token (second half at +SN)
-                const int rr = q * 32 + lane;
-                const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16);
-                const bool f32 = p.mode == EPI_DOWN || p.mode == EPI_PARTIAL_F32;
-                float *fout = static_cast<float *>(p.out) +
-                              (p.mode == EPI_PARTIAL_F32 ? (size_t)t.ks * p.out_split_stride : 0);
-                uint16_t *hout = static_cast<uint16_t *>(p.out);
 #pragma unroll 1
-                for (int c = 0; c < SN; c += 16) {
-                    uint32_t v0[16], v1[16];
-                    tmem_ld16(tb + c, v0);
-                    tmem_ld16(tb + SN + c, v1);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int z = 0; z < 16; ++z) {
-                        const int tok = t.m0 + c + z;
-                        if (tok >= t.Me) break;
-                        const size_t prow = (size_t)(t.seg0 + tok);
-                        if (p.mode == EPI_GATEUP) {
-                            // h in the operand's column order: column x at 16 (x / 16) + perm16(x mod 16)
-                            const int r = localA + rr;
-                            if (r < p.I) {
-                                const float h = silu(__uint_as_float(v0[z])) * __uint_as_float(v1[z]);
-                                hout[prow * p.out_ld + (r & ~15) + perm16(r & 15)] = float_to_bf16_bits(h);
-                            }
-                            continue;
-                        }
-                        const float rwv = p.mode == EPI_DOWN ? __ldg(p.rw + prow) : 1.0f;
-#pragma unroll
-                        for (int hf = 0; hf < 2; ++hf) {
-                            const int row = localA + hf * p.half_stride + rr;
-                            if (row >= p.N) continue;
-                            const float v = __uint_as_float(hf ? v1[z] : v0[z]);
-                            if (f32) fout[prow * p.out_ld + row] = rwv * v;
-                            else hout[prow * p.out_ld + row] = float_to_bf16_bits(v);
-                        }
-                    }
-                }
-            }
-#pragma unroll 1
-            for (int j = 0; j < (SN ? 0 : MT); ++j) {
+            for (int j = 0; j < MT; ++j) {
                 const int tok = t.m0 + j * 128 + m;
                 const bool live = tok < t.Me;
                 const size_t prow = (size_t)(t.seg0 + tok);
@@ -774,23 +706,6 @@ __global__ void pack_xt_kernel(const uint16_t *__restrict__ x, const int *__rest
     }
 }
 
-template <int EMB, int SN>
-cudaError_t launch_tc_sn(const TcGemmParams &p, const CUtensorMap &ta, const CUtensorMap &tc, int grid, cudaStream_t s) {
-    auto kern = tc_gemm_w2_kernel<1, false, false, false, EMB, SN>;
-    const int smem = TcSmem<1, EMB>::kTotal;
-    cudaError_t err = kernel_setup(reinterpret_cast<const void *>(kern), smem, kTcThreads, 0, nullptr);
-    if (err != cudaSuccess) return err;
-    kern<<<grid, kTcThreads, smem, s>>>(ta, tc, p);
-    return cudaGetLastError();
-}
-
-template <int EMB>
-cudaError_t launch_tc_sn_any(const TcGemmParams &p, const CUtensorMap &ta, const CUtensorMap &tc, int grid,
-                             cudaStream_t s) {
-    if (p.sn != 64) return cudaErrorInvalidValue;  // (the only width the dispatch uses)
-    return launch_tc_sn<EMB, 64>(p, ta, tc, grid, s);
-}
-
 template <int MT>
 cudaError_t launch_tc_mt(const TcGemmParams &p, const CUtensorMap &ta, const CUtensorMap &tc, int grid, cudaStream_t s) {
     auto kern = p.emb == 1 ? tc_gemm_w2_kernel<MT, false, false, false, 1>
@@ -810,12 +725,6 @@ cudaError_t launch_tc_mt(const TcGemmParams &p, const CUtensorMap &ta, const CUt
 
 cudaError_t launch_tc_gemm_w2(const TcGemmParams &p, const CUtensorMap &tm_a, const CUtensorMap &tm_codes, int mt,
                               int grid, cudaStream_t s) {
-    if (p.sn) {  // small-token tiles: the formats with the scale in the code stream only
-        if (mt != 1 || p.m_tile != p.sn) return cudaErrorInvalidValue;
-        if (p.emb == 1) return launch_tc_sn_any<1>(p, tm_a, tm_codes, grid, s);
-        if (p.emb == 2) return launch_tc_sn_any<2>(p, tm_a, tm_codes, grid, s);
-        return cudaErrorInvalidValue;
-    }
     if (mt == 1) return launch_tc_mt<1>(p, tm_a, tm_codes, grid, s);
     if (mt == 2) return launch_tc_mt<2>(p, tm_a, tm_codes, grid, s);
     return cudaErrorInvalidValue;

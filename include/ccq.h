@@ -85,7 +85,7 @@ typedef enum {
  *     63 in its top 3 bits and the 13-bit scale q in its low 13 bits.  Zero-point 4.  k must be a
  *     multiple of 256.
  *   Weight: w = bf16_rn((u - zp) * bf16_rn(fl32(q * super_scale[n]))).
- *   Every matmul with these formats runs on the tcgen05 kernel (any m).
+ *   They run on both matmul kernels, chosen by token count as for the other formats.
  */
 enum {
     CCQ_FMT_W2_CCQ_G64 = 1,
@@ -213,8 +213,8 @@ size_t ccq_gemm_workspace_size(const ccq_weight *w, int32_t m);
  *   x_bf16 (device) BF16 [m][k], 16-byte aligned;  m >= 0 (m == 0 is a no-op)
  *   y_bf16 (device) BF16 [m][n], 16-byte aligned
  *   ws     (device) workspace of ccq_gemm_workspace_size(w, m) bytes (may be NULL if that is 0)
- * Dispatch: small m runs the register-decode tensor-core kernel (decoded weights go straight into
- * mma operands in registers); large m runs the tcgen05/TMEM kernel (decoded weights go to shared
+ * Dispatch: m <= 32 runs the register-decode tensor-core kernel (decoded weights go straight into
+ * mma operands in registers); m >= 33 runs the tcgen05/TMEM kernel (decoded weights go to shared
  * memory tiles that the tensor core reads). */
 ccq_status ccq_w2a16_gemm(const ccq_weight *w, const void *x_bf16, int32_t m, void *y_bf16, void *ws,
                           size_t ws_bytes, ccq_stream_t stream);
@@ -252,7 +252,8 @@ size_t ccq_moe_workspace_size(int32_t T, int32_t topk, int32_t H, int32_t I, int
  *   expert_ids (device) int32 [T][topk], each in [0, E) and distinct within a token
  *   routing_w  (device) fp32 [T][topk], used as given (no renormalisation)
  *   ws         (device) workspace of ccq_moe_workspace_size(...) bytes
- * The formats may be mixed (w13 and w2 need not share a format). */
+ * The formats may be mixed (w13 and w2 need not share a format).  Dispatch by the mean rows per
+ * expert, T * topk / E: below 28 the register-decode kernel, from 28 the tcgen05 kernel. */
 ccq_status ccq_moe_w2a16_forward(const ccq_weight *w13, const ccq_weight *w2, int32_t num_experts,
                                  const void *x_bf16, int32_t T, const int32_t *expert_ids,
                                  const float *routing_w, int32_t topk, void *y_bf16, void *ws,

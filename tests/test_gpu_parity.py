@@ -98,7 +98,7 @@ def test_gemm_one_hot_identity_small_m(ccq):
 
 
 def test_gemm_one_hot_identity_tcgen05(ccq):
-    # x = I_K with K >= 48 rows runs the tcgen05 kernel: decoded BF16 weights in shared memory
+    # x = I_K with K >= 33 rows runs the tcgen05 kernel: decoded BF16 weights in shared memory
     n, k = 528, 576
     codes, scales, alpha, beta = synth.w2_format_random(n, k, 1401)
     W = w2_weight(ccq, codes, scales, alpha, beta)
@@ -167,7 +167,9 @@ def run_moe(ccq, W13, W2, x, ids, rw):
     return y.float().cpu().numpy(), st
 
 
-@pytest.mark.parametrize("T,E,topk", [(5, 8, 2), (40, 4, 1), (24, 16, 4)])
+# (104, 8, 2): 26 rows per expert, the decode-sized kernel with experts over one 32-token chunk;
+# (112, 8, 2): 28 rows per expert, the smallest MoE layer on the tcgen05 kernel
+@pytest.mark.parametrize("T,E,topk", [(5, 8, 2), (40, 4, 1), (24, 16, 4), (104, 8, 2), (112, 8, 2)])
 def test_moe_small_full(ccq, T, E, topk):
     H, I = 256, 128
     W13, W2, d13, d2 = moe_weights(ccq, E, H, I, 2000 + T)
@@ -255,7 +257,7 @@ def test_moe_decode_layer_full_size_sampled(ccq):
 @pytest.mark.parametrize("T,E,topk,H,I,zipf", [(256, 8, 2, 256, 128, False), (512, 16, 4, 1024, 512, True),
                                                (700, 4, 1, 576, 192, False)])
 def test_moe_prefill_full(ccq, T, E, topk, H, I, zipf):
-    # prefill-sized (>= 48 rows per expert on average): tcgen05 grouped GEMMs
+    # prefill-sized (>= 28 rows per expert on average): tcgen05 grouped GEMMs
     W13, W2, d13, d2 = moe_weights(ccq, E, H, I, 2400 + T)
     x = synth.activations(T, H, 2401 + T, outlier_frac=0.01)
     ids, rw = (synth.routing_zipf(T, E, topk, 2402 + T) if zipf else synth.routing_uniform(T, E, topk, 2402 + T))
@@ -575,7 +577,8 @@ def test_moe_std_quantized_layer_matches_oracle(ccq):
 
 # ----------------------------------------------------------------------------------------------
 # formats with the scale in the redundant bits (CCQ §3.5 Algorithm 2): (4,3,2) 2.75 bpw and
-# hybrid (3,3,2)+(3,4,2) 2.5 bpw; every matmul runs on the tcgen05 kernel
+# hybrid (3,3,2)+(3,4,2) 2.5 bpw; decode-sized token counts run the register-decode kernel, larger
+# ones the tcgen05 kernel
 # ----------------------------------------------------------------------------------------------
 def emb_weight(ccq, kind, codes, sup, experts=1):
     fmt = ccq.CCQ_FMT_W275_432 if kind == 1 else ccq.CCQ_FMT_W25_HYBRID
@@ -617,7 +620,7 @@ def test_gemm_emb_one_hot_identity(ccq, kind):
     W = emb_weight(ccq, kind, codes, sup)
     ref = oracle.bf16_to_f64(emb_oracle(kind, codes, sup)).T.astype(np.float32)
     eye = synth.one_hot_rows(k).cuda()
-    for j in range(0, 64, 16):  # small m: still the tcgen05 kernel
+    for j in range(0, 64, 16):  # 16 tokens: the register-decode kernel; all k rows: the tcgen05 kernel
         y = ccq.ccq_w2a16_gemm(W, eye[j:j + 16].contiguous()).float().cpu().numpy()
         assert np.array_equal(y, ref[j:j + 16]), j
     y = ccq.ccq_w2a16_gemm(W, eye).float().cpu().numpy()
@@ -655,7 +658,7 @@ def test_moe_emb_formats(ccq, fmts, T):
 
 @pytest.mark.parametrize("kind", [1, 2])
 def test_moe_emb_encoded_layer_matches_oracle(ccq, kind):
-    # weights through the device encoder, decode-sized token count (still the tcgen05 kernel)
+    # weights through the device encoder, decode-sized token count (the register-decode kernel)
     E, H, I, topk, T = 8, 1024, 512, 2, 16
     fmt = ccq.CCQ_FMT_W275_432 if kind == 1 else ccq.CCQ_FMT_W25_HYBRID
 
@@ -675,9 +678,9 @@ def test_moe_emb_encoded_layer_matches_oracle(ccq, kind):
 
 
 @pytest.mark.parametrize("kind", [1, 2])
-@pytest.mark.parametrize("m", [17, 40, 48, 57, 64])
-def test_gemm_emb_small_token_tiles(ccq, kind, m):
-    # below 48 tokens the decode-sized kernel; 48-64: one 64-token tile on the tcgen05 kernel's N side
+@pytest.mark.parametrize("m", [17, 32, 33, 40, 48, 57, 64])
+def test_gemm_emb_path_boundary(ccq, kind, m):
+    # up to 32 tokens the decode-sized kernel; from 33 one 128-token tile on the tcgen05 kernel
     n, k = 512, 1024
     codes, sup = synth.emb_format_random(kind, n, k, 9600 + m + kind)
     W = emb_weight(ccq, kind, codes, sup)
@@ -688,10 +691,11 @@ def test_gemm_emb_small_token_tiles(ccq, kind, m):
 
 
 @pytest.mark.parametrize("fmts", [("w275", "w275"), ("w25", "w25")])
-@pytest.mark.parametrize("T,zipf", [(48, False), (200, False), (240, True)])
-def test_moe_emb_small_token_tiles(ccq, fmts, T, zipf):
-    # 12 rows per expert on average (decode-sized kernel), 50 and 60 (64-token tiles on the tcgen05
-    # kernel's N side), with experts that span several tiles (and, under Zipf routing, experts with none)
+@pytest.mark.parametrize("T,zipf", [(48, False), (104, False), (112, False), (200, False), (240, True)])
+def test_moe_emb_path_boundary(ccq, fmts, T, zipf):
+    # 12 and 26 rows per expert on average (decode-sized kernel, some experts over one 32-token chunk
+    # at 26), 28, 50 and 60 (tcgen05 kernel), with experts that span several chunks (and, under Zipf
+    # routing, experts with none)
     E, H, I, topk = 8, 1024, 512, 2
     W13, W2, d13, d2 = moe_weights_fmt(ccq, E, H, I, 9700 + T + FMT_SEED[fmts[0]], *fmts)
     x = synth.activations(T, H, 9701 + T)
