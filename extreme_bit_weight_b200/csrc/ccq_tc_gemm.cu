@@ -34,11 +34,12 @@ namespace {
 constexpr int kDecWarps = 16;  // two threads per weight row of the 256-row tile
 constexpr int kEpiWarps = 4;
 constexpr int kTcThreads = (2 + kDecWarps + kEpiWarps) * 32;  // 704
-// Ring depths.  Activation stages: 3 with 128-token tiles, 2 with 256-token tiles.  Decoded-weight
-// stages: as many as shared memory leaves (4 / 3; 3 with 128-token tiles of the embedded-scale
-// formats, whose code ring is wider), so that the decoders can run ahead of the MMA.
-template <int MT>
-constexpr int kSAof = MT == 1 ? 3 : 2;
+// Ring depths.  Activation stages: 4 with 128-token tiles, 3 with 256-token tiles (2 for the
+// embedded-scale formats, whose code ring is wider), so that enough activation loads are in flight
+// to cover their latency.  Decoded-weight stages: 4 / 3 (3 with 128-token tiles of the
+// embedded-scale formats), so that the decoders can run ahead of the MMA.
+template <int MT, int EMB>
+constexpr int kSAof = MT == 1 ? 4 : (EMB ? 2 : 3);
 template <int MT, int EMB>
 constexpr int kSBof = MT == 1 ? (EMB ? 3 : 4) : 3;
 constexpr int kSC = 2;   // code stages (4 groups each)
@@ -55,7 +56,7 @@ constexpr int kCTileOf = 2 * 128 * kCRowOf<EMB>;  // two 128-row halves
 
 template <int MT, int EMB = 0>
 struct TcSmem {
-    static constexpr int kA = kSAof<MT> * MT * kATile;
+    static constexpr int kA = kSAof<MT, EMB> * MT * kATile;
     static constexpr int kB = kSBof<MT, EMB> * kBTile;
     static constexpr int kC = kSC * kCTileOf<EMB>;
     static constexpr int kTotal = kA + kB + kC + 1024;
@@ -297,7 +298,7 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     using S = TcSmem<MT, EMB>;
     constexpr int kCRow = kCRowOf<EMB>;
     constexpr int kCTile = kCTileOf<EMB>;
-    constexpr int kSA = kSAof<MT>;
+    constexpr int kSA = kSAof<MT, EMB>;
     constexpr int kSB = kSBof<MT, EMB>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned start, kept as an offset from the shared array so that loads and stores
