@@ -119,8 +119,9 @@ def test_gemm_small_linear(ccq):
     assert e <= 4e-3  # fp32 accumulation + one BF16 output rounding
 
 
+# m = 32: the largest call on the decode-sized kernel (one 32-token chunk); 33: the smallest on tcgen05
 @pytest.mark.parametrize("m,n,k", [(1, 16, 64), (3, 48, 192), (8, 256, 512), (9, 272, 576), (17, 128, 1088),
-                                   (33, 256, 1024), (1, 8192, 8192), (16, 8192, 8192),
+                                   (32, 256, 1024), (33, 256, 1024), (1, 8192, 8192), (16, 8192, 8192),
                                    (48, 256, 256), (130, 272, 576), (300, 512, 1088), (128, 8192, 8192)])
 def test_gemm_shapes(ccq, m, n, k):
     codes, scales, alpha, beta = synth.w2_format_random(n, k, 1500 + m + n + k)
