@@ -129,20 +129,27 @@ __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t e) {
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(m), "r"(e));
     return d;
 }
+// (a & m) | E, E an immediate: the logic op reads two registers
+template <uint32_t E>
+__device__ __forceinline__ uint32_t and_or_e(uint32_t a, uint32_t m) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(m), "n"(E));
+    return d;
+}
 
 struct RowDecode {
     uint64_t ab;    // {alpha, alpha}: code scale of the row
     uint64_t bb;    // {beta, beta}: code zero-point of the row
 };
 
-// The constants of the decode, held in registers: the integer multiply stays a multiply and the
-// window mask/exponent pair feeds one three-input logic op.
+// The constants of the decode, held in registers: the integer multiply stays a multiply, and the
+// window mask is the logic op's register operand while the BF16 exponent pattern is its immediate
+// (a logic op that reads three registers, mask and exponent both in registers, was 2-3% slower).
 struct DecodeConsts {
     uint64_t neg_magic;  // {-2^23, -2^23}: byte value from its 0x4B0000bb bit pattern
     uint64_t round_mag;  // {1.5*2^23, 1.5*2^23 - 0x4B40}: round to integer; second byte pre-cancels
     uint32_t mul16;      // 65536
     uint32_t wmask;      // 0x003F003F: one 6-bit state window per 16-bit half
-    uint32_t wexp;       // 0x43004300: BF16 exponent of 128 in both halves
 };
 
 // Decode one 32-bit word (4 consecutive bytes of one row) into the eight BF16x2 registers
@@ -164,24 +171,25 @@ __device__ __forceinline__ void decode_word(uint32_t w, const RowDecode &rd, con
     uint32_t X01, X23;
     asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(X01) : "r"(r1), "r"(k.mul16), "r"(r0));
     asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(X23) : "r"(r3), "r"(k.mul16), "r"(r2));
-    R[0] = and_or(X01 >> 9, k.wmask, k.wexp);
-    R[1] = and_or(X23 >> 9, k.wmask, k.wexp);
-    R[2] = and_or(X01 >> 6, k.wmask, k.wexp);
-    R[3] = and_or(X23 >> 6, k.wmask, k.wexp);
-    R[4] = and_or(X01 >> 3, k.wmask, k.wexp);
-    R[5] = and_or(X23 >> 3, k.wmask, k.wexp);
-    R[6] = and_or(X01, k.wmask, k.wexp);
-    R[7] = and_or(X23, k.wmask, k.wexp);
+    R[0] = and_or_e<0x43004300u>(X01 >> 9, k.wmask);
+    R[1] = and_or_e<0x43004300u>(X23 >> 9, k.wmask);
+    R[2] = and_or_e<0x43004300u>(X01 >> 6, k.wmask);
+    R[3] = and_or_e<0x43004300u>(X23 >> 6, k.wmask);
+    R[4] = and_or_e<0x43004300u>(X01 >> 3, k.wmask);
+    R[5] = and_or_e<0x43004300u>(X23 >> 3, k.wmask);
+    R[6] = and_or_e<0x43004300u>(X01, k.wmask);
+    R[7] = and_or_e<0x43004300u>(X23, k.wmask);
 }
 
 // W4: one 32-bit word = 8 signed 4-bit codes (first of a pair in the low nibble).  Register i holds
 // codes i and i+4 as BF16 (128 + (q + 8)) -- the sign bit of each nibble flipped, OR-ed into the
 // exponent pattern of 128 -- so one shift and one three-input logic op per register.
-__device__ __forceinline__ void decode_word_w4(uint32_t w, uint32_t m4, uint32_t x4, uint32_t R[4]) {
-    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[0]) : "r"(w), "r"(m4), "r"(x4));
-    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[1]) : "r"(w >> 4), "r"(m4), "r"(x4));
-    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[2]) : "r"(w >> 8), "r"(m4), "r"(x4));
-    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[3]) : "r"(w >> 12), "r"(m4), "r"(x4));
+__device__ __forceinline__ void decode_word_w4(uint32_t w, uint32_t m4, uint32_t R[4]) {
+    constexpr uint32_t x4 = 0x43084308u;  // BF16 128 in both halves, and the nibble sign flip
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[0]) : "r"(w), "r"(m4), "n"(x4));
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[1]) : "r"(w >> 4), "r"(m4), "n"(x4));
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[2]) : "r"(w >> 8), "r"(m4), "n"(x4));
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(R[3]) : "r"(w >> 12), "r"(m4), "n"(x4));
 }
 
 // WINT2-Standard: one 32-bit word = 16 plain 2-bit fields (field i of byte j at bits 2i of the byte),
@@ -189,14 +197,14 @@ __device__ __forceinline__ void decode_word_w4(uint32_t w, uint32_t m4, uint32_t
 // byte3).  Bytes 0,1 and 2,3 are first spread into the two 16-bit halves of one register each.
 __device__ __forceinline__ void decode_word_std(uint32_t w, const DecodeConsts &k, uint32_t R[8]) {
     const uint32_t X01 = prmt(w, 0u, 0x4140u), X23 = prmt(w, 0u, 0x4342u);
-    R[0] = and_or(X01, k.wmask, k.wexp);
-    R[1] = and_or(X23, k.wmask, k.wexp);
-    R[2] = and_or(X01 >> 2, k.wmask, k.wexp);
-    R[3] = and_or(X23 >> 2, k.wmask, k.wexp);
-    R[4] = and_or(X01 >> 4, k.wmask, k.wexp);
-    R[5] = and_or(X23 >> 4, k.wmask, k.wexp);
-    R[6] = and_or(X01 >> 6, k.wmask, k.wexp);
-    R[7] = and_or(X23 >> 6, k.wmask, k.wexp);
+    R[0] = and_or_e<0x43004300u>(X01, k.wmask);
+    R[1] = and_or_e<0x43004300u>(X23, k.wmask);
+    R[2] = and_or_e<0x43004300u>(X01 >> 2, k.wmask);
+    R[3] = and_or_e<0x43004300u>(X23 >> 2, k.wmask);
+    R[4] = and_or_e<0x43004300u>(X01 >> 4, k.wmask);
+    R[5] = and_or_e<0x43004300u>(X23 >> 4, k.wmask);
+    R[6] = and_or_e<0x43004300u>(X01 >> 6, k.wmask);
+    R[7] = and_or_e<0x43004300u>(X23 >> 6, k.wmask);
 }
 
 __device__ __forceinline__ void mma_bf16(float *c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -321,9 +329,9 @@ __device__ __forceinline__ void group_w4(uint32_t ca, uint32_t xs, uint32_t gs, 
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         uint32_t t[4];
-        decode_word_w4(q[r].x, kc.wmask, kc.wexp, t);
+        decode_word_w4(q[r].x, kc.wmask, t);
         R[r][0] = t[0]; R[r][2] = t[1]; R[r][4] = t[2]; R[r][6] = t[3];
-        decode_word_w4(q[r].y, kc.wmask, kc.wexp, t);
+        decode_word_w4(q[r].y, kc.wmask, t);
         R[r][1] = t[0]; R[r][3] = t[1]; R[r][5] = t[2]; R[r][7] = t[3];
     }
     group_mma<NT, G>(R[0], R[1], R[2], R[3], xs, gs, sc, acc);
@@ -746,7 +754,6 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
     kc.mul16 = 65536u + opaque;
     // one state window / one nibble / one 2-bit field per half
     kc.wmask = (W4 ? 0x000F000Fu : STD ? 0x00030003u : 0x003F003Fu) ^ opaque;
-    kc.wexp = (W4 ? 0x43084308u : 0x43004300u) ^ opaque;   // BF16 128 (W4: and the nibble sign flip)
 
     // per-thread shared-memory offsets inside a stage, for this warp's groups Gh..Gh+kGroups-1
     constexpr int kG = C::kGroups;
