@@ -151,7 +151,16 @@ __device__ __forceinline__ uint64_t fpk2(float lo, float hi) { return pk2(__floa
 struct RowCodeParams {
     uint64_t ab, bb;         // {alpha, alpha}, {beta, beta}
     uint64_t neg, rnd;       // {-2^23, -2^23}; {1.5*2^23, 1.5*2^23 - 0x4B40} (second byte pre-cancels)
+    uint32_t mask;           // the state-window mask in a register (0x003F003F; STD: 0x00030003)
 };
+
+// (a & m) | E in one logic op: the mask m in a register, the exponent pattern E its immediate
+template <uint32_t E>
+__device__ __forceinline__ uint32_t and_or_e(uint32_t a, uint32_t m) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(m), "n"(E));
+    return d;
+}
 
 // One 4-byte word of a row -> 16 BF16 weights (u - 32) * s in window-major order, as 8 registers:
 // out[2i], out[2i+1] = window i of bytes (0,1) and (2,3).  Byte value, q*alpha + beta (one fp32
@@ -169,15 +178,16 @@ __device__ __forceinline__ void decode_word_bf16(uint32_t w, const RowCodeParams
     upk2(c23, r2, r3);
     const uint32_t X01 = r1 * 65536u + r0;
     const uint32_t X23 = r3 * 65536u + r2;
-    const uint32_t M = 0x003F003Fu, E = 0x43004300u, Z = 0x43204320u;  // Z = bf16x2(160, 160)
-    out[0] = bmul2(bsub2(((X01 >> 9) & M) | E, Z), s2);
-    out[1] = bmul2(bsub2(((X23 >> 9) & M) | E, Z), s2);
-    out[2] = bmul2(bsub2(((X01 >> 6) & M) | E, Z), s2);
-    out[3] = bmul2(bsub2(((X23 >> 6) & M) | E, Z), s2);
-    out[4] = bmul2(bsub2(((X01 >> 3) & M) | E, Z), s2);
-    out[5] = bmul2(bsub2(((X23 >> 3) & M) | E, Z), s2);
-    out[6] = bmul2(bsub2((X01 & M) | E, Z), s2);
-    out[7] = bmul2(bsub2((X23 & M) | E, Z), s2);
+    const uint32_t M = rp.mask, Z = 0x43204320u;  // Z = bf16x2(160, 160)
+    constexpr uint32_t E = 0x43004300u;
+    out[0] = bmul2(bsub2(and_or_e<E>(X01 >> 9, M), Z), s2);
+    out[1] = bmul2(bsub2(and_or_e<E>(X23 >> 9, M), Z), s2);
+    out[2] = bmul2(bsub2(and_or_e<E>(X01 >> 6, M), Z), s2);
+    out[3] = bmul2(bsub2(and_or_e<E>(X23 >> 6, M), Z), s2);
+    out[4] = bmul2(bsub2(and_or_e<E>(X01 >> 3, M), Z), s2);
+    out[5] = bmul2(bsub2(and_or_e<E>(X23 >> 3, M), Z), s2);
+    out[6] = bmul2(bsub2(and_or_e<E>(X01, M), Z), s2);
+    out[7] = bmul2(bsub2(and_or_e<E>(X23, M), Z), s2);
 }
 
 // W4: one word = 8 signed 4-bit codes (low nibble first).  out[i] = BF16 (q_i * s, q_{i+4} * s):
@@ -194,13 +204,13 @@ __device__ __forceinline__ void decode_word_w4_bf16(uint32_t w, uint32_t s2, uin
 
 // WINT2-Standard: one word = 16 plain 2-bit fields, in the same window-major order as a CCQ word:
 // out[2i], out[2i+1] = field i of bytes (0,1) and (2,3), each 128 + q minus 130 exactly, times s.
-__device__ __forceinline__ void decode_word_std_bf16(uint32_t w, uint32_t s2, uint32_t out[8]) {
+__device__ __forceinline__ void decode_word_std_bf16(uint32_t w, uint32_t M, uint32_t s2, uint32_t out[8]) {
     const uint32_t X01 = prmt(w, 0u, 0x4140u), X23 = prmt(w, 0u, 0x4342u);
-    const uint32_t M = 0x00030003u, E = 0x43004300u, Z = 0x43024302u;  // Z = bf16x2(130, 130)
+    const uint32_t Z = 0x43024302u;  // Z = bf16x2(130, 130)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        out[2 * i] = bmul2(bsub2(((X01 >> (2 * i)) & M) | E, Z), s2);
-        out[2 * i + 1] = bmul2(bsub2(((X23 >> (2 * i)) & M) | E, Z), s2);
+        out[2 * i] = bmul2(bsub2(and_or_e<0x43004300u>(X01 >> (2 * i), M), Z), s2);
+        out[2 * i + 1] = bmul2(bsub2(and_or_e<0x43004300u>(X23 >> (2 * i), M), Z), s2);
     }
 }
 
@@ -434,6 +444,8 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         RowCodeParams rp;
         rp.neg = fpk2(-8388608.0f, -8388608.0f);
         rp.rnd = fpk2(12582912.0f, 12582912.0f - 19264.0f);
+        // (an opaque zero keeps the mask in a register, so the logic op's immediate is the exponent)
+        rp.mask = (STD ? 0x00030003u : 0x003F003Fu) ^ (uint32_t)(p.K >> 30);
         for (int w = blockIdx.x; w < total_work && ok; w += gridDim.x) {
             TileInfo t;
             tile_of(p, w, t);
@@ -533,8 +545,8 @@ tc_gemm_w2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                     const float sc = bf16_bits_to_float(float_to_bf16_bits(sraw));
                     const uint32_t s2 = pack_bf16x2(sc, sc);
                     if constexpr (STD) {
-                        decode_word_std_bf16(q2w.x, s2, o[0]);
-                        decode_word_std_bf16(q2w.y, s2, o[1]);
+                        decode_word_std_bf16(q2w.x, rp.mask, s2, o[0]);
+                        decode_word_std_bf16(q2w.y, rp.mask, s2, o[1]);
                     } else {
                         decode_word_bf16(q2w.x, rp, s2, o[0]);
                         decode_word_bf16(q2w.y, rp, s2, o[1]);
