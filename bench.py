@@ -133,10 +133,10 @@ def tensor_peak():
 
 # DRAM bytes (read + write) per touched expert of the fused decode launch, from the ncu capture of
 # the same kernel on the 16-expert small case (profiles/decode_gemm_w2_moe_decode_T8_E16_full.md:
-# 457.8 MB over 16 experts); each expert's weights cost the same bytes at any expert count, so the
+# 459.4 MB over 16 experts); each expert's weights cost the same bytes at any expert count, so the
 # full workload's traffic is this times the touched experts.  Retake the capture (and update this
 # figure) whenever the kernel changes.
-FUSED_DECODE_DRAM_BYTES_PER_EXPERT = 457_765_888 / 16
+FUSED_DECODE_DRAM_BYTES_PER_EXPERT = 459_449_856 / 16
 
 
 def config_dict():
