@@ -2,16 +2,18 @@
 // the small-M grouped GEMM of Table 5), sm_100a.
 //
 // Work unit = one expert x two 128-row halves of its weight x one k range (split-K) x all of the
-// expert's tokens (in chunks of 8*NT).  The kernel is persistent: CTA b takes units b,
-// b + gridDim.x, ... and one producer thread streams every 512-column stage of all of them through
-// one shared-memory ring (so the next unit's first stages load while the current unit finishes):
+// expert's tokens (in chunks of 8*NT).  The kernel is persistent: each CTA takes its next unit from
+// the launch's work counter (without one: units b, b + gridDim.x, ...), and one producer thread
+// streams every 512-column stage of all of them through one shared-memory ring (so the next unit's
+// first stages load while the current unit finishes):
 //   * the two halves' code bytes, [128 rows][128 B] each, by TMA with the 128-byte swizzle;
 //   * their group scales, the activation operand slice in the XA layout (see ccq_kernels.cuh)
 //     and its gsq group-sum table;
 //   * with a unit's first stage, the unit's per-row alpha/beta (or W4 channel scales).
-// Sixteen consumer warps decode the bytes in registers and feed them straight into
-// mma.sync.m16n8k16 (BF16 in, fp32 accumulate) as the A operand -- weights on the M side, tokens
-// on the N side -- so no decoded weight is ever written to memory.  The producer warpgroup gives
+// Eight consumer warps, one per 16-row slot of both halves (sixteen, two per slot splitting a stage's
+// groups, when the scale rows cannot be staged by TMA), decode the bytes in registers and feed them
+// straight into mma.sync.m16n8k16 (BF16 in, fp32 accumulate) as the A operand -- weights on the M
+// side, tokens on the N side -- so no decoded weight is ever written to memory.  The producer warpgroup gives
 // its registers to the consumer warpgroups (setmaxnreg), so the issue work never slows a consumer.
 //
 // Decode (CCQ §3.3 Eq. 1 inverted and §3.5 Algorithm 3, Table 1 row (6,4,3)):
@@ -467,11 +469,12 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
     return v;
 }
 
-// Persistent: CTA b walks units b, b + gridDim.x, ...; its producer streams every stage of every
-// unit through one ring, so the next unit's first stages load while this unit finishes.
+// Persistent: each CTA takes units from the work counter (or walks units b, b + gridDim.x, ...); its
+// producer streams every stage of every unit through one ring, so the next unit's first stages load
+// while this unit finishes.
 // FUSED: the launch holds the MoE gate/up units (p, m1) followed by the down units (p2, m2).
-// STD: WINT2-Standard plain 2-bit fields (no per-row constants).  KH: consumer layout (Cfg; KH = 1
-// only with TMA-staged fp32 scales).
+// STD: WINT2-Standard plain 2-bit fields (no per-row constants).  KH: consumer layout (Cfg; KH = 2
+// only for fp32 scales that TMA does not stage).  EMBK: 1 / 2 = the (4,3,2) / hybrid formats.
 template <int NT, bool TMA_SC, bool W4, bool FUSED, bool Q4 = false, bool STD = false, int KH = 2,
           int EMBK = 0>
 __global__ void __launch_bounds__(Cfg<KH>::kThreads, 1)
