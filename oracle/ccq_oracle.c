@@ -112,10 +112,10 @@ int32_t oracle_cluster_code(uint8_t q, float code_scale, float code_zero)
  * W2 dequantization, (L,N,S) = (6,4,3) with code cluster, group size g, [CCQ] §3.5 Algorithm 3
  * and Table 1 row (6,4,3).
  *
- * Layout ([WINT2] "4 weights packed into each INT8"; [CCQ] Algorithm 1 reshape to groups of
- * g/N vectors of N): codes[n][k/4], byte j of row n holds weights k = 4j .. 4j+3, one (6,4,3)
- * code of 4 states; scales[n][k/g]; code_scale[n], code_zero[n] per output channel (§3.3,
- * "along the dimension of output channels").
+ * Layout ([WINT2]: four weights per 8-bit storage element; [CCQ] Algorithm 1 reshape to groups
+ * of g/N vectors of N): codes[n][k/4], byte j of row n holds weights k = 4j .. 4j+3, one (6,4,3)
+ * code of 4 states; scales[n][k/g]; code_scale[n], code_zero[n] per output channel (§3.3
+ * clusters the codes channel by channel).
  *
  * Per weight: C = cluster code of the byte; the codebook row of C (reduced mod 2^15, since the
  * state windows only cover the low T bits) gives the 4 states u_0..u_3; the weight is
