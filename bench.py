@@ -297,7 +297,9 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # raw nvidia-smi samples; the JSON line carries their summary
+        log_dir = os.environ.get("CCQ_BENCH_LOG_DIR", os.path.join(ROOT, "bench_logs"))
+        self.path = os.path.join(log_dir, f"clocks_rank{gpu_index}.csv")
 
     def start(self):
         try:
