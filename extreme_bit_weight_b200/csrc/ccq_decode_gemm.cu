@@ -691,7 +691,8 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
             }
         } else if (Q4 && warp > C::kConsumerWarps) {
             // scale expanders: for each slot in ring order, the 4-bit scales of the stage's rows ->
-            // fp32 s = fl32(q4 * super[row]) in the [half][row][8 groups] layout the consumers read
+            // bf16(fl32(q4 * super[row])) as fp32 in the [half][row][8 groups] layout the consumers
+            // read (rounded here once per scale, so the consumers use them as they are)
             const int et = (warp - C::kConsumerWarps - 1) * 32 + lane;  // 0..95
             for (int j = 0;; ++j) {
                 const int slot = j % kStages;
@@ -726,8 +727,8 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                         float v[8];
 #pragma unroll
                         for (int b = 0; b < 4; ++b) {
-                            v[2 * b] = __fmul_rn((float)(bytes[k][b] & 0xFu), sup[k]);
-                            v[2 * b + 1] = __fmul_rn((float)(bytes[k][b] >> 4), sup[k]);
+                            v[2 * b] = round_bf16(__fmul_rn((float)(bytes[k][b] & 0xFu), sup[k]));
+                            v[2 * b + 1] = round_bf16(__fmul_rn((float)(bytes[k][b] >> 4), sup[k]));
                         }
                         float4 *dst = reinterpret_cast<float4 *>(sc + idx * 8);  // [half][row][8]
                         dst[0] = make_float4(v[0], v[1], v[2], v[3]);
@@ -880,7 +881,9 @@ decode_gemm_w2_kernel(const __grid_constant__ MapSet m1, const __grid_constant__
                 const float v2[4] = {s2.x, s2.y, s2.z, s2.w}, v3[4] = {s3.x, s3.y, s3.z, s3.w};
                 static_for<4>([&](auto Gc) {
                     constexpr int G = decltype(Gc)::value;
-                    const float sc[4] = {round_bf16(v0[G]), round_bf16(v1[G]), round_bf16(v2[G]), round_bf16(v3[G])};
+                    // (4-bit scales arrive rounded by the expanders)
+                    const float sc[4] = {Q4 ? v0[G] : round_bf16(v0[G]), Q4 ? v1[G] : round_bf16(v1[G]),
+                                         Q4 ? v2[G] : round_bf16(v2[G]), Q4 ? v3[G] : round_bf16(v3[G])};
                     group_w2<NT, G, STD>(sb + (coff[G] ^ cflip), xs, gs, sc, rd, kc, acc);
                 });
             };
