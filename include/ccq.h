@@ -264,7 +264,7 @@ ccq_status ccq_moe_w2a16_forward(const ccq_weight *w13, const ccq_weight *w2, in
  * [2] after activation packing, [3] after the gate/up kernel, [4] after the group-sum kernel,
  * [5] after the down kernel, [6] after the combine.  When the decode-sized path runs both
  * projections as one fused launch (the same 2-bit format on both: CCQ or STD with fp32 group-scale
- * rows a multiple of 16 bytes, or CCQ with 4-bit scales),
+ * rows a multiple of 16 bytes, CCQ with 4-bit scales, or the same (4,3,2) / hybrid format),
  * [3], [4] and [5] are all recorded after that launch.  `events` (host) holds
  * CCQ_MOE_TRACE_POINTS cudaEvent_t handles created by the caller (NULL: no events).  No paper
  * counterpart: a measurement hook. */
