@@ -103,10 +103,15 @@ def _np_ptr(a: np.ndarray):
 
 
 def _dptr(t):
+    """Device address of a tensor (None and raw integer addresses pass through).  A host tensor is
+    refused here: every pointer the library's compute entry points take is device memory, and the
+    C ABI cannot tell a host address from a device one without a driver query per call."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise CcqError(CCQ_ERR_INVALID_ARG, "host tensor passed where device memory is required")
     return t.data_ptr()
 
 
@@ -277,7 +282,7 @@ def ccq_w2a16_gemm(w: CcqWeight, x: torch.Tensor, y: torch.Tensor = None, ws: to
         y = torch.empty((m, w.n), dtype=torch.bfloat16, device=x.device)
     if ws is None:  # (a caller's workspace is size-checked by the library)
         ws = workspace(ccq_gemm_workspace_size(w, m), x.device)
-    _check(_lib.ccq_w2a16_gemm(w._ref, x.data_ptr(), m, y.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
+    _check(_lib.ccq_w2a16_gemm(w._ref, _dptr(x), m, _dptr(y), _dptr(ws), ws.numel(), _stream(stream)),
            "ccq_w2a16_gemm")
     return y
 

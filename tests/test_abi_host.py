@@ -149,3 +149,16 @@ def test_w4_quantizer_matches_oracle(ccq):
     c, s = ccq.ccq_quantize_w4_host(w, threads=3)
     oc, os_ = oracle.quantize_w4(w)
     assert np.array_equal(c, oc) and np.array_equal(s, os_)
+
+
+def test_binding_refuses_host_tensors(ccq):
+    # every compute entry point takes device memory; a host tensor is refused before any call
+    import torch
+
+    with pytest.raises(ccq.CcqError):
+        ccq.CcqWeight(ccq.CCQ_FMT_W2_CCQ_G64, 16, 64, np.zeros((16, 16), np.uint8), np.zeros((16, 1), np.float32),
+                      np.zeros(16, np.float32), np.zeros(16, np.float32), device="cpu")
+    with pytest.raises(ccq.CcqError):
+        ccq.ccq_check_device_error(torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ccq.CcqError):
+        ccq.ccq_selftest_bounded_wait(torch.zeros(256, dtype=torch.uint8), 0)
